@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Throughput of the block-quantised routed MoE layer on B200.
+
+One step = one forward (route, plan, gate/up + SwiGLU, down, combine) of each
+of L distinct synthetic layers on its own batch of T tokens, replayed as one
+CUDA graph.  The L layers' selected experts (L x ~23.7 MB for the
+model-shaped decode layer) are far larger than the 126 MB L2, so no step finds
+its weights in L2.  value = layer-tokens per second = K * L * T / time (max
+over ranks); the expert-weight GB/s and the roofline of the dominant kernel
+come from the same inputs.  Everything is seeded and synthetic (synth/).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+STAGES = ["route_plan", "gate_up", "down", "combine"]
+KERNEL_NAMES = {"route_plan": "route_kernel", "gate_up": "matvec_kernel<gate/up>",
+                "down": "matvec_kernel<down>", "combine": "combine_kernel"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="model_decode", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--layers", type=int, default=48, help="distinct layers per step")
+    ap.add_argument("--tokens", type=int, default=0, help="override tokens per layer")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="for profiler runs: few steps, no baselines")
+    return ap.parse_args()
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, index):
+        self.samples = []
+        self.stop_ev = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report it rather than guess
+            self.err = str(e)
+
+    def _run(self):
+        while not self.stop_ev.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop_ev.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"nvml unavailable: {self.err}"]}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = statistics.median(s[0] for s in self.samples)
+        seen = set()
+        for _, rs in self.samples:
+            for name, bit in self.REASONS.items():
+                if rs & bit:
+                    seen.add(name)
+        return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": sorted(seen),
+                "samples": len(self.samples)}
+
+
+def peaks():
+    try:
+        p = json.load(open(PEAKS_FILE))
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_traffic(stage, wl_name):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path)).get(f"{stage}:{wl_name}")
+    except Exception:
+        return None
+    if not rec:
+        return None
+    if rec.get("source_sha") != kernel_source_sha():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_quantized_expert_moe_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+
+def oracle_rate(li, wl, budget_s, max_s=30.0):
+    """Oracle layer-tokens/s on a bounded sample of the workload's tokens."""
+    import oracle
+    ex = oracle.Experts.from_layer(li)
+    done, spent, n, step = 0, 0.0, 4, 0
+    while spent < budget_s:
+        x = synth.tokens(wl, li.router, li.layer, 1000 + step, n)
+        t0 = time.perf_counter()
+        ex.layer(synth.tokens_f64(wl, x), li.router, wl.top_k)
+        dt = time.perf_counter() - t0
+        done += n
+        spent += dt
+        step += 1
+        rate = n / max(dt, 1e-9)
+        n = int(max(1, min(rate * (budget_s - spent), rate * (max_s - spent), 4096)))
+        if spent >= max_s or n < 1:
+            break
+    return done / spent, done, spent, oracle.threads()
+
+
+def reference_arm(a, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    li = synth.layer_inputs(wl, 0)
+    import oracle
+    ex = oracle.Experts.from_layer(li)
+    n = max(1, wl.tokens)
+    per_step = []
+    total_tok = 0
+    for s in range(a.warmup + a.steps):
+        x = synth.tokens(wl, li.router, 0, 2000 + s, n)
+        t0 = time.perf_counter()
+        ex.layer(synth.tokens_f64(wl, x), li.router, wl.top_k)
+        dt = time.perf_counter() - t0
+        if s >= a.warmup:
+            per_step.append(dt)
+            total_tok += n
+    secs = sum(per_step)
+    v = total_tok / secs
+    sample = f"{a.steps} steps x {n} tokens of layer 0 ({wl.name}), fp64 oracle"
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s",
+            "impl": "reference", "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "tokens_per_layer": n, "parallelism": "replicas"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+
+METRIC = "MoE layer tokens/s and expert-weight HBM GB/s (% of roofline), 1 B200"
+
+
+def _to_dev_x(x_np):
+    import torch
+    if x_np.dtype == np.uint16:
+        return torch.from_numpy(x_np.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x_np)).cuda()
+
+
+def ours_arm(a, wl):
+    import torch
+    import block_quantized_expert_moe_b200 as bq
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.cuda.current_device()
+    T = a.tokens or wl.tokens
+    L = a.layers
+    k = wl.top_k
+    H, E = wl.hidden, wl.n_experts
+    xbytes = 2 if wl.x_dtype == synth.DT_BF16 else 4
+
+    t0 = time.time()
+    layers = []
+    li0 = None
+    for l in range(L):
+        li = synth.layer_inputs(wl, l)
+        x = synth.tokens(wl, li.router, l, 0, T)
+        pack = bq.pack_layer(li, max_tokens=T, max_top_k=k, device=dev)
+        layers.append({"pack": pack, "x": _to_dev_x(x), "xh": x,
+                       "wr": torch.from_numpy(li.router.view(np.int16)).cuda(),
+                       "out": torch.empty(T, H, device="cuda")})
+        if l == 0:
+            li0 = li
+        del li
+    gen_s = time.time() - t0
+    log(f"[bench] rank {rank}: built {L} layers of {wl.name} in {gen_s:.1f} s")
+    info = layers[0]["pack"].info()
+
+    def fwd(ly):
+        bq.moe_layer_forward(ly["x"], ly["wr"], ly["pack"], bq.MOE_FMT_FROM_PACK, k, ly["out"])
+
+    # routing of every layer (deterministic): active experts and slots
+    n_active, slots = [], []
+    for ly in layers:
+        fwd(ly)
+        idx, gate, counts = bq.moe_read_routing(ly["pack"], T, k)
+        n_active.append(int((counts[:E] > 0).sum()) + (1 if wl.has_shared else 0))
+        slots.append(T * k + (T if wl.has_shared else 0))
+    torch.cuda.synchronize()
+    gu_b, dn_b = info["gate_up_bytes_per_expert"], info["down_bytes_per_expert"]
+    exp_b = info["expert_bytes"]
+    I = wl.inter
+    stage_bytes = {
+        "route_plan": [E * H * 2 + T * H * xbytes + 2 * T * E * 4 for _ in layers],
+        "gate_up": [na * gu_b + T * H * xbytes + s * I * 4 for na, s in zip(n_active, slots)],
+        "down": [na * dn_b + s * I * 4 + s * H * 4 for na, s in zip(n_active, slots)],
+        "combine": [s * H * 4 + T * H * 4 for s in slots],
+    }
+    unique_bytes_step = sum(na * exp_b + E * H * 2 for na in n_active)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- timed region: K replays of the one-step graph
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for ly in layers:
+            fwd(ly)
+    for _ in range(max(a.warmup, 3)):
+        g.replay()
+    barrier()
+    st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        st.record()
+        for _ in range(a.steps):
+            g.replay()
+        en.record()
+        en.synchronize()
+    ms = max_over_ranks(st.elapsed_time(en))
+    barrier()
+    value = world * a.steps * L * T / (ms / 1e3)
+    expert_gbs = world * a.steps * unique_bytes_step / (ms / 1e3) / 1e9
+
+    # ---- kernel-stage durations: the same work with event records around each kernel
+    kp = max(1, min(a.steps, 10))
+    for ly in layers:
+        bq.moe_profile_begin(ly["pack"], kp)
+    gp = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gp):
+        for _ in range(kp):
+            for ly in layers:
+                fwd(ly)
+    gp.replay()
+    torch.cuda.synchronize()
+    stage_ms = np.zeros(4)
+    nf = 0
+    for ly in layers:
+        m, n = bq.moe_profile_end(ly["pack"])
+        stage_ms += m
+        nf += n
+    stage_us = {s: float(stage_ms[i] / nf * 1e3) for i, s in enumerate(STAGES)}
+    dom = max(STAGES, key=lambda s: stage_us[s])
+    dom_bytes = float(np.mean(stage_bytes[dom]))
+    hbm, peak_src = peaks()
+    achieved = dom_bytes / (stage_us[dom] * 1e-6) / 1e9
+    traffic = kernel_traffic(dom, wl.name)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": traffic, "kernel": KERNEL_NAMES[dom],
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                else "fallback 6650 GB/s",
+                "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": stage_us[dom]}
+    del gp
+
+    # ---- end to end: pinned host input -> forward -> host output, every layer, every step
+    e2e = None
+    if not a.no_e2e:
+        xh = [torch.from_numpy(ly["xh"].view(np.int16) if ly["xh"].dtype == np.uint16 else ly["xh"]).pin_memory()
+              for ly in layers]
+        oh = [torch.empty(T, H, dtype=torch.float32).pin_memory() for _ in layers]
+        ge = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ge):
+            for ly, xin, o in zip(layers, xh, oh):
+                ly["x"].view(xin.dtype).copy_(xin, non_blocking=True)
+                fwd(ly)
+                o.copy_(ly["out"], non_blocking=True)
+        for _ in range(max(a.warmup, 3)):
+            ge.replay()
+        barrier()
+        st.record()
+        for _ in range(a.steps):
+            ge.replay()
+        en.record()
+        en.synchronize()
+        ems = max_over_ranks(st.elapsed_time(en))
+        barrier()
+        e2e = {"value": world * a.steps * L * T / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": L * T * H * xbytes, "d2h_bytes_per_step": L * T * H * 4,
+               "ms_per_step": ems / a.steps}
+        del ge
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and not a.quick:
+        v, n, secs, cores = oracle_rate(li0, wl, a.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} tokens of layer 0 ({wl.name}) in {secs:.1f} s, fp64 oracle, "
+                         f"OpenMP over tokens"}
+
+    del g
+    for ly in layers:
+        ly["pack"].free()
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": wl.name, "layers_per_step": L, "tokens_per_layer": T,
+                           "hidden": H, "experts": E, "inter": I, "top_k": k,
+                           "shared_expert": wl.has_shared,
+                           "formats": f"{synth.FMT_NAMES[wl.fmt_gate_up]}/{synth.FMT_NAMES[wl.fmt_down]}",
+                           "parallelism": f"replicas x{world}",
+                           "l2": f"inputs larger than L2: {L} distinct layers, "
+                                 f"{unique_bytes_step / 1e6:.0f} MB of selected expert weights per step"},
+                "expert_gbs": expert_gbs, "expert_gbs_frac": expert_gbs / hbm,
+                "unique_expert_bytes_per_step": unique_bytes_step,
+                "active_experts_per_layer": float(np.mean(n_active)),
+                "stage_us": stage_us, "roofline": roofline, "clocks": clk.summary(),
+                "e2e": e2e, "gpu_launches": 4 * L * a.steps, "cpu_baseline": cpu,
+                "gen_seconds": gen_s}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    a = parse()
+    wl = synth.WORKLOADS[a.workload]
+    if a.quick:
+        a.no_e2e = True
+        a.no_cpu_baseline = True
+    if a.impl == "reference":
+        reference_arm(a, wl)
+    else:
+        ours_arm(a, wl)
+
+
+if __name__ == "__main__":
+    main()

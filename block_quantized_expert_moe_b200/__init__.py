@@ -1,0 +1,241 @@
+"""Python binding of libmoe, the C-ABI library of the block-quantised routed
+MoE layer for B200 (include/moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  Device buffers are torch CUDA tensors (PyTorch provides memory and
+streams); weights enter as canonical blocks in host numpy arrays.  The library
+must be built (build.py, or __graft_entry__.build()); importing this module
+without it raises, there is no other implementation.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_FMT_MISMATCH = 0, 1, 2, 3
+MOE_ERR_OOM, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE = 4, 5, 6, 7
+MOE_FMT_FROM_PACK, MOE_FMT_Q8_0, MOE_FMT_Q5_1, MOE_FMT_IQ4_NL, MOE_FMT_NVFP4 = 0, 1, 2, 3, 4
+MOE_DT_F32, MOE_DT_BF16 = 1, 2
+MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_DENSE = 0, 1, 2, 3
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {moe_status_string(status)} ({status})")
+
+
+class moe_pack_desc(ctypes.Structure):
+    _fields_ = [("n_experts", ctypes.c_int), ("hidden", ctypes.c_int), ("inter", ctypes.c_int),
+                ("has_shared", ctypes.c_int), ("max_tokens", ctypes.c_int),
+                ("max_top_k", ctypes.c_int), ("fmt_gate_up", ctypes.c_int),
+                ("fmt_down", ctypes.c_int), ("gate_up_blocks", ctypes.c_void_p),
+                ("down_blocks", ctypes.c_void_p), ("gate_up_tensor_scale", ctypes.c_void_p),
+                ("down_tensor_scale", ctypes.c_void_p), ("iq4nl_table", ctypes.c_void_p),
+                ("shared_gate_up_blocks", ctypes.c_void_p),
+                ("shared_down_blocks", ctypes.c_void_p)]
+
+
+class moe_pack_info(ctypes.Structure):
+    _fields_ = [("gate_up_bytes_per_expert", ctypes.c_int64),
+                ("down_bytes_per_expert", ctypes.c_int64), ("expert_bytes", ctypes.c_int64),
+                ("arena_bytes", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64),
+                ("device", ctypes.c_int)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmoe.so is not built ({LIB_PATH}); run block_quantized_expert_moe_b200/build.py")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_status_string.argtypes = [i32]
+    L.moe_pack_experts.restype = i32
+    L.moe_pack_experts.argtypes = [ctypes.POINTER(moe_pack_desc), i32, ctypes.POINTER(vp)]
+    L.moe_pack_free.restype = i32
+    L.moe_pack_free.argtypes = [vp]
+    L.moe_pack_query.restype = i32
+    L.moe_pack_query.argtypes = [vp, ctypes.POINTER(moe_pack_info)]
+    L.moe_route_workspace_bytes.restype = sz
+    L.moe_route_workspace_bytes.argtypes = [i32, i32]
+    L.moe_route_topk.restype = i32
+    L.moe_route_topk.argtypes = [vp, i32, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+    L.moe_layer_forward.restype = i32
+    L.moe_layer_forward.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, vp]
+    L.moe_layer_forward_ex.restype = i32
+    L.moe_layer_forward_ex.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, i32, vp]
+    L.moe_read_routing.restype = i32
+    L.moe_read_routing.argtypes = [vp, i32, i32, vp, vp, vp, vp]
+    L.moe_profile_begin.restype = i32
+    L.moe_profile_begin.argtypes = [vp, i32]
+    L.moe_profile_end.restype = i32
+    L.moe_profile_end.argtypes = [vp, vp, vp]
+    L.moe_get_device_error.restype = i32
+    L.moe_get_device_error.argtypes = [vp]
+    return L
+
+
+lib = _load()
+
+
+def moe_status_string(status):
+    return lib.moe_status_string(int(status)).decode()
+
+
+def _check(status, what):
+    if status != MOE_OK:
+        raise MoeError(status, what)
+
+
+def _np_ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float32:
+        return MOE_DT_F32
+    if t.dtype == torch.bfloat16:
+        return MOE_DT_BF16
+    raise TypeError(f"activations must be float32 or bfloat16, not {t.dtype}")
+
+
+class Pack:
+    """An uploaded expert pack (owns device memory until free())."""
+
+    def __init__(self, handle, desc):
+        self.handle = handle
+        self.n_experts = desc.n_experts
+        self.hidden = desc.hidden
+        self.inter = desc.inter
+        self.has_shared = bool(desc.has_shared)
+        self.max_tokens = desc.max_tokens
+        self.max_top_k = desc.max_top_k
+        self.fmt_gate_up = desc.fmt_gate_up
+        self.fmt_down = desc.fmt_down
+
+    def info(self):
+        return moe_pack_query(self)
+
+    def free(self):
+        if self.handle:
+            _check(lib.moe_pack_free(self.handle), "moe_pack_free")
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def moe_pack_experts(n_experts, hidden, inter, fmt_gate_up, fmt_down, gate_up_blocks, down_blocks,
+                     gate_up_tensor_scale=None, down_tensor_scale=None, iq4nl_table=None,
+                     shared_gate_up_blocks=None, shared_down_blocks=None, max_tokens=64,
+                     max_top_k=None, device=0):
+    """Upload a layer's experts.  Blocks are host uint8 arrays in the canonical
+    layout of include/moe.h (expert-major); NVFP4 scales float32 [E(+1)]."""
+    keep = [np.ascontiguousarray(gate_up_blocks, np.uint8), np.ascontiguousarray(down_blocks, np.uint8)]
+    opt = lambda a, dt: None if a is None else np.ascontiguousarray(a, dt)
+    gts, dts = opt(gate_up_tensor_scale, np.float32), opt(down_tensor_scale, np.float32)
+    tab = opt(iq4nl_table, np.int8)
+    sgu, sdn = opt(shared_gate_up_blocks, np.uint8), opt(shared_down_blocks, np.uint8)
+    keep += [gts, dts, tab, sgu, sdn]
+    d = moe_pack_desc(n_experts, hidden, inter, 1 if sgu is not None else 0, max_tokens,
+                      max_top_k if max_top_k is not None else n_experts, fmt_gate_up, fmt_down,
+                      _np_ptr(keep[0]), _np_ptr(keep[1]), _np_ptr(gts), _np_ptr(dts), _np_ptr(tab),
+                      _np_ptr(sgu), _np_ptr(sdn))
+    h = ctypes.c_void_p()
+    _check(lib.moe_pack_experts(ctypes.byref(d), device, ctypes.byref(h)), "moe_pack_experts")
+    return Pack(h, d)
+
+
+def moe_pack_free(pack):
+    pack.free()
+
+
+def moe_pack_query(pack):
+    info = moe_pack_info()
+    _check(lib.moe_pack_query(pack.handle, ctypes.byref(info)), "moe_pack_query")
+    return {f: getattr(info, f) for f, _ in moe_pack_info._fields_}
+
+
+def moe_route_workspace_bytes(n_tokens, n_experts):
+    return lib.moe_route_workspace_bytes(n_tokens, n_experts)
+
+
+def moe_route_topk(x, router_w, top_k, idx_out, gate_out, workspace, stream=None):
+    """x: CUDA [T, H] float32/bfloat16; router_w: CUDA [E, H] bf16 bits (bfloat16,
+    int16 or uint16 tensor); idx_out int32 [T, k]; gate_out float32 [T, k];
+    workspace: CUDA uint8 tensor of moe_route_workspace_bytes(T, E) bytes."""
+    T, H = x.shape
+    E = router_w.shape[0]
+    _check(lib.moe_route_topk(x.data_ptr(), _dtype_code(x), router_w.data_ptr(), T, H, E, top_k,
+                              idx_out.data_ptr(), gate_out.data_ptr(), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
+           "moe_route_topk")
+
+
+def moe_layer_forward(x, router_w, pack, fmt, top_k, out, stream=None):
+    """out[T, H] (float32 CUDA) = the MoE layer on x[T, H] (float32/bfloat16 CUDA)."""
+    _check(lib.moe_layer_forward(x.data_ptr(), _dtype_code(x), router_w.data_ptr(), pack.handle,
+                                 fmt, x.shape[0], top_k, out.data_ptr(), _stream_ptr(stream)),
+           "moe_layer_forward")
+
+
+def moe_layer_forward_ex(x, router_w, pack, fmt, top_k, out, path, stream=None):
+    _check(lib.moe_layer_forward_ex(x.data_ptr(), _dtype_code(x), router_w.data_ptr(), pack.handle,
+                                    fmt, x.shape[0], top_k, out.data_ptr(), path,
+                                    _stream_ptr(stream)),
+           "moe_layer_forward_ex")
+
+
+def moe_read_routing(pack, n_tokens, top_k, stream=None):
+    """Routing of the last forward on `pack`, to host: (idx [T,k], gate [T,k], counts [E+1])."""
+    idx = np.empty((n_tokens, top_k), np.int32)
+    gate = np.empty((n_tokens, top_k), np.float32)
+    counts = np.empty(pack.n_experts + 1, np.int32)
+    _check(lib.moe_read_routing(pack.handle, n_tokens, top_k, _np_ptr(idx), _np_ptr(gate),
+                                _np_ptr(counts), _stream_ptr(stream)), "moe_read_routing")
+    return idx, gate, counts
+
+
+def moe_profile_begin(pack, max_forwards):
+    _check(lib.moe_profile_begin(pack.handle, max_forwards), "moe_profile_begin")
+
+
+def moe_profile_end(pack):
+    """-> (ms per stage [route+plan, gate/up, down, combine] summed, n_forwards)."""
+    ms = np.zeros(4, np.float64)
+    n = ctypes.c_int(0)
+    _check(lib.moe_profile_end(pack.handle, _np_ptr(ms), ctypes.byref(n)), "moe_profile_end")
+    return ms, n.value
+
+
+def moe_get_device_error(pack):
+    return lib.moe_get_device_error(pack.handle)
+
+
+def pack_layer(li, max_tokens=64, max_top_k=None, device=0):
+    """Pack a synth.LayerInputs-like object (router, gate_up, down, scales, table)."""
+    wl = li.wl
+    E = wl.n_experts
+    gs = li.gate_up_scale
+    ds = li.down_scale
+    return moe_pack_experts(E, wl.hidden, wl.inter, wl.fmt_gate_up, wl.fmt_down, li.gate_up[:E],
+                            li.down[:E], gs, ds, li.table,
+                            li.gate_up[E] if wl.has_shared else None,
+                            li.down[E] if wl.has_shared else None, max_tokens,
+                            max_top_k if max_top_k is not None else wl.top_k, device)

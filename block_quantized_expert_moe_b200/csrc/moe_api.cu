@@ -1,0 +1,619 @@
+// Host side of the C ABI in include/moe.h: argument checks, the expert pack
+// (repack of canonical blocks into the device planes + upload), workspace
+// management and the enqueueing of each forward's kernels.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <thread>
+#include <vector>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+cudaError_t route_set_attributes();
+cudaError_t matvec_set_attributes();
+}  // namespace moe
+
+using namespace moe;
+
+struct moe_pack {
+    int device = 0;
+    int num_sms = 0;
+    int E = 0, H = 0, I = 0, has_shared = 0, max_tokens = 0, max_top_k = 0;
+    int fmt_gu = 0, fmt_dn = 0;
+    DevProj gu, dn;
+    uint32_t tab[4] = {0, 0, 0, 0};
+    std::vector<void *> allocations;
+    Workspace ws;
+    int64_t arena_bytes = 0, workspace_bytes = 0;
+    int grid_cache[2][2];  // [gateup][tt==8]
+    // kernel-stage timing (moe_profile_begin/end)
+    bool prof_on = false;
+    std::vector<cudaEvent_t> prof_ev;
+    int prof_used = 0;
+};
+
+namespace {
+
+const uint32_t kNvfp4Tab[4] = {
+    // 2*e2m1 for codes 0..15, each stored as value + 128
+    0x83828180u,  // 0, 1, 2, 3
+    0x8C888684u,  // 4, 6, 8, 12
+    0x7D7E7F80u,  // -0, -1, -2, -3
+    0x74787A7Cu,  // -4, -6, -8, -12
+};
+
+std::mutex g_dev_mutex;
+bool g_dev_ready[64];
+
+moe_status init_device(int dev)
+{
+    std::lock_guard<std::mutex> lk(g_dev_mutex);
+    if (dev < 0 || dev >= 64) return MOE_ERR_INVALID_ARG;
+    if (g_dev_ready[dev]) return MOE_OK;
+    if (route_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
+    if (matvec_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
+    g_dev_ready[dev] = true;
+    return MOE_OK;
+}
+
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev)
+    {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
+    }
+    ~DeviceGuard()
+    {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_fmt(int f) { return f >= MOE_FMT_Q8_0 && f <= MOE_FMT_NVFP4; }
+
+int64_t canon_row_bytes(int fmt, int64_t cols)
+{
+    switch (fmt) {
+    case MOE_FMT_Q8_0: return cols / 32 * 34;
+    case MOE_FMT_Q5_1: return cols / 32 * 24;
+    case MOE_FMT_IQ4_NL: return cols / 32 * 18;
+    case MOE_FMT_NVFP4: return cols / 16 * 9;
+    default: return -1;
+    }
+}
+
+// Device plane sizes of one row of `cols` weights.
+void plane_rows(int fmt, int cols, int &qs_row, int &sc_row, int &qh_row)
+{
+    qh_row = 0;
+    switch (fmt) {
+    case MOE_FMT_Q8_0: qs_row = cols; sc_row = cols / 32 * 2; break;
+    case MOE_FMT_Q5_1: qs_row = cols / 2; sc_row = cols / 32 * 4; qh_row = cols / 32 * 4; break;
+    case MOE_FMT_IQ4_NL: qs_row = cols / 2; sc_row = cols / 32 * 2; break;
+    default: qs_row = cols / 2; sc_row = cols / 16; break;  // NVFP4
+    }
+}
+
+int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+// Repack one expert's projection (rows x cols canonical blocks) into planes.
+// Returns false on an invalid NVFP4 block scale.
+bool repack_expert(int fmt, const uint8_t *src, int rows, int cols, uint8_t *qs, uint8_t *sc,
+                   uint8_t *qh)
+{
+    const int64_t rb = canon_row_bytes(fmt, cols);
+    int qs_row, sc_row, qh_row;
+    plane_rows(fmt, cols, qs_row, sc_row, qh_row);
+    for (int r = 0; r < rows; ++r) {
+        const uint8_t *row = src + (int64_t)r * rb;
+        uint8_t *q = qs + (int64_t)r * qs_row;
+        uint8_t *s = sc + (int64_t)r * sc_row;
+        if (fmt == MOE_FMT_Q8_0) {
+            for (int b = 0; b < cols / 32; ++b) {
+                const uint8_t *blk = row + b * 34;
+                s[2 * b] = blk[0];
+                s[2 * b + 1] = blk[1];
+                for (int j = 0; j < 32; ++j) q[b * 32 + j] = blk[2 + j] ^ 0x80u;  // bias by +128
+            }
+        } else if (fmt == MOE_FMT_Q5_1) {
+            uint8_t *h = qh + (int64_t)r * qh_row;
+            for (int b = 0; b < cols / 32; ++b) {
+                const uint8_t *blk = row + b * 24;
+                std::memcpy(s + 4 * b, blk, 4);      // d, m
+                std::memcpy(h + 4 * b, blk + 4, 4);  // qh
+                std::memcpy(q + 16 * b, blk + 8, 16);
+            }
+        } else if (fmt == MOE_FMT_IQ4_NL) {
+            for (int b = 0; b < cols / 32; ++b) {
+                const uint8_t *blk = row + b * 18;
+                s[2 * b] = blk[0];
+                s[2 * b + 1] = blk[1];
+                std::memcpy(q + 16 * b, blk + 2, 16);
+            }
+        } else {
+            for (int b = 0; b < cols / 16; ++b) {
+                const uint8_t *blk = row + b * 9;
+                if (blk[0] >= 0x7Fu) return false;  // negative scale or NaN
+                s[b] = blk[0];
+                std::memcpy(q + 8 * b, blk + 1, 8);
+            }
+        }
+    }
+    return true;
+}
+
+template <class F>
+void parallel_for(int n, F f)
+{
+    unsigned hw = std::thread::hardware_concurrency();
+    int nt = (int)std::min<unsigned>(hw ? hw : 1, 64u);
+    nt = std::min(nt, n);
+    if (nt <= 1) {
+        for (int i = 0; i < n; ++i) f(i);
+        return;
+    }
+    std::vector<std::thread> th;
+    for (int t = 0; t < nt; ++t)
+        th.emplace_back([&, t] {
+            for (int i = t; i < n; i += nt) f(i);
+        });
+    for (auto &x : th) x.join();
+}
+
+void free_pack_memory(moe_pack *p)
+{
+    for (void *a : p->allocations) cudaFree(a);
+    p->allocations.clear();
+}
+
+moe_status dev_alloc(moe_pack *p, size_t bytes, void **out)
+{
+    void *ptr = nullptr;
+    if (cudaMalloc(&ptr, bytes ? bytes : 16) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_OOM;
+    }
+    p->allocations.push_back(ptr);
+    *out = ptr;
+    return MOE_OK;
+}
+
+// Build one projection's planes for all slots (routed experts + shared).
+moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, const uint8_t *blocks,
+                      const uint8_t *shared_blocks, const float *ts, int n_slots)
+{
+    dp.fmt = fmt;
+    dp.rows = rows;
+    dp.cols = cols;
+    plane_rows(fmt, cols, dp.qs_row, dp.sc_row, dp.qh_row);
+    dp.qs_stride = round_up((int64_t)rows * dp.qs_row, 256);
+    dp.sc_stride = round_up((int64_t)rows * dp.sc_row, 256);
+    dp.qh_stride = round_up((int64_t)rows * dp.qh_row, 256);
+    const int64_t canon = canon_row_bytes(fmt, cols) * rows;
+    std::vector<uint8_t> hq, hs, hh;
+    try {
+        hq.assign((size_t)dp.qs_stride * n_slots, 0);
+        hs.assign((size_t)dp.sc_stride * n_slots, 0);
+        if (dp.qh_row) hh.assign((size_t)dp.qh_stride * n_slots, 0);
+    } catch (const std::bad_alloc &) {
+        return MOE_ERR_OOM;
+    }
+    std::vector<char> ok((size_t)n_slots, 1);
+    parallel_for(n_slots, [&](int s) {
+        const uint8_t *src = s < p->E ? blocks + (int64_t)s * canon : shared_blocks;
+        ok[s] = repack_expert(fmt, src, rows, cols, hq.data() + (int64_t)s * dp.qs_stride,
+                              hs.data() + (int64_t)s * dp.sc_stride,
+                              dp.qh_row ? hh.data() + (int64_t)s * dp.qh_stride : nullptr);
+    });
+    for (char c : ok)
+        if (!c) return MOE_ERR_INVALID_ARG;
+    void *dq, *ds, *dh = nullptr, *dt = nullptr;
+    moe_status st;
+    if ((st = dev_alloc(p, hq.size(), &dq)) != MOE_OK) return st;
+    if ((st = dev_alloc(p, hs.size(), &ds)) != MOE_OK) return st;
+    if (cudaMemcpy(dq, hq.data(), hq.size(), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpy(ds, hs.data(), hs.size(), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    if (dp.qh_row) {
+        if ((st = dev_alloc(p, hh.size(), &dh)) != MOE_OK) return st;
+        if (cudaMemcpy(dh, hh.data(), hh.size(), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if (fmt == MOE_FMT_NVFP4) {
+        for (int s = 0; s < n_slots; ++s)
+            if (!(ts[s] >= 0.f) || ts[s] > 3.0e38f) return MOE_ERR_INVALID_ARG;
+        if ((st = dev_alloc(p, sizeof(float) * n_slots, &dt)) != MOE_OK) return st;
+        if (cudaMemcpy(dt, ts, sizeof(float) * n_slots, cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    dp.qs = static_cast<const uint8_t *>(dq);
+    dp.sc = static_cast<const uint8_t *>(ds);
+    dp.qh = static_cast<const uint8_t *>(dh);
+    dp.ts = static_cast<const float *>(dt);
+    p->arena_bytes += (int64_t)(hq.size() + hs.size() + hh.size()) + (dt ? 4 * n_slots : 0);
+    return MOE_OK;
+}
+
+moe_status build_workspace(moe_pack *p)
+{
+    const int64_t T = p->max_tokens, k = p->max_top_k, E = p->E;
+    const int64_t slots = T * (k + 1);
+    Workspace &w = p->ws;
+    w.max_groups = (int)(slots + E + 2);
+    struct Item { void **dst; int64_t bytes; };
+    Item items[] = {
+        {(void **)&w.logits, T * E * 4}, {(void **)&w.idx, T * k * 4}, {(void **)&w.gate, T * k * 4},
+        {(void **)&w.cnt, (E + 1) * 4}, {(void **)&w.off, (E + 1) * 4}, {(void **)&w.perm_tok, slots * 4},
+        {(void **)&w.slot_pos, T * k * 4}, {(void **)&w.groups, (int64_t)w.max_groups * 16},
+        {(void **)&w.n_groups, 4}, {(void **)&w.ticket, 4}, {(void **)&w.err, 4},
+        {(void **)&w.h, slots * p->I * 4}, {(void **)&w.y, slots * p->H * 4},
+    };
+    int64_t total = 0;
+    for (auto &it : items) total += round_up(it.bytes, 256);
+    void *base;
+    moe_status st = dev_alloc(p, (size_t)total, &base);
+    if (st != MOE_OK) return st;
+    if (cudaMemset(base, 0, (size_t)total) != cudaSuccess) return MOE_ERR_CUDA;
+    int64_t o = 0;
+    for (auto &it : items) {
+        *it.dst = static_cast<char *>(base) + o;
+        o += round_up(it.bytes, 256);
+    }
+    p->workspace_bytes = total;
+    return MOE_OK;
+}
+
+moe_status check_launch(cudaError_t e)
+{
+    if (e == cudaSuccess) return MOE_OK;
+    return MOE_ERR_CUDA;
+}
+
+// Record profiling event i of the current forward (no-op when profiling is off
+// or the event budget is used up).
+void prof_mark(moe_pack *p, int base, int i, cudaStream_t s)
+{
+    if (base < 0) return;
+    cudaEvent_t ev = p->prof_ev[(size_t)base + i];
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &cs);
+    if (cs == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+    else cudaEventRecord(ev, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_status_string(moe_status s)
+{
+    switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported";
+    case MOE_ERR_FMT_MISMATCH: return "format does not match the pack";
+    case MOE_ERR_OOM: return "out of memory";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_DEVICE: return "device-side plan error";
+    default: return "unknown status";
+    }
+}
+
+moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
+{
+    if (!d || !out) return MOE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (d->n_experts < 1 || d->n_experts > 1024) return MOE_ERR_INVALID_ARG;
+    if (d->hidden < 32 || d->hidden > 16384 || d->hidden % 32) return MOE_ERR_INVALID_ARG;
+    if (d->inter < 32 || d->inter > 16384 || d->inter % 32) return MOE_ERR_INVALID_ARG;
+    if (d->max_tokens < 1 || d->max_tokens > 65536) return MOE_ERR_INVALID_ARG;
+    if (d->max_top_k < 1 || d->max_top_k > d->n_experts) return MOE_ERR_INVALID_ARG;
+    if (!valid_fmt(d->fmt_gate_up) || !valid_fmt(d->fmt_down)) return MOE_ERR_INVALID_ARG;
+    if (!d->gate_up_blocks || !d->down_blocks) return MOE_ERR_INVALID_ARG;
+    if ((d->fmt_gate_up == MOE_FMT_IQ4_NL || d->fmt_down == MOE_FMT_IQ4_NL) && !d->iq4nl_table)
+        return MOE_ERR_INVALID_ARG;
+    if (d->fmt_gate_up == MOE_FMT_NVFP4 && !d->gate_up_tensor_scale) return MOE_ERR_INVALID_ARG;
+    if (d->fmt_down == MOE_FMT_NVFP4 && !d->down_tensor_scale) return MOE_ERR_INVALID_ARG;
+    if (d->has_shared && (!d->shared_gate_up_blocks || !d->shared_down_blocks)) return MOE_ERR_INVALID_ARG;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (device < 0 || device >= ndev) return MOE_ERR_INVALID_ARG;
+    DeviceGuard g(device);
+    if (!g.ok) return MOE_ERR_CUDA;
+    moe_status st = init_device(device);
+    if (st != MOE_OK) return st;
+    moe_pack *p = new (std::nothrow) moe_pack();
+    if (!p) return MOE_ERR_OOM;
+    p->device = device;
+    cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, device);
+    p->E = d->n_experts;
+    p->H = d->hidden;
+    p->I = d->inter;
+    p->has_shared = d->has_shared ? 1 : 0;
+    p->max_tokens = d->max_tokens;
+    p->max_top_k = d->max_top_k;
+    p->fmt_gu = d->fmt_gate_up;
+    p->fmt_dn = d->fmt_down;
+    if (d->iq4nl_table)
+        for (int c = 0; c < 16; ++c)
+            p->tab[c / 4] |= (uint32_t)((uint8_t)d->iq4nl_table[c] ^ 0x80u) << (8 * (c % 4));
+    for (auto &row : p->grid_cache) row[0] = row[1] = 0;
+    const int n_slots = p->E + p->has_shared;
+    std::vector<float> gts, dts;
+    if (p->fmt_gu == MOE_FMT_NVFP4) gts.assign(d->gate_up_tensor_scale, d->gate_up_tensor_scale + n_slots);
+    if (p->fmt_dn == MOE_FMT_NVFP4) dts.assign(d->down_tensor_scale, d->down_tensor_scale + n_slots);
+    st = build_proj(p, p->gu, p->fmt_gu, 2 * p->I, p->H, static_cast<const uint8_t *>(d->gate_up_blocks),
+                    static_cast<const uint8_t *>(d->shared_gate_up_blocks), gts.data(), n_slots);
+    if (st == MOE_OK)
+        st = build_proj(p, p->dn, p->fmt_dn, p->H, p->I, static_cast<const uint8_t *>(d->down_blocks),
+                        static_cast<const uint8_t *>(d->shared_down_blocks), dts.data(), n_slots);
+    if (st == MOE_OK) st = build_workspace(p);
+    if (st == MOE_OK && cudaDeviceSynchronize() != cudaSuccess) st = MOE_ERR_CUDA;
+    if (st != MOE_OK) {
+        free_pack_memory(p);
+        delete p;
+        return st;
+    }
+    *out = p;
+    return MOE_OK;
+}
+
+moe_status moe_pack_free(moe_pack *p)
+{
+    if (!p) return MOE_OK;
+    DeviceGuard g(p->device);
+    cudaDeviceSynchronize();
+    free_pack_memory(p);
+    delete p;
+    return MOE_OK;
+}
+
+moe_status moe_pack_query(const moe_pack *p, moe_pack_info *info)
+{
+    if (!p || !info) return MOE_ERR_INVALID_ARG;
+    info->gate_up_bytes_per_expert = (int64_t)p->gu.rows * (p->gu.qs_row + p->gu.sc_row + p->gu.qh_row);
+    info->down_bytes_per_expert = (int64_t)p->dn.rows * (p->dn.qs_row + p->dn.sc_row + p->dn.qh_row);
+    info->expert_bytes = info->gate_up_bytes_per_expert + info->down_bytes_per_expert +
+                         (p->fmt_gu == MOE_FMT_NVFP4 ? 4 : 0) + (p->fmt_dn == MOE_FMT_NVFP4 ? 4 : 0);
+    info->arena_bytes = p->arena_bytes;
+    info->workspace_bytes = p->workspace_bytes;
+    info->device = p->device;
+    return MOE_OK;
+}
+
+size_t moe_route_workspace_bytes(int n_tokens, int n_experts)
+{
+    if (n_tokens < 1 || n_experts < 1) return 0;
+    return 256 + (size_t)n_tokens * n_experts * sizeof(float);
+}
+
+moe_status moe_route_topk(const void *x, moe_dtype x_dtype, const uint16_t *router_w, int n_tokens,
+                          int hidden, int n_experts, int top_k, int32_t *idx_out, float *gate_out,
+                          void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!x || !router_w || !idx_out || !gate_out || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
+    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+    if (n_tokens < 1 || hidden < 8 || hidden % 8 || hidden > 16384) return MOE_ERR_INVALID_ARG;
+    if (n_experts < 1 || n_experts > 1024 || top_k < 1 || top_k > n_experts) return MOE_ERR_INVALID_ARG;
+    if (workspace_bytes < moe_route_workspace_bytes(n_tokens, n_experts)) return MOE_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    moe_status st = init_device(dev);
+    if (st != MOE_OK) return st;
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    RouteArgs a{};
+    a.x = x;
+    a.x_dtype = x_dtype;
+    a.wr = router_w;
+    a.T = n_tokens;
+    a.H = hidden;
+    a.E = n_experts;
+    a.k = top_k;
+    a.rt = route_tokens_per_pass(hidden);
+    a.ticket = static_cast<int32_t *>(workspace);
+    a.logits = reinterpret_cast<float *>(static_cast<char *>(workspace) + 256);
+    a.idx = idx_out;
+    a.gate = gate_out;
+    a.do_plan = 0;
+    if (cudaMemsetAsync(a.ticket, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return check_launch(launch_route(a, route_grid(n_experts, sms), s));
+}
+
+moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
+                                const moe_pack *p, moe_fmt fmt, int n_tokens, int top_k, float *out,
+                                moe_path path, void *stream)
+{
+    if (!p || !x || !router_w || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+    if (n_tokens < 1 || n_tokens > p->max_tokens) return MOE_ERR_INVALID_ARG;
+    if (top_k < 1 || top_k > p->max_top_k) return MOE_ERR_INVALID_ARG;
+    if (fmt != MOE_FMT_FROM_PACK && fmt != p->fmt_gu) return MOE_ERR_FMT_MISMATCH;
+    if (path == MOE_PATH_AUTO) path = MOE_PATH_DECODE;
+    if (path != MOE_PATH_DECODE) return MOE_ERR_UNSUPPORTED;
+    DeviceGuard g(p->device);
+    if (!g.ok) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    moe_pack *pm = const_cast<moe_pack *>(p);
+    const Workspace &w = p->ws;
+    const int T = n_tokens, k = top_k;
+    // tokens per work group: 8 unless a single token, or 8 staged fp32 rows of
+    // the longer reduction would not fit in shared memory
+    const int kmax = std::max(p->H, p->I);
+    const int tt = (T == 1 || (size_t)8 * kmax * 4 * 33 / 32 > 200 * 1024) ? 1 : 8;
+    int pbase = -1;
+    if (pm->prof_on && (size_t)pm->prof_used + 5 <= pm->prof_ev.size()) {
+        pbase = pm->prof_used;
+        pm->prof_used += 5;
+    }
+    prof_mark(pm, pbase, 0, s);
+
+    RouteArgs ra{};
+    ra.x = x;
+    ra.x_dtype = x_dtype;
+    ra.wr = router_w;
+    ra.T = T;
+    ra.H = p->H;
+    ra.E = p->E;
+    ra.k = k;
+    ra.rt = route_tokens_per_pass(p->H);
+    ra.logits = w.logits;
+    ra.ticket = w.ticket;
+    ra.idx = w.idx;
+    ra.gate = w.gate;
+    ra.do_plan = 1;
+    ra.has_shared = p->has_shared;
+    ra.tt = tt;
+    ra.cnt = w.cnt;
+    ra.off = w.off;
+    ra.perm_tok = w.perm_tok;
+    ra.slot_pos = w.slot_pos;
+    ra.n_groups = w.n_groups;
+    ra.err = w.err;
+    ra.groups = w.groups;
+    ra.max_groups = w.max_groups;
+    moe_status st = check_launch(launch_route(ra, route_grid(p->E, p->num_sms), s));
+    if (st != MOE_OK) return st;
+    prof_mark(pm, pbase, 1, s);
+
+    MatvecArgs gu{};
+    gu.w = p->gu;
+    gu.groups = w.groups;
+    gu.n_groups = w.n_groups;
+    gu.perm_tok = w.perm_tok;
+    gu.x = x;
+    gu.x_dtype = x_dtype;
+    gu.out = w.h;
+    gu.out_stride = p->I;
+    gu.rows_out = p->I;
+    std::memcpy(gu.tab, p->fmt_gu == MOE_FMT_NVFP4 ? kNvfp4Tab : p->tab, sizeof(gu.tab));
+    int &ggu = pm->grid_cache[1][tt == 8];
+    if (!ggu) ggu = matvec_grid(gu, true, tt, p->num_sms);
+    st = check_launch(launch_matvec(gu, true, tt, ggu, s));
+    if (st != MOE_OK) return st;
+    prof_mark(pm, pbase, 2, s);
+
+    MatvecArgs dn{};
+    dn.w = p->dn;
+    dn.groups = w.groups;
+    dn.n_groups = w.n_groups;
+    dn.perm_tok = w.perm_tok;
+    dn.x = w.h;
+    dn.x_dtype = MOE_DT_F32;
+    dn.out = w.y;
+    dn.out_stride = p->H;
+    dn.rows_out = p->H;
+    std::memcpy(dn.tab, p->fmt_dn == MOE_FMT_NVFP4 ? kNvfp4Tab : p->tab, sizeof(dn.tab));
+    int &gdn = pm->grid_cache[0][tt == 8];
+    if (!gdn) gdn = matvec_grid(dn, false, tt, p->num_sms);
+    st = check_launch(launch_matvec(dn, false, tt, gdn, s));
+    if (st != MOE_OK) return st;
+    prof_mark(pm, pbase, 3, s);
+
+    CombineArgs ca{};
+    ca.y = w.y;
+    ca.slot_pos = w.slot_pos;
+    ca.gate = w.gate;
+    ca.T = T;
+    ca.k = k;
+    ca.H = p->H;
+    ca.has_shared = p->has_shared;
+    ca.out = out;
+    st = check_launch(launch_combine(ca, s));
+    prof_mark(pm, pbase, 4, s);
+    return st;
+}
+
+moe_status moe_layer_forward(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
+                             const moe_pack *pack, moe_fmt fmt, int n_tokens, int top_k, float *out,
+                             void *stream)
+{
+    return moe_layer_forward_ex(x, x_dtype, router_w, pack, fmt, n_tokens, top_k, out, MOE_PATH_AUTO,
+                                stream);
+}
+
+moe_status moe_read_routing(const moe_pack *p, int n_tokens, int top_k, int32_t *idx, float *gate,
+                            int32_t *counts, void *stream)
+{
+    if (!p || n_tokens < 1 || n_tokens > p->max_tokens || top_k < 1 || top_k > p->max_top_k)
+        return MOE_ERR_INVALID_ARG;
+    DeviceGuard g(p->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = (size_t)n_tokens * top_k;
+    if (idx && cudaMemcpyAsync(idx, p->ws.idx, n * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (gate && cudaMemcpyAsync(gate, p->ws.gate, n * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (counts && cudaMemcpyAsync(counts, p->ws.cnt, (size_t)(p->E + 1) * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_profile_begin(moe_pack *p, int max_forwards)
+{
+    if (!p || max_forwards < 1 || max_forwards > (1 << 20) || p->prof_on) return MOE_ERR_INVALID_ARG;
+    DeviceGuard g(p->device);
+    p->prof_ev.assign((size_t)max_forwards * 5, nullptr);
+    for (auto &e : p->prof_ev)
+        if (cudaEventCreate(&e) != cudaSuccess) {
+            for (auto &f : p->prof_ev)
+                if (f) cudaEventDestroy(f);
+            p->prof_ev.clear();
+            return MOE_ERR_CUDA;
+        }
+    p->prof_used = 0;
+    p->prof_on = true;
+    return MOE_OK;
+}
+
+moe_status moe_profile_end(moe_pack *p, double *ms, int *n_forwards)
+{
+    if (!p || !p->prof_on) return MOE_ERR_INVALID_ARG;
+    DeviceGuard g(p->device);
+    moe_status st = cudaDeviceSynchronize() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    double acc[4] = {0, 0, 0, 0};
+    const int n = p->prof_used / 5;
+    for (int f = 0; f < n && st == MOE_OK; ++f)
+        for (int i = 0; i < 4; ++i) {
+            float v = 0.f;
+            if (cudaEventElapsedTime(&v, p->prof_ev[(size_t)5 * f + i], p->prof_ev[(size_t)5 * f + i + 1]) !=
+                cudaSuccess) {
+                st = MOE_ERR_CUDA;
+                break;
+            }
+            acc[i] += v;
+        }
+    for (auto &e : p->prof_ev) cudaEventDestroy(e);
+    p->prof_ev.clear();
+    p->prof_on = false;
+    p->prof_used = 0;
+    if (ms)
+        for (int i = 0; i < 4; ++i) ms[i] = acc[i];
+    if (n_forwards) *n_forwards = n;
+    return st;
+}
+
+moe_status moe_get_device_error(const moe_pack *p)
+{
+    if (!p) return MOE_ERR_INVALID_ARG;
+    DeviceGuard g(p->device);
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    int32_t e = 0;
+    if (cudaMemcpy(&e, p->ws.err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (e) cudaMemset(p->ws.err, 0, 4);
+    return static_cast<moe_status>(e);
+}
+
+}  // extern "C"

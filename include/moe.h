@@ -1,0 +1,208 @@
+/*
+ * moe.h - C ABI of the block-quantised routed mixture-of-experts FFN layer,
+ * for one NVIDIA B200 (sm_100a).
+ *
+ * The layer is the routed MoE FFN of a Qwen3.8-Flash-Next-style model: the
+ * model card "Qwen3.8-Flash-Next-Basalt" and the "llms-full.txt" FAQ describe
+ * a mixture-of-experts model whose tokens each use only their selected
+ * experts, and the "Qwen3.8-Flash-Next UD-IQ2_XS (L4 fix) for Basalt" model
+ * card, section "What was changed", names the fast path a device-planned MoE
+ * tail with grouped kernels over routed experts stored as IQ4_NL, NVFP4, Q5_1
+ * or Q8_0.  Per token t the layer computes
+ *
+ *   l_e   = sum_h Wr[e,h] x[t,h]                    router logits (fp32 accumulate)
+ *   S     = the top_k largest l_e, ties to the lower expert index
+ *   g_e   = exp(l_e - max l) / sum_{j in S} exp(l_j - max l)   (softmax renormalised over S)
+ *   y_e   = D_e (silu(G_e x) * (U_e x))              SwiGLU expert, fp32 accumulate
+ *   out_t = sum_{e in S} g_e y_e  (+ y_shared when the pack has a shared expert)
+ *
+ * Memory: every pointer argument named "device" is CUDA device memory of the
+ * pack's device (torch tensors qualify); "host" pointers are ordinary host
+ * memory.  Device pointers must be 16-byte aligned.  The caller owns x,
+ * router weights, outputs and the stream; the library owns each pack (its
+ * device weight arena and a workspace sized at pack time).
+ *
+ * Streams and errors: argument errors return synchronously before anything is
+ * enqueued.  Forward and route calls only enqueue work on `stream`; they do
+ * not synchronise the host and do not allocate.  A launch failure returns
+ * MOE_ERR_CUDA.  Errors raised inside kernels (a bounded wait that ran out, a
+ * plan overflow) set a sticky word that moe_get_device_error() returns.
+ * One pack runs one forward at a time: two forwards on one pack must be
+ * ordered (same stream, or events); concurrent streams need separate packs.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, top_k out of range */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid but not implemented (format/shape combination) */
+    MOE_ERR_FMT_MISMATCH = 3, /* fmt argument disagrees with the pack */
+    MOE_ERR_OOM = 4,          /* device or host allocation failed (pack only) */
+    MOE_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+    MOE_ERR_TIMEOUT = 6,      /* a bounded device-side wait ran out */
+    MOE_ERR_DEVICE = 7        /* a kernel detected an inconsistent plan */
+} moe_status;
+
+/* Block formats, each along the reduction (K) dimension of a weight row:
+ *   Q8_0   32 weights in 34 B: fp16 d, int8 q[32]                 w = d*q
+ *   Q5_1   32 weights in 24 B: fp16 d, fp16 m, u32 qh, qs[16]     w = d*q + m, q in [0,31]
+ *   IQ4_NL 32 weights in 18 B: fp16 d, qs[16] (4-bit indices)     w = d*T[i], T from the pack desc
+ *   NVFP4  16 weights in  9 B: E4M3 scale, 8 B of E2M1 codes, and one fp32
+ *          scale s per matrix                                     w = s*e4m3*e2m1
+ * Byte order inside a block (little endian):
+ *   Q8_0   [0,2) d  [2,34) q
+ *   Q5_1   [0,2) d  [2,4) m  [4,8) qh (bit j is bit 4 of element j)  [8,24) qs
+ *   IQ4_NL [0,2) d  [2,18) qs
+ *   for Q5_1 and IQ4_NL element j < 16 is the low nibble of qs[j] and element
+ *   j >= 16 the high nibble of qs[j-16];
+ *   NVFP4  [0] E4M3 scale  [1,9) codes: element 2i is the low, 2i+1 the high
+ *   nibble of byte 1+i.
+ * IQ4_NL is 4.5 bits per weight, the size the UD-IQ2_XS model card ("What was
+ * changed") gives when it requantises a Q5_0 tensor (5.5 bits) to IQ4_NL. */
+typedef enum {
+    MOE_FMT_FROM_PACK = 0, /* forward: accept the pack's formats */
+    MOE_FMT_Q8_0 = 1,
+    MOE_FMT_Q5_1 = 2,
+    MOE_FMT_IQ4_NL = 3,
+    MOE_FMT_NVFP4 = 4
+} moe_fmt;
+
+typedef enum { MOE_DT_F32 = 1, MOE_DT_BF16 = 2 } moe_dtype;
+
+/* Kernel path of a forward.  AUTO picks DECODE for n_tokens <= 64 (decode and
+ * speculative-verify batches) and PREFILL above.  DENSE is the dense-batched
+ * comparison variant: every active expert multiplies the whole batch, with a
+ * zero gate for tokens not routed to it. */
+typedef enum {
+    MOE_PATH_AUTO = 0,
+    MOE_PATH_DECODE = 1,
+    MOE_PATH_PREFILL = 2,
+    MOE_PATH_DENSE = 3
+} moe_path;
+
+/* Description of one layer's experts, all in HOST memory; moe_pack_experts
+ * copies what it needs, the caller keeps ownership.
+ *   gate_up_blocks  n_experts x [2*inter rows x hidden] canonical blocks, rows
+ *                   0..inter-1 are the gate projection G, inter..2*inter-1 the
+ *                   up projection U, expert after expert
+ *   down_blocks     n_experts x [hidden rows x inter] blocks (D)
+ *   *_tensor_scale  NVFP4 only: one fp32 scale per expert, n_experts entries
+ *                   (+1 for the shared expert, at index n_experts); else NULL
+ *   iq4nl_table     16 int8 entries, required when a projection is IQ4_NL
+ *   shared_*_blocks the always-on shared expert (gate 1), same shapes and
+ *                   formats, required iff has_shared
+ *   max_tokens, max_top_k  size the pack's workspace (forward refuses more)
+ * Constraints: hidden and inter are multiples of 32 (all formats), hidden <=
+ * 16384, inter <= 16384, 1 <= n_experts <= 1024, 1 <= max_top_k <= n_experts,
+ * 1 <= max_tokens <= 65536. */
+typedef struct {
+    int n_experts;
+    int hidden;
+    int inter;
+    int has_shared;
+    int max_tokens;
+    int max_top_k;
+    moe_fmt fmt_gate_up;
+    moe_fmt fmt_down;
+    const void *gate_up_blocks;
+    const void *down_blocks;
+    const float *gate_up_tensor_scale;
+    const float *down_tensor_scale;
+    const int8_t *iq4nl_table;
+    const void *shared_gate_up_blocks;
+    const void *shared_down_blocks;
+} moe_pack_desc;
+
+typedef struct moe_pack moe_pack; /* opaque; owns device memory */
+
+/* Sizes of a pack, for accounting (bytes are HBM bytes of the packed blocks). */
+typedef struct {
+    int64_t gate_up_bytes_per_expert;
+    int64_t down_bytes_per_expert;
+    int64_t expert_bytes;         /* gate_up + down (+ NVFP4 matrix scales) */
+    int64_t arena_bytes;          /* all experts incl. shared */
+    int64_t workspace_bytes;
+    int device;
+} moe_pack_info;
+
+/* Validate `desc`, repack every expert's blocks into the device layout (scales
+ * split from codes, 16-byte aligned rows) and upload them to `device`; also
+ * allocate the forward workspace.  Synchronous.  Rejects NVFP4 block scales
+ * that are negative or NaN (MOE_ERR_INVALID_ARG).  On success *out owns the
+ * device memory until moe_pack_free. */
+moe_status moe_pack_experts(const moe_pack_desc *desc, int device, moe_pack **out);
+
+/* Free a pack (synchronises its device).  NULL is accepted. */
+moe_status moe_pack_free(moe_pack *pack);
+
+moe_status moe_pack_query(const moe_pack *pack, moe_pack_info *info);
+
+/* Workspace bytes moe_route_topk needs for n_tokens x n_experts. */
+size_t moe_route_workspace_bytes(int n_tokens, int n_experts);
+
+/* Router GEMV, softmax and top-k of n_tokens tokens.
+ *   x         device, [n_tokens x hidden], fp32 or bf16 (x_dtype), row-major
+ *   router_w  device, [n_experts x hidden] bf16 bits, row-major
+ *   idx_out   device, [n_tokens x top_k] int32: selected experts by descending
+ *             logit, ties to the lower index
+ *   gate_out  device, [n_tokens x top_k] fp32 gates (sum to 1 per token)
+ *   workspace device, moe_route_workspace_bytes(n_tokens, n_experts) bytes,
+ *             owned by the caller; its contents need no initialisation
+ * hidden % 8 == 0, 1 <= top_k <= n_experts <= 1024. */
+moe_status moe_route_topk(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
+                          int n_tokens, int hidden, int n_experts, int top_k, int32_t *idx_out,
+                          float *gate_out, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/* The whole layer: route, plan, grouped gate/up + SwiGLU, down, combine.
+ *   x        device [n_tokens x hidden] fp32 or bf16
+ *   router_w device [n_experts x hidden] bf16 bits
+ *   fmt      MOE_FMT_FROM_PACK, or the pack's gate/up format (checked)
+ *   out      device [n_tokens x hidden] fp32
+ * 1 <= n_tokens <= max_tokens, 1 <= top_k <= max_top_k.  Enqueues on `stream`
+ * (a cudaStream_t; NULL is the legacy default stream). */
+moe_status moe_layer_forward(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
+                             const moe_pack *pack, moe_fmt fmt, int n_tokens, int top_k,
+                             float *out, void *stream);
+
+/* As moe_layer_forward with an explicit kernel path (see moe_path). */
+moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
+                                const moe_pack *pack, moe_fmt fmt, int n_tokens, int top_k,
+                                float *out, moe_path path, void *stream);
+
+/* After a forward: copy its routing and plan to HOST memory (synchronises
+ * `stream`).  Any pointer may be NULL.
+ *   idx   [n_tokens x top_k] int32, gate [n_tokens x top_k] fp32,
+ *   counts [n_experts + 1] int32 tokens per expert (last entry: shared). */
+moe_status moe_read_routing(const moe_pack *pack, int n_tokens, int top_k, int32_t *idx,
+                            float *gate, int32_t *counts, void *stream);
+
+/* Kernel timing of forwards, for measurement.  moe_profile_begin creates
+ * CUDA events for up to max_forwards forwards (this allocates: call it before
+ * a timed region or a stream capture); each later forward on the pack then
+ * records an event before each of its kernels and after the last one
+ * (captured as event-record nodes when the stream is capturing).
+ * moe_profile_end synchronises the device, adds the elapsed times per kernel
+ * stage over all recorded forwards into ms[4] (route+plan, gate/up, down,
+ * combine; host memory), stores the forward count in *n_forwards, and frees
+ * the events.  Forwards beyond max_forwards are not recorded. */
+moe_status moe_profile_begin(moe_pack *pack, int max_forwards);
+moe_status moe_profile_end(moe_pack *pack, double *ms, int *n_forwards);
+
+/* Sticky device-side error of the pack (synchronises its device), then clears it. */
+moe_status moe_get_device_error(const moe_pack *pack);
+
+const char *moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

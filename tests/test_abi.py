@@ -1,0 +1,90 @@
+"""The C-ABI library loads, exports every function include/moe.h declares, and
+rejects bad arguments before touching a device.  CPU only."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import block_quantized_expert_moe_b200 as bq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_function_is_exported():
+    names = declared_functions()
+    assert "moe_layer_forward" in names and "moe_pack_experts" in names and "moe_route_topk" in names
+    out = subprocess.run(["nm", "-D", "--defined-only", bq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r" T (moe_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(bq.lib, n)
+
+
+def test_status_strings():
+    assert bq.moe_status_string(bq.MOE_OK) == "ok"
+    assert "argument" in bq.moe_status_string(bq.MOE_ERR_INVALID_ARG)
+    assert bq.moe_status_string(99) == "unknown status"
+
+
+def test_route_workspace_size():
+    assert bq.moe_route_workspace_bytes(1, 512) == 256 + 512 * 4
+    assert bq.moe_route_workspace_bytes(0, 512) == 0
+
+
+def _desc(**kw):
+    base = dict(n_experts=4, hidden=64, inter=32, has_shared=0, max_tokens=8, max_top_k=2,
+                fmt_gate_up=bq.MOE_FMT_Q8_0, fmt_down=bq.MOE_FMT_Q8_0)
+    base.update(kw)
+    d = bq.moe_pack_desc()
+    for k, v in base.items():
+        setattr(d, k, v)
+    return d
+
+
+@pytest.mark.parametrize("kw", [
+    dict(n_experts=0), dict(n_experts=2000), dict(hidden=48), dict(inter=40), dict(max_tokens=0),
+    dict(max_top_k=5), dict(fmt_gate_up=9), dict(fmt_down=0),
+])
+def test_pack_rejects_bad_descriptions_without_a_device(kw):
+    buf = np.zeros(1 << 16, np.uint8)
+    d = _desc(**kw)
+    d.gate_up_blocks = buf.ctypes.data
+    d.down_blocks = buf.ctypes.data
+    h = ctypes.c_void_p()
+    assert bq.lib.moe_pack_experts(ctypes.byref(d), 0, ctypes.byref(h)) == bq.MOE_ERR_INVALID_ARG
+    assert not h.value
+
+
+def test_pack_requires_tables_scales_and_shared_blocks():
+    buf = np.zeros(1 << 16, np.uint8)
+    for kw in (dict(fmt_gate_up=bq.MOE_FMT_IQ4_NL), dict(fmt_down=bq.MOE_FMT_NVFP4), dict(has_shared=1)):
+        d = _desc(**kw)
+        d.gate_up_blocks = buf.ctypes.data
+        d.down_blocks = buf.ctypes.data
+        h = ctypes.c_void_p()
+        assert bq.lib.moe_pack_experts(ctypes.byref(d), 0, ctypes.byref(h)) == bq.MOE_ERR_INVALID_ARG
+    h = ctypes.c_void_p()
+    assert bq.lib.moe_pack_experts(None, 0, ctypes.byref(h)) == bq.MOE_ERR_INVALID_ARG
+
+
+def test_forward_and_route_reject_null_and_misaligned_pointers():
+    assert bq.lib.moe_layer_forward(None, 1, None, None, 0, 1, 1, None, None) == bq.MOE_ERR_INVALID_ARG
+    buf = np.zeros(4096, np.uint8)
+    p = buf.ctypes.data + 8 if buf.ctypes.data % 16 == 0 else buf.ctypes.data
+    assert bq.lib.moe_route_topk(p, 2, p, 1, 64, 4, 2, p, p, p, 4096, None) == bq.MOE_ERR_INVALID_ARG
+    a = buf.ctypes.data + (-buf.ctypes.data % 16)
+    # top_k > n_experts and hidden not a multiple of 8
+    assert bq.lib.moe_route_topk(a, 2, a, 1, 64, 4, 5, a, a, a, 4096, None) == bq.MOE_ERR_INVALID_ARG
+    assert bq.lib.moe_route_topk(a, 2, a, 1, 60, 4, 2, a, a, a, 4096, None) == bq.MOE_ERR_INVALID_ARG
+    assert bq.lib.moe_route_topk(a, 2, a, 1, 64, 4, 2, a, a, a, 16, None) == bq.MOE_ERR_INVALID_ARG

@@ -1,0 +1,123 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Routing: the selected expert set of every token must equal the oracle's
+(inputs carry a top-k logit margin >= 1e-3) and gates agree within 1e-5.
+Outputs: normwise max relative error per token <= 2e-3 (fp32-accumulate
+decode kernels).
+"""
+import numpy as np
+import pytest
+
+import synth
+from harness import (DECODE_TOL, assert_routing_equal, expected_counts, gpu_layer, normwise_err,
+                     oracle_layer, router_to_device, to_device)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def _layer(name, layer=0, **kw):
+    wl = synth.WORKLOADS[name].with_(**kw) if kw else synth.WORKLOADS[name]
+    return wl, synth.layer_inputs(wl, layer)
+
+
+def _check(li, x, k, tol=DECODE_TOL, path=None):
+    out, idx, gate, counts = gpu_layer(li, x, k, path=path)
+    ref, ridx, rgate = oracle_layer(li, x, k)
+    assert_routing_equal(idx, gate, ridx, rgate)
+    assert np.array_equal(counts, expected_counts(ridx, li.wl.n_experts, x.shape[0], li.wl.has_shared))
+    err = normwise_err(out, ref)
+    assert err <= tol, err
+    return err
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2])
+def test_tiny_q8_decode_one_token(layer):
+    wl, li = _layer("tiny_q8", layer)
+    _check(li, synth.tokens(wl, li.router, layer), wl.top_k)
+
+
+@pytest.mark.parametrize("step", [0, 1])
+def test_model_decode_iq4nl_q51_shared_one_token(step):
+    wl, li = _layer("model_decode")
+    _check(li, synth.tokens(wl, li.router, 0, step), wl.top_k)
+
+
+def test_spec_verify_eight_correlated_tokens():
+    wl, li = _layer("spec_verify", layer=5)
+    _check(li, synth.tokens(wl, li.router, 5), wl.top_k)
+
+
+def test_zipf_batch_nvfp4_64_tokens():
+    wl, li = _layer("zipf_batch", layer=2)
+    _check(li, synth.tokens(wl, li.router, 2), wl.top_k)
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_Q8_0, synth.FMT_Q5_1, synth.FMT_IQ4_NL, synth.FMT_NVFP4])
+def test_every_format_on_both_projections(fmt):
+    wl = synth.Workload("fmt", 1024, 32, 256, 4, True, fmt, fmt, synth.DT_BF16, 13, seed=fmt)
+    li = synth.layer_inputs(wl)
+    _check(li, synth.tokens(wl, li.router), wl.top_k)
+
+
+def test_ragged_shapes_and_k_equals_E():
+    # hidden 96 (3 units per row), inter 64, top_k = E, shared expert, 3 tokens
+    wl = synth.Workload("ragged", 96, 5, 64, 5, True, synth.FMT_IQ4_NL, synth.FMT_Q5_1, synth.DT_F32, 3,
+                        seed=4)
+    li = synth.layer_inputs(wl)
+    _check(li, synth.tokens(wl, li.router), 5)
+    # hidden 1056 (33 units: one lane of 32 takes two), top_k = 1
+    wl = synth.Workload("odd", 1056, 9, 96, 1, False, synth.FMT_Q8_0, synth.FMT_NVFP4, synth.DT_BF16, 17,
+                        seed=5)
+    li = synth.layer_inputs(wl)
+    _check(li, synth.tokens(wl, li.router), 1)
+
+
+def test_route_topk_bit_exact_sets_and_gates():
+    import block_quantized_expert_moe_b200 as bq
+    for name, T in (("tiny_q8", 1), ("model_decode", 1), ("zipf_batch", 64), ("spec_verify", 8)):
+        wl, li = _layer(name)
+        x = synth.tokens(wl, li.router, 0, 0, T)
+        xt, wr = to_device(x), router_to_device(li.router)
+        idx = torch.empty(T, wl.top_k, dtype=torch.int32, device="cuda")
+        gate = torch.empty(T, wl.top_k, dtype=torch.float32, device="cuda")
+        ws = torch.empty(bq.moe_route_workspace_bytes(T, wl.n_experts), dtype=torch.uint8, device="cuda")
+        bq.moe_route_topk(xt, wr, wl.top_k, idx, gate, ws)
+        torch.cuda.synchronize()
+        import oracle
+        ridx, rgate, _ = oracle.route(synth.tokens_f64(wl, x), li.router, wl.top_k)
+        assert np.array_equal(idx.cpu().numpy(), ridx)  # margin-guarded: order is unique too
+        assert np.abs(gate.cpu().numpy() - rgate).max() <= 1e-5
+
+
+def test_outputs_are_bitwise_reproducible():
+    wl, li = _layer("zipf_batch")
+    x = synth.tokens(wl, li.router)
+    outs, _, _, _ = gpu_layer(li, x, wl.top_k, repeat=3)
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+
+
+def test_fmt_argument_is_checked():
+    import block_quantized_expert_moe_b200 as bq
+    wl, li = _layer("tiny_q8")
+    pack = bq.pack_layer(li, max_tokens=4)
+    x = to_device(synth.tokens(wl, li.router))
+    out = torch.empty(1, wl.hidden, device="cuda")
+    with pytest.raises(bq.MoeError) as e:
+        bq.moe_layer_forward(x, router_to_device(li.router), pack, bq.MOE_FMT_NVFP4, wl.top_k, out)
+    assert e.value.status == bq.MOE_ERR_FMT_MISMATCH
+    with pytest.raises(bq.MoeError) as e:  # more tokens than the pack was sized for
+        bq.moe_layer_forward(torch.zeros(5, wl.hidden, device="cuda"), router_to_device(li.router), pack,
+                             0, wl.top_k, torch.empty(5, wl.hidden, device="cuda"))
+    assert e.value.status == bq.MOE_ERR_INVALID_ARG
+    pack.free()
+
+
+def test_pack_rejects_nan_block_scale():
+    import block_quantized_expert_moe_b200 as bq
+    wl = synth.Workload("nan", 64, 4, 32, 2, False, synth.FMT_NVFP4, synth.FMT_NVFP4, synth.DT_BF16, 1)
+    li = synth.layer_inputs(wl)
+    li.gate_up[1, 9 * 3] = 0x7F  # E4M3 NaN scale in expert 1
+    with pytest.raises(bq.MoeError) as e:
+        bq.pack_layer(li)
+    assert e.value.status == bq.MOE_ERR_INVALID_ARG
