@@ -63,6 +63,8 @@ def _load():
     L.moe_route_workspace_bytes.argtypes = [i32, i32]
     L.moe_route_topk.restype = i32
     L.moe_route_topk.argtypes = [vp, i32, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+    L.moe_route_topk_noalloc.restype = i32
+    L.moe_route_topk_noalloc.argtypes = [vp, i32, vp, i32, i32, i32, i32, vp, vp, vp]
     L.moe_layer_forward.restype = i32
     L.moe_layer_forward.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, vp]
     L.moe_layer_forward_ex.restype = i32
@@ -186,6 +188,17 @@ def moe_route_topk(x, router_w, top_k, idx_out, gate_out, workspace, stream=None
                               idx_out.data_ptr(), gate_out.data_ptr(), workspace.data_ptr(),
                               workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
            "moe_route_topk")
+
+
+def moe_route_topk_noalloc(x, router_w, top_k, idx_out, gate_out, stream=None):
+    """moe_route_topk for callers that cannot allocate: the scratch is a fixed
+    array inside the library (n_tokens * n_experts <= 65536; calls that overlap
+    on the GPU race; the first call on a device must precede any capture)."""
+    T, H = x.shape
+    E = router_w.shape[0]
+    _check(lib.moe_route_topk_noalloc(x.data_ptr(), _dtype_code(x), router_w.data_ptr(), T, H, E, top_k,
+                                      idx_out.data_ptr(), gate_out.data_ptr(), _stream_ptr(stream)),
+           "moe_route_topk_noalloc")
 
 
 def moe_layer_forward(x, router_w, pack, fmt, top_k, out, stream=None):

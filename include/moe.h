@@ -162,6 +162,25 @@ moe_status moe_route_topk(const void *x, moe_dtype x_dtype, const uint16_t *rout
                           float *gate_out, void *workspace, size_t workspace_bytes,
                           void *stream);
 
+/* moe_route_topk without a workspace argument.  This entry point has no
+ * counterpart in the pages; it exists for callers that cannot allocate device
+ * memory (code running while a global-mode stream capture is open, where
+ * cudaMalloc is illegal, or a host framework that forbids allocation after
+ * start-up because cudaMalloc/cudaFree can synchronise the device).  Its
+ * scratch is a fixed array inside the library, present on every device that
+ * loads it until the process exits:
+ *   n_tokens * n_experts <= 65536 (e.g. 64 x 1024), else MOE_ERR_INVALID_ARG;
+ *   nothing is allocated; the ticket it needs at zero is cleared on `stream`
+ *   by each call;
+ *   all calls on a device share the scratch: calls that overlap on the GPU
+ *   (unordered streams) race and give wrong results;
+ *   the first call on a device looks up the scratch address - make it before
+ *   any stream capture starts.
+ * Other arguments, layouts and outputs as moe_route_topk. */
+moe_status moe_route_topk_noalloc(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
+                                  int n_tokens, int hidden, int n_experts, int top_k,
+                                  int32_t *idx_out, float *gate_out, void *stream);
+
 /* The whole layer: route, plan, grouped gate/up + SwiGLU, down, combine.
  *   x        device [n_tokens x hidden] fp32 or bf16
  *   router_w device [n_experts x hidden] bf16 bits
