@@ -30,9 +30,10 @@ import synth  # noqa: E402
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
-STAGES = ["route_plan", "gate_up", "down", "combine"]
+STAGES = ["route_plan", "gate_up", "down", "combine", "fused", "prefill"]
 KERNEL_NAMES = {"route_plan": "route_kernel", "gate_up": "matvec_kernel<gate/up>",
-                "down": "matvec_kernel<down>", "combine": "combine_kernel"}
+                "down": "matvec_kernel<down>", "combine": "combine_kernel",
+                "fused": "fused_decode_kernel", "prefill": "prefill sequence"}
 
 
 def parse():
@@ -120,6 +121,17 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak(kind):
+    """Dense tensor peak in TFLOP/s for bf16 or fp4 (fp4 = bf16 x 4, the nominal
+    2.25 -> 9 PFLOP/s ratio), sustained figure (prefill runs inside long steps)."""
+    try:
+        p = json.load(open(PEAKS_FILE))
+        bf16, src = float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured sustained bf16"
+    except Exception:
+        bf16, src = 1400.0, "fallback sustained bf16"
+    return (bf16 * 4.0, src + " x4 (nominal fp4/bf16)") if kind == "fp4" else (bf16, src)
 
 
 def kernel_traffic(stage, wl_name):
@@ -273,6 +285,12 @@ def ours_arm(a, wl):
         "down": [na * dn_b + s * I * 4 + s * H * 4 for na, s in zip(n_active, slots)],
         "combine": [s * H * 4 + T * H * 4 for s in slots],
     }
+    # the fused kernel reads the router, every active expert's blocks and x,
+    # writes and re-reads h, and writes out
+    stage_bytes["fused"] = [E * H * 2 + na * exp_b + T * H * xbytes + 2 * s * I * 4 + T * H * 4
+                            for na, s in zip(n_active, slots)]
+    # prefill: tensor work of the router and both expert GEMMs
+    prefill_flops = [2.0 * T * H * E + 2.0 * s * H * 2 * I + 2.0 * s * I * H for s in slots]
     unique_bytes_step = sum(na * exp_b + E * H * 2 for na in n_active)
 
     def barrier():
@@ -319,23 +337,34 @@ def ours_arm(a, wl):
                 fwd(ly)
     gp.replay()
     torch.cuda.synchronize()
-    stage_ms = np.zeros(4)
+    stage_ms = np.zeros(6)
     nf = 0
     for ly in layers:
         m, n = bq.moe_profile_end(ly["pack"])
         stage_ms += m
         nf += n
-    stage_us = {s: float(stage_ms[i] / nf * 1e3) for i, s in enumerate(STAGES)}
-    dom = max(STAGES, key=lambda s: stage_us[s])
-    dom_bytes = float(np.mean(stage_bytes[dom]))
+    prefill_kernels = 7 if wl.fmt_gate_up == synth.FMT_NVFP4 else 6  # route GEMM, top-k, plan, gather, GEMMs (+ h quant)
+    launches_per_fwd = 1 if stage_ms[4] > 0 else (prefill_kernels if stage_ms[5] > 0 else 4)
+    stage_us = {s: float(stage_ms[i] / nf * 1e3) for i, s in enumerate(STAGES) if stage_ms[i] > 0}
+    dom = max(stage_us, key=lambda s: stage_us[s])
     hbm, peak_src = peaks()
-    achieved = dom_bytes / (stage_us[dom] * 1e-6) / 1e9
     traffic = kernel_traffic(dom, wl.name)
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": traffic, "kernel": KERNEL_NAMES[dom],
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
-                else "fallback 6650 GB/s",
-                "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": stage_us[dom]}
+    if dom == "prefill":
+        kind = "fp4" if wl.fmt_gate_up == synth.FMT_NVFP4 else "bf16"
+        tpk, tsrc = tensor_peak(kind)
+        fl = float(np.mean(prefill_flops))
+        achieved = fl / (stage_us[dom] * 1e-6) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": tpk, "unit": "TFLOP/s",
+                    "frac": achieved / tpk, "traffic": traffic, "kernel": KERNEL_NAMES[dom],
+                    "peak_source": tsrc, "algorithmic_flops_per_launch": fl, "avg_launch_us": stage_us[dom]}
+    else:
+        dom_bytes = float(np.mean(stage_bytes[dom]))
+        achieved = dom_bytes / (stage_us[dom] * 1e-6) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "traffic": traffic, "kernel": KERNEL_NAMES[dom],
+                    "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                    else "fallback 6650 GB/s",
+                    "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": stage_us[dom]}
     del gp
 
     # ---- end to end: pinned host input -> forward -> host output, every layer, every step
@@ -390,7 +419,7 @@ def ours_arm(a, wl):
                 "unique_expert_bytes_per_step": unique_bytes_step,
                 "active_experts_per_layer": float(np.mean(n_active)),
                 "stage_us": stage_us, "roofline": roofline, "clocks": clk.summary(),
-                "e2e": e2e, "gpu_launches": 4 * L * a.steps, "cpu_baseline": cpu,
+                "e2e": e2e, "gpu_launches": launches_per_fwd * L * a.steps, "cpu_baseline": cpu,
                 "gen_seconds": gen_s}
         print(json.dumps(line), flush=True)
     if dist is not None:

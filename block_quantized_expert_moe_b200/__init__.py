@@ -19,7 +19,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_FMT_MISMATCH = 0, 1, 2
 MOE_ERR_OOM, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE = 4, 5, 6, 7
 MOE_FMT_FROM_PACK, MOE_FMT_Q8_0, MOE_FMT_Q5_1, MOE_FMT_IQ4_NL, MOE_FMT_NVFP4 = 0, 1, 2, 3, 4
 MOE_DT_F32, MOE_DT_BF16 = 1, 2
-MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_DENSE = 0, 1, 2, 3
+MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_DENSE, MOE_PATH_GROUPED = 0, 1, 2, 3, 4
 
 
 class MoeError(RuntimeError):
@@ -230,8 +230,8 @@ def moe_profile_begin(pack, max_forwards):
 
 
 def moe_profile_end(pack):
-    """-> (ms per stage [route+plan, gate/up, down, combine] summed, n_forwards)."""
-    ms = np.zeros(4, np.float64)
+    """-> (ms per kernel [route+plan, gate/up, down, combine, fused, prefill] summed, n_forwards)."""
+    ms = np.zeros(6, np.float64)
     n = ctypes.c_int(0)
     _check(lib.moe_profile_end(pack.handle, _np_ptr(ms), ctypes.byref(n)), "moe_profile_end")
     return ms, n.value

@@ -18,6 +18,10 @@ cudaError_t route_set_attributes();
 cudaError_t matvec_set_attributes();
 }  // namespace moe
 
+// kernel-stage slots of the profiling API (moe_profile_end's ms[])
+enum { PROF_ROUTE = 0, PROF_GATE_UP = 1, PROF_DOWN = 2, PROF_COMBINE = 3, PROF_FUSED = 4, PROF_PREFILL = 5,
+       PROF_STAGES = 6 };
+
 using namespace moe;
 
 struct moe_pack {
@@ -31,10 +35,15 @@ struct moe_pack {
     Workspace ws;
     int64_t arena_bytes = 0, workspace_bytes = 0;
     int grid_cache[2][2];  // [gateup][tt==8]
-    // kernel-stage timing (moe_profile_begin/end)
+    // kernel-stage timing (moe_profile_begin/end): per recorded forward, the
+    // first event index and its path (fused: 2 events, grouped: 5)
     bool prof_on = false;
     std::vector<cudaEvent_t> prof_ev;
+    std::vector<std::pair<int, int>> prof_fwd;
     int prof_used = 0;
+    int fused_grid[2] = {0, 0};   // [tt==8]
+    bool has_prefill = false;     // tensor-core prefill workspace present
+    PrefillWorkspace pws;
 };
 
 namespace {
@@ -57,6 +66,10 @@ moe_status init_device(int dev)
     if (g_dev_ready[dev]) return MOE_OK;
     if (route_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (matvec_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
+    if (fused_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
+    if (prefill_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
+    if (prefill_nvfp4_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
+    if (prefill_q8_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     g_dev_ready[dev] = true;
     return MOE_OK;
 }
@@ -99,9 +112,14 @@ void plane_rows(int fmt, int cols, int &qs_row, int &sc_row, int &qh_row)
     case MOE_FMT_Q8_0: qs_row = cols; sc_row = cols / 32 * 2; break;
     case MOE_FMT_Q5_1: qs_row = cols / 2; sc_row = cols / 32 * 4; qh_row = cols / 32 * 4; break;
     case MOE_FMT_IQ4_NL: qs_row = cols / 2; sc_row = cols / 32 * 2; break;
-    default: qs_row = cols / 2; sc_row = cols / 16; break;  // NVFP4
+    default: qs_row = cols / 2; sc_row = 0; break;  // NVFP4: scales in the block-scale layout
     }
 }
+
+int nvfp4_ksteps(int cols) { return (cols + 63) / 64; }
+
+// bytes of one expert's NVFP4 scale plane: 128-row blocks x K steps x 512
+int64_t nvfp4_sf_bytes(int rows, int cols) { return (int64_t)((rows + 127) / 128) * nvfp4_ksteps(cols) * 512; }
 
 int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
@@ -140,10 +158,11 @@ bool repack_expert(int fmt, const uint8_t *src, int rows, int cols, uint8_t *qs,
                 std::memcpy(q + 16 * b, blk + 2, 16);
             }
         } else {
+            const int ks = nvfp4_ksteps(cols);
             for (int b = 0; b < cols / 16; ++b) {
                 const uint8_t *blk = row + b * 9;
                 if (blk[0] >= 0x7Fu) return false;  // negative scale or NaN
-                s[b] = blk[0];
+                sc[sf_offset(r, b >> 2, b & 3, ks)] = blk[0];
                 std::memcpy(q + 8 * b, blk + 1, 8);
             }
         }
@@ -196,7 +215,8 @@ moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, con
     dp.cols = cols;
     plane_rows(fmt, cols, dp.qs_row, dp.sc_row, dp.qh_row);
     dp.qs_stride = round_up((int64_t)rows * dp.qs_row, 256);
-    dp.sc_stride = round_up((int64_t)rows * dp.sc_row, 256);
+    dp.sc_stride = round_up(fmt == MOE_FMT_NVFP4 ? nvfp4_sf_bytes(rows, cols) : (int64_t)rows * dp.sc_row, 256);
+    dp.ksteps = fmt == MOE_FMT_NVFP4 ? nvfp4_ksteps(cols) : 0;
     dp.qh_stride = round_up((int64_t)rows * dp.qh_row, 256);
     const int64_t canon = canon_row_bytes(fmt, cols) * rows;
     std::vector<uint8_t> hq, hs, hh;
@@ -251,7 +271,7 @@ moe_status build_workspace(moe_pack *p)
         {(void **)&w.logits, T * E * 4}, {(void **)&w.idx, T * k * 4}, {(void **)&w.gate, T * k * 4},
         {(void **)&w.cnt, (E + 1) * 4}, {(void **)&w.off, (E + 1) * 4}, {(void **)&w.perm_tok, slots * 4},
         {(void **)&w.slot_pos, T * k * 4}, {(void **)&w.groups, (int64_t)w.max_groups * 16},
-        {(void **)&w.n_groups, 4}, {(void **)&w.ticket, 4}, {(void **)&w.err, 4},
+        {(void **)&w.n_groups, 4}, {(void **)&w.ticket, 4}, {(void **)&w.err, 4}, {(void **)&w.bar, 8},
         {(void **)&w.h, slots * p->I * 4}, {(void **)&w.y, slots * p->H * 4},
     };
     int64_t total = 0;
@@ -266,6 +286,44 @@ moe_status build_workspace(moe_pack *p)
         o += round_up(it.bytes, 256);
     }
     p->workspace_bytes = total;
+    return MOE_OK;
+}
+
+// Buffers of the tensor-core prefill (NVFP4 experts, more than 64 tokens).
+moe_status build_prefill_workspace(moe_pack *p)
+{
+    const int64_t T = p->max_tokens, k = p->max_top_k, E = p->E, H = p->H, I = p->I;
+    const int64_t rows = round_up(T * k + T + (E + 1) * 127, 128);
+    PrefillWorkspace &w = p->pws;
+    w.logits = p->ws.logits;
+    w.idx = p->ws.idx;
+    w.gate = p->ws.gate;
+    w.slot_pos = p->ws.slot_pos;
+    w.cnt = p->ws.cnt;
+    w.max_rows = (int)rows;
+    struct Item { void **dst; int64_t bytes; };
+    Item items[] = {
+        {(void **)&w.pad_off, (E + 2) * 4}, {(void **)&w.fill, (E + 2) * 4}, {(void **)&w.tiles, rows / 128 * 8 + 64},
+        {(void **)&w.ptiles, rows / 128 * 16 + 64}, {(void **)&w.n_ptiles, 4},
+        {(void **)&w.n_tiles, 4}, {(void **)&w.total_rows, 4}, {(void **)&w.perm_tok, rows * 4},
+        {(void **)&w.row_gate, rows * 4}, {(void **)&w.row_scale_x, rows * 4}, {(void **)&w.row_scale_h, rows * 4},
+        {(void **)&w.a_q, p->fmt_gu == MOE_FMT_Q8_0 ? rows * H * 2 : rows * H / 2},
+        {(void **)&w.sfa, rows / 128 * (H / 64) * 512},
+        {(void **)&w.h, rows * I * 4}, {(void **)&w.h_q, rows * I / 2}, {(void **)&w.sfh, rows / 128 * (I / 64) * 512},
+    };
+    int64_t total = 0;
+    for (auto &it : items) total += round_up(it.bytes, 256);
+    void *base;
+    moe_status st = dev_alloc(p, (size_t)total, &base);
+    if (st != MOE_OK) return st;
+    if (cudaMemset(base, 0, (size_t)total) != cudaSuccess) return MOE_ERR_CUDA;
+    int64_t o = 0;
+    for (auto &it : items) {
+        *it.dst = static_cast<char *>(base) + o;
+        o += round_up(it.bytes, 256);
+    }
+    p->workspace_bytes += total;
+    p->has_prefill = true;
     return MOE_OK;
 }
 
@@ -358,6 +416,11 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
         st = build_proj(p, p->dn, p->fmt_dn, p->H, p->I, static_cast<const uint8_t *>(d->down_blocks),
                         static_cast<const uint8_t *>(d->shared_down_blocks), dts.data(), n_slots);
     if (st == MOE_OK) st = build_workspace(p);
+    const bool nv = p->fmt_gu == MOE_FMT_NVFP4 && p->fmt_dn == MOE_FMT_NVFP4 &&
+                    prefill_nvfp4_supported(p->H, p->I, p->E, p->max_top_k);
+    const bool q8 = p->fmt_gu == MOE_FMT_Q8_0 && p->fmt_dn == MOE_FMT_Q8_0 &&
+                    prefill_q8_supported(p->H, p->I, p->E, p->max_top_k);
+    if (st == MOE_OK && p->max_tokens > kDecodeMaxTokens && (nv || q8)) st = build_prefill_workspace(p);
     if (st == MOE_OK && cudaDeviceSynchronize() != cudaSuccess) st = MOE_ERR_CUDA;
     if (st != MOE_OK) {
         free_pack_memory(p);
@@ -381,8 +444,13 @@ moe_status moe_pack_free(moe_pack *p)
 moe_status moe_pack_query(const moe_pack *p, moe_pack_info *info)
 {
     if (!p || !info) return MOE_ERR_INVALID_ARG;
-    info->gate_up_bytes_per_expert = (int64_t)p->gu.rows * (p->gu.qs_row + p->gu.sc_row + p->gu.qh_row);
-    info->down_bytes_per_expert = (int64_t)p->dn.rows * (p->dn.qs_row + p->dn.sc_row + p->dn.qh_row);
+    // HBM bytes one expert's blocks occupy (the NVFP4 scale bytes as stored: K/16 per row)
+    auto proj_bytes = [](const DevProj &d) {
+        const int64_t sc = d.fmt == MOE_FMT_NVFP4 ? (int64_t)d.cols / 16 : d.sc_row;
+        return (int64_t)d.rows * (d.qs_row + sc + d.qh_row);
+    };
+    info->gate_up_bytes_per_expert = proj_bytes(p->gu);
+    info->down_bytes_per_expert = proj_bytes(p->dn);
     info->expert_bytes = info->gate_up_bytes_per_expert + info->down_bytes_per_expert +
                          (p->fmt_gu == MOE_FMT_NVFP4 ? 4 : 0) + (p->fmt_dn == MOE_FMT_NVFP4 ? 4 : 0);
     info->arena_bytes = p->arena_bytes;
@@ -428,6 +496,14 @@ moe_status moe_route_topk(const void *x, moe_dtype x_dtype, const uint16_t *rout
     a.idx = idx_out;
     a.gate = gate_out;
     a.do_plan = 0;
+    if (x_dtype == MOE_DT_BF16 && n_tokens > kDecodeMaxTokens) {
+        // many tokens: the router as a tensor-core GEMM (word 1 of the workspace
+        // records a timed-out wait), then top-k per token
+        int32_t *werr = a.ticket + 1;
+        if (cudaMemsetAsync(werr, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+        return check_launch(prefill_route(x, router_w, n_tokens, hidden, n_experts, top_k, a.logits, idx_out,
+                                          gate_out, nullptr, werr, s));
+    }
     if (cudaMemsetAsync(a.ticket, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
     return check_launch(launch_route(a, route_grid(n_experts, sms), s));
 }
@@ -442,14 +518,89 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     if (n_tokens < 1 || n_tokens > p->max_tokens) return MOE_ERR_INVALID_ARG;
     if (top_k < 1 || top_k > p->max_top_k) return MOE_ERR_INVALID_ARG;
     if (fmt != MOE_FMT_FROM_PACK && fmt != p->fmt_gu) return MOE_ERR_FMT_MISMATCH;
-    if (path == MOE_PATH_AUTO) path = MOE_PATH_DECODE;
-    if (path != MOE_PATH_DECODE) return MOE_ERR_UNSUPPORTED;
+    const bool prefill_ok = p->has_prefill && x_dtype == MOE_DT_BF16 && top_k <= 32;
+    if (path == MOE_PATH_AUTO)
+        path = n_tokens <= kDecodeMaxTokens ? MOE_PATH_DECODE : (prefill_ok ? MOE_PATH_PREFILL : MOE_PATH_GROUPED);
+    if (path == MOE_PATH_PREFILL && !prefill_ok) return MOE_ERR_UNSUPPORTED;
+    if (path != MOE_PATH_DECODE && path != MOE_PATH_GROUPED && path != MOE_PATH_PREFILL) return MOE_ERR_UNSUPPORTED;
     DeviceGuard g(p->device);
     if (!g.ok) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     moe_pack *pm = const_cast<moe_pack *>(p);
     const Workspace &w = p->ws;
     const int T = n_tokens, k = top_k;
+    if (path == MOE_PATH_PREFILL) {
+        PrefillNvArgs pa{};
+        pa.x = x;
+        pa.wr = router_w;
+        pa.T = T;
+        pa.H = p->H;
+        pa.I = p->I;
+        pa.E = p->E;
+        pa.k = k;
+        pa.has_shared = p->has_shared;
+        pa.gu = &p->gu;
+        pa.dn = &p->dn;
+        pa.out = out;
+        pa.err = w.err;
+        pa.ws = &p->pws;
+        pa.num_sms = p->num_sms;
+        int pbase = -1;
+        if (pm->prof_on && (size_t)pm->prof_used + 2 <= pm->prof_ev.size()) {
+            pbase = pm->prof_used;
+            pm->prof_used += 2;
+            pm->prof_fwd.push_back({pbase, 2});
+        }
+        prof_mark(pm, pbase, 0, s);
+        moe_status st = check_launch(p->fmt_gu == MOE_FMT_Q8_0 ? prefill_q8_forward(pa, s) : prefill_nvfp4_forward(pa, s));
+        prof_mark(pm, pbase, 1, s);
+        return st;
+    }
+    if (path == MOE_PATH_DECODE && T <= kFusedMaxT && k <= kFusedMaxK) {
+        FusedArgs fa{};
+        fa.x = x;
+        fa.x_dtype = x_dtype;
+        fa.wr = router_w;
+        fa.T = T;
+        fa.H = p->H;
+        fa.E = p->E;
+        fa.I = p->I;
+        fa.k = k;
+        fa.has_shared = p->has_shared;
+        fa.gu = p->gu;
+        fa.dn = p->dn;
+        std::memcpy(fa.tab_gu, p->fmt_gu == MOE_FMT_NVFP4 ? kNvfp4Tab : p->tab, sizeof(fa.tab_gu));
+        std::memcpy(fa.tab_dn, p->fmt_dn == MOE_FMT_NVFP4 ? kNvfp4Tab : p->tab, sizeof(fa.tab_dn));
+        fa.logits = w.logits;
+        fa.h = w.h;
+        fa.y = w.y;
+        fa.out = out;
+        fa.idx_out = w.idx;
+        fa.gate_out = w.gate;
+        fa.cnt_out = w.cnt;
+        fa.bar = w.bar;
+        fa.err = w.err;
+        const int tt = T == 1 ? 1 : 8;
+        const size_t limit = 220 * 1024;
+        fa.rowsplit = fused_smem_bytes(fa, tt, 1) <= limit ? 1 : 0;
+        const size_t smem = fused_smem_bytes(fa, tt, fa.rowsplit);
+        if (smem <= limit) {
+            int &grid = pm->fused_grid[tt == 8];
+            if (!grid) grid = fused_grid(tt, 220 * 1024, p->num_sms);
+            if (grid > 0) {
+                int pbase = -1;
+                if (pm->prof_on && (size_t)pm->prof_used + 2 <= pm->prof_ev.size()) {
+                    pbase = pm->prof_used;
+                    pm->prof_used += 2;
+                    pm->prof_fwd.push_back({pbase, 1});
+                }
+                prof_mark(pm, pbase, 0, s);
+                moe_status st = check_launch(launch_fused(fa, tt, grid, smem, s));
+                prof_mark(pm, pbase, 1, s);
+                return st;
+            }
+        }
+    }
     // tokens per work group: 8 unless a single token, or 8 staged fp32 rows of
     // the longer reduction would not fit in shared memory
     const int kmax = std::max(p->H, p->I);
@@ -458,6 +609,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     if (pm->prof_on && (size_t)pm->prof_used + 5 <= pm->prof_ev.size()) {
         pbase = pm->prof_used;
         pm->prof_used += 5;
+        pm->prof_fwd.push_back({pbase, 0});
     }
     prof_mark(pm, pbase, 0, s);
 
@@ -573,6 +725,7 @@ moe_status moe_profile_begin(moe_pack *p, int max_forwards)
             p->prof_ev.clear();
             return MOE_ERR_CUDA;
         }
+    p->prof_fwd.clear();
     p->prof_used = 0;
     p->prof_on = true;
     return MOE_OK;
@@ -583,24 +736,28 @@ moe_status moe_profile_end(moe_pack *p, double *ms, int *n_forwards)
     if (!p || !p->prof_on) return MOE_ERR_INVALID_ARG;
     DeviceGuard g(p->device);
     moe_status st = cudaDeviceSynchronize() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-    double acc[4] = {0, 0, 0, 0};
-    const int n = p->prof_used / 5;
-    for (int f = 0; f < n && st == MOE_OK; ++f)
-        for (int i = 0; i < 4; ++i) {
+    double acc[PROF_STAGES] = {0, 0, 0, 0, 0, 0};
+    for (const auto &f : p->prof_fwd) {
+        if (st != MOE_OK) break;
+        const int nint = f.second ? 1 : 4;
+        for (int i = 0; i < nint; ++i) {
             float v = 0.f;
-            if (cudaEventElapsedTime(&v, p->prof_ev[(size_t)5 * f + i], p->prof_ev[(size_t)5 * f + i + 1]) !=
+            if (cudaEventElapsedTime(&v, p->prof_ev[(size_t)f.first + i], p->prof_ev[(size_t)f.first + i + 1]) !=
                 cudaSuccess) {
                 st = MOE_ERR_CUDA;
                 break;
             }
-            acc[i] += v;
+            acc[f.second == 1 ? PROF_FUSED : f.second == 2 ? PROF_PREFILL : i] += v;
         }
+    }
     for (auto &e : p->prof_ev) cudaEventDestroy(e);
+    const int n = (int)p->prof_fwd.size();
     p->prof_ev.clear();
+    p->prof_fwd.clear();
     p->prof_on = false;
     p->prof_used = 0;
     if (ms)
-        for (int i = 0; i < 4; ++i) ms[i] = acc[i];
+        for (int i = 0; i < PROF_STAGES; ++i) ms[i] = acc[i];
     if (n_forwards) *n_forwards = n;
     return st;
 }

@@ -20,8 +20,10 @@ constexpr int kDecodeMaxTokens = 64;
 //   Q5_1    qs: rows x K/2 (16 B per 32-block, canonical nibble order)
 //           qh: rows x K/32 u32, sc: rows x K/32 {fp16 d, fp16 m}
 //   IQ4_NL  qs: rows x K/2, sc: rows x K/32 fp16 d
-//   NVFP4   qs: rows x K/2 (8 B per 16-block), sc: rows x K/16 E4M3 scales,
-//           ts: one fp32 matrix scale per expert
+//   NVFP4   qs: rows x K/2 (8 B per 16-block); sc: E4M3 block scales in the
+//           tcgen05 block-scale layout (see sf_offset), shared by the decode
+//           kernels and the block-scaled prefill MMA; ts: one fp32 matrix
+//           scale per expert
 // Expert e's plane starts at base + e * stride.
 struct DevProj {
     int fmt = 0, rows = 0, cols = 0;
@@ -30,8 +32,18 @@ struct DevProj {
     const uint8_t *qh = nullptr;
     const float *ts = nullptr;
     int64_t qs_stride = 0, sc_stride = 0, qh_stride = 0;  // bytes per expert
-    int qs_row = 0, sc_row = 0, qh_row = 0;               // bytes per row
+    int qs_row = 0, sc_row = 0, qh_row = 0;               // bytes per row (sc_row: not NVFP4)
+    int ksteps = 0;                                       // NVFP4: 64-wide K steps per row
 };
+
+// Byte offset of E4M3 scale q (0..3) of row r in 64-wide K step s, in the
+// block-scale layout of the tcgen05 block-scaled MMA: atoms of 512 bytes hold
+// 128 rows x 4 scales, row r at (r % 32) * 16 + ((r / 32) % 4) * 4; atoms run
+// over K steps first, then over 128-row blocks.
+__host__ __device__ inline int64_t sf_offset(int r, int s, int q, int ksteps)
+{
+    return ((int64_t)(r >> 7) * ksteps + s) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + q;
+}
 
 // Forward workspace (device), sized at pack time for max_tokens x max_top_k.
 struct Workspace {
@@ -45,6 +57,7 @@ struct Workspace {
     int4 *groups = nullptr;      // {expert, first slot, tokens, 0}
     int32_t *n_groups = nullptr;
     int32_t *ticket = nullptr;   // last-CTA counter of the route kernel
+    unsigned *bar = nullptr;     // grid barrier of the fused decode kernel {count, gen}
     int32_t *err = nullptr;      // sticky device error (moe_status)
     float *h = nullptr;          // [slots x I]
     float *y = nullptr;          // [slots x H]
@@ -102,5 +115,74 @@ size_t matvec_smem_bytes(const MatvecArgs &a, bool gateup, int tt);
 int matvec_grid(const MatvecArgs &a, bool gateup, int tt, int num_sms);
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
+
+// Fused decode (one cooperative launch per layer, n_tokens <= 8).
+constexpr int kFusedMaxT = 8;
+constexpr int kFusedMaxK = 16;
+
+struct FusedArgs {
+    const void *x;
+    int x_dtype;
+    const uint16_t *wr;
+    int T, H, E, I, k, has_shared;
+    DevProj gu, dn;
+    uint32_t tab_gu[4], tab_dn[4];
+    float *logits;      // [T x E]
+    float *h;           // [slots x I]
+    float *y;           // [slots x H] (when not rowsplit)
+    float *out;         // [T x H]
+    int32_t *idx_out;   // routing readback, written by CTA 0
+    float *gate_out;
+    int32_t *cnt_out;
+    unsigned *bar;      // {arrive count, generation}
+    int32_t *err;
+    int rowsplit;       // down + combine by output rows in one phase
+};
+
+// tensor-core prefill
+struct PrefillWorkspace {
+    float *logits = nullptr;   // [T x E]
+    int32_t *idx = nullptr;    // [T x k]
+    float *gate = nullptr;     // [T x k]
+    int32_t *slot_pos = nullptr;
+    int32_t *cnt = nullptr;    // [E + 1]
+    int32_t *pad_off = nullptr, *fill = nullptr;  // [E + 1]
+    int2 *tiles = nullptr;     // [max_rows / 128]  128-row M tiles
+    int4 *ptiles = nullptr;    // [max_rows / 128]  pairs of M tiles of one expert (bf16 path)
+    int32_t *n_tiles = nullptr, *total_rows = nullptr, *n_ptiles = nullptr;
+    int32_t *perm_tok = nullptr;  // [max_rows]
+    float *row_gate = nullptr, *row_scale_x = nullptr, *row_scale_h = nullptr;  // [max_rows]
+    uint8_t *a_q = nullptr, *sfa = nullptr;  // gate/up activations: NVFP4 codes + scales, or bf16 rows (Q8_0)
+    float *h = nullptr;                      // [max_rows x I]
+    uint8_t *h_q = nullptr, *sfh = nullptr;  // NVFP4 activations of the down GEMM
+    int max_rows = 0;
+};
+
+struct PrefillNvArgs {
+    const void *x;  // bf16 [T x H]
+    const uint16_t *wr;
+    int T, H, I, E, k, has_shared;
+    const DevProj *gu, *dn;
+    float *out;
+    int32_t *err;
+    const PrefillWorkspace *ws;
+    int num_sms;
+};
+
+cudaError_t prefill_set_attributes();
+cudaError_t prefill_nvfp4_set_attributes();
+bool prefill_nvfp4_supported(int H, int I, int E, int k);
+cudaError_t prefill_nvfp4_forward(const PrefillNvArgs &a, cudaStream_t s);
+cudaError_t prefill_plan_launch(const PrefillWorkspace &w, int E, int T, int has_shared, int32_t *err, cudaStream_t s);
+cudaError_t prefill_q8_set_attributes();
+bool prefill_q8_supported(int H, int I, int E, int k);
+cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s);
+cudaError_t prefill_route(const void *x_bf16, const uint16_t *wr, int T, int H, int E, int k, float *logits,
+                          int32_t *idx, float *gate, int32_t *cnt, int32_t *err, cudaStream_t s);
+
+size_t fused_smem_bytes(const FusedArgs &a, int tt, int rowsplit);
+cudaError_t fused_set_attributes();
+int fused_grid(int tt, size_t smem, int num_sms);
+cudaError_t launch_fused(const FusedArgs &a, int tt, int grid, size_t smem, cudaStream_t s);
 
 }  // namespace moe

@@ -1,0 +1,388 @@
+// Tensor-core prefill for Q8_0 experts: the weight blocks are dequantised to
+// bf16 in shared memory and multiplied with tcgen05.mma kind::f16.
+//
+// The same padded slot space as the NVFP4 prefill (every 128-row M tile
+// belongs to one expert).  A CTA tile is up to two consecutive M tiles of one
+// expert (256 rows) by 256 weight rows: each dequantised weight stage then feeds
+// two 128 x 256 MMAs, halving the dequantisation work per multiply-add, and the
+// two f32 accumulators fill the 512 tensor-memory columns.
+//
+//   warps 0-3    epilogue (one accumulator row per thread and half)
+//   warp 4       TMA producer of the activation tiles (bf16, 128-byte swizzle)
+//   warp 5       MMA issuer (one elected thread)
+//   warps 6-13   dequantisers: thread n owns weight row n of the stage; it
+//                loads the row's 64 int8 codes and two fp16 scales (the next
+//                stage's already in flight), converts q*d to bf16 and stores
+//                the eight 16-byte chunks at their 128-byte-swizzle positions,
+//                then makes them visible to the tensor core (fence.proxy.async)
+//
+//   gate/up  A = x rows gathered into slot order (bf16); B rows 0..127 the gate
+//            rows n0..n0+127, rows 128..255 the up rows I+n0..;
+//            epilogue h = silu(d_g) * d_u, stored bf16 for the down GEMM
+//   down     A = h (bf16); B = D_e rows n0..n0+255;
+//            epilogue out[token] += gate * d (fp32 vector reductions)
+// All mbarrier waits are bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "moe_internal.cuh"
+#include "tc_common.cuh"
+#include "tma_maps.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace tc;
+using namespace tmaps;
+
+constexpr int kQ8Threads = 448;  // 14 warps
+constexpr int kQ8Stages = 3;
+constexpr int kQ8A = 128 * 128;  // one 128-row half: 128 rows x 64 bf16
+constexpr int kQ8B = 256 * 128;  // 256 weight rows x 64 bf16
+constexpr int kQ8Stage = 2 * kQ8A + kQ8B;
+constexpr size_t kQ8Smem = (size_t)kQ8Stages * kQ8Stage + 1024;
+
+struct Q8GemmArgs {
+    const int4 *ptiles;        // {expert, first padded row, halves (1|2), 0}
+    const int32_t *n_ptiles;
+    int NT;                    // weight-row tiles of 256 (gate/up: I/128 pairs of 128)
+    int K;                     // reduction length
+    const uint8_t *qs;         // Q8_0 codes plane (stored +128), rows x K bytes per expert
+    int64_t qs_stride;
+    const uint8_t *sc;         // fp16 scale plane, rows x K/32 per expert
+    int64_t sc_stride;
+    int sc_row;
+    int up_off;                // gate/up: row offset of U (= I); down: 0
+    const int32_t *perm_tok;
+    const float *row_gate;
+    __nv_bfloat16 *h;          // gate/up output [rows x I] bf16
+    int I;
+    float *out;                // down output [T x H]
+    int H;
+    int32_t *err;
+};
+
+__device__ __forceinline__ float byte_f(uint32_t w, int i)  // biased int8 -> float
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(w), "r"(0x4B000000u), "r"(0x7650u + i));
+    return __uint_as_float(d) - 8388736.f;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kQ8Threads, 1)
+    q8_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const Q8GemmArgs g)
+{
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t fa_bar[kQ8Stages], fb_bar[kQ8Stages], empty_bar[kQ8Stages], accf_bar, acce_bar;
+    __shared__ uint32_t tmem_base;
+    __shared__ volatile int abort_flag;
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = *g.n_ptiles * g.NT;
+    const int KT = g.K / 64;
+
+    if (warp == 5) {
+        tmem_alloc(&tmem_base, 512);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kQ8Stages; ++s) {
+            mbar_init(&fa_bar[s], 1);
+            mbar_init(&fb_bar[s], 8);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&accf_bar, 1);
+        mbar_init(&acce_bar, 4);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 4) {  // ---- activation producer
+        if (lane == 0) {
+            prefetch_tmap(&tmA);
+            int it = 0;
+            for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
+                const int4 pt = g.ptiles[tile / g.NT];
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = it % kQ8Stages, u = it / kQ8Stages;
+                    if (u > 0 && !mbar_wait(&empty_bar[s], (u - 1) & 1)) {
+                        abort_flag = 1;
+                        break;
+                    }
+                    uint8_t *a_s = smem + s * kQ8Stage;
+                    mbar_arrive_expect_tx(&fa_bar[s], pt.z * kQ8A);
+                    tma_load_2d(a_s, &tmA, &fa_bar[s], kt * 64, pt.y);
+                    if (pt.z == 2) tma_load_2d(a_s + kQ8A, &tmA, &fa_bar[s], kt * 64, pt.y + 128);
+                }
+            }
+        }
+    } else if (warp == 5) {  // ---- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(128, 256);
+            int it = 0, tcount = 0;
+            for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x, ++tcount) {
+                const int nh = g.ptiles[tile / g.NT].z;
+                if (tcount > 0 && !mbar_wait(&acce_bar, (tcount - 1) & 1)) {
+                    abort_flag = 1;
+                    break;
+                }
+                tc_fence_after_sync();
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = it % kQ8Stages, u = it / kQ8Stages;
+                    if (!mbar_wait(&fa_bar[s], u & 1) || !mbar_wait(&fb_bar[s], u & 1)) {
+                        abort_flag = 1;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    uint8_t *a_s = smem + s * kQ8Stage, *b_s = a_s + 2 * kQ8A;
+                    const uint64_t bd = desc_kmajor_sw128(b_s);
+                    for (int hh = 0; hh < nh; ++hh) {
+                        const uint64_t ad = desc_kmajor_sw128(a_s + hh * kQ8A);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_f16(tmem + hh * 256, ad + 2 * kk, bd + 2 * kk, idesc, (kt | kk) != 0);
+                    }
+                    mma_commit(&empty_bar[s]);
+                }
+                mma_commit(&accf_bar);
+            }
+        }
+    } else if (warp >= 6) {  // ---- weight dequantisers: thread n owns weight row n
+        const int n = threadIdx.x - 192;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
+            const int mt = tile / g.NT, nt = tile % g.NT;
+            const int e = g.ptiles[mt].x;
+            const int row = GATEUP ? (n < 128 ? nt * 128 + n : g.up_off + nt * 128 + (n - 128)) : nt * 256 + n;
+            const uint8_t *qrow = g.qs + (int64_t)e * g.qs_stride + (int64_t)row * g.K;
+            const uint8_t *srow = g.sc + (int64_t)e * g.sc_stride + (int64_t)row * g.sc_row;
+            uint4 q[4];
+            uint32_t sc2;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) q[i] = __ldg(reinterpret_cast<const uint4 *>(qrow) + i);
+            sc2 = __ldg(reinterpret_cast<const uint32_t *>(srow));
+            for (int kt = 0; kt < KT; ++kt, ++it) {
+                const int s = it % kQ8Stages, u = it / kQ8Stages;
+                uint4 qn[4];
+                uint32_t scn = 0;
+                if (kt + 1 < KT) {  // next K slice of this row, in flight while we convert
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) qn[i] = __ldg(reinterpret_cast<const uint4 *>(qrow + (kt + 1) * 64) + i);
+                    scn = __ldg(reinterpret_cast<const uint32_t *>(srow + (kt + 1) * 4));
+                }
+                if (u > 0) {
+                    bool ok = true;
+                    if (lane == 0) ok = mbar_wait(&empty_bar[s], (u - 1) & 1);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) {
+                        abort_flag = 1;
+                        break;
+                    }
+                }
+                const float d0 = __half2float(__ushort_as_half((unsigned short)(sc2 & 0xFFFFu)));
+                const float d1 = __half2float(__ushort_as_half((unsigned short)(sc2 >> 16)));
+                uint8_t *b_row = smem + s * kQ8Stage + 2 * kQ8A + (n >> 3) * 1024 + (n & 7) * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {  // chunk c: 8 codes, k = 8c .. 8c+7
+                    const uint32_t w0 = (&q[c >> 1].x)[(c & 1) * 2], w1 = (&q[c >> 1].x)[(c & 1) * 2 + 1];
+                    const float d = c < 4 ? d0 : d1;
+                    uint4 o;
+                    o.x = pack_bf16x2(byte_f(w0, 0) * d, byte_f(w0, 1) * d);
+                    o.y = pack_bf16x2(byte_f(w0, 2) * d, byte_f(w0, 3) * d);
+                    o.z = pack_bf16x2(byte_f(w1, 0) * d, byte_f(w1, 1) * d);
+                    o.w = pack_bf16x2(byte_f(w1, 2) * d, byte_f(w1, 3) * d);
+                    *reinterpret_cast<uint4 *>(b_row + ((c ^ (n & 7)) << 4)) = o;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&fb_bar[s]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) q[i] = qn[i];
+                sc2 = scn;
+            }
+        }
+    } else {  // ---- epilogue, warps 0-3
+        int tcount = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tcount) {
+            const bool ok = mbar_wait(&accf_bar, tcount & 1);
+            tc_fence_after_sync();
+            if (!ok || abort_flag) {
+                if (threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+                break;
+            }
+            const int mt = tile / g.NT, nt = tile % g.NT;
+            const int4 pt = g.ptiles[mt];
+            for (int hh = 0; hh < pt.z; ++hh) {
+                const int row = pt.y + hh * 128 + warp * 32 + lane;
+                const int tok = g.perm_tok[row];
+                const uint32_t tl = tmem + hh * 256 + ((uint32_t)(warp * 32) << 16);
+                if (GATEUP) {
+#pragma unroll 1
+                    for (int c = 0; c < 128; c += 16) {
+                        float vg[16], vu[16];
+                        tmem_ld16(tl + c, vg);
+                        tmem_ld16(tl + 128 + c, vu);
+                        if (tok >= 0) {
+                            uint32_t o[8];
+#pragma unroll
+                            for (int i = 0; i < 16; i += 2) {
+                                const float a0 = vg[i], a1 = vg[i + 1];
+                                o[i / 2] = pack_bf16x2(a0 / (1.f + expf(-a0)) * vu[i], a1 / (1.f + expf(-a1)) * vu[i + 1]);
+                            }
+                            uint4 *dst = reinterpret_cast<uint4 *>(g.h + (size_t)row * g.I + nt * 128 + c);
+                            dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                            dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                        }
+                    }
+                } else {
+                    const float gt = tok >= 0 ? g.row_gate[row] : 0.f;
+#pragma unroll 1
+                    for (int c = 0; c < 256; c += 16) {
+                        float v[16];
+                        tmem_ld16(tl + c, v);
+                        if (tok >= 0) {
+                            float *dst = g.out + (size_t)tok * g.H + nt * 256 + c;
+#pragma unroll
+                            for (int i = 0; i < 16; i += 4)
+                                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + i),
+                                             "f"(v[i] * gt), "f"(v[i + 1] * gt), "f"(v[i + 2] * gt), "f"(v[i + 3] * gt)
+                                             : "memory");
+                        }
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce_bar);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (abort_flag && threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+    if (warp == 5) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// One warp per token: copy x[t] (bf16) into its k routed slot rows (and the
+// shared slot) of the padded slot space.
+__global__ void __launch_bounds__(256) gather_scatter_kernel(const uint16_t *x, int T, int H, int k, int E,
+                                                             int has_shared, const int32_t *idx, const float *gate,
+                                                             const int32_t *pad_off, int32_t *fill, uint16_t *xp,
+                                                             int32_t *perm_tok, float *row_gate, int32_t *slot_pos,
+                                                             int max_rows)
+{
+    __shared__ int s_pos[8][33];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int t = blockIdx.x * 8 + wib;
+    if (t >= T) return;
+    const int nd = k + (has_shared ? 1 : 0);
+    for (int j = 0; j < nd; ++j) {
+        int pos = 0;
+        if (lane == 0) {
+            const int e = j < k ? idx[(size_t)t * k + j] : E;
+            pos = pad_off[e] + atomicAdd(&fill[e], 1);
+            if (pos >= max_rows) pos = -1;
+            s_pos[wib][j] = pos;
+            if (pos >= 0) {
+                perm_tok[pos] = t;
+                row_gate[pos] = j < k ? gate[(size_t)t * k + j] : 1.f;
+                if (j < k) slot_pos[(size_t)t * k + j] = pos;
+            }
+        }
+    }
+    __syncwarp();
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+    for (int c = lane; c < H / 8; c += 32) {
+        const uint4 v = __ldg(src + c);
+        for (int j = 0; j < nd; ++j) {
+            const int pos = s_pos[wib][j];
+            if (pos >= 0) reinterpret_cast<uint4 *>(xp + (size_t)pos * H)[c] = v;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t prefill_q8_set_attributes()
+{
+    cudaError_t e = cudaFuncSetAttribute(q8_grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kQ8Smem);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(q8_grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kQ8Smem);
+}
+
+bool prefill_q8_supported(int H, int I, int E, int k)
+{
+    return H % 256 == 0 && I % 256 == 0 && E <= 1023 && k <= 32;
+}
+
+cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s)
+{
+    const int H = a.H, I = a.I, E = a.E, k = a.k, T = a.T;
+    const PrefillWorkspace &w = *a.ws;
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(w.cnt, 0, sizeof(int32_t) * (E + 1), s)) != cudaSuccess) return e;
+    if ((e = prefill_route(a.x, a.wr, T, H, E, k, w.logits, w.idx, w.gate, w.cnt, a.err, s)) != cudaSuccess) return e;
+    if ((e = prefill_plan_launch(w, E, T, a.has_shared, a.err, s)) != cudaSuccess) return e;
+    uint16_t *xp = reinterpret_cast<uint16_t *>(w.a_q);  // bf16 slot rows, sized for the Q8_0 path
+    gather_scatter_kernel<<<(T + 7) / 8, 256, 0, s>>>(reinterpret_cast<const uint16_t *>(a.x), T, H, k, E,
+                                                       a.has_shared, w.idx, w.gate, w.pad_off, w.fill, xp, w.perm_tok,
+                                                       w.row_gate, w.slot_pos, w.max_rows);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    CUtensorMap ma;
+    if (!make_map_bf16(&ma, xp, w.max_rows, H, 128)) return cudaErrorInvalidValue;
+    Q8GemmArgs g{};
+    g.ptiles = w.ptiles;
+    g.n_ptiles = w.n_ptiles;
+    g.NT = I / 128;
+    g.K = H;
+    g.qs = a.gu->qs;
+    g.qs_stride = a.gu->qs_stride;
+    g.sc = a.gu->sc;
+    g.sc_stride = a.gu->sc_stride;
+    g.sc_row = a.gu->sc_row;
+    g.up_off = I;
+    g.perm_tok = w.perm_tok;
+    g.row_gate = w.row_gate;
+    g.h = reinterpret_cast<__nv_bfloat16 *>(w.h);
+    g.I = I;
+    g.out = a.out;
+    g.H = H;
+    g.err = a.err;
+    q8_grouped_gemm_kernel<true><<<a.num_sms, kQ8Threads, kQ8Smem, s>>>(ma, g);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.out, 0, sizeof(float) * (size_t)T * H, s)) != cudaSuccess) return e;
+    CUtensorMap mh;
+    if (!make_map_bf16(&mh, w.h, w.max_rows, I, 128)) return cudaErrorInvalidValue;
+    Q8GemmArgs d = g;
+    d.NT = H / 256;
+    d.K = I;
+    d.qs = a.dn->qs;
+    d.qs_stride = a.dn->qs_stride;
+    d.sc = a.dn->sc;
+    d.sc_stride = a.dn->sc_stride;
+    d.sc_row = a.dn->sc_row;
+    d.up_off = 0;
+    q8_grouped_gemm_kernel<false><<<a.num_sms, kQ8Threads, kQ8Smem, s>>>(mh, d);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -78,14 +78,19 @@ typedef enum {
 typedef enum { MOE_DT_F32 = 1, MOE_DT_BF16 = 2 } moe_dtype;
 
 /* Kernel path of a forward.  AUTO picks DECODE for n_tokens <= 64 (decode and
- * speculative-verify batches) and PREFILL above.  DENSE is the dense-batched
+ * speculative-verify batches) and PREFILL above when the pack can run it (both
+ * projections NVFP4 - native block-scaled FP4 MMA with the activations rounded
+ * to NVFP4 per token - or both Q8_0 - weights dequantised to bf16 for bf16 MMA;
+ * hidden and inter multiples of 256, bf16 activations, top_k <= 32; its
+ * buffers are sized at pack time when max_tokens > 64), else GROUPED.  DENSE is the dense-batched
  * comparison variant: every active expert multiplies the whole batch, with a
  * zero gate for tokens not routed to it. */
 typedef enum {
     MOE_PATH_AUTO = 0,
-    MOE_PATH_DECODE = 1,
+    MOE_PATH_DECODE = 1,   /* one fused launch for n_tokens <= 8, top_k <= 16, else GROUPED */
     MOE_PATH_PREFILL = 2,
-    MOE_PATH_DENSE = 3
+    MOE_PATH_DENSE = 3,
+    MOE_PATH_GROUPED = 4   /* decode as separate route / gate-up / down / combine launches */
 } moe_path;
 
 /* Description of one layer's experts, all in HOST memory; moe_pack_experts
@@ -156,7 +161,9 @@ size_t moe_route_workspace_bytes(int n_tokens, int n_experts);
  *   gate_out  device, [n_tokens x top_k] fp32 gates (sum to 1 per token)
  *   workspace device, moe_route_workspace_bytes(n_tokens, n_experts) bytes,
  *             owned by the caller; its contents need no initialisation
- * hidden % 8 == 0, 1 <= top_k <= n_experts <= 1024. */
+ * hidden % 8 == 0, 1 <= top_k <= n_experts <= 1024.  More than 64 bf16 tokens
+ * run the router as a tensor-core GEMM; if one of its bounded waits runs out,
+ * int32 word 1 of the workspace holds MOE_ERR_TIMEOUT afterwards. */
 moe_status moe_route_topk(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
                           int n_tokens, int hidden, int n_experts, int top_k, int32_t *idx_out,
                           float *gate_out, void *workspace, size_t workspace_bytes,
@@ -210,9 +217,11 @@ moe_status moe_read_routing(const moe_pack *pack, int n_tokens, int top_k, int32
  * records an event before each of its kernels and after the last one
  * (captured as event-record nodes when the stream is capturing).
  * moe_profile_end synchronises the device, adds the elapsed times per kernel
- * stage over all recorded forwards into ms[4] (route+plan, gate/up, down,
- * combine; host memory), stores the forward count in *n_forwards, and frees
- * the events.  Forwards beyond max_forwards are not recorded. */
+ * over all recorded forwards into ms[6] (host memory: route+plan, gate/up,
+ * down, combine of the grouped path, the fused decode kernel, and the whole
+ * tensor-core prefill sequence), stores the
+ * forward count in *n_forwards, and frees the events.  Forwards beyond
+ * max_forwards are not recorded. */
 moe_status moe_profile_begin(moe_pack *pack, int max_forwards);
 moe_status moe_profile_end(moe_pack *pack, double *ms, int *n_forwards);
 

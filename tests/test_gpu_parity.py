@@ -121,3 +121,53 @@ def test_pack_rejects_nan_block_scale():
     with pytest.raises(bq.MoeError) as e:
         bq.pack_layer(li)
     assert e.value.status == bq.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name,layer,T", [("tiny_q8", 3, 1), ("model_decode", 1, 1), ("spec_verify", 2, 8),
+                                          ("model_decode", 4, 3)])
+def test_fused_and_grouped_decode_paths_both_match_the_oracle(name, layer, T):
+    import block_quantized_expert_moe_b200 as bq
+    wl, li = _layer(name, layer)
+    x = synth.tokens(wl, li.router, layer, 7, T)
+    ref, ridx, rgate = oracle_layer(li, x, wl.top_k)
+    outs = {}
+    for path in (bq.MOE_PATH_DECODE, bq.MOE_PATH_GROUPED):
+        out, idx, gate, counts = gpu_layer(li, x, wl.top_k, path=path)
+        assert_routing_equal(idx, gate, ridx, rgate)
+        assert np.array_equal(counts, expected_counts(ridx, wl.n_experts, T, wl.has_shared))
+        err = normwise_err(out, ref)
+        assert err <= DECODE_TOL, (path, err)
+        outs[path] = out
+    # same fp32 arithmetic in a different order: close, not necessarily bitwise
+    assert normwise_err(outs[bq.MOE_PATH_DECODE], outs[bq.MOE_PATH_GROUPED]) <= 1e-5
+
+
+def test_fused_decode_ragged_shapes():
+    for T in (1, 3, 5, 8):
+        wl = synth.Workload("ragged_fused", 96, 7, 64, 3, True, synth.FMT_NVFP4, synth.FMT_Q5_1, synth.DT_BF16,
+                            T, seed=10 + T)
+        li = synth.layer_inputs(wl)
+        _check(li, synth.tokens(wl, li.router), wl.top_k)
+
+
+@pytest.mark.parametrize("name,T,kw", [("prefill_nvfp4", 300, {}),
+                                       ("prefill_nvfp4", 130, dict(n_experts=200, hidden=96, top_k=5))])
+def test_tensor_core_router_matches_oracle(name, T, kw):
+    """More than 64 bf16 tokens: the router runs as a tcgen05 GEMM (ragged M, N and K tiles here)."""
+    import block_quantized_expert_moe_b200 as bq
+    import oracle
+    wl = synth.WORKLOADS[name].with_(**kw)
+    wr_np, _ = synth.router(wl)
+    x = synth.tokens(wl, wr_np, 0, 0, T)
+    xt, wr = to_device(x), router_to_device(wr_np)
+    idx = torch.empty(T, wl.top_k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, wl.top_k, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(bq.moe_route_workspace_bytes(T, wl.n_experts), dtype=torch.uint8, device="cuda")
+    bq.moe_route_topk(xt, wr, wl.top_k, idx, gate, ws)
+    torch.cuda.synchronize()
+    assert ws[4:8].view(torch.int32).item() == 0  # no timed-out wait
+    ridx, rgate, rlog = oracle.route(synth.tokens_f64(wl, x), wr_np, wl.top_k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.abs(gate.cpu().numpy() - rgate).max() <= 1e-5
+    logits = ws[256:256 + 4 * T * wl.n_experts].view(torch.float32).view(T, wl.n_experts).cpu().numpy()
+    assert np.abs(logits - rlog).max() <= 1e-4 * np.abs(rlog).max()
