@@ -337,7 +337,7 @@ def ours_arm(a, wl):
                 fwd(ly)
     gp.replay()
     torch.cuda.synchronize()
-    stage_ms = np.zeros(6)
+    stage_ms = np.zeros(15)
     nf = 0
     for ly in layers:
         m, n = bq.moe_profile_end(ly["pack"])
@@ -346,6 +346,9 @@ def ours_arm(a, wl):
     prefill_kernels = 7 if wl.fmt_gate_up == synth.FMT_NVFP4 else 6  # route GEMM, top-k, plan, gather, GEMMs (+ h quant)
     launches_per_fwd = 1 if stage_ms[4] > 0 else (prefill_kernels if stage_ms[5] > 0 else 4)
     stage_us = {s: float(stage_ms[i] / nf * 1e3) for i, s in enumerate(STAGES) if stage_ms[i] > 0}
+    phase_names = ["stage_x", "router", "barrier1", "plan", "gate_up", "barrier2", "down", "barrier3", "combine"]
+    fused_phase_us = ({n: float(stage_ms[6 + i] / nf * 1e3) for i, n in enumerate(phase_names)}
+                      if stage_ms[4] > 0 else None)
     dom = max(stage_us, key=lambda s: stage_us[s])
     hbm, peak_src = peaks()
     traffic = kernel_traffic(dom, wl.name)
@@ -418,7 +421,8 @@ def ours_arm(a, wl):
                 "expert_gbs": expert_gbs, "expert_gbs_frac": expert_gbs / hbm,
                 "unique_expert_bytes_per_step": unique_bytes_step,
                 "active_experts_per_layer": float(np.mean(n_active)),
-                "stage_us": stage_us, "roofline": roofline, "clocks": clk.summary(),
+                "stage_us": stage_us, "fused_phase_us": fused_phase_us, "roofline": roofline,
+                "clocks": clk.summary(),
                 "e2e": e2e, "gpu_launches": launches_per_fwd * L * a.steps, "cpu_baseline": cpu,
                 "gen_seconds": gen_s}
         print(json.dumps(line), flush=True)

@@ -230,8 +230,9 @@ def moe_profile_begin(pack, max_forwards):
 
 
 def moe_profile_end(pack):
-    """-> (ms per kernel [route+plan, gate/up, down, combine, fused, prefill] summed, n_forwards)."""
-    ms = np.zeros(6, np.float64)
+    """-> (ms[15] summed over recorded forwards: route+plan, gate/up, down, combine,
+    fused, prefill, then the fused kernel's nine phases; n_forwards)."""
+    ms = np.zeros(15, np.float64)
     n = ctypes.c_int(0)
     _check(lib.moe_profile_end(pack.handle, _np_ptr(ms), ctypes.byref(n)), "moe_profile_end")
     return ms, n.value

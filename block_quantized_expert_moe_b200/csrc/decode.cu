@@ -102,7 +102,7 @@ __device__ __forceinline__ void reduce_lanes(float (&v)[TT], int lpr)
 }
 
 template <int FMT, bool GATEUP, int TT>
-__global__ void __launch_bounds__(kThreads) matvec_kernel(const MatvecArgs a)
+__global__ void __launch_bounds__(kThreads, 1) matvec_kernel(const MatvecArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     float4 *xs4 = reinterpret_cast<float4 *>(smem);

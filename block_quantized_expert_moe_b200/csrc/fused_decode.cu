@@ -356,6 +356,51 @@ __device__ void phase_gateup(const FusedArgs &a, const Plan &pl, const float4 *x
     const int ng = *pl.n_groups;
     const long long total = (long long)ng * tpg;
     const long long t0 = total * blockIdx.x / gridDim.x, t1 = total * (blockIdx.x + 1) / gridDim.x;
+    if constexpr (TT == 1) {
+        if (NU <= 2 * LPR) {  // one token: this lane's x units live in registers for every task
+            const int u = sl, u2 = sl + LPR;
+            const bool has2 = u2 < NU;
+            float4 xr0[8], xr1[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                xr0[j] = u < NU ? xs4[u * 8 + (j ^ (u & 7))] : make_float4(0.f, 0.f, 0.f, 0.f);
+                xr1[j] = has2 ? xs4[u2 * 8 + (j ^ (u2 & 7))] : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            const float xs0 = FMT == MOE_FMT_Q5_1 && u < NU ? xsum[u] : 0.f;
+            const float xs1 = FMT == MOE_FMT_Q5_1 && has2 ? xsum[u2] : 0.f;
+            for (long long tk = t0 + warp; tk < t1; tk += NW) {
+                const int g = (int)(tk / tpg);
+                const int r = (int)(tk - (long long)g * tpg) * RPW + sub;
+                const bool valid = r < rows;
+                const int rr = valid ? r : rows - 1;
+                const int4 gd = pl.groups[g];
+                const int e = gd.x, slot0 = gd.y;
+                const float half_ts = FMT == MOE_FMT_NVFP4 ? 0.5f * __ldg(w.ts + e) : 0.5f;
+                float s0 = 0.f, s1 = 0.f;
+                if (u < NU) {
+                    const Raw g0 = load_unit<FMT>(w, e, rr, u);
+                    const Raw v0 = load_unit<FMT>(w, e, rows + rr, u);
+                    Raw g1 = g0, v1 = v0;
+                    if (has2) {
+                        g1 = load_unit<FMT>(w, e, rr, u2);
+                        v1 = load_unit<FMT>(w, e, rows + rr, u2);
+                    }
+                    s0 = unit_dot_reg<FMT>(g0, xr0, xs0, a.tab_gu, half_ts, s0);
+                    s1 = unit_dot_reg<FMT>(v0, xr0, xs0, a.tab_gu, half_ts, s1);
+                    if (has2) {
+                        s0 = unit_dot_reg<FMT>(g1, xr1, xs1, a.tab_gu, half_ts, s0);
+                        s1 = unit_dot_reg<FMT>(v1, xr1, xs1, a.tab_gu, half_ts, s1);
+                    }
+                }
+                for (int o = LPR >> 1; o >= 1; o >>= 1) {
+                    s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+                    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+                }
+                if (valid && sl == 0) a.h[(size_t)slot0 * a.I + r] = s0 / (1.f + expf(-s0)) * s1;
+            }
+            return;
+        }
+    }
     for (long long tk = t0 + warp; tk < t1; tk += NW) {
         const int g = (int)(tk / tpg);
         const int r = (int)(tk - (long long)g * tpg) * RPW + sub;
@@ -673,6 +718,7 @@ __global__ void __launch_bounds__(FT, 1) fused_decode_kernel(const FusedArgs a)
     pl.scan_tmp = reinterpret_cast<int *>(smem + L.scan);
     pl.n_groups = reinterpret_cast<int *>(smem + L.ng);
 
+    if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[0] = clock64();
     // the shared expert's weights do not depend on routing: start them into L2
     if (a.has_shared) {
         int turn = 0;
@@ -687,9 +733,13 @@ __global__ void __launch_bounds__(FT, 1) fused_decode_kernel(const FusedArgs a)
     }
     stage_tokens<FT>(a, xs4, xsum, a.gu.fmt == MOE_FMT_Q5_1);
     __syncthreads();
+    if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[1] = clock64();
     phase_router<FT, TT>(a, xs4);
+    if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[2] = clock64();
     if (!grid_sync(a.bar, a.err)) return;
+    if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[3] = clock64();
     phase_plan<FT>(a, pl);
+    if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[4] = clock64();
 
     if (a.rowsplit) {  // start this CTA's down rows into L2 while gate/up runs
         const int NU = a.I >> 5;
@@ -718,7 +768,9 @@ __global__ void __launch_bounds__(FT, 1) fused_decode_kernel(const FusedArgs a)
     case MOE_FMT_IQ4_NL: run_gateup<MOE_FMT_IQ4_NL, FT, TT>(a, pl, xs4, xsum); break;
     default: run_gateup<MOE_FMT_NVFP4, FT, TT>(a, pl, xs4, xsum); break;
     }
+    if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[5] = clock64();
     if (!grid_sync(a.bar, a.err)) return;
+    if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[6] = clock64();
     if (a.rowsplit) {
         switch (a.dn.fmt) {
         case MOE_FMT_Q8_0: phase_down_rows<MOE_FMT_Q8_0, FT, TT>(a, pl, hs4, hsum); break;
@@ -726,6 +778,7 @@ __global__ void __launch_bounds__(FT, 1) fused_decode_kernel(const FusedArgs a)
         case MOE_FMT_IQ4_NL: phase_down_rows<MOE_FMT_IQ4_NL, FT, TT>(a, pl, hs4, hsum); break;
         default: phase_down_rows<MOE_FMT_NVFP4, FT, TT>(a, pl, hs4, hsum); break;
         }
+    if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[7] = clock64();
     } else {
         switch (a.dn.fmt) {
         case MOE_FMT_Q8_0: phase_down_slots<MOE_FMT_Q8_0, FT, TT>(a, pl, hs4, hsum); break;
@@ -733,12 +786,15 @@ __global__ void __launch_bounds__(FT, 1) fused_decode_kernel(const FusedArgs a)
         case MOE_FMT_IQ4_NL: phase_down_slots<MOE_FMT_IQ4_NL, FT, TT>(a, pl, hs4, hsum); break;
         default: phase_down_slots<MOE_FMT_NVFP4, FT, TT>(a, pl, hs4, hsum); break;
         }
+        if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[7] = clock64();
         if (!grid_sync(a.bar, a.err)) return;
+        if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[8] = clock64();
         phase_combine<FT>(a, pl);
     }
+    if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[9] = clock64();
 }
 
-constexpr int kFT1 = 512;  // threads per CTA, one-token kernel
+constexpr int kFT1 = 384;  // threads per CTA, one-token kernel
 constexpr int kFT8 = 256;  // threads per CTA, up-to-8-token kernel
 
 }  // namespace

@@ -20,7 +20,7 @@ cudaError_t matvec_set_attributes();
 
 // kernel-stage slots of the profiling API (moe_profile_end's ms[])
 enum { PROF_ROUTE = 0, PROF_GATE_UP = 1, PROF_DOWN = 2, PROF_COMBINE = 3, PROF_FUSED = 4, PROF_PREFILL = 5,
-       PROF_STAGES = 6 };
+       PROF_STAGES = 6, PROF_PHASES = 9, PROF_OUT = PROF_STAGES + PROF_PHASES };
 
 using namespace moe;
 
@@ -30,7 +30,8 @@ struct moe_pack {
     int E = 0, H = 0, I = 0, has_shared = 0, max_tokens = 0, max_top_k = 0;
     int fmt_gu = 0, fmt_dn = 0;
     DevProj gu, dn;
-    uint32_t tab[4] = {0, 0, 0, 0};
+    CodeTable ct_gu{}, ct_dn{};
+    uint8_t perm_gu[16], perm_dn[16];  // stored position of each 4-bit code
     std::vector<void *> allocations;
     Workspace ws;
     int64_t arena_bytes = 0, workspace_bytes = 0;
@@ -41,6 +42,8 @@ struct moe_pack {
     std::vector<cudaEvent_t> prof_ev;
     std::vector<std::pair<int, int>> prof_fwd;
     int prof_used = 0;
+    long long *prof_stamps = nullptr;  // device, 16 clock64 stamps per recorded fused forward
+    int prof_nstamp = 0, prof_stamp_cap = 0;
     int fused_grid[2] = {0, 0};   // [tt==8]
     bool has_prefill = false;     // tensor-core prefill workspace present
     PrefillWorkspace pws;
@@ -48,13 +51,78 @@ struct moe_pack {
 
 namespace {
 
-const uint32_t kNvfp4Tab[4] = {
-    // 2*e2m1 for codes 0..15, each stored as value + 128
-    0x83828180u,  // 0, 1, 2, 3
-    0x8C888684u,  // 4, 6, 8, 12
-    0x7D7E7F80u,  // -0, -1, -2, -3
-    0x74787A7Cu,  // -4, -6, -8, -12
-};
+// Code table of a 4-bit format for the decode kernels' byte-permute lookup.
+// Entry bytes are value + bias; when every position pair (i, i+8) can be given
+// entries whose biased bytes share their top bit, the table is laid out for the
+// XOR-combined lookup (two permutes and one XOR per four nibbles) and perm[c]
+// is the position code c is stored as; otherwise the masked lookup with the
+// identity position.  NVFP4 entries are 2*e2m1(c) (integers -12..12), so its
+// block scales carry the factor 1/2.
+CodeTable build_code_table(int fmt, const int8_t *iq4, uint8_t perm[16])
+{
+    CodeTable ct{};
+    for (int c = 0; c < 16; ++c) perm[c] = (uint8_t)c;
+    if (fmt != MOE_FMT_IQ4_NL && fmt != MOE_FMT_NVFP4) return ct;
+    int v[16];
+    if (fmt == MOE_FMT_NVFP4) {
+        const int mag[8] = {0, 1, 2, 3, 4, 6, 8, 12};
+        for (int c = 0; c < 16; ++c) v[c] = (c & 8) ? -mag[c & 7] : mag[c & 7];
+    } else {
+        for (int c = 0; c < 16; ++c) v[c] = iq4[c];
+    }
+    int lo = 127, hi = -128;
+    for (int c = 0; c < 16; ++c) {
+        lo = std::min(lo, v[c]);
+        hi = std::max(hi, v[c]);
+    }
+    // candidate biases keeping every byte in [0, 255]; prefer one with an even
+    // split of top bits (all-equal counts as even)
+    int bias = -1;
+    for (int b : {192, 128, 127, 129, 126, 130}) {
+        if (lo + b < 0 || hi + b > 255) continue;
+        int n1 = 0;
+        for (int c = 0; c < 16; ++c) n1 += (v[c] + b) >= 128;
+        if (n1 % 2 == 0) {
+            bias = b;
+            break;
+        }
+    }
+    uint8_t pos_code[16];
+    if (bias >= 0) {
+        int ones[16], zeros[16], n1 = 0, n0 = 0;
+        for (int c = 0; c < 16; ++c) {
+            if (v[c] + bias >= 128) ones[n1++] = c;
+            else zeros[n0++] = c;
+        }
+        int p = 0;
+        for (int i = 0; i + 1 < n1; i += 2, ++p) {
+            pos_code[p] = (uint8_t)ones[i];
+            pos_code[p + 8] = (uint8_t)ones[i + 1];
+        }
+        for (int i = 0; i + 1 < n0; i += 2, ++p) {
+            pos_code[p] = (uint8_t)zeros[i];
+            pos_code[p + 8] = (uint8_t)zeros[i + 1];
+        }
+        if (fmt == MOE_FMT_NVFP4)  // native codes stay in place (the prefill MMA reads them); bias 192
+            for (int q = 0; q < 16; ++q) pos_code[q] = (uint8_t)q;  // makes every top bit equal
+        for (int q = 0; q < 16; ++q) perm[pos_code[q]] = (uint8_t)q;
+        uint8_t bytes[16];
+        for (int i = 0; i < 8; ++i) {
+            const uint8_t l = (uint8_t)(v[pos_code[i]] + bias);
+            const uint8_t h = (uint8_t)(v[pos_code[i + 8]] + bias);
+            bytes[i] = l;
+            bytes[i + 8] = (uint8_t)(h ^ ((l & 0x80) ? 0xFF : 0x00));
+        }
+        for (int i = 0; i < 16; ++i) ct.t[i / 4] |= (uint32_t)bytes[i] << (8 * (i % 4));
+        ct.xor_mode = 1;
+    } else {
+        bias = 128;
+        for (int c = 0; c < 16; ++c) ct.t[c / 4] |= (uint32_t)(uint8_t)(v[c] + bias) << (8 * (c % 4));
+        ct.xor_mode = 0;
+    }
+    ct.magic = 8388608.f + (float)bias;
+    return ct;
+}
 
 std::mutex g_dev_mutex;
 bool g_dev_ready[64];
@@ -126,8 +194,10 @@ int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 // Repack one expert's projection (rows x cols canonical blocks) into planes.
 // Returns false on an invalid NVFP4 block scale.
 bool repack_expert(int fmt, const uint8_t *src, int rows, int cols, uint8_t *qs, uint8_t *sc,
-                   uint8_t *qh)
+                   uint8_t *qh, const uint8_t *perm)
 {
+    uint8_t pbyte[256];  // both nibbles of a code byte through the position map
+    for (int b = 0; b < 256; ++b) pbyte[b] = (uint8_t)(perm[b & 15] | (perm[b >> 4] << 4));
     const int64_t rb = canon_row_bytes(fmt, cols);
     int qs_row, sc_row, qh_row;
     plane_rows(fmt, cols, qs_row, sc_row, qh_row);
@@ -155,7 +225,7 @@ bool repack_expert(int fmt, const uint8_t *src, int rows, int cols, uint8_t *qs,
                 const uint8_t *blk = row + b * 18;
                 s[2 * b] = blk[0];
                 s[2 * b + 1] = blk[1];
-                std::memcpy(q + 16 * b, blk + 2, 16);
+                for (int i = 0; i < 16; ++i) q[16 * b + i] = pbyte[blk[2 + i]];
             }
         } else {
             const int ks = nvfp4_ksteps(cols);
@@ -208,7 +278,7 @@ moe_status dev_alloc(moe_pack *p, size_t bytes, void **out)
 
 // Build one projection's planes for all slots (routed experts + shared).
 moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, const uint8_t *blocks,
-                      const uint8_t *shared_blocks, const float *ts, int n_slots)
+                      const uint8_t *shared_blocks, const float *ts, int n_slots, const uint8_t *perm)
 {
     dp.fmt = fmt;
     dp.rows = rows;
@@ -232,7 +302,7 @@ moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, con
         const uint8_t *src = s < p->E ? blocks + (int64_t)s * canon : shared_blocks;
         ok[s] = repack_expert(fmt, src, rows, cols, hq.data() + (int64_t)s * dp.qs_stride,
                               hs.data() + (int64_t)s * dp.sc_stride,
-                              dp.qh_row ? hh.data() + (int64_t)s * dp.qh_stride : nullptr);
+                              dp.qh_row ? hh.data() + (int64_t)s * dp.qh_stride : nullptr, perm);
     });
     for (char c : ok)
         if (!c) return MOE_ERR_INVALID_ARG;
@@ -402,19 +472,18 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
     p->max_top_k = d->max_top_k;
     p->fmt_gu = d->fmt_gate_up;
     p->fmt_dn = d->fmt_down;
-    if (d->iq4nl_table)
-        for (int c = 0; c < 16; ++c)
-            p->tab[c / 4] |= (uint32_t)((uint8_t)d->iq4nl_table[c] ^ 0x80u) << (8 * (c % 4));
+    p->ct_gu = build_code_table(p->fmt_gu, d->iq4nl_table, p->perm_gu);
+    p->ct_dn = build_code_table(p->fmt_dn, d->iq4nl_table, p->perm_dn);
     for (auto &row : p->grid_cache) row[0] = row[1] = 0;
     const int n_slots = p->E + p->has_shared;
     std::vector<float> gts, dts;
     if (p->fmt_gu == MOE_FMT_NVFP4) gts.assign(d->gate_up_tensor_scale, d->gate_up_tensor_scale + n_slots);
     if (p->fmt_dn == MOE_FMT_NVFP4) dts.assign(d->down_tensor_scale, d->down_tensor_scale + n_slots);
     st = build_proj(p, p->gu, p->fmt_gu, 2 * p->I, p->H, static_cast<const uint8_t *>(d->gate_up_blocks),
-                    static_cast<const uint8_t *>(d->shared_gate_up_blocks), gts.data(), n_slots);
+                    static_cast<const uint8_t *>(d->shared_gate_up_blocks), gts.data(), n_slots, p->perm_gu);
     if (st == MOE_OK)
         st = build_proj(p, p->dn, p->fmt_dn, p->H, p->I, static_cast<const uint8_t *>(d->down_blocks),
-                        static_cast<const uint8_t *>(d->shared_down_blocks), dts.data(), n_slots);
+                        static_cast<const uint8_t *>(d->shared_down_blocks), dts.data(), n_slots, p->perm_dn);
     if (st == MOE_OK) st = build_workspace(p);
     const bool nv = p->fmt_gu == MOE_FMT_NVFP4 && p->fmt_dn == MOE_FMT_NVFP4 &&
                     prefill_nvfp4_supported(p->H, p->I, p->E, p->max_top_k);
@@ -569,8 +638,8 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
         fa.has_shared = p->has_shared;
         fa.gu = p->gu;
         fa.dn = p->dn;
-        std::memcpy(fa.tab_gu, p->fmt_gu == MOE_FMT_NVFP4 ? kNvfp4Tab : p->tab, sizeof(fa.tab_gu));
-        std::memcpy(fa.tab_dn, p->fmt_dn == MOE_FMT_NVFP4 ? kNvfp4Tab : p->tab, sizeof(fa.tab_dn));
+        fa.tab_gu = p->ct_gu;
+        fa.tab_dn = p->ct_dn;
         fa.logits = w.logits;
         fa.h = w.h;
         fa.y = w.y;
@@ -593,6 +662,8 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
                     pbase = pm->prof_used;
                     pm->prof_used += 2;
                     pm->prof_fwd.push_back({pbase, 1});
+                    if (pm->prof_stamps && pm->prof_nstamp < pm->prof_stamp_cap)
+                        fa.stamps = pm->prof_stamps + 16 * (size_t)pm->prof_nstamp++;
                 }
                 prof_mark(pm, pbase, 0, s);
                 moe_status st = check_launch(launch_fused(fa, tt, grid, smem, s));
@@ -651,7 +722,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     gu.out = w.h;
     gu.out_stride = p->I;
     gu.rows_out = p->I;
-    std::memcpy(gu.tab, p->fmt_gu == MOE_FMT_NVFP4 ? kNvfp4Tab : p->tab, sizeof(gu.tab));
+    gu.tab = p->ct_gu;
     int &ggu = pm->grid_cache[1][tt == 8];
     if (!ggu) ggu = matvec_grid(gu, true, tt, p->num_sms);
     st = check_launch(launch_matvec(gu, true, tt, ggu, s));
@@ -668,7 +739,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     dn.out = w.y;
     dn.out_stride = p->H;
     dn.rows_out = p->H;
-    std::memcpy(dn.tab, p->fmt_dn == MOE_FMT_NVFP4 ? kNvfp4Tab : p->tab, sizeof(dn.tab));
+    dn.tab = p->ct_dn;
     int &gdn = pm->grid_cache[0][tt == 8];
     if (!gdn) gdn = matvec_grid(dn, false, tt, p->num_sms);
     st = check_launch(launch_matvec(dn, false, tt, gdn, s));
@@ -727,6 +798,14 @@ moe_status moe_profile_begin(moe_pack *p, int max_forwards)
         }
     p->prof_fwd.clear();
     p->prof_used = 0;
+    p->prof_nstamp = 0;
+    p->prof_stamp_cap = max_forwards;
+    if (cudaMalloc(&p->prof_stamps, sizeof(long long) * 16 * (size_t)max_forwards) != cudaSuccess ||
+        cudaMemset(p->prof_stamps, 0, sizeof(long long) * 16 * (size_t)max_forwards) != cudaSuccess) {
+        cudaGetLastError();
+        p->prof_stamps = nullptr;
+        p->prof_stamp_cap = 0;
+    }
     p->prof_on = true;
     return MOE_OK;
 }
@@ -736,7 +815,7 @@ moe_status moe_profile_end(moe_pack *p, double *ms, int *n_forwards)
     if (!p || !p->prof_on) return MOE_ERR_INVALID_ARG;
     DeviceGuard g(p->device);
     moe_status st = cudaDeviceSynchronize() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-    double acc[PROF_STAGES] = {0, 0, 0, 0, 0, 0};
+    double acc[PROF_OUT] = {};
     for (const auto &f : p->prof_fwd) {
         if (st != MOE_OK) break;
         const int nint = f.second ? 1 : 4;
@@ -750,6 +829,28 @@ moe_status moe_profile_end(moe_pack *p, double *ms, int *n_forwards)
             acc[f.second == 1 ? PROF_FUSED : f.second == 2 ? PROF_PREFILL : i] += v;
         }
     }
+    if (p->prof_stamps && p->prof_nstamp > 0 && st == MOE_OK) {
+        // fused-kernel phases (CTA 0's clock): stage, router, barrier, plan,
+        // gate/up, barrier, down, barrier, combine/tail
+        std::vector<long long> h((size_t)16 * p->prof_nstamp);
+        int khz = 0;
+        cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, p->device);
+        if (khz > 0 && cudaMemcpy(h.data(), p->prof_stamps, h.size() * sizeof(long long), cudaMemcpyDeviceToHost) ==
+                           cudaSuccess) {
+            for (int f = 0; f < p->prof_nstamp; ++f) {
+                const long long *c = h.data() + 16 * (size_t)f;
+                auto span = [&](int a, int b) { return (c[a] && c[b] && c[b] > c[a]) ? (double)(c[b] - c[a]) : 0.0; };
+                double ph[PROF_PHASES];
+                for (int i = 0; i < 7; ++i) ph[i] = span(i, i + 1);
+                ph[7] = span(7, 8);
+                ph[8] = c[8] ? span(8, 9) : span(7, 9);
+                for (int i = 0; i < PROF_PHASES; ++i) acc[PROF_STAGES + i] += ph[i] / khz;  // cycles / kHz = ms
+            }
+        }
+    }
+    if (p->prof_stamps) cudaFree(p->prof_stamps);
+    p->prof_stamps = nullptr;
+    p->prof_nstamp = p->prof_stamp_cap = 0;
     for (auto &e : p->prof_ev) cudaEventDestroy(e);
     const int n = (int)p->prof_fwd.size();
     p->prof_ev.clear();
@@ -757,7 +858,7 @@ moe_status moe_profile_end(moe_pack *p, double *ms, int *n_forwards)
     p->prof_on = false;
     p->prof_used = 0;
     if (ms)
-        for (int i = 0; i < PROF_STAGES; ++i) ms[i] = acc[i];
+        for (int i = 0; i < PROF_OUT; ++i) ms[i] = acc[i];
     if (n_forwards) *n_forwards = n;
     return st;
 }

@@ -81,6 +81,15 @@ struct RouteArgs {
     int max_groups;
 };
 
+// 16-entry code table of a 4-bit format, built on the host by build_code_table:
+// entry bytes (value + bias) in t[0..3], magic = 2^23 + bias, xor_mode when the
+// halves were arranged for the XOR-combined lookup (else masked select).
+struct CodeTable {
+    uint32_t t[4];
+    float magic;
+    int xor_mode;
+};
+
 struct MatvecArgs {
     DevProj w;
     const int4 *groups;
@@ -91,8 +100,7 @@ struct MatvecArgs {
     float *out;               // gate/up: h [slots x I]; down: y [slots x H]
     int out_stride;
     int rows_out;             // gate/up: I (row pairs); down: H
-    uint32_t tab[4];          // 16-entry code table, bytes biased by +128
-    float ts_mul;             // NVFP4: folded into the block scale decode
+    CodeTable tab;            // 4-bit formats' code table
 };
 
 struct CombineArgs {
@@ -126,7 +134,7 @@ struct FusedArgs {
     const uint16_t *wr;
     int T, H, E, I, k, has_shared;
     DevProj gu, dn;
-    uint32_t tab_gu[4], tab_dn[4];
+    CodeTable tab_gu, tab_dn;
     float *logits;      // [T x E]
     float *h;           // [slots x I]
     float *y;           // [slots x H] (when not rowsplit)
@@ -137,6 +145,7 @@ struct FusedArgs {
     unsigned *bar;      // {arrive count, generation}
     int32_t *err;
     int rowsplit;       // down + combine by output rows in one phase
+    long long *stamps;  // optional: clock64 of CTA 0 at each phase boundary
 };
 
 // tensor-core prefill

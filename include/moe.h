@@ -212,14 +212,18 @@ moe_status moe_read_routing(const moe_pack *pack, int n_tokens, int top_k, int32
                             float *gate, int32_t *counts, void *stream);
 
 /* Kernel timing of forwards, for measurement.  moe_profile_begin creates
- * CUDA events for up to max_forwards forwards (this allocates: call it before
- * a timed region or a stream capture); each later forward on the pack then
+ * CUDA events (and a small device buffer) for up to max_forwards forwards
+ * (this allocates: call it before a timed region or a stream capture); each
+ * later forward on the pack then
  * records an event before each of its kernels and after the last one
  * (captured as event-record nodes when the stream is capturing).
  * moe_profile_end synchronises the device, adds the elapsed times per kernel
- * over all recorded forwards into ms[6] (host memory: route+plan, gate/up,
- * down, combine of the grouped path, the fused decode kernel, and the whole
- * tensor-core prefill sequence), stores the
+ * over all recorded forwards into ms[15] (host memory): [0..5] route+plan,
+ * gate/up, down, combine of the grouped path, the fused decode kernel, the
+ * whole tensor-core prefill sequence; [6..14] the fused kernel's phases as seen
+ * by its first CTA (token staging, router, barrier, plan, gate/up, barrier,
+ * down, barrier, combine), from its SM clock at the device's nominal rate.  It
+ * stores the
  * forward count in *n_forwards, and frees the events.  Forwards beyond
  * max_forwards are not recorded. */
 moe_status moe_profile_begin(moe_pack *pack, int max_forwards);
