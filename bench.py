@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--quick", action="store_true", help="for profiler runs: few steps, no baselines")
+    ap.add_argument("--path", choices=["auto", "grouped", "dense"], default="auto",
+                    help="decode kernel path (dense: the dense-batched comparison variant)")
     return ap.parse_args()
 
 
@@ -213,6 +215,32 @@ def reference_arm(a, wl):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- replicas across ranks
+
+
+def sync_barrier(dist, device_sync):
+    """Device sync, then a process barrier, then device sync (no-op barrier at N=1)."""
+    device_sync()
+    if dist is not None:
+        dist.barrier()
+    device_sync()
+
+
+def reduce_max(dist, v, device):
+    """Maximum of a per-rank float over all ranks (the slowest replica times the job)."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, steps, layers, tokens, ms_max):
+    """Whole-job layer-tokens/s: every rank runs its own replica of the step."""
+    return world * steps * layers * tokens / (ms_max / 1e3)
+
+
 # ---------------------------------------------------------------- GPU arm
 
 
@@ -254,7 +282,8 @@ def ours_arm(a, wl):
     for l in range(L):
         li = synth.layer_inputs(wl, l)
         x = synth.tokens(wl, li.router, l, 0, T)
-        pack = bq.pack_layer(li, max_tokens=T, max_top_k=k, device=dev)
+        pack = bq.pack_layer(li, max_tokens=T, max_top_k=k, device=dev,
+                             flags=bq.MOE_PACK_DENSE if a.path == "dense" else 0)
         layers.append({"pack": pack, "x": _to_dev_x(x), "xh": x,
                        "wr": torch.from_numpy(li.router.view(np.int16)).cuda(),
                        "out": torch.empty(T, H, device="cuda")})
@@ -265,8 +294,10 @@ def ours_arm(a, wl):
     log(f"[bench] rank {rank}: built {L} layers of {wl.name} in {gen_s:.1f} s")
     info = layers[0]["pack"].info()
 
+    path = {"auto": bq.MOE_PATH_AUTO, "grouped": bq.MOE_PATH_GROUPED, "dense": bq.MOE_PATH_DENSE}[a.path]
+
     def fwd(ly):
-        bq.moe_layer_forward(ly["x"], ly["wr"], ly["pack"], bq.MOE_FMT_FROM_PACK, k, ly["out"])
+        bq.moe_layer_forward_ex(ly["x"], ly["wr"], ly["pack"], bq.MOE_FMT_FROM_PACK, k, ly["out"], path)
 
     # routing of every layer (deterministic): active experts and slots
     n_active, slots = [], []
@@ -294,17 +325,10 @@ def ours_arm(a, wl):
     unique_bytes_step = sum(na * exp_b + E * H * 2 for na in n_active)
 
     def barrier():
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        torch.cuda.synchronize()
+        sync_barrier(dist, torch.cuda.synchronize)
 
     def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(dist, v, "cuda")
 
     # ---- timed region: K replays of the one-step graph
     g = torch.cuda.CUDAGraph()
@@ -323,7 +347,7 @@ def ours_arm(a, wl):
         en.synchronize()
     ms = max_over_ranks(st.elapsed_time(en))
     barrier()
-    value = world * a.steps * L * T / (ms / 1e3)
+    value = job_throughput(world, a.steps, L, T, ms)
     expert_gbs = world * a.steps * unique_bytes_step / (ms / 1e3) / 1e9
 
     # ---- kernel-stage durations: the same work with event records around each kernel
@@ -415,7 +439,7 @@ def ours_arm(a, wl):
                            "hidden": H, "experts": E, "inter": I, "top_k": k,
                            "shared_expert": wl.has_shared,
                            "formats": f"{synth.FMT_NAMES[wl.fmt_gate_up]}/{synth.FMT_NAMES[wl.fmt_down]}",
-                           "parallelism": f"replicas x{world}",
+                           "parallelism": f"replicas x{world}", "path": a.path,
                            "l2": f"inputs larger than L2: {L} distinct layers, "
                                  f"{unique_bytes_step / 1e6:.0f} MB of selected expert weights per step"},
                 "expert_gbs": expert_gbs, "expert_gbs_frac": expert_gbs / hbm,

@@ -36,7 +36,10 @@ class moe_pack_desc(ctypes.Structure):
                 ("down_blocks", ctypes.c_void_p), ("gate_up_tensor_scale", ctypes.c_void_p),
                 ("down_tensor_scale", ctypes.c_void_p), ("iq4nl_table", ctypes.c_void_p),
                 ("shared_gate_up_blocks", ctypes.c_void_p),
-                ("shared_down_blocks", ctypes.c_void_p)]
+                ("shared_down_blocks", ctypes.c_void_p), ("flags", ctypes.c_int)]
+
+
+MOE_PACK_DENSE = 1
 
 
 class moe_pack_info(ctypes.Structure):
@@ -146,7 +149,7 @@ class Pack:
 def moe_pack_experts(n_experts, hidden, inter, fmt_gate_up, fmt_down, gate_up_blocks, down_blocks,
                      gate_up_tensor_scale=None, down_tensor_scale=None, iq4nl_table=None,
                      shared_gate_up_blocks=None, shared_down_blocks=None, max_tokens=64,
-                     max_top_k=None, device=0):
+                     max_top_k=None, device=0, flags=0):
     """Upload a layer's experts.  Blocks are host uint8 arrays in the canonical
     layout of include/moe.h (expert-major); NVFP4 scales float32 [E(+1)]."""
     keep = [np.ascontiguousarray(gate_up_blocks, np.uint8), np.ascontiguousarray(down_blocks, np.uint8)]
@@ -158,7 +161,7 @@ def moe_pack_experts(n_experts, hidden, inter, fmt_gate_up, fmt_down, gate_up_bl
     d = moe_pack_desc(n_experts, hidden, inter, 1 if sgu is not None else 0, max_tokens,
                       max_top_k if max_top_k is not None else n_experts, fmt_gate_up, fmt_down,
                       _np_ptr(keep[0]), _np_ptr(keep[1]), _np_ptr(gts), _np_ptr(dts), _np_ptr(tab),
-                      _np_ptr(sgu), _np_ptr(sdn))
+                      _np_ptr(sgu), _np_ptr(sdn), flags)
     h = ctypes.c_void_p()
     _check(lib.moe_pack_experts(ctypes.byref(d), device, ctypes.byref(h)), "moe_pack_experts")
     return Pack(h, d)
@@ -242,7 +245,7 @@ def moe_get_device_error(pack):
     return lib.moe_get_device_error(pack.handle)
 
 
-def pack_layer(li, max_tokens=64, max_top_k=None, device=0):
+def pack_layer(li, max_tokens=64, max_top_k=None, device=0, flags=0):
     """Pack a synth.LayerInputs-like object (router, gate_up, down, scales, table)."""
     wl = li.wl
     E = wl.n_experts
@@ -252,4 +255,4 @@ def pack_layer(li, max_tokens=64, max_top_k=None, device=0):
                             li.down[:E], gs, ds, li.table,
                             li.gate_up[E] if wl.has_shared else None,
                             li.down[E] if wl.has_shared else None, max_tokens,
-                            max_top_k if max_top_k is not None else wl.top_k, device)
+                            max_top_k if max_top_k is not None else wl.top_k, device, flags)

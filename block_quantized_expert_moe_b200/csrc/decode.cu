@@ -203,6 +203,29 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
     }
 }
 
+// Dense-batched combine: out[t] = sum over active experts a of dgate[a*T+t] *
+// y[a*T+t] (the shared expert's gate is 1), in expert order.
+__global__ void __launch_bounds__(kThreads) combine_dense_kernel(const float *y, const float *dgate,
+                                                                 const int32_t *n_rows, int T, int H, float *out)
+{
+    const int t = blockIdx.y;
+    const int H4 = H >> 2;
+    const int n_act = __ldg(n_rows) / T;
+    for (int c = blockIdx.x * kThreads + threadIdx.x; c < H4; c += gridDim.x * kThreads) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int a = 0; a < n_act; ++a) {
+            const float g = __ldcg(dgate + (size_t)a * T + t);
+            if (g == 0.f) continue;
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(y + ((size_t)a * T + t) * H) + c);
+            acc.x = fmaf(g, v.x, acc.x);
+            acc.y = fmaf(g, v.y, acc.y);
+            acc.z = fmaf(g, v.z, acc.z);
+            acc.w = fmaf(g, v.w, acc.w);
+        }
+        reinterpret_cast<float4 *>(out + (size_t)t * H)[c] = acc;
+    }
+}
+
 using KernelFn = void (*)(MatvecArgs);
 
 template <int FMT>
@@ -263,6 +286,14 @@ cudaError_t launch_matvec(const MatvecArgs &a, bool gateup, int tt, int grid, cu
     KernelFn f = pick(a.w.fmt, gateup, tt);
     if (!f) return cudaErrorInvalidValue;
     f<<<grid, kThreads, matvec_smem_bytes(a, gateup, tt), s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine_dense(const float *y, const float *dgate, const int32_t *n_rows, int T, int H,
+                                 float *out, cudaStream_t s)
+{
+    dim3 grid((H / 4 + kThreads - 1) / kThreads, T);
+    combine_dense_kernel<<<grid, kThreads, 0, s>>>(y, dgate, n_rows, T, H, out);
     return cudaGetLastError();
 }
 

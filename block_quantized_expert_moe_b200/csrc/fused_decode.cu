@@ -245,52 +245,62 @@ __device__ void phase_router(const FusedArgs &a, const float4 *xs4)
 }
 
 // ---- P2: top-k and the plan, in this CTA's shared memory ----------------------
+// Order-preserving key of a float (larger float -> larger unsigned key).
+__device__ __forceinline__ unsigned fkey(float f)
+{
+    const unsigned u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Top-k of one token's logits by warp `warp`: k rounds of (lane-local best,
+// warp max of the order-preserving key with redux, lowest index among the
+// lanes holding it).  Writes the selected experts (descending logit) and gates.
+__device__ void warp_topk(const FusedArgs &a, int t, int *sel_e, float *sel_g)
+{
+    const int lane = threadIdx.x & 31;
+    const int E = a.E, k = a.k;
+    float v[32];
+    uint32_t taken = 0u;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) v[i] = __ldcg(a.logits + (size_t)t * E + e);
+        else { v[i] = -INFINITY; taken |= 1u << i; }
+    }
+    float vmax = 0.f, den = 0.f;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 32;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (!((taken >> i) & 1u) && (bi == 32 || v[i] > bv)) {
+                bv = v[i];
+                bi = i;
+            }
+        const unsigned key = bi < 32 ? fkey(bv) : 0u;
+        const unsigned kmax = __reduce_max_sync(0xffffffffu, key);
+        const unsigned cand = (key == kmax && bi < 32) ? (unsigned)(lane + 32 * bi) : 0xffffffffu;
+        const unsigned win = __reduce_min_sync(0xffffffffu, cand);
+        if ((int)(win & 31) == lane) taken |= 1u << (win >> 5);
+        const float wv = __shfl_sync(0xffffffffu, bv, win & 31);
+        if (j == 0) vmax = wv;
+        den += expf(wv - vmax);
+        if (lane == 0) {
+            sel_e[t * k + j] = (int)win;
+            sel_g[t * k + j] = wv;  // logit for now, gate below
+        }
+    }
+    __syncwarp();
+    if (lane < k) sel_g[t * k + lane] = expf(sel_g[t * k + lane] - vmax) / den;
+    __syncwarp();
+}
+
 template <int FT>
 __device__ void phase_plan(const FusedArgs &a, const Plan &pl)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = a.E, k = a.k, T = a.T;
-    if (warp < T) {
-        const int t = warp;
-        float v[32];
-        uint32_t taken = 0u;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E) v[i] = __ldcg(a.logits + (size_t)t * E + e);
-            else { v[i] = -INFINITY; taken |= 1u << i; }
-        }
-        float vmax = 0.f, den = 0.f;
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int bi = INT_MAX;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if (!((taken >> i) & 1u) && (bi == INT_MAX || v[i] > bv)) {
-                    bv = v[i];
-                    bi = lane + 32 * i;
-                }
-            }
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (oi != INT_MAX && (bi == INT_MAX || ov > bv || (ov == bv && oi < bi))) {
-                    bv = ov;
-                    bi = oi;
-                }
-            }
-            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-            if (j == 0) vmax = bv;
-            den += expf(bv - vmax);
-            if (lane == 0) {
-                pl.sel_e[t * k + j] = bi;
-                pl.sel_g[t * k + j] = bv;  // logit for now, gate below
-            }
-        }
-        __syncwarp();
-        if (lane < k) pl.sel_g[t * k + lane] = expf(pl.sel_g[t * k + lane] - vmax) / den;
-    }
+    if (warp < T) warp_topk(a, warp, pl.sel_e, pl.sel_g);
     for (int e = threadIdx.x; e < E; e += FT) {
         pl.cnt[e] = 0;
         pl.mask[e] = 0u;
@@ -336,6 +346,45 @@ __device__ void phase_plan(const FusedArgs &a, const Plan &pl)
     __syncthreads();
 }
 
+// Plan of a single token: the k experts in ascending id order, one slot and one
+// group each, the shared expert's group last.  Warp 0 only; no block scans.
+template <int FT>
+__device__ void phase_plan_t1(const FusedArgs &a, const Plan &pl)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int k = a.k, E = a.E;
+    if (warp == 0) {
+        warp_topk(a, 0, pl.sel_e, pl.sel_g);
+        const int me = lane < k ? pl.sel_e[lane] : INT_MAX;
+        int rank = 0;
+        for (int i = 0; i < k; ++i) rank += __shfl_sync(0xffffffffu, me, i) < me;
+        if (lane < k) {
+            pl.groups[rank] = make_int4(me, rank, 1, 0);
+            pl.perm_tok[rank] = 0;
+            pl.slot_gate[rank] = pl.sel_g[lane];
+            pl.slot_of[lane] = rank;
+        }
+        if (lane == 0) {
+            if (a.has_shared) {
+                pl.groups[k] = make_int4(E, k, 1, 0);
+                pl.perm_tok[k] = 0;
+                pl.slot_gate[k] = 1.f;
+            }
+            *pl.n_groups = k + (a.has_shared ? 1 : 0);
+        }
+    }
+    if (blockIdx.x == 0) {
+        for (int e = threadIdx.x; e <= E; e += FT) a.cnt_out[e] = e < E ? 0 : (a.has_shared ? 1 : 0);
+        __syncthreads();
+        if (warp == 0 && lane < k) {
+            a.idx_out[lane] = pl.sel_e[lane];
+            a.gate_out[lane] = pl.sel_g[lane];
+            a.cnt_out[pl.sel_e[lane]] = 1;
+        }
+    }
+    __syncthreads();
+}
+
 __device__ __forceinline__ int lanes_per_row(int NU)
 {
     return NU >= 32 ? 32 : NU >= 16 ? 16 : NU >= 8 ? 8 : NU >= 4 ? 4 : NU >= 2 ? 2 : 1;
@@ -368,35 +417,68 @@ __device__ void phase_gateup(const FusedArgs &a, const Plan &pl, const float4 *x
             }
             const float xs0 = FMT == MOE_FMT_Q5_1 && u < NU ? xsum[u] : 0.f;
             const float xs1 = FMT == MOE_FMT_Q5_1 && has2 ? xsum[u2] : 0.f;
-            for (long long tk = t0 + warp; tk < t1; tk += NW) {
+            // one task of look-ahead: the next task's code loads are in flight
+            // while this one is decoded
+            auto task_of = [&](long long tk, int &e, int &rr, int &r, int &slot0) {
                 const int g = (int)(tk / tpg);
-                const int r = (int)(tk - (long long)g * tpg) * RPW + sub;
-                const bool valid = r < rows;
-                const int rr = valid ? r : rows - 1;
+                r = (int)(tk - (long long)g * tpg) * RPW + sub;
+                rr = r < rows ? r : rows - 1;
                 const int4 gd = pl.groups[g];
-                const int e = gd.x, slot0 = gd.y;
-                const float half_ts = FMT == MOE_FMT_NVFP4 ? 0.5f * __ldg(w.ts + e) : 0.5f;
+                e = gd.x;
+                slot0 = gd.y;
+            };
+            Raw c0, c1, c2, c3;  // gate u, up u, gate u2, up u2 of the current task
+            int ce = 0, crr = 0, cr = rows, cslot = 0;
+            long long tk = t0 + warp;
+            if (tk < t1) {
+                task_of(tk, ce, crr, cr, cslot);
+                if (u < NU) {
+                    c0 = load_unit<FMT>(w, ce, crr, u);
+                    c1 = load_unit<FMT>(w, ce, rows + crr, u);
+                    if (has2) {
+                        c2 = load_unit<FMT>(w, ce, crr, u2);
+                        c3 = load_unit<FMT>(w, ce, rows + crr, u2);
+                    }
+                }
+            }
+            for (; tk < t1; tk += NW) {
+                const long long tn = tk + NW;
+                Raw n0, n1, n2, n3;
+                int ne = 0, nrr = 0, nr = rows, nslot = 0;
+                if (tn < t1) {
+                    task_of(tn, ne, nrr, nr, nslot);
+                    if (u < NU) {
+                        n0 = load_unit<FMT>(w, ne, nrr, u);
+                        n1 = load_unit<FMT>(w, ne, rows + nrr, u);
+                        if (has2) {
+                            n2 = load_unit<FMT>(w, ne, nrr, u2);
+                            n3 = load_unit<FMT>(w, ne, rows + nrr, u2);
+                        }
+                    }
+                }
+                const float half_ts = FMT == MOE_FMT_NVFP4 ? 0.5f * __ldg(w.ts + ce) : 0.5f;
                 float s0 = 0.f, s1 = 0.f;
                 if (u < NU) {
-                    const Raw g0 = load_unit<FMT>(w, e, rr, u);
-                    const Raw v0 = load_unit<FMT>(w, e, rows + rr, u);
-                    Raw g1 = g0, v1 = v0;
+                    s0 = unit_dot_reg<FMT>(c0, xr0, xs0, a.tab_gu, half_ts, s0);
+                    s1 = unit_dot_reg<FMT>(c1, xr0, xs0, a.tab_gu, half_ts, s1);
                     if (has2) {
-                        g1 = load_unit<FMT>(w, e, rr, u2);
-                        v1 = load_unit<FMT>(w, e, rows + rr, u2);
-                    }
-                    s0 = unit_dot_reg<FMT>(g0, xr0, xs0, a.tab_gu, half_ts, s0);
-                    s1 = unit_dot_reg<FMT>(v0, xr0, xs0, a.tab_gu, half_ts, s1);
-                    if (has2) {
-                        s0 = unit_dot_reg<FMT>(g1, xr1, xs1, a.tab_gu, half_ts, s0);
-                        s1 = unit_dot_reg<FMT>(v1, xr1, xs1, a.tab_gu, half_ts, s1);
+                        s0 = unit_dot_reg<FMT>(c2, xr1, xs1, a.tab_gu, half_ts, s0);
+                        s1 = unit_dot_reg<FMT>(c3, xr1, xs1, a.tab_gu, half_ts, s1);
                     }
                 }
                 for (int o = LPR >> 1; o >= 1; o >>= 1) {
                     s0 += __shfl_xor_sync(0xffffffffu, s0, o);
                     s1 += __shfl_xor_sync(0xffffffffu, s1, o);
                 }
-                if (valid && sl == 0) a.h[(size_t)slot0 * a.I + r] = s0 / (1.f + expf(-s0)) * s1;
+                if (cr < rows && sl == 0) a.h[(size_t)cslot * a.I + cr] = s0 / (1.f + expf(-s0)) * s1;
+                c0 = n0;
+                c1 = n1;
+                c2 = n2;
+                c3 = n3;
+                ce = ne;
+                crr = nrr;
+                cr = nr;
+                cslot = nslot;
             }
             return;
         }
@@ -738,7 +820,8 @@ __global__ void __launch_bounds__(FT, 1) fused_decode_kernel(const FusedArgs a)
     if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[2] = clock64();
     if (!grid_sync(a.bar, a.err)) return;
     if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[3] = clock64();
-    phase_plan<FT>(a, pl);
+    if (a.T == 1) phase_plan_t1<FT>(a, pl);
+    else phase_plan<FT>(a, pl);
     if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[4] = clock64();
 
     if (a.rowsplit) {  // start this CTA's down rows into L2 while gate/up runs

@@ -27,7 +27,7 @@ using namespace moe;
 struct moe_pack {
     int device = 0;
     int num_sms = 0;
-    int E = 0, H = 0, I = 0, has_shared = 0, max_tokens = 0, max_top_k = 0;
+    int E = 0, H = 0, I = 0, has_shared = 0, max_tokens = 0, max_top_k = 0, flags = 0;
     int fmt_gu = 0, fmt_dn = 0;
     DevProj gu, dn;
     CodeTable ct_gu{}, ct_dn{};
@@ -333,7 +333,8 @@ moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, con
 moe_status build_workspace(moe_pack *p)
 {
     const int64_t T = p->max_tokens, k = p->max_top_k, E = p->E;
-    const int64_t slots = T * (k + 1);
+    int64_t slots = T * (k + 1);
+    if ((p->flags & MOE_PACK_DENSE) && T <= kDecodeMaxTokens) slots = std::max(slots, (E + 1) * T);
     Workspace &w = p->ws;
     w.max_groups = (int)(slots + E + 2);
     struct Item { void **dst; int64_t bytes; };
@@ -343,6 +344,7 @@ moe_status build_workspace(moe_pack *p)
         {(void **)&w.slot_pos, T * k * 4}, {(void **)&w.groups, (int64_t)w.max_groups * 16},
         {(void **)&w.n_groups, 4}, {(void **)&w.ticket, 4}, {(void **)&w.err, 4}, {(void **)&w.bar, 8},
         {(void **)&w.h, slots * p->I * 4}, {(void **)&w.y, slots * p->H * 4},
+        {(void **)&w.dgate, slots * 4}, {(void **)&w.n_dense_rows, 4},
     };
     int64_t total = 0;
     for (auto &it : items) total += round_up(it.bytes, 256);
@@ -470,6 +472,7 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
     p->has_shared = d->has_shared ? 1 : 0;
     p->max_tokens = d->max_tokens;
     p->max_top_k = d->max_top_k;
+    p->flags = d->flags;
     p->fmt_gu = d->fmt_gate_up;
     p->fmt_dn = d->fmt_down;
     p->ct_gu = build_code_table(p->fmt_gu, d->iq4nl_table, p->perm_gu);
@@ -591,7 +594,10 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     if (path == MOE_PATH_AUTO)
         path = n_tokens <= kDecodeMaxTokens ? MOE_PATH_DECODE : (prefill_ok ? MOE_PATH_PREFILL : MOE_PATH_GROUPED);
     if (path == MOE_PATH_PREFILL && !prefill_ok) return MOE_ERR_UNSUPPORTED;
-    if (path != MOE_PATH_DECODE && path != MOE_PATH_GROUPED && path != MOE_PATH_PREFILL) return MOE_ERR_UNSUPPORTED;
+    if (path == MOE_PATH_DENSE && (!(p->flags & MOE_PACK_DENSE) || n_tokens > kDecodeMaxTokens))
+        return MOE_ERR_UNSUPPORTED;
+    if (path != MOE_PATH_DECODE && path != MOE_PATH_GROUPED && path != MOE_PATH_PREFILL && path != MOE_PATH_DENSE)
+        return MOE_ERR_UNSUPPORTED;
     DeviceGuard g(p->device);
     if (!g.ok) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -708,6 +714,9 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     ra.err = w.err;
     ra.groups = w.groups;
     ra.max_groups = w.max_groups;
+    ra.dense = path == MOE_PATH_DENSE;
+    ra.dgate = w.dgate;
+    ra.n_dense_rows = w.n_dense_rows;
     moe_status st = check_launch(launch_route(ra, route_grid(p->E, p->num_sms), s));
     if (st != MOE_OK) return st;
     prof_mark(pm, pbase, 1, s);
@@ -746,6 +755,11 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     if (st != MOE_OK) return st;
     prof_mark(pm, pbase, 3, s);
 
+    if (path == MOE_PATH_DENSE) {
+        st = check_launch(launch_combine_dense(w.y, w.dgate, w.n_dense_rows, T, p->H, out, s));
+        prof_mark(pm, pbase, 4, s);
+        return st;
+    }
     CombineArgs ca{};
     ca.y = w.y;
     ca.slot_pos = w.slot_pos;

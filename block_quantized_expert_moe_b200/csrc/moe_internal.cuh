@@ -59,6 +59,8 @@ struct Workspace {
     int32_t *ticket = nullptr;   // last-CTA counter of the route kernel
     unsigned *bar = nullptr;     // grid barrier of the fused decode kernel {count, gen}
     int32_t *err = nullptr;      // sticky device error (moe_status)
+    float *dgate = nullptr;      // dense-batched plan: per slot gate (0 when not routed)
+    int32_t *n_dense_rows = nullptr;
     float *h = nullptr;          // [slots x I]
     float *y = nullptr;          // [slots x H]
     int max_groups = 0;
@@ -79,6 +81,10 @@ struct RouteArgs {
     int32_t *cnt, *off, *perm_tok, *slot_pos, *n_groups, *err;
     int4 *groups;
     int max_groups;
+    // dense-batched plan: every active expert takes the whole batch
+    int dense;
+    float *dgate;           // [slots] gate of (active expert, token), 0 if not routed
+    int32_t *n_dense_rows;  // active experts (incl. shared) x T
 };
 
 // 16-entry code table of a 4-bit format, built on the host by build_code_table:
@@ -123,6 +129,8 @@ size_t matvec_smem_bytes(const MatvecArgs &a, bool gateup, int tt);
 int matvec_grid(const MatvecArgs &a, bool gateup, int tt, int num_sms);
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
+cudaError_t launch_combine_dense(const float *y, const float *dgate, const int32_t *n_rows, int T, int H,
+                                 float *out, cudaStream_t s);
 
 // Fused decode (one cooperative launch per layer, n_tokens <= 8).
 constexpr int kFusedMaxT = 8;

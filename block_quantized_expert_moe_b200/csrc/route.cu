@@ -128,6 +128,57 @@ __device__ void topk_phase(const RouteArgs &a, unsigned char *smem)
     }
 }
 
+// Dense-batched plan: active expert a (ascending id, the shared expert last)
+// owns slots a*T .. a*T+T-1, one per token of the batch; its gate for token t is
+// the routing gate if t selected it, else 0.
+__device__ void plan_dense(const RouteArgs &a, unsigned char *smem)
+{
+    const int tid = threadIdx.x;
+    const int E = a.E, k = a.k, T = a.T, tt = a.tt;
+    int *cnt = reinterpret_cast<int *>(smem);
+    int *act = cnt + (E + 1);
+    int *tmp = act + (E + 1);
+    for (int e = tid; e < E; e += kThreads) cnt[e] = 0;
+    __syncthreads();
+    for (int i = tid; i < T * k; i += kThreads) atomicAdd(&cnt[__ldcg(a.idx + i)], 1);
+    __syncthreads();
+    for (int e = tid; e < E; e += kThreads) act[e] = cnt[e] > 0 ? 1 : 0;
+    __syncthreads();
+    const int n_routed = block_exclusive_scan(act, E, tmp);
+    const int n_act = n_routed + (a.has_shared ? 1 : 0);
+    const int chunks = (T + tt - 1) / tt;
+    if (n_act * chunks > a.max_groups) {
+        if (tid == 0) {
+            atomicExch(a.err, (int)MOE_ERR_DEVICE);
+            *a.n_groups = 0;
+        }
+        return;
+    }
+    for (int i = tid; i < n_act * T; i += kThreads) {
+        a.perm_tok[i] = i % T;
+        a.dgate[i] = (a.has_shared && i >= n_routed * T) ? 1.f : 0.f;
+    }
+    for (int e = tid; e < E; e += kThreads) {
+        a.cnt[e] = cnt[e];
+        if (cnt[e] > 0)
+            for (int c = 0; c < chunks; ++c)
+                a.groups[act[e] * chunks + c] = make_int4(e, act[e] * T + c * tt, min(tt, T - c * tt), 0);
+    }
+    if (a.has_shared)
+        for (int c = tid; c < chunks; c += kThreads)
+            a.groups[n_routed * chunks + c] = make_int4(E, n_routed * T + c * tt, min(tt, T - c * tt), 0);
+    __syncthreads();  // dgate zeroed before the routed gates land
+    for (int i = tid; i < T * k; i += kThreads) {
+        const int e = __ldcg(a.idx + i);
+        a.dgate[act[e] * T + i / k] = __ldcg(a.gate + i);
+    }
+    if (tid == 0) {
+        a.cnt[E] = a.has_shared ? T : 0;
+        *a.n_groups = n_act * chunks;
+        *a.n_dense_rows = n_act * T;
+    }
+}
+
 __device__ void plan_phase(const RouteArgs &a, unsigned char *smem)
 {
     const int tid = threadIdx.x;
@@ -282,7 +333,8 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const RouteArgs a)
     topk_phase(a, smem);
     if (a.do_plan) {
         __syncthreads();
-        plan_phase(a, smem);
+        if (a.dense) plan_dense(a, smem);
+        else plan_phase(a, smem);
     }
     __syncthreads();
     if (threadIdx.x == 0) *a.ticket = 0;

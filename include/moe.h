@@ -83,8 +83,9 @@ typedef enum { MOE_DT_F32 = 1, MOE_DT_BF16 = 2 } moe_dtype;
  * to NVFP4 per token - or both Q8_0 - weights dequantised to bf16 for bf16 MMA;
  * hidden and inter multiples of 256, bf16 activations, top_k <= 32; its
  * buffers are sized at pack time when max_tokens > 64), else GROUPED.  DENSE is the dense-batched
- * comparison variant: every active expert multiplies the whole batch, with a
- * zero gate for tokens not routed to it. */
+ * comparison variant (pack created with MOE_PACK_DENSE, n_tokens <= 64): every
+ * active expert multiplies the whole batch, with a zero gate for the tokens not
+ * routed to it. */
 typedef enum {
     MOE_PATH_AUTO = 0,
     MOE_PATH_DECODE = 1,   /* one fused launch for n_tokens <= 8, top_k <= 16, else GROUPED */
@@ -124,7 +125,12 @@ typedef struct {
     const int8_t *iq4nl_table;
     const void *shared_gate_up_blocks;
     const void *shared_down_blocks;
+    int flags;            /* MOE_PACK_* bits, 0 for none */
 } moe_pack_desc;
+
+/* moe_pack_desc.flags: size the workspace for MOE_PATH_DENSE as well (every
+ * active expert times the whole batch: (n_experts + 1) * max_tokens slots). */
+#define MOE_PACK_DENSE 1
 
 typedef struct moe_pack moe_pack; /* opaque; owns device memory */
 

@@ -22,14 +22,14 @@ def router_to_device(wr):
     return torch.from_numpy(np.ascontiguousarray(wr).view(np.int16)).cuda()
 
 
-def gpu_layer(li, x_np, k, path=None, pack=None, repeat=1):
+def gpu_layer(li, x_np, k, path=None, pack=None, repeat=1, flags=0):
     """Run the layer through the C ABI.  Returns (out [T,H] float64, idx, gate, counts)."""
     import torch
     import block_quantized_expert_moe_b200 as bq
     T = x_np.shape[0]
     own = pack is None
     if own:
-        pack = bq.pack_layer(li, max_tokens=T, max_top_k=k)
+        pack = bq.pack_layer(li, max_tokens=T, max_top_k=k, flags=flags)
     xt = to_device(x_np)
     wr = router_to_device(li.router)
     out = torch.full((T, li.wl.hidden), float("nan"), device="cuda")

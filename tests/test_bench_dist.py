@@ -1,0 +1,59 @@
+"""The benchmark's multi-rank logic (replicas, max-over-ranks timing, rank-0
+output) on two gloo ranks on the CPU."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.sync_barrier(dist, lambda: None)
+        ms = 10.0 + 5.0 * rank                      # rank 1 is the slow replica
+        ms_max = bench.reduce_max(dist, ms, "cpu")
+        value = bench.job_throughput(world, steps=4, layers=3, tokens=2, ms_max=ms_max)
+        q.put((rank, ms_max, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_replicas_take_the_slowest_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [15.0, 15.0]
+    # 2 ranks x 4 steps x 3 layers x 2 tokens in 15 ms
+    assert all(abs(r[2] - 48 / 0.015) < 1e-6 for r in res)
+
+
+def test_single_rank_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.reduce_max(None, 3.5, "cpu") == 3.5
+    bench.sync_barrier(None, lambda: None)
+    assert bench.job_throughput(1, 10, 48, 1, 100.0) == 4800.0

@@ -171,3 +171,15 @@ def test_tensor_core_router_matches_oracle(name, T, kw):
     assert np.abs(gate.cpu().numpy() - rgate).max() <= 1e-5
     logits = ws[256:256 + 4 * T * wl.n_experts].view(torch.float32).view(T, wl.n_experts).cpu().numpy()
     assert np.abs(logits - rlog).max() <= 1e-4 * np.abs(rlog).max()
+
+
+@pytest.mark.parametrize("name,T", [("zipf_batch", 64), ("model_decode", 5)])
+def test_dense_batched_variant_matches_oracle(name, T):
+    """Every active expert multiplies the whole batch (zero gates where not routed)."""
+    import block_quantized_expert_moe_b200 as bq
+    wl, li = _layer(name, 1)
+    x = synth.tokens(wl, li.router, 1, 3, T)
+    out, idx, gate, counts = gpu_layer(li, x, wl.top_k, path=bq.MOE_PATH_DENSE, flags=bq.MOE_PACK_DENSE)
+    ref, ridx, rgate = oracle_layer(li, x, wl.top_k)
+    assert_routing_equal(idx, gate, ridx, rgate)
+    assert normwise_err(out, ref) <= DECODE_TOL
