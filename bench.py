@@ -361,7 +361,7 @@ def ours_arm(a, wl):
                 fwd(ly)
     gp.replay()
     torch.cuda.synchronize()
-    stage_ms = np.zeros(15)
+    stage_ms = np.zeros(32)
     nf = 0
     for ly in layers:
         m, n = bq.moe_profile_end(ly["pack"])
@@ -370,10 +370,21 @@ def ours_arm(a, wl):
     prefill_kernels = 7 if wl.fmt_gate_up == synth.FMT_NVFP4 else 6  # route GEMM, top-k, plan, gather, GEMMs (+ h quant)
     launches_per_fwd = 1 if stage_ms[4] > 0 else (prefill_kernels if stage_ms[5] > 0 else 4)
     stage_us = {s: float(stage_ms[i] / nf * 1e3) for i, s in enumerate(STAGES) if stage_ms[i] > 0}
-    phase_names = ["stage_x", "router", "barrier1", "plan", "gate_up", "barrier2", "down", "barrier3", "combine"]
-    fused_phase_us = ({n: float(stage_ms[6 + i] / nf * 1e3) for i, n in enumerate(phase_names)}
+    phase_names = (["stage_x", "router", "logit_poll_topk", "issue", "gate_up", "h_poll", "down", "-", "tail"]
+                   if T == 1 else
+                   ["stage_x", "router", "barrier1", "plan", "gate_up", "barrier2", "down", "barrier3", "combine"])
+    fused_phase_us = ({n: float(stage_ms[6 + i] / nf * 1e3) for i, n in enumerate(phase_names) if n != "-"}
                       if stage_ms[4] > 0 else None)
+    # streaming kernel: first/last CTA reaching each grid event, from the first CTA's start
+    grid_names = ["last_start", "first_router", "last_router", "first_issue", "last_issue",
+                  "first_gate_up", "last_gate_up", "first_end", "last_end"]
+    grid_event_us = ({n: float(stage_ms[15 + i] / nf * 1e3) for i, n in enumerate(grid_names)}
+                     if stage_ms[4] > 0 and T == 1 else None)
+    if grid_event_us is not None:
+        grid_event_us["cta0_points"] = [round(float(v / nf * 1e3), 3) for v in stage_ms[24:32]]
     dom = max(stage_us, key=lambda s: stage_us[s])
+    # one token: the streaming kernel (whole-row bulk copies) runs in place of the fused one
+    kname = "stream1_kernel" if dom == "fused" and T == 1 else KERNEL_NAMES[dom]
     hbm, peak_src = peaks()
     traffic = kernel_traffic(dom, wl.name)
     if dom == "prefill":
@@ -388,7 +399,7 @@ def ours_arm(a, wl):
         dom_bytes = float(np.mean(stage_bytes[dom]))
         achieved = dom_bytes / (stage_us[dom] * 1e-6) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                    "frac": achieved / hbm, "traffic": traffic, "kernel": KERNEL_NAMES[dom],
+                    "frac": achieved / hbm, "traffic": traffic, "kernel": kname,
                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                     else "fallback 6650 GB/s",
                     "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": stage_us[dom]}
@@ -445,7 +456,7 @@ def ours_arm(a, wl):
                 "expert_gbs": expert_gbs, "expert_gbs_frac": expert_gbs / hbm,
                 "unique_expert_bytes_per_step": unique_bytes_step,
                 "active_experts_per_layer": float(np.mean(n_active)),
-                "stage_us": stage_us, "fused_phase_us": fused_phase_us, "roofline": roofline,
+                "stage_us": stage_us, "fused_phase_us": fused_phase_us, "grid_event_us": grid_event_us, "roofline": roofline,
                 "clocks": clk.summary(),
                 "e2e": e2e, "gpu_launches": launches_per_fwd * L * a.steps, "cpu_baseline": cpu,
                 "gen_seconds": gen_s}

@@ -233,9 +233,10 @@ def moe_profile_begin(pack, max_forwards):
 
 
 def moe_profile_end(pack):
-    """-> (ms[15] summed over recorded forwards: route+plan, gate/up, down, combine,
-    fused, prefill, then the fused kernel's nine phases; n_forwards)."""
-    ms = np.zeros(15, np.float64)
+    """-> (ms[32] summed over recorded forwards: route+plan, gate/up, down, combine,
+    fused, prefill, the fused kernel's nine phases, then the streaming kernel's
+    grid events and its first CTA's sub-step times; n_forwards)."""
+    ms = np.zeros(32, np.float64)
     n = ctypes.c_int(0)
     _check(lib.moe_profile_end(pack.handle, _np_ptr(ms), ctypes.byref(n)), "moe_profile_end")
     return ms, n.value

@@ -20,7 +20,9 @@ cudaError_t matvec_set_attributes();
 
 // kernel-stage slots of the profiling API (moe_profile_end's ms[])
 enum { PROF_ROUTE = 0, PROF_GATE_UP = 1, PROF_DOWN = 2, PROF_COMBINE = 3, PROF_FUSED = 4, PROF_PREFILL = 5,
-       PROF_STAGES = 6, PROF_PHASES = 9, PROF_OUT = PROF_STAGES + PROF_PHASES };
+       PROF_STAGES = 6, PROF_PHASES = 9, PROF_GRID = 9, PROF_SUB = 8,
+       PROF_OUT = PROF_STAGES + PROF_PHASES + PROF_GRID + PROF_SUB };
+constexpr int kStampStride = 32;  // device stamps per recorded forward (see FusedArgs::stamps)
 
 using namespace moe;
 
@@ -45,6 +47,9 @@ struct moe_pack {
     long long *prof_stamps = nullptr;  // device, 16 clock64 stamps per recorded fused forward
     int prof_nstamp = 0, prof_stamp_cap = 0;
     int fused_grid[2] = {0, 0};   // [tt==8]
+    int stream1 = -1;             // single-token streaming kernel usable (-1: not yet checked)
+    size_t stream1_smem = 0;
+    int pdl = 1;                  // launch it as a programmatic dependent of the previous kernel
     bool has_prefill = false;     // tensor-core prefill workspace present
     PrefillWorkspace pws;
 };
@@ -135,6 +140,7 @@ moe_status init_device(int dev)
     if (route_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (matvec_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (fused_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
+    if (stream1_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_nvfp4_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_q8_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
@@ -194,7 +200,7 @@ int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 // Repack one expert's projection (rows x cols canonical blocks) into planes.
 // Returns false on an invalid NVFP4 block scale.
 bool repack_expert(int fmt, const uint8_t *src, int rows, int cols, uint8_t *qs, uint8_t *sc,
-                   uint8_t *qh, const uint8_t *perm)
+                   uint8_t *qh, uint8_t *sr, const uint8_t *perm)
 {
     uint8_t pbyte[256];  // both nibbles of a code byte through the position map
     for (int b = 0; b < 256; ++b) pbyte[b] = (uint8_t)(perm[b & 15] | (perm[b >> 4] << 4));
@@ -233,6 +239,7 @@ bool repack_expert(int fmt, const uint8_t *src, int rows, int cols, uint8_t *qs,
                 const uint8_t *blk = row + b * 9;
                 if (blk[0] >= 0x7Fu) return false;  // negative scale or NaN
                 sc[sf_offset(r, b >> 2, b & 3, ks)] = blk[0];
+                sr[(int64_t)r * (cols / 16) + b] = blk[0];
                 std::memcpy(q + 8 * b, blk + 1, 8);
             }
         }
@@ -288,12 +295,16 @@ moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, con
     dp.sc_stride = round_up(fmt == MOE_FMT_NVFP4 ? nvfp4_sf_bytes(rows, cols) : (int64_t)rows * dp.sc_row, 256);
     dp.ksteps = fmt == MOE_FMT_NVFP4 ? nvfp4_ksteps(cols) : 0;
     dp.qh_stride = round_up((int64_t)rows * dp.qh_row, 256);
+    const bool nv = fmt == MOE_FMT_NVFP4;
+    dp.sr_row = nv ? cols / 16 : dp.sc_row;
+    dp.sr_stride = nv ? round_up((int64_t)rows * dp.sr_row, 256) : dp.sc_stride;
     const int64_t canon = canon_row_bytes(fmt, cols) * rows;
-    std::vector<uint8_t> hq, hs, hh;
+    std::vector<uint8_t> hq, hs, hh, hr;
     try {
         hq.assign((size_t)dp.qs_stride * n_slots, 0);
         hs.assign((size_t)dp.sc_stride * n_slots, 0);
         if (dp.qh_row) hh.assign((size_t)dp.qh_stride * n_slots, 0);
+        if (nv) hr.assign((size_t)dp.sr_stride * n_slots, 0);
     } catch (const std::bad_alloc &) {
         return MOE_ERR_OOM;
     }
@@ -302,7 +313,8 @@ moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, con
         const uint8_t *src = s < p->E ? blocks + (int64_t)s * canon : shared_blocks;
         ok[s] = repack_expert(fmt, src, rows, cols, hq.data() + (int64_t)s * dp.qs_stride,
                               hs.data() + (int64_t)s * dp.sc_stride,
-                              dp.qh_row ? hh.data() + (int64_t)s * dp.qh_stride : nullptr, perm);
+                              dp.qh_row ? hh.data() + (int64_t)s * dp.qh_stride : nullptr,
+                              nv ? hr.data() + (int64_t)s * dp.sr_stride : nullptr, perm);
     });
     for (char c : ok)
         if (!c) return MOE_ERR_INVALID_ARG;
@@ -322,11 +334,17 @@ moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, con
         if ((st = dev_alloc(p, sizeof(float) * n_slots, &dt)) != MOE_OK) return st;
         if (cudaMemcpy(dt, ts, sizeof(float) * n_slots, cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
     }
+    void *dr = ds;
+    if (nv) {
+        if ((st = dev_alloc(p, hr.size(), &dr)) != MOE_OK) return st;
+        if (cudaMemcpy(dr, hr.data(), hr.size(), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     dp.qs = static_cast<const uint8_t *>(dq);
     dp.sc = static_cast<const uint8_t *>(ds);
     dp.qh = static_cast<const uint8_t *>(dh);
     dp.ts = static_cast<const float *>(dt);
-    p->arena_bytes += (int64_t)(hq.size() + hs.size() + hh.size()) + (dt ? 4 * n_slots : 0);
+    dp.sr = static_cast<const uint8_t *>(dr);
+    p->arena_bytes += (int64_t)(hq.size() + hs.size() + hh.size() + hr.size()) + (dt ? 4 * n_slots : 0);
     return MOE_OK;
 }
 
@@ -345,6 +363,7 @@ moe_status build_workspace(moe_pack *p)
         {(void **)&w.n_groups, 4}, {(void **)&w.ticket, 4}, {(void **)&w.err, 4}, {(void **)&w.bar, 8},
         {(void **)&w.h, slots * p->I * 4}, {(void **)&w.y, slots * p->H * 4},
         {(void **)&w.dgate, slots * 4}, {(void **)&w.n_dense_rows, 4},
+        {(void **)&w.xcnt, 16},
     };
     int64_t total = 0;
     for (auto &it : items) total += round_up(it.bytes, 256);
@@ -655,6 +674,31 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
         fa.cnt_out = w.cnt;
         fa.bar = w.bar;
         fa.err = w.err;
+        fa.xcnt = w.xcnt;
+        if (T == 1) {
+            if (pm->stream1 < 0) {
+                // probe with the pack's largest top-k: the layout only grows with k
+                FusedArgs probe = fa;
+                probe.k = p->max_top_k;
+                pm->stream1 = stream1_supported(probe, p->num_sms, 226 * 1024) ? 1 : 0;
+                pm->stream1_smem = pm->stream1 ? stream1_smem_bytes(probe, p->num_sms) : 0;
+            }
+            if (pm->stream1 && p->max_top_k <= kFusedMaxK) {
+                int pbase = -1;
+                if (pm->prof_on && (size_t)pm->prof_used + 2 <= pm->prof_ev.size()) {
+                    pbase = pm->prof_used;
+                    pm->prof_used += 2;
+                    pm->prof_fwd.push_back({pbase, 1});
+                    if (pm->prof_stamps && pm->prof_nstamp < pm->prof_stamp_cap)
+                        fa.stamps = pm->prof_stamps + kStampStride * (size_t)pm->prof_nstamp++;
+                }
+                prof_mark(pm, pbase, 0, s);
+                moe_status st = check_launch(launch_stream1(fa, p->num_sms, stream1_smem_bytes(fa, p->num_sms),
+                                                            pm->pdl && pbase < 0, s));
+                prof_mark(pm, pbase, 1, s);
+                return st;
+            }
+        }
         const int tt = T == 1 ? 1 : 8;
         const size_t limit = 220 * 1024;
         fa.rowsplit = fused_smem_bytes(fa, tt, 1) <= limit ? 1 : 0;
@@ -669,7 +713,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
                     pm->prof_used += 2;
                     pm->prof_fwd.push_back({pbase, 1});
                     if (pm->prof_stamps && pm->prof_nstamp < pm->prof_stamp_cap)
-                        fa.stamps = pm->prof_stamps + 16 * (size_t)pm->prof_nstamp++;
+                        fa.stamps = pm->prof_stamps + kStampStride * (size_t)pm->prof_nstamp++;
                 }
                 prof_mark(pm, pbase, 0, s);
                 moe_status st = check_launch(launch_fused(fa, tt, grid, smem, s));
@@ -814,8 +858,8 @@ moe_status moe_profile_begin(moe_pack *p, int max_forwards)
     p->prof_used = 0;
     p->prof_nstamp = 0;
     p->prof_stamp_cap = max_forwards;
-    if (cudaMalloc(&p->prof_stamps, sizeof(long long) * 16 * (size_t)max_forwards) != cudaSuccess ||
-        cudaMemset(p->prof_stamps, 0, sizeof(long long) * 16 * (size_t)max_forwards) != cudaSuccess) {
+    if (cudaMalloc(&p->prof_stamps, sizeof(long long) * kStampStride * (size_t)max_forwards) != cudaSuccess ||
+        cudaMemset(p->prof_stamps, 0, sizeof(long long) * kStampStride * (size_t)max_forwards) != cudaSuccess) {
         cudaGetLastError();
         p->prof_stamps = nullptr;
         p->prof_stamp_cap = 0;
@@ -846,19 +890,36 @@ moe_status moe_profile_end(moe_pack *p, double *ms, int *n_forwards)
     if (p->prof_stamps && p->prof_nstamp > 0 && st == MOE_OK) {
         // fused-kernel phases (CTA 0's clock): stage, router, barrier, plan,
         // gate/up, barrier, down, barrier, combine/tail
-        std::vector<long long> h((size_t)16 * p->prof_nstamp);
+        std::vector<long long> h((size_t)kStampStride * p->prof_nstamp);
         int khz = 0;
         cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, p->device);
         if (khz > 0 && cudaMemcpy(h.data(), p->prof_stamps, h.size() * sizeof(long long), cudaMemcpyDeviceToHost) ==
                            cudaSuccess) {
             for (int f = 0; f < p->prof_nstamp; ++f) {
-                const long long *c = h.data() + 16 * (size_t)f;
+                const long long *c = h.data() + kStampStride * (size_t)f;
                 auto span = [&](int a, int b) { return (c[a] && c[b] && c[b] > c[a]) ? (double)(c[b] - c[a]) : 0.0; };
                 double ph[PROF_PHASES];
                 for (int i = 0; i < 7; ++i) ph[i] = span(i, i + 1);
                 ph[7] = span(7, 8);
                 ph[8] = c[8] ? span(8, 9) : span(7, 9);
                 for (int i = 0; i < PROF_PHASES; ++i) acc[PROF_STAGES + i] += ph[i] / khz;  // cycles / kHz = ms
+                // grid-wide events (global timer, ns): first and last CTA of each,
+                // relative to the first CTA's start; the first start is stored as
+                // 2^62 - t so that one atomic maximum serves both
+                // CTA 0 sub-steps of the streaming kernel (clock64 at [24..31]), from its start
+                for (int i = 0; i < PROF_SUB; ++i)
+                    if (c[24 + i] > c[0] && c[0])
+                        acc[PROF_STAGES + PROF_PHASES + PROF_GRID + i] += (double)(c[24 + i] - c[0]) / khz;
+                if (c[11] > 0) {
+                    const long long t0 = (1ll << 62) - c[10];
+                    double *gx = acc + PROF_STAGES + PROF_PHASES;
+                    gx[0] += (c[11] - t0) * 1e-6;
+                    for (int ev = 1; ev < 5; ++ev) {
+                        if (c[11 + 2 * ev] <= 0) continue;
+                        gx[2 * ev - 1] += ((1ll << 62) - c[10 + 2 * ev] - t0) * 1e-6;
+                        gx[2 * ev] += (c[11 + 2 * ev] - t0) * 1e-6;
+                    }
+                }
             }
         }
     }

@@ -34,6 +34,12 @@ struct DevProj {
     int64_t qs_stride = 0, sc_stride = 0, qh_stride = 0;  // bytes per expert
     int qs_row = 0, sc_row = 0, qh_row = 0;               // bytes per row (sc_row: not NVFP4)
     int ksteps = 0;                                       // NVFP4: 64-wide K steps per row
+    // scales row by row (2 bytes per 32 weights, 4 for Q5_1): the sc plane
+    // itself, except for NVFP4, which keeps a second, row-major copy of its
+    // E4M3 scales for the streaming decode kernel's bulk row copies
+    const uint8_t *sr = nullptr;
+    int64_t sr_stride = 0;
+    int sr_row = 0;
 };
 
 // Byte offset of E4M3 scale q (0..3) of row r in 64-wide K step s, in the
@@ -64,6 +70,9 @@ struct Workspace {
     float *h = nullptr;          // [slots x I]
     float *y = nullptr;          // [slots x H]
     int max_groups = 0;
+    // single-token streaming kernel: {finished-CTA ticket, logits arrivals, h
+    // arrivals}; all zero between launches (the last CTA to finish resets them)
+    unsigned *xcnt = nullptr;
 };
 
 struct RouteArgs {
@@ -153,7 +162,9 @@ struct FusedArgs {
     unsigned *bar;      // {arrive count, generation}
     int32_t *err;
     int rowsplit;       // down + combine by output rows in one phase
-    long long *stamps;  // optional: clock64 of CTA 0 at each phase boundary
+    long long *stamps;  // optional: [0..9] clock64 of CTA 0 at each phase boundary; [10..19]
+                        // streaming kernel: per grid event {2^62 - first, last} global timer
+    unsigned *xcnt;     // streaming kernel's hand-over counters (see Workspace)
 };
 
 // tensor-core prefill
@@ -196,6 +207,14 @@ bool prefill_q8_supported(int H, int I, int E, int k);
 cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s);
 cudaError_t prefill_route(const void *x_bf16, const uint16_t *wr, int T, int H, int E, int k, float *logits,
                           int32_t *idx, float *gate, int32_t *cnt, int32_t *err, cudaStream_t s);
+
+// Single-token streaming decode (stream_decode.cu): same arguments as the
+// fused kernel; every weight byte a CTA needs is requested by bulk copies into
+// shared memory as soon as it is known.
+size_t stream1_smem_bytes(const FusedArgs &a, int grid);
+bool stream1_supported(const FusedArgs &a, int grid, size_t smem_limit);
+cudaError_t stream1_set_attributes();
+cudaError_t launch_stream1(const FusedArgs &a, int grid, size_t smem, int pdl, cudaStream_t s);
 
 size_t fused_smem_bytes(const FusedArgs &a, int tt, int rowsplit);
 cudaError_t fused_set_attributes();

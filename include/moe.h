@@ -224,11 +224,15 @@ moe_status moe_read_routing(const moe_pack *pack, int n_tokens, int top_k, int32
  * records an event before each of its kernels and after the last one
  * (captured as event-record nodes when the stream is capturing).
  * moe_profile_end synchronises the device, adds the elapsed times per kernel
- * over all recorded forwards into ms[15] (host memory): [0..5] route+plan,
+ * over all recorded forwards into ms[32] (host memory): [0..5] route+plan,
  * gate/up, down, combine of the grouped path, the fused decode kernel, the
  * whole tensor-core prefill sequence; [6..14] the fused kernel's phases as seen
  * by its first CTA (token staging, router, barrier, plan, gate/up, barrier,
- * down, barrier, combine), from its SM clock at the device's nominal rate.  It
+ * down, barrier, combine), from its SM clock at the device's nominal rate;
+ * [15..23] single-token streaming kernel only, from the global timer, relative
+ * to the first CTA's start: last CTA start, first and last CTA to publish its
+ * router rows, to issue its routed copies, to finish gate/up, to end;
+ * [24..31] its first CTA's time at eight internal points (kernel-specific).  It
  * stores the
  * forward count in *n_forwards, and frees the events.  Forwards beyond
  * max_forwards are not recorded. */

@@ -60,6 +60,25 @@ def test_every_format_on_both_projections(fmt):
     _check(li, synth.tokens(wl, li.router), wl.top_k)
 
 
+@pytest.mark.parametrize("fmt_gu,fmt_dn", [(synth.FMT_Q8_0, synth.FMT_Q8_0), (synth.FMT_Q5_1, synth.FMT_Q5_1),
+                                           (synth.FMT_IQ4_NL, synth.FMT_IQ4_NL), (synth.FMT_NVFP4, synth.FMT_NVFP4),
+                                           (synth.FMT_NVFP4, synth.FMT_Q5_1)])
+def test_single_token_streaming_kernel_every_format(fmt_gu, fmt_dn):
+    """One token with whole-row bulk copies (hidden and inter multiples of 256):
+    fewer experts than SMs, so many CTAs own no router row and a few pairs."""
+    wl = synth.Workload("s1", 1024, 32, 256, 4, True, fmt_gu, fmt_dn, synth.DT_BF16, 1, seed=20 + fmt_gu)
+    li = synth.layer_inputs(wl)
+    for step in range(2):
+        _check(li, synth.tokens(wl, li.router, 0, step), wl.top_k)
+
+
+def test_single_token_streaming_kernel_sixteen_experts_no_shared():
+    wl = synth.Workload("s1k16", 512, 64, 256, 16, False, synth.FMT_IQ4_NL, synth.FMT_Q8_0, synth.DT_F32, 1,
+                        seed=31)
+    li = synth.layer_inputs(wl)
+    _check(li, synth.tokens(wl, li.router), 16)
+
+
 def test_ragged_shapes_and_k_equals_E():
     # hidden 96 (3 units per row), inter 64, top_k = E, shared expert, 3 tokens
     wl = synth.Workload("ragged", 96, 5, 64, 5, True, synth.FMT_IQ4_NL, synth.FMT_Q5_1, synth.DT_F32, 3,
