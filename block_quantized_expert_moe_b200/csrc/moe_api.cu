@@ -50,6 +50,8 @@ struct moe_pack {
     int stream1 = -1;             // single-token streaming kernel usable (-1: not yet checked)
     size_t stream1_smem = 0;
     int pdl = 1;                  // launch it as a programmatic dependent of the previous kernel
+    int sgm = -1;                 // streamed grouped matvecs usable (-1: not yet checked)
+    SgmProj sg_gu{}, sg_dn{};
     bool has_prefill = false;     // tensor-core prefill workspace present
     PrefillWorkspace pws;
 };
@@ -141,6 +143,7 @@ moe_status init_device(int dev)
     if (matvec_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (fused_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (stream1_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
+    if (sgm_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_nvfp4_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_q8_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
@@ -650,7 +653,19 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
         prof_mark(pm, pbase, 1, s);
         return st;
     }
-    if (path == MOE_PATH_DECODE && T <= kFusedMaxT && k <= kFusedMaxK) {
+    // two or more tokens: the streamed grouped matvecs (rows per lane, TMA-fed),
+    // when the planes' rows fit their tile loads
+    if (pm->sgm < 0) {
+        const int slots = p->E + (p->has_shared ? 1 : 0);
+        pm->sgm = (w.max_groups <= sgm_max_groups() && p->I % 16 == 0 && p->H % 32 == 0 &&
+                   sgm_prepare(p->gu, slots, true, &pm->sg_gu) && sgm_prepare(p->dn, slots, false, &pm->sg_dn) &&
+                   sgm_stages(pm->sg_gu, p->H) >= 2 && sgm_stages(pm->sg_dn, p->I) >= 2)
+                      ? 1
+                      : 0;
+    }
+    // one token: the single-token kernels; 2..8 tokens: the fused kernel unless
+    // the streamed grouped matvecs apply
+    if (path == MOE_PATH_DECODE && T <= kFusedMaxT && k <= kFusedMaxK && (T == 1 || pm->sgm != 1)) {
         FusedArgs fa{};
         fa.x = x;
         fa.x_dtype = x_dtype;
@@ -765,6 +780,16 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     if (st != MOE_OK) return st;
     prof_mark(pm, pbase, 1, s);
 
+    if (path == MOE_PATH_DECODE && T >= 2 && tt == 8 && pm->sgm == 1) {
+        st = check_launch(launch_sgm(pm->sg_gu, p->gu, w.groups, w.n_groups, w.perm_tok, x, x_dtype, w.h, p->I,
+                                     p->I, true, p->ct_gu, w.err, p->num_sms, s));
+        if (st != MOE_OK) return st;
+        prof_mark(pm, pbase, 2, s);
+        st = check_launch(launch_sgm(pm->sg_dn, p->dn, w.groups, w.n_groups, w.perm_tok, w.h, MOE_DT_F32, w.y,
+                                     p->H, p->H, false, p->ct_dn, w.err, p->num_sms, s));
+        if (st != MOE_OK) return st;
+        prof_mark(pm, pbase, 3, s);
+    } else {
     MatvecArgs gu{};
     gu.w = p->gu;
     gu.groups = w.groups;
@@ -798,6 +823,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     st = check_launch(launch_matvec(dn, false, tt, gdn, s));
     if (st != MOE_OK) return st;
     prof_mark(pm, pbase, 3, s);
+    }
 
     if (path == MOE_PATH_DENSE) {
         st = check_launch(launch_combine_dense(w.y, w.dgate, w.n_dense_rows, T, p->H, out, s));

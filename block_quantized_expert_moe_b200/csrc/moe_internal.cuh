@@ -3,6 +3,7 @@
 // blocks.  Nothing here is part of the public C ABI (include/moe.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -207,6 +208,22 @@ bool prefill_q8_supported(int H, int I, int E, int k);
 cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s);
 cudaError_t prefill_route(const void *x_bf16, const uint16_t *wr, int T, int H, int E, int k, float *logits,
                           int32_t *idx, float *gate, int32_t *cnt, int32_t *err, cudaStream_t s);
+
+// Streamed grouped matvec (stream_group.cu): per projection, TMA maps of the
+// code / scale / fifth-bit planes (3-D: row bytes x rows x expert slots) and
+// the stage layout of a 32-row block.
+struct SgmProj {
+    CUtensorMap map[3];
+    int row_bytes[3], w[3], off[3];
+    int stage_bytes, tx_bytes, fmt, ok;
+};
+bool sgm_prepare(const DevProj &w, int n_slots, bool gateup, SgmProj *out);
+int sgm_max_groups();
+int sgm_stages(const SgmProj &p, int K);
+cudaError_t sgm_set_attributes();
+cudaError_t launch_sgm(const SgmProj &p, const DevProj &w, const int4 *groups, const int32_t *n_groups,
+                       const int32_t *perm_tok, const void *x, int x_dtype, float *out, int out_stride, int rows_out,
+                       bool gateup, const CodeTable &tab, int32_t *err, int grid, cudaStream_t s);
 
 // Single-token streaming decode (stream_decode.cu): same arguments as the
 // fused kernel; every weight byte a CTA needs is requested by bulk copies into

@@ -22,6 +22,7 @@
 // ever waits on another.
 #include <climits>
 
+#include "decode_common.cuh"
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -89,6 +90,26 @@ __device__ void topk_phase(const RouteArgs &a, unsigned char *smem)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nw = kThreads / 32;
     const int E = a.E, k = a.k;
+    if (k <= 32 && E <= 1024) {
+        // one warp per token: the row into shared memory, then the threshold
+        // selection (candidates at or above the k-th largest lane maximum)
+        float *row = reinterpret_cast<float *>(smem) + (size_t)warp * (E + 128);
+        unsigned *cand = reinterpret_cast<unsigned *>(row + E);
+        for (int t = warp; t < a.T; t += nw) {
+            for (int e = lane; e < E; e += 32) row[e] = __ldcg(a.logits + (size_t)t * E + e);
+            __syncwarp();
+            int me;
+            float mg;
+            if (E <= 512) topk_threshold<16>(row, E, k, me, mg, cand);
+            else topk_threshold<32>(row, E, k, me, mg, cand);
+            if (lane < k) {
+                a.idx[(size_t)t * k + lane] = me;
+                a.gate[(size_t)t * k + lane] = mg;
+            }
+            __syncwarp();
+        }
+        return;
+    }
     float *row = reinterpret_cast<float *>(smem) + warp * E;
     float *selv = reinterpret_cast<float *>(smem) + nw * E + warp * E;
     uint32_t *taken = reinterpret_cast<uint32_t *>(smem + (size_t)2 * nw * E * sizeof(float)) + warp * 32;
@@ -261,22 +282,33 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const RouteArgs a)
     for (int t0 = 0; t0 < a.T; t0 += a.rt) {
         const int nt = min(a.rt, a.T - t0);
         __syncthreads();
-        for (int i = threadIdx.x; i < nt * nch; i += kThreads) {
-            int t = i / nch, c = i - t * nch;
-            float4 lo, hi;
-            if (a.x_dtype == MOE_DT_BF16) {
-                uint4 v = ldg_nc16(reinterpret_cast<const uint16_t *>(a.x) + (size_t)(t0 + t) * H + c * 8);
-                lo = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
-                hi = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
-            } else {
-                const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(a.x) +
-                                                                   (size_t)(t0 + t) * H + c * 8);
-                lo = __ldg(p);
-                hi = __ldg(p + 1);
+        for (int i0 = threadIdx.x; i0 < nt * nch; i0 += 4 * kThreads) {
+            float4 lo[4], hi[4];  // four chunks' loads in flight before any store
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int i = i0 + q * kThreads;
+                if (i >= nt * nch) break;
+                const int t = i / nch, c = i - t * nch;
+                if (a.x_dtype == MOE_DT_BF16) {
+                    uint4 v = ldg_nc16(reinterpret_cast<const uint16_t *>(a.x) + (size_t)(t0 + t) * H + c * 8);
+                    lo[q] = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
+                    hi[q] = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
+                } else {
+                    const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(a.x) +
+                                                                       (size_t)(t0 + t) * H + c * 8);
+                    lo[q] = __ldg(p);
+                    hi[q] = __ldg(p + 1);
+                }
             }
-            float4 *d = reinterpret_cast<float4 *>(xs + (size_t)t * H + c * 8);
-            d[0] = lo;
-            d[1] = hi;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int i = i0 + q * kThreads;
+                if (i >= nt * nch) break;
+                const int t = i / nch, c = i - t * nch;
+                float4 *d = reinterpret_cast<float4 *>(xs + (size_t)t * H + c * 8);
+                d[0] = lo[q];
+                d[1] = hi[q];
+            }
         }
         __syncthreads();
         for (int e = e0 + warp; e < e1; e += nw) {
@@ -352,6 +384,8 @@ size_t route_smem_bytes(int H, int rt, int E)
 {
     size_t stage = (size_t)rt * H * sizeof(float);
     size_t topk = (size_t)2 * (kThreads / 32) * E * sizeof(float) + (kThreads / 32) * 32 * sizeof(uint32_t);
+    const size_t topk_thr = (size_t)(kThreads / 32) * (E + 128) * sizeof(float);  // row + candidates per warp
+    if (topk_thr > topk) topk = topk_thr;
     size_t plan = (size_t)E * 8 + (size_t)4 * (E + 1) * sizeof(int) + 64 * sizeof(int);
     size_t m = stage > topk ? stage : topk;
     return m > plan ? m : plan;
