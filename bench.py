@@ -385,6 +385,8 @@ def ours_arm(a, wl):
     dom = max(stage_us, key=lambda s: stage_us[s])
     # one token: the streaming kernel (whole-row bulk copies) runs in place of the fused one
     kname = "stream1_kernel" if dom == "fused" and T == 1 else KERNEL_NAMES[dom]
+    if a.path == "auto" and T >= 2 and dom in ("gate_up", "down"):
+        kname = f"sgm_kernel<{dom.replace('_', '/')}>"  # streamed grouped matvec (row per lane)
     hbm, peak_src = peaks()
     traffic = kernel_traffic(dom, wl.name)
     if dom == "prefill":
