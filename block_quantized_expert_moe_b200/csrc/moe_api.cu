@@ -363,7 +363,7 @@ moe_status build_workspace(moe_pack *p)
         {(void **)&w.logits, T * E * 4}, {(void **)&w.idx, T * k * 4}, {(void **)&w.gate, T * k * 4},
         {(void **)&w.cnt, (E + 1) * 4}, {(void **)&w.off, (E + 1) * 4}, {(void **)&w.perm_tok, slots * 4},
         {(void **)&w.slot_pos, T * k * 4}, {(void **)&w.groups, (int64_t)w.max_groups * 16},
-        {(void **)&w.n_groups, 4}, {(void **)&w.ticket, 4}, {(void **)&w.err, 4}, {(void **)&w.bar, 8},
+        {(void **)&w.n_groups, 4}, {(void **)&w.ticket, 64}, {(void **)&w.err, 4}, {(void **)&w.bar, 8},
         {(void **)&w.h, slots * p->I * 4}, {(void **)&w.y, slots * p->H * 4},
         {(void **)&w.dgate, slots * 4}, {(void **)&w.n_dense_rows, 4},
         {(void **)&w.xcnt, 16},
@@ -598,8 +598,9 @@ moe_status moe_route_topk(const void *x, moe_dtype x_dtype, const uint16_t *rout
         return check_launch(prefill_route(x, router_w, n_tokens, hidden, n_experts, top_k, a.logits, idx_out,
                                           gate_out, nullptr, werr, s));
     }
-    if (cudaMemsetAsync(a.ticket, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-    return check_launch(launch_route(a, route_grid(n_experts, sms), s));
+    // tickets: word 0 and words 2.. (one per 8-token block); the kernel leaves them zero
+    if (cudaMemsetAsync(a.ticket, 0, 64, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return check_launch(launch_route(a, route_grid(n_experts, n_tokens, a.rt, sms), s));
 }
 
 moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
@@ -776,7 +777,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     ra.dense = path == MOE_PATH_DENSE;
     ra.dgate = w.dgate;
     ra.n_dense_rows = w.n_dense_rows;
-    moe_status st = check_launch(launch_route(ra, route_grid(p->E, p->num_sms), s));
+    moe_status st = check_launch(launch_route(ra, route_grid(p->E, T, ra.rt, p->num_sms), s));
     if (st != MOE_OK) return st;
     prof_mark(pm, pbase, 1, s);
 

@@ -63,7 +63,7 @@ struct Workspace {
     int32_t *slot_pos = nullptr; // [T x k]   (t, j) -> slot
     int4 *groups = nullptr;      // {expert, first slot, tokens, 0}
     int32_t *n_groups = nullptr;
-    int32_t *ticket = nullptr;   // last-CTA counter of the route kernel
+    int32_t *ticket = nullptr;   // route kernel tickets: [0] token blocks done, [2 + b] CTAs of block b
     unsigned *bar = nullptr;     // grid barrier of the fused decode kernel {count, gen}
     int32_t *err = nullptr;      // sticky device error (moe_status)
     float *dgate = nullptr;      // dense-batched plan: per slot gate (0 when not routed)
@@ -132,7 +132,7 @@ size_t route_smem_bytes(int H, int rt, int E);
 void init_device_attributes();  // once per device, with that device current
 int route_tokens_per_pass(int H);
 cudaError_t launch_route(const RouteArgs &a, int grid, cudaStream_t s);
-int route_grid(int E, int num_sms);
+int route_grid(int E, int T, int rt, int num_sms);
 
 cudaError_t launch_matvec(const MatvecArgs &a, bool gateup, int tt, int grid, cudaStream_t s);
 size_t matvec_smem_bytes(const MatvecArgs &a, bool gateup, int tt);

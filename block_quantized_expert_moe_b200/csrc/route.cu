@@ -3,14 +3,17 @@
 // The "Qwen3.8-Flash-Next UD-IQ2_XS (L4 fix) for Basalt" model card, section
 // "What was changed", calls its fast decode path a device-planned MoE tail:
 // the per-expert token lists are built on the GPU, with no host round trip.
-// Here the plan is built by the last CTA of the router launch:
+// Here the plan is built at the end of the router launch:
 //
 //   phase 1 (all CTAs)   logits[t][e] = sum_h Wr[e][h] x[t][h], fp32 accumulate;
-//                        CTA b owns experts [E*b/G, E*(b+1)/G), one warp per
-//                        expert row, x staged in shared memory as fp32
-//   phase 2 (last CTA)   per token: k rounds of warp arg-max (ties to the lower
-//                        expert index), then gates exp(l - lmax) / sum over S
-//   phase 3 (last CTA)   plan: per-expert counts by shared-memory atomics, an
+//                        CTA b takes token block b % ntb (8 tokens, staged in
+//                        shared memory as fp32 once) and a slice of the expert
+//                        rows, one warp per row
+//   phase 2 (last CTA of each token block)  one warp per token: the threshold
+//                        top-k (candidates at or above the k-th largest lane
+//                        maximum, ranked in one pass; ties to the lower expert
+//                        index), gates exp(l - lmax) / sum over the selected
+//   phase 3 (last block) plan: per-expert counts by shared-memory atomics, an
 //                        exclusive scan to slot offsets, and a stable slot
 //                        order (tokens ascending inside an expert) from 64-bit
 //                        token masks and popcounts, so the plan is identical
@@ -18,8 +21,8 @@
 //                        {expert, first slot, tokens <= tt} for the grouped
 //                        matvecs, the shared expert's groups last.
 //
-// The last CTA is found with a global ticket (atomicAdd after a fence); no CTA
-// ever waits on another.
+// "Last" is decided by global tickets (atomicAdd after a fence: one per token
+// block, one over blocks); no CTA ever waits on another.
 #include <climits>
 
 #include "decode_common.cuh"
@@ -28,6 +31,8 @@
 namespace moe {
 
 namespace {
+
+constexpr int kRouteMaxBlockGroups = 14;  // per-group tickets at words 2..15 of the ticket area
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
@@ -85,7 +90,7 @@ __device__ int block_exclusive_scan(int *v, int n, int *tmp)
     return total;
 }
 
-__device__ void topk_phase(const RouteArgs &a, unsigned char *smem)
+__device__ void topk_phase(const RouteArgs &a, unsigned char *smem, int t_begin, int t_end)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nw = kThreads / 32;
@@ -95,7 +100,7 @@ __device__ void topk_phase(const RouteArgs &a, unsigned char *smem)
         // selection (candidates at or above the k-th largest lane maximum)
         float *row = reinterpret_cast<float *>(smem) + (size_t)warp * (E + 128);
         unsigned *cand = reinterpret_cast<unsigned *>(row + E);
-        for (int t = warp; t < a.T; t += nw) {
+        for (int t = t_begin + warp; t < t_end; t += nw) {
             for (int e = lane; e < E; e += 32) row[e] = __ldcg(a.logits + (size_t)t * E + e);
             __syncwarp();
             int me;
@@ -113,7 +118,7 @@ __device__ void topk_phase(const RouteArgs &a, unsigned char *smem)
     float *row = reinterpret_cast<float *>(smem) + warp * E;
     float *selv = reinterpret_cast<float *>(smem) + nw * E + warp * E;
     uint32_t *taken = reinterpret_cast<uint32_t *>(smem + (size_t)2 * nw * E * sizeof(float)) + warp * 32;
-    for (int t = warp; t < a.T; t += nw) {
+    for (int t = t_begin + warp; t < t_end; t += nw) {
         for (int e = lane; e < E; e += 32) row[e] = __ldcg(a.logits + (size_t)t * E + e);
         taken[lane] = 0u;
         __syncwarp();
@@ -276,10 +281,16 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const RouteArgs a)
     float *xs = reinterpret_cast<float *>(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = kThreads / 32;
     const int H = a.H, E = a.E;
-    const int e0 = (int)((long long)E * blockIdx.x / gridDim.x);
-    const int e1 = (int)((long long)E * (blockIdx.x + 1) / gridDim.x);
+    // CTA b takes token block b % ntb (rt tokens) and a slice of the expert rows,
+    // so every CTA stages its tokens once and the grid covers all SMs
+    // token blocks of rt tokens, dealt to NB block groups (more blocks than
+    // groups: a CTA handles blocks j, j + NB, ...)
+    const int ntb = (a.T + a.rt - 1) / a.rt, NB = min(ntb, kRouteMaxBlockGroups), per = gridDim.x / NB;
+    const int tb = blockIdx.x % NB, slice = blockIdx.x / NB;
+    const int e0 = slice < per ? (int)((long long)E * slice / per) : E;
+    const int e1 = slice < per ? (int)((long long)E * (slice + 1) / per) : E;
     const int nch = H >> 3;  // 16-byte chunks of 8 bf16 in a router row
-    for (int t0 = 0; t0 < a.T; t0 += a.rt) {
+    for (int t0 = tb * a.rt; t0 < a.T && e1 > e0; t0 += NB * a.rt) {
         const int nt = min(a.rt, a.T - t0);
         __syncthreads();
         for (int i0 = threadIdx.x; i0 < nt * nch; i0 += 4 * kThreads) {
@@ -353,16 +364,28 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const RouteArgs a)
             }
         }
     }
+    // the last CTA of this token block selects its tokens' experts; the last
+    // token block to finish builds the plan (tickets: [0] blocks, [2 + tb] CTAs)
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        int ticket = atomicAdd(a.ticket, 1);
-        s_last = ticket == (int)gridDim.x - 1;
+        const int ticket = atomicAdd(a.ticket + 2 + tb, 1);
+        s_last = ticket == per - 1;
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    topk_phase(a, smem);
+    for (int t0 = tb * a.rt; t0 < a.T; t0 += NB * a.rt) topk_phase(a, smem, t0, min(a.T, t0 + a.rt));
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        a.ticket[2 + tb] = 0;
+        __threadfence();
+        const int ticket = atomicAdd(a.ticket, 1);
+        s_last = ticket == NB - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
     if (a.do_plan) {
         __syncthreads();
         if (a.dense) plan_dense(a, smem);
@@ -391,10 +414,12 @@ size_t route_smem_bytes(int H, int rt, int E)
     return m > plan ? m : plan;
 }
 
-int route_grid(int E, int num_sms)
+int route_grid(int E, int T, int rt, int num_sms)
 {
-    int g = (E + (kThreads / 32) - 1) / (kThreads / 32);
-    return g < num_sms ? g : num_sms;
+    const int ntb = min((T + rt - 1) / rt, kRouteMaxBlockGroups);  // block groups
+    int per = (E + (kThreads / 32) - 1) / (kThreads / 32);  // row slices: >= one warp's row each
+    if (per * ntb > num_sms) per = num_sms / ntb > 0 ? num_sms / ntb : 1;
+    return per * ntb;
 }
 
 cudaError_t route_set_attributes()

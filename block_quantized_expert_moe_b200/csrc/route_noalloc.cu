@@ -101,6 +101,6 @@ extern "C" moe_status moe_route_topk_noalloc(const void *x, moe_dtype x_dtype, c
     a.idx = idx_out;
     a.gate = gate_out;
     a.do_plan = 0;
-    if (cudaMemsetAsync(a.ticket, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-    return launch_route(a, route_grid(n_experts, sms), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (cudaMemsetAsync(a.ticket, 0, 64, s) != cudaSuccess) return MOE_ERR_CUDA;  // the tickets (words 0, 2..)
+    return launch_route(a, route_grid(n_experts, n_tokens, a.rt, sms), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

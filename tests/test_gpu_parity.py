@@ -94,7 +94,8 @@ def test_ragged_shapes_and_k_equals_E():
 
 def test_route_topk_bit_exact_sets_and_gates():
     import block_quantized_expert_moe_b200 as bq
-    for name, T in (("tiny_q8", 1), ("model_decode", 1), ("zipf_batch", 64), ("spec_verify", 8)):
+    # fp32 x with 200 tokens stays on the CUDA-core router: 25 token blocks over 14 block groups
+    for name, T in (("tiny_q8", 1), ("model_decode", 1), ("zipf_batch", 64), ("spec_verify", 8), ("tiny_q8", 200)):
         wl, li = _layer(name)
         x = synth.tokens(wl, li.router, 0, 0, T)
         xt, wr = to_device(x), router_to_device(li.router)
