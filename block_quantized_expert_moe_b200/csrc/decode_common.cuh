@@ -160,8 +160,8 @@ __device__ void topk_threshold(const float *lg, int E, int k, int &my_e, float &
 #pragma unroll
     for (int i = 0; i < NPL; ++i) lm = max(lm, key[i]);
     int lrank = 0;
-#pragma unroll 4
-    for (int l = 0; l < 32; ++l) {
+#pragma unroll
+    for (int l = 0; l < 32; ++l) {  // independent shuffles: fully unrolled
         const unsigned o = __shfl_sync(0xffffffffu, lm, l);
         lrank += (o > lm || (o == lm && l < lane)) ? 1 : 0;
     }
@@ -189,9 +189,11 @@ __device__ void topk_threshold(const float *lg, int E, int k, int &my_e, float &
             }
         __syncwarp();
         const unsigned ck = lane < total ? cand[lane] : 0u, ce = lane < total ? cand[32 + lane] : 0xffffffffu;
+        // lanes >= total hold key 0 / id ~0, which never outrank a candidate:
+        // a fixed 32-step, fully unrolled loop needs no bound
         int r = 0;
-#pragma unroll 1
-        for (int q = 0; q < total; ++q) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
             const unsigned qk = __shfl_sync(0xffffffffu, ck, q), qe = __shfl_sync(0xffffffffu, ce, q);
             r += (qk > ck || (qk == ck && qe < ce)) ? 1 : 0;
         }

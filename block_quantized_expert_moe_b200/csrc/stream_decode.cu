@@ -73,7 +73,7 @@ constexpr int kS1NumBars = kS1BarH + 1;  // 32: one bit each in the armed mask
 constexpr long long kS1PollLimit = 1ll << 31;     // clocks
 
 __host__ __device__ inline size_t s1_al16(size_t v) { return (v + 15) & ~(size_t)15; }
-__host__ __device__ inline int s1_cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+__host__ __device__ inline int s1_cdiv(int a, int b) { return (a + b - 1) / b; }  // 32-bit: shapes are small
 
 // Shared-memory layout; host and device compute it from the same arguments.
 struct S1Layout {
@@ -91,7 +91,7 @@ __host__ __device__ inline S1Layout s1_layout(const FusedArgs &a, int G)
     S1Layout L;
     L.ng = a.k + (a.has_shared ? 1 : 0);
     L.rr = s1_cdiv(a.E, G);
-    L.gp = s1_cdiv((long long)L.ng * a.I, G);
+    L.gp = s1_cdiv(L.ng * a.I, G);
     L.dr = s1_cdiv(a.H, G);
     L.gu_pair = 2 * (a.gu.qs_row + a.gu.sr_row + a.gu.qh_row);
     L.dn_row = a.dn.qs_row + a.dn.sr_row + a.dn.qh_row;
@@ -320,6 +320,23 @@ __device__ void s1_gateup(const FusedArgs &a, const S1Layout &L, uint8_t *smem, 
     const int LPR = lanes_per_row(NU), RPW = 32 / LPR;
     const int sub = lane / LPR, sl = lane - sub * LPR;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
+    // each lane owns at most two units of x (H <= 64 * lanes per row): keep them in registers
+    const bool xreg = NU <= 2 * LPR;
+    const int u = sl, u2 = sl + LPR;
+    const bool has1 = u < NU, has2 = u2 < NU;
+    float4 xr0[8], xr1[8];
+    float xs0 = 0.f, xs1 = 0.f;
+    if (xreg) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            xr0[j] = has1 ? xs4[u * 8 + (j ^ (u & 7))] : make_float4(0.f, 0.f, 0.f, 0.f);
+            xr1[j] = has2 ? xs4[u2 * 8 + (j ^ (u2 & 7))] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (FMT == MOE_FMT_Q5_1) {
+            xs0 = has1 ? xsum[u] : 0.f;
+            xs1 = has2 ? xsum[u2] : 0.f;
+        }
+    }
 #pragma unroll 1
     for (int base = warp * RPW; base < npairs; base += kS1Warps * RPW) {
         const int q = base + sub;
@@ -338,15 +355,31 @@ __device__ void s1_gateup(const FusedArgs &a, const S1Layout &L, uint8_t *smem, 
                       *uh = gh + (size_t)n * w.qh_row;
         const float half_ts = FMT == MOE_FMT_NVFP4 ? 0.5f * __ldg(w.ts + grp_e[sg.g]) : 0.5f;
         float s0 = 0.f, s1 = 0.f;
-        if (ok) {
+        if (ok && xreg) {
+            // all four unit loads of the pair first, then four independent dot products
+            const Raw g0 = lds_unit<FMT>(gq, gs, gh, u), u0r = lds_unit<FMT>(uq, us, uh, u);
+            Raw g1 = g0, u1r = u0r;
+            if (has2) {
+                g1 = lds_unit<FMT>(gq, gs, gh, u2);
+                u1r = lds_unit<FMT>(uq, us, uh, u2);
+            }
+            if (has1) {
+                s0 = unit_dot_reg<FMT>(g0, xr0, xs0, a.tab_gu, half_ts, s0);
+                s1 = unit_dot_reg<FMT>(u0r, xr0, xs0, a.tab_gu, half_ts, s1);
+            }
+            if (has2) {
+                s0 = unit_dot_reg<FMT>(g1, xr1, xs1, a.tab_gu, half_ts, s0);
+                s1 = unit_dot_reg<FMT>(u1r, xr1, xs1, a.tab_gu, half_ts, s1);
+            }
+        } else if (ok) {
 #pragma unroll 1
-            for (int u = sl; u < NU; u += LPR) {
+            for (int v = sl; v < NU; v += LPR) {
                 float4 xr[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) xr[j] = xs4[u * 8 + (j ^ (u & 7))];
-                const float xs = FMT == MOE_FMT_Q5_1 ? xsum[u] : 0.f;
-                s0 = unit_dot_reg<FMT>(lds_unit<FMT>(gq, gs, gh, u), xr, xs, a.tab_gu, half_ts, s0);
-                s1 = unit_dot_reg<FMT>(lds_unit<FMT>(uq, us, uh, u), xr, xs, a.tab_gu, half_ts, s1);
+                for (int j = 0; j < 8; ++j) xr[j] = xs4[v * 8 + (j ^ (v & 7))];
+                const float xs = FMT == MOE_FMT_Q5_1 ? xsum[v] : 0.f;
+                s0 = unit_dot_reg<FMT>(lds_unit<FMT>(gq, gs, gh, v), xr, xs, a.tab_gu, half_ts, s0);
+                s1 = unit_dot_reg<FMT>(lds_unit<FMT>(uq, us, uh, v), xr, xs, a.tab_gu, half_ts, s1);
             }
         }
         for (int o = LPR >> 1; o >= 1; o >>= 1) {
@@ -388,62 +421,79 @@ __device__ void s1_h_sums(const S1Layout &L, uint8_t *smem, int I)
 }
 
 // ---- down + combine over this CTA's output rows -----------------------------------
-// Task = (group g, block of rows): the warp keeps its lanes' 32-weight units of
-// h_g in registers for every row of the block (LPR lanes per row, RPW rows at
-// a time); gate_g * (D_g h_g)[r] goes to part[g][r], summed over g in order.
+// Row-dots (group g, output row i) are dealt round-robin: step s of the CTA is
+// row-dots s*RPW .. s*RPW + RPW - 1 (LPR lanes each), warp w takes steps w,
+// w + W, ... two at a time so two independent decode chains are in flight; each
+// step reads its group's h unit (one per lane) and writes gate_g * (D_g h_g)[i]
+// to part[g][i], summed over g in the layer's order at the end.
+template <int FMT>
+__device__ __forceinline__ float s1_row_dot(const FusedArgs &a, const S1Layout &L, const uint8_t *smem, int nd,
+                                            int rd, int sl, int LPR, int NU, float half_ts_base, const int *grp_e,
+                                            const uint64_t *bars, int *fail, bool &ok)
+{
+    const DevProj &w = a.dn;
+    const int nc = a.I >> 2;
+    const int g = rd / nd, i = rd - g * nd;
+    ok = s1_wait(const_cast<uint64_t *>(bars) + kS1BarDown + g, a.err, fail);
+    const float4 *hs4 = reinterpret_cast<const float4 *>(smem + L.h);
+    const float *hsum = reinterpret_cast<const float *>(smem + L.hsum);
+    const uint8_t *b = smem + L.dn + (size_t)g * L.dr * L.dn_row;
+    const uint8_t *q = b + (size_t)i * w.qs_row, *sc = b + (size_t)nd * w.qs_row + (size_t)i * w.sr_row,
+                  *qh = b + (size_t)nd * (w.qs_row + w.sr_row) + (size_t)i * w.qh_row;
+    const float half_ts = FMT == MOE_FMT_NVFP4 ? half_ts_base * __ldg(w.ts + grp_e[g]) : 0.5f;
+    float v = 0.f;
+    if (!ok) return v;
+    if (NU <= LPR) {  // one unit per lane
+        float4 hr[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hr[j] = hs4[g * nc + sl * 8 + (j ^ (sl & 7))];
+        const float hsr = FMT == MOE_FMT_Q5_1 ? hsum[g * NU + sl] : 0.f;
+        v = unit_dot_reg<FMT>(lds_unit<FMT>(q, sc, qh, sl), hr, hsr, a.tab_dn, half_ts, 0.f);
+    } else {
+        const int xoff[1] = {g * nc}, xsoff[1] = {g * NU};
+        float acc[1] = {0.f};
+        for (int u = sl; u < NU; u += LPR)
+            unit_dot<FMT, 1>(lds_unit<FMT>(q, sc, qh, u), u, hs4, hsum, xoff, xsoff, 1, a.tab_dn, half_ts, acc);
+        v = acc[0];
+    }
+    return v;
+}
+
 template <int FMT>
 __device__ void s1_down(const FusedArgs &a, const S1Layout &L, uint8_t *smem, int r0, int nd, const int *grp_e,
                         const float *grp_gate, int *fail)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const DevProj &w = a.dn;
-    const int K = a.I, nc = K >> 2, NU = K >> 5;
+    const int NU = a.I >> 5;
     const int ng = L.ng;
-    const float4 *hs4 = reinterpret_cast<const float4 *>(smem + L.h);
-    const float *hsum = reinterpret_cast<const float *>(smem + L.hsum);
     float *part = reinterpret_cast<float *>(smem + L.part);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
+    const uint64_t *bars = reinterpret_cast<const uint64_t *>(smem + L.bars);
     const int LPR = lanes_per_row(NU), RPW = 32 / LPR;
     const int sub = lane / LPR, sl = lane - sub * LPR;
-    const bool hreg = NU <= LPR;  // one unit per lane
-    // row blocks per group: enough tasks for every warp
-    const int nb = min(nd, (kS1Warps + ng - 1) / ng);
-    const int rb = (nd + nb - 1) / nb;
-    for (int task = warp; task < ng * nb; task += kS1Warps) {
-        const int g = task / nb, blk = task - g * nb;
-        const int i0 = blk * rb, i1 = min(nd, i0 + rb);
-        const bool ok = s1_wait(bars + kS1BarDown + g, a.err, fail);
-        const float half_ts = FMT == MOE_FMT_NVFP4 ? 0.5f * __ldg(w.ts + grp_e[g]) : 0.5f;
-        const float gg = grp_gate[g];
-        const uint8_t *b = smem + L.dn + (size_t)g * L.dr * L.dn_row;
-        const uint8_t *qb = b, *sb = b + (size_t)nd * w.qs_row, *hb = b + (size_t)nd * (w.qs_row + w.sr_row);
-        float4 hr[8];
-        float hsr = 0.f;
-        if (hreg) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) hr[j] = hs4[g * nc + sl * 8 + (j ^ (sl & 7))];
-            if (FMT == MOE_FMT_Q5_1) hsr = hsum[g * NU + sl];
+    const int nrd = ng * nd, nsteps = (nrd + RPW - 1) / RPW;
+#pragma unroll 1
+    for (int s0 = warp; s0 < nsteps; s0 += 2 * kS1Warps) {
+        const int s1 = s0 + kS1Warps;
+        const int rd0 = s0 * RPW + sub, rd1 = s1 * RPW + sub;
+        const bool v0ok = rd0 < nrd, v1ok = s1 < nsteps && rd1 < nrd;
+        bool ok0 = false, ok1 = false;
+        float v0 = s1_row_dot<FMT>(a, L, smem, nd, v0ok ? rd0 : nrd - 1, sl, LPR, NU, 0.5f, grp_e, bars, fail, ok0);
+        float v1 = 0.f;
+        if (s1 < nsteps)  // warp-uniform
+            v1 = s1_row_dot<FMT>(a, L, smem, nd, v1ok ? rd1 : nrd - 1, sl, LPR, NU, 0.5f, grp_e, bars, fail, ok1);
+        for (int o = LPR >> 1; o >= 1; o >>= 1) {
+            v0 += __shfl_xor_sync(0xffffffffu, v0, o);
+            v1 += __shfl_xor_sync(0xffffffffu, v1, o);
         }
-        const int xoff[1] = {g * nc}, xsoff[1] = {g * NU};
-        for (int i = i0 + sub; i - sub < i1; i += RPW) {
-            const bool valid = i < i1;
-            const int ii = valid ? i : i1 - 1;
-            const uint8_t *q = qb + (size_t)ii * w.qs_row, *sc = sb + (size_t)ii * w.sr_row,
-                          *qh = hb + (size_t)ii * w.qh_row;
-            float v = 0.f;
-            if (ok) {
-                if (hreg) {
-                    v = unit_dot_reg<FMT>(lds_unit<FMT>(q, sc, qh, sl), hr, hsr, a.tab_dn, half_ts, 0.f);
-                } else {
-                    float acc[1] = {0.f};
-                    for (int u = sl; u < NU; u += LPR)
-                        unit_dot<FMT, 1>(lds_unit<FMT>(q, sc, qh, u), u, hs4, hsum, xoff, xsoff, 1, a.tab_dn, half_ts,
-                                         acc);
-                    v = acc[0];
-                }
+        if (sl == 0) {
+            if (v0ok) {
+                const int g = rd0 / nd;
+                part[g * L.dr + rd0 - g * nd] = grp_gate[g] * v0;
             }
-            for (int o = LPR >> 1; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (valid && sl == 0) part[g * L.dr + ii] = gg * v;
+            if (v1ok) {
+                const int g = rd1 / nd;
+                part[g * L.dr + rd1 - g * nd] = grp_gate[g] * v1;
+            }
         }
     }
     if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) a.stamps[30] = clock64();
@@ -472,10 +522,11 @@ __global__ void __launch_bounds__(kS1Threads, 1) stream1_kernel(const FusedArgs 
     if (stamp) a.stamps[0] = clock64();
 
     const int k = a.k, hs = a.has_shared ? 1 : 0;
-    const int e0 = (int)((long long)a.E * c / G), e1 = (int)((long long)a.E * (c + 1) / G);
-    const long long P = (long long)L.ng * a.I;
-    const int p0 = (int)(P * c / G), p1 = (int)(P * (c + 1) / G);
-    const int r0 = (int)((long long)a.H * c / G), r1 = (int)((long long)a.H * (c + 1) / G);
+    // 32-bit products: E, ng * I and H times the grid stay far below 2^31 for the shapes taken
+    const int e0 = a.E * c / G, e1 = a.E * (c + 1) / G;
+    const int P = L.ng * a.I;
+    const int p0 = P * c / G, p1 = P * (c + 1) / G;
+    const int r0 = a.H * c / G, r1 = a.H * (c + 1) / G;
     const int nd = r1 - r0;
     Seg *seg = reinterpret_cast<Seg *>(flags + 8 + 128);  // this CTA's gate/up chunks
     // copy sources and the layout, for the issuing code (256-byte slots after the chunks)
@@ -692,6 +743,8 @@ size_t stream1_smem_bytes(const FusedArgs &a, int grid) { return s1_layout(a, gr
 bool stream1_supported(const FusedArgs &a, int grid, size_t smem_limit)
 {
     if (a.T != 1 || grid < 1 || a.k > kFusedMaxK || a.E > 1024) return false;
+    // 32-bit work splits in the kernel: every product (size x grid) must fit
+    if ((long long)(kFusedMaxK + 1) * a.I * grid >= (1ll << 31) || (long long)a.H * grid >= (1ll << 31)) return false;
     if (!a.xcnt || !a.logits || !a.h) return false;
     // bulk copies move whole rows: every plane's row must be a multiple of 16 bytes
     const DevProj *ps[2] = {&a.gu, &a.dn};
