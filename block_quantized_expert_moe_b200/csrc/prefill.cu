@@ -20,6 +20,7 @@
 #include <climits>
 #include <mutex>
 
+#include "decode_common.cuh"
 #include "moe_internal.cuh"
 #include "tc_common.cuh"
 #include "tma_maps.cuh"
@@ -151,9 +152,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 __global__ void __launch_bounds__(256) topk_rows_kernel(const float *logits, int T, int E, int k, int32_t *idx,
                                                         float *gate, int32_t *cnt)
 {
+    extern __shared__ float topk_smem[];
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= T) return;
+    if (k <= 32 && E <= 1024) {
+        // the token's logits into shared memory, then the one-pass threshold selection
+        float *row = topk_smem + (size_t)(threadIdx.x >> 5) * (E + 128);
+        for (int e = lane; e < E; e += 32) row[e] = __ldg(logits + (size_t)t * E + e);
+        __syncwarp();
+        int me;
+        float mg;
+        if (E <= 512) topk_threshold<16>(row, E, k, me, mg, reinterpret_cast<unsigned *>(row + E));
+        else topk_threshold<32>(row, E, k, me, mg, reinterpret_cast<unsigned *>(row + E));
+        if (lane < k) {
+            idx[(size_t)t * k + lane] = me;
+            gate[(size_t)t * k + lane] = mg;
+            if (cnt) atomicAdd(&cnt[me], 1);
+        }
+        return;
+    }
     float v[32];
     uint32_t taken = 0u;
 #pragma unroll
@@ -228,7 +246,7 @@ cudaError_t prefill_route(const void *x_bf16, const uint16_t *wr, int T, int H, 
     gemm_bf16_tn_kernel<kRouterBN, kRouterStages><<<grid, kGemmThreads, kRouterSmem, s>>>(ma, mb, g);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    topk_rows_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, T, E, k, idx, gate, cnt);
+    topk_rows_kernel<<<(T + 7) / 8, 256, (size_t)8 * (E + 128) * sizeof(float), s>>>(logits, T, E, k, idx, gate, cnt);
     return cudaGetLastError();
 }
 
@@ -683,6 +701,9 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(const uint16_t *x, i
 
 // One warp per padded row: quantise h (fp32) of real rows to NVFP4 with a
 // per-row scale (the activation of the down GEMM).
+// Row quantisation of h for the down GEMM: one warp per row, one lane per
+// 16-value block (the same per-block rule as quant_step, so every code and
+// scale is bit-identical to it); I/16 blocks per row, 32 at I = 512.
 __global__ void __launch_bounds__(256) quant_rows_kernel(const float *h, int rows_cap, const int32_t *n_rows_dev,
                                                          int I, const int32_t *perm_tok, uint8_t *h_q, uint8_t *sfh,
                                                          int ksteps, float *row_scale)
@@ -692,26 +713,46 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const float *h, int row
     if (r >= rows_cap || r >= *n_rows_dev) return;
     if (perm_tok[r] < 0) return;
     const float *hr = h + (size_t)r * I;
+    const int nb = I >> 4;
     float amax = 0.f;
-    for (int c = lane * 4; c < I; c += 128) {
-        const float4 q = __ldcg(reinterpret_cast<const float4 *>(hr + c));
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
+    for (int b = lane; b < nb; b += 32) {
+        const float4 *p = reinterpret_cast<const float4 *>(hr + b * 16);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = __ldcg(p + q);
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float s = amax / (6.f * 448.f);
     if (lane == 0) row_scale[r] = s;
-    for (int st = lane; st < ksteps; st += 32) {
-        float v[64];
+    for (int b = lane; b < nb; b += 32) {
+        float v[16];
+        const float4 *p = reinterpret_cast<const float4 *>(hr + b * 16);
 #pragma unroll
-        for (int i = 0; i < 64; i += 4) {
-            const float4 q = __ldcg(reinterpret_cast<const float4 *>(hr + st * 64 + i));
-            v[i] = q.x;
-            v[i + 1] = q.y;
-            v[i + 2] = q.z;
-            v[i + 3] = q.w;
+        for (int q = 0; q < 4; ++q) {
+            const float4 w = __ldcg(p + q);
+            v[4 * q] = w.x;
+            v[4 * q + 1] = w.y;
+            v[4 * q + 2] = w.z;
+            v[4 * q + 3] = w.w;
         }
-        quant_step(v, s, h_q + (size_t)r * (I / 2) + st * 32, sfh + sf_offset(r, st, 0, ksteps));
+        float bmax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+        const uint32_t sb = s > 0.f ? e4m3_rn_sat(bmax / (6.f * s)) : 0u;
+        const float sbv = e4m3_val(sb);
+        const float den = s * sbv;
+        uint2 cw = make_uint2(0u, 0u);
+        if (sbv > 0.f) {
+            cw.x = e2m1x8(v[0] / den, v[1] / den, v[2] / den, v[3] / den, v[4] / den, v[5] / den, v[6] / den,
+                          v[7] / den);
+            cw.y = e2m1x8(v[8] / den, v[9] / den, v[10] / den, v[11] / den, v[12] / den, v[13] / den, v[14] / den,
+                          v[15] / den);
+        }
+        *reinterpret_cast<uint2 *>(h_q + (size_t)r * (I / 2) + b * 8) = cw;
+        sfh[sf_offset(r, b >> 2, b & 3, ksteps)] = (uint8_t)sb;
     }
 }
 
