@@ -282,6 +282,10 @@ constexpr int kNvSfA = 4 * 512, kNvSfB = 2 * 4 * 512;       // four K steps
 constexpr int kNvStage = kNvStageA + kNvStageB + kNvSfA + kNvSfB;
 constexpr size_t kNvSmem = (size_t)kNvStages * kNvStage + 1024;
 constexpr uint32_t kNvTmemCols = 512;  // accumulator 256 + scales 48 (+ unused)
+constexpr int kNvEpiWarps = 16;         // warps 0-15: epilogue (four per TMEM lane quarter)
+constexpr int kNvEpiParts = kNvEpiWarps / 4;
+constexpr int kNvTmaWarp = kNvEpiWarps, kNvMmaWarp = kNvEpiWarps + 1;
+constexpr int kNvThreads = 32 * (kNvEpiWarps + 2);
 
 struct NvGemmArgs {
     const int2 *tiles;        // M tiles: {expert, first padded row}
@@ -320,7 +324,7 @@ __device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, 
 }
 
 template <bool GATEUP>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kNvThreads, 1)
     nvfp4_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                               const NvGemmArgs g)
 {
@@ -333,7 +337,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int n_tiles = *g.n_tiles * g.NT;
     const int KT = g.K / 256;  // stages per tile
 
-    if (warp == 5) {
+    if (warp == kNvMmaWarp) {
         tmem_alloc(&tmem_base, kNvTmemCols);
         tmem_relinquish();
     }
@@ -343,7 +347,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&accf_bar, 1);
-        mbar_init(&acce_bar, 4);
+        mbar_init(&acce_bar, kNvEpiWarps);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -353,7 +357,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = tmem_base;
     const uint32_t t_acc = tmem, t_sfa = tmem + 256, t_sfb = tmem + 256 + 16;
 
-    if (warp == 4) {
+    if (warp == kNvTmaWarp) {
         if (lane == 0) {
             prefetch_tmap(&tmA);
             prefetch_tmap(&tmB);
@@ -392,7 +396,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kNvMmaWarp) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_nvf4(128, 256);
             int it = 0, tcount = 0;
@@ -436,13 +440,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             const int mt = tile / g.NT, nt = tile % g.NT;
             const int2 td = g.tiles[mt];
-            const int e = td.x, row = td.y + warp * 32 + lane;
+            // warps q, q + 4, ... read TMEM lanes 32 q .. 32 q + 31 and split the columns
+            const int quarter = warp & 3, part = warp >> 2;
+            const int e = td.x, row = td.y + quarter * 32 + lane;
             const int tok = g.perm_tok[row];
             const float sc = g.row_scale[row] * g.ts[e];
-            const uint32_t tl = t_acc + ((uint32_t)(warp * 32) << 16);
+            const uint32_t tl = t_acc + ((uint32_t)(quarter * 32) << 16);
             if (GATEUP) {
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 16) {
+                for (int c = part * (128 / kNvEpiParts); c < (part + 1) * (128 / kNvEpiParts); c += 16) {
                     float vg[16], vu[16];
                     tmem_ld16(tl + c, vg);
                     tmem_ld16(tl + 128 + c, vu);
@@ -454,7 +460,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                             for (int q = 0; q < 4; ++q) {
                                 const float a = vg[i + q] * sc, b = vu[i + q] * sc;
-                                o[q] = a / (1.f + expf(-a)) * b;
+                                // silu with the fast exponential (ex2-based; well inside the prefill tolerance)
+                                o[q] = a * __frcp_rn(1.f + __expf(-a)) * b;
                             }
                             *reinterpret_cast<float4 *>(dst + i) = make_float4(o[0], o[1], o[2], o[3]);
                         }
@@ -463,7 +470,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             } else {
                 const float gsc = tok >= 0 ? sc * g.row_gate[row] : 0.f;
 #pragma unroll 1
-                for (int c = 0; c < 256; c += 16) {
+                for (int c = part * (256 / kNvEpiParts); c < (part + 1) * (256 / kNvEpiParts); c += 16) {
                     float v[16];
                     tmem_ld16(tl + c, v);
                     if (tok >= 0) {
@@ -482,7 +489,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_before_sync();
     __syncthreads();
     if (abort_flag && threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
-    if (warp == 5) {
+    if (warp == kNvMmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, kNvTmemCols);
     }
@@ -819,7 +826,7 @@ cudaError_t prefill_nvfp4_forward(const PrefillNvArgs &a, cudaStream_t s)
     g.out = a.out;
     g.H = H;
     g.err = a.err;
-    nvfp4_grouped_gemm_kernel<true><<<a.num_sms, kGemmThreads, kNvSmem, s>>>(ma, mb, g);
+    nvfp4_grouped_gemm_kernel<true><<<a.num_sms, kNvThreads, kNvSmem, s>>>(ma, mb, g);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     quant_rows_kernel<<<(w.max_rows + 7) / 8, 256, 0, s>>>(w.h, w.max_rows, w.total_rows, I, w.perm_tok, w.h_q,
                                                            w.sfh, ks_i, w.row_scale_h);
@@ -839,7 +846,7 @@ cudaError_t prefill_nvfp4_forward(const PrefillNvArgs &a, cudaStream_t s)
     d.ksteps_b = a.dn->ksteps;
     d.ts = a.dn->ts;
     d.row_scale = w.row_scale_h;
-    nvfp4_grouped_gemm_kernel<false><<<a.num_sms, kGemmThreads, kNvSmem, s>>>(ma2, mb2, d);
+    nvfp4_grouped_gemm_kernel<false><<<a.num_sms, kNvThreads, kNvSmem, s>>>(ma2, mb2, d);
     return cudaGetLastError();
 }
 
