@@ -7,10 +7,11 @@
 // two 128 x 256 MMAs, halving the dequantisation work per multiply-add, and the
 // two f32 accumulators fill the 512 tensor-memory columns.
 //
-//   warps 0-3    epilogue (one accumulator row per thread and half)
-//   warp 4       TMA producer of the activation tiles (bf16, 128-byte swizzle)
-//   warp 5       MMA issuer (one elected thread)
-//   warps 6-13   dequantisers: thread n owns weight row n of the stage; it
+//   warps 0-7    epilogue (warps q and q + 4 read accumulator lanes 32q..32q+31
+//                and split the columns)
+//   warp 8       TMA producer of the activation tiles (bf16, 128-byte swizzle)
+//   warp 9       MMA issuer (one elected thread)
+//   warps 10-17  dequantisers: thread n owns weight row n of the stage; it
 //                loads the row's 64 int8 codes and two fp16 scales (the next
 //                stage's already in flight), converts q*d to bf16 and stores
 //                the eight 16-byte chunks at their 128-byte-swizzle positions,
@@ -38,7 +39,9 @@ namespace {
 using namespace tc;
 using namespace tmaps;
 
-constexpr int kQ8Threads = 448;  // 14 warps
+constexpr int kQ8EpiWarps = 8;
+constexpr int kQ8TmaWarp = kQ8EpiWarps, kQ8MmaWarp = kQ8EpiWarps + 1, kQ8DeqWarp0 = kQ8EpiWarps + 2;
+constexpr int kQ8Threads = 32 * (kQ8DeqWarp0 + 8);  // 18 warps
 constexpr int kQ8Stages = 3;
 constexpr int kQ8A = 128 * 128;  // one 128-row half: 128 rows x 64 bf16
 constexpr int kQ8B = 256 * 128;  // 256 weight rows x 64 bf16
@@ -92,7 +95,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     const int n_tiles = *g.n_ptiles * g.NT;
     const int KT = g.K / 64;
 
-    if (warp == 5) {
+    if (warp == kQ8MmaWarp) {
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
@@ -103,7 +106,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&accf_bar, 1);
-        mbar_init(&acce_bar, 4);
+        mbar_init(&acce_bar, kQ8EpiWarps);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     tc_fence_after_sync();
     const uint32_t tmem = tmem_base;
 
-    if (warp == 4) {  // ---- activation producer
+    if (warp == kQ8TmaWarp) {  // ---- activation producer
         if (lane == 0) {
             prefetch_tmap(&tmA);
             int it = 0;
@@ -131,7 +134,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
                 }
             }
         }
-    } else if (warp == 5) {  // ---- MMA issuer
+    } else if (warp == kQ8MmaWarp) {  // ---- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(128, 256);
             int it = 0, tcount = 0;
@@ -162,8 +165,8 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
                 mma_commit(&accf_bar);
             }
         }
-    } else if (warp >= 6) {  // ---- weight dequantisers: thread n owns weight row n
-        const int n = threadIdx.x - 192;
+    } else if (warp >= kQ8DeqWarp0) {  // ---- weight dequantisers: thread n owns weight row n
+        const int n = threadIdx.x - 32 * kQ8DeqWarp0;
         int it = 0;
         for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
             const int mt = tile / g.NT, nt = tile % g.NT;
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
                 sc2 = scn;
             }
         }
-    } else {  // ---- epilogue, warps 0-3
+    } else {  // ---- epilogue, warps 0-7
         int tcount = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tcount) {
             const bool ok = mbar_wait(&accf_bar, tcount & 1);
@@ -227,13 +230,14 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
             }
             const int mt = tile / g.NT, nt = tile % g.NT;
             const int4 pt = g.ptiles[mt];
+            const int quarter = warp & 3, part = warp >> 2;
             for (int hh = 0; hh < pt.z; ++hh) {
-                const int row = pt.y + hh * 128 + warp * 32 + lane;
+                const int row = pt.y + hh * 128 + quarter * 32 + lane;
                 const int tok = g.perm_tok[row];
-                const uint32_t tl = tmem + hh * 256 + ((uint32_t)(warp * 32) << 16);
+                const uint32_t tl = tmem + hh * 256 + ((uint32_t)(quarter * 32) << 16);
                 if (GATEUP) {
 #pragma unroll 1
-                    for (int c = 0; c < 128; c += 16) {
+                    for (int c = part * 64; c < part * 64 + 64; c += 16) {
                         float vg[16], vu[16];
                         tmem_ld16(tl + c, vg);
                         tmem_ld16(tl + 128 + c, vu);
@@ -242,7 +246,9 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
 #pragma unroll
                             for (int i = 0; i < 16; i += 2) {
                                 const float a0 = vg[i], a1 = vg[i + 1];
-                                o[i / 2] = pack_bf16x2(a0 / (1.f + expf(-a0)) * vu[i], a1 / (1.f + expf(-a1)) * vu[i + 1]);
+                                // silu with the fast exponential (well inside the prefill tolerance)
+                                o[i / 2] = pack_bf16x2(a0 * __frcp_rn(1.f + __expf(-a0)) * vu[i],
+                                                       a1 * __frcp_rn(1.f + __expf(-a1)) * vu[i + 1]);
                             }
                             uint4 *dst = reinterpret_cast<uint4 *>(g.h + (size_t)row * g.I + nt * 128 + c);
                             dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -252,7 +258,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
                 } else {
                     const float gt = tok >= 0 ? g.row_gate[row] : 0.f;
 #pragma unroll 1
-                    for (int c = 0; c < 256; c += 16) {
+                    for (int c = part * 128; c < part * 128 + 128; c += 16) {
                         float v[16];
                         tmem_ld16(tl + c, v);
                         if (tok >= 0) {
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     tc_fence_before_sync();
     __syncthreads();
     if (abort_flag && threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
-    if (warp == 5) {
+    if (warp == kQ8MmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
     }
