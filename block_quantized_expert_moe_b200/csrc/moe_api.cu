@@ -401,7 +401,7 @@ moe_status build_prefill_workspace(moe_pack *p)
         {(void **)&w.ptiles, rows / 128 * 16 + 64}, {(void **)&w.n_ptiles, 4},
         {(void **)&w.n_tiles, 4}, {(void **)&w.total_rows, 4}, {(void **)&w.perm_tok, rows * 4},
         {(void **)&w.row_gate, rows * 4}, {(void **)&w.row_scale_x, rows * 4}, {(void **)&w.row_scale_h, rows * 4},
-        {(void **)&w.a_q, p->fmt_gu == MOE_FMT_Q8_0 ? rows * H * 2 : rows * H / 2},
+        {(void **)&w.a_q, p->fmt_gu != MOE_FMT_NVFP4 ? rows * H * 2 : rows * H / 2},
         {(void **)&w.sfa, rows / 128 * (H / 64) * 512},
         {(void **)&w.h, rows * I * 4}, {(void **)&w.h_q, rows * I / 2}, {(void **)&w.sfh, rows / 128 * (I / 64) * 512},
     };
@@ -512,8 +512,8 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
     if (st == MOE_OK) st = build_workspace(p);
     const bool nv = p->fmt_gu == MOE_FMT_NVFP4 && p->fmt_dn == MOE_FMT_NVFP4 &&
                     prefill_nvfp4_supported(p->H, p->I, p->E, p->max_top_k);
-    const bool q8 = p->fmt_gu == MOE_FMT_Q8_0 && p->fmt_dn == MOE_FMT_Q8_0 &&
-                    prefill_q8_supported(p->H, p->I, p->E, p->max_top_k);
+    // bf16-dequantising tensor-core prefill: Q8_0, IQ4_NL and Q5_1, in any mix
+    const bool q8 = prefill_q8_supported(p->fmt_gu, p->fmt_dn, p->H, p->I, p->E, p->max_top_k);
     if (st == MOE_OK && p->max_tokens > kDecodeMaxTokens && (nv || q8)) st = build_prefill_workspace(p);
     if (st == MOE_OK && cudaDeviceSynchronize() != cudaSuccess) st = MOE_ERR_CUDA;
     if (st != MOE_OK) {
@@ -639,6 +639,8 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
         pa.has_shared = p->has_shared;
         pa.gu = &p->gu;
         pa.dn = &p->dn;
+        pa.tab_gu = p->ct_gu;
+        pa.tab_dn = p->ct_dn;
         pa.out = out;
         pa.err = w.err;
         pa.ws = &p->pws;
@@ -650,7 +652,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
             pm->prof_fwd.push_back({pbase, 2});
         }
         prof_mark(pm, pbase, 0, s);
-        moe_status st = check_launch(p->fmt_gu == MOE_FMT_Q8_0 ? prefill_q8_forward(pa, s) : prefill_nvfp4_forward(pa, s));
+        moe_status st = check_launch(p->fmt_gu == MOE_FMT_NVFP4 ? prefill_nvfp4_forward(pa, s) : prefill_q8_forward(pa, s));
         prof_mark(pm, pbase, 1, s);
         return st;
     }

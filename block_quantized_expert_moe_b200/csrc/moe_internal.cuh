@@ -192,6 +192,7 @@ struct PrefillNvArgs {
     const uint16_t *wr;
     int T, H, I, E, k, has_shared;
     const DevProj *gu, *dn;
+    CodeTable tab_gu, tab_dn;  // 4-bit formats (the dequantising path)
     float *out;
     int32_t *err;
     const PrefillWorkspace *ws;
@@ -204,7 +205,7 @@ bool prefill_nvfp4_supported(int H, int I, int E, int k);
 cudaError_t prefill_nvfp4_forward(const PrefillNvArgs &a, cudaStream_t s);
 cudaError_t prefill_plan_launch(const PrefillWorkspace &w, int E, int T, int has_shared, int32_t *err, cudaStream_t s);
 cudaError_t prefill_q8_set_attributes();
-bool prefill_q8_supported(int H, int I, int E, int k);
+bool prefill_q8_supported(int fmt_gu, int fmt_dn, int H, int I, int E, int k);  // Q8_0 / IQ4_NL / Q5_1
 cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s);
 cudaError_t prefill_route(const void *x_bf16, const uint16_t *wr, int T, int H, int E, int k, float *logits,
                           int32_t *idx, float *gate, int32_t *cnt, int32_t *err, cudaStream_t s);

@@ -29,6 +29,7 @@
 #include <cuda_runtime.h>
 
 #include "moe_internal.cuh"
+#include "quant_dot.cuh"
 #include "tc_common.cuh"
 #include "tma_maps.cuh"
 
@@ -53,11 +54,16 @@ struct Q8GemmArgs {
     const int32_t *n_ptiles;
     int NT;                    // weight-row tiles of 256 (gate/up: I/128 pairs of 128)
     int K;                     // reduction length
-    const uint8_t *qs;         // Q8_0 codes plane (stored +128), rows x K bytes per expert
+    const uint8_t *qs;         // codes plane: Q8_0 K bytes per row (stored +128), 4-bit K/2
     int64_t qs_stride;
-    const uint8_t *sc;         // fp16 scale plane, rows x K/32 per expert
+    int qs_row;
+    const uint8_t *sc;         // scale plane: fp16 d per 32 (Q5_1: {d, m})
     int64_t sc_stride;
     int sc_row;
+    const uint8_t *qh;         // Q5_1 fifth bits, u32 per 32
+    int64_t qh_stride;
+    int qh_row;
+    CodeTable tab;             // IQ4_NL table (biased bytes; the pack's code positions)
     int up_off;                // gate/up: row offset of U (= I); down: 0
     const int32_t *perm_tok;
     const float *row_gate;
@@ -82,9 +88,89 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return r;
 }
 
-template <bool GATEUP>
+// One 64-wide K slice (two 32-weight blocks) of a weight row, as loaded.
+template <int FMT>
+struct DqSlice {
+    uint4 q[FMT == MOE_FMT_Q8_0 ? 4 : 2];  // codes
+    uint32_t s0, s1;                       // block scales (Q8_0 / IQ4_NL: fp16 d; Q5_1: {d, m})
+    uint32_t h0, h1;                       // Q5_1 fifth bits
+};
+
+template <int FMT>
+__device__ __forceinline__ DqSlice<FMT> dq_load(const uint8_t *qrow, const uint8_t *srow, const uint8_t *hrow, int kt)
+{
+    DqSlice<FMT> r;
+    r.h0 = r.h1 = 0;
+    if constexpr (FMT == MOE_FMT_Q8_0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r.q[i] = __ldg(reinterpret_cast<const uint4 *>(qrow + kt * 64) + i);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) r.q[i] = __ldg(reinterpret_cast<const uint4 *>(qrow + kt * 32) + i);
+    }
+    if constexpr (FMT == MOE_FMT_Q5_1) {
+        const uint2 sv = __ldg(reinterpret_cast<const uint2 *>(srow + kt * 8));
+        const uint2 hv = __ldg(reinterpret_cast<const uint2 *>(hrow + kt * 8));
+        r.s0 = sv.x;
+        r.s1 = sv.y;
+        r.h0 = hv.x;
+        r.h1 = hv.y;
+    } else {
+        const uint32_t sv = __ldg(reinterpret_cast<const uint32_t *>(srow + kt * 4));
+        r.s0 = sv & 0xFFFFu;
+        r.s1 = sv >> 16;
+    }
+    return r;
+}
+
+__device__ __forceinline__ float half_bits(uint32_t b) { return __half2float(__ushort_as_half((unsigned short)b)); }
+
+// The 32 weights of block u of the slice, in element order.
+template <int FMT>
+__device__ __forceinline__ void dq_block(const DqSlice<FMT> &r, int u, const CodeTable &ct, float (&v)[32])
+{
+    if constexpr (FMT == MOE_FMT_Q8_0) {
+        const float d = half_bits(u ? r.s1 : r.s0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t w = (&r.q[2 * u].x)[i];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) v[4 * i + b] = byte_f(w, b) * d;
+        }
+    } else if constexpr (FMT == MOE_FMT_IQ4_NL) {
+        // element j < 16: low nibble of byte j; j >= 16: high nibble of byte j - 16
+        const float d = half_bits(u ? r.s1 : r.s0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            uint32_t o0, o1;
+            qd::lut16((&r.q[u].x)[s], ct, o0, o1);  // o0 = [lo0 hi0 lo1 hi1], o1 = [lo2 hi2 lo3 hi3] of bytes 4s..
+            const uint32_t oo[2] = {o0, o1};
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t o = oo[b >> 1];
+                const float lo = __uint_as_float(qd::prmt(o, 0x4B000000u, 0x7650u + 2 * (b & 1))) - ct.magic;
+                const float hi = __uint_as_float(qd::prmt(o, 0x4B000000u, 0x7650u + 2 * (b & 1) + 1)) - ct.magic;
+                v[4 * s + b] = lo * d;
+                v[16 + 4 * s + b] = hi * d;
+            }
+        }
+    } else {  // Q5_1: q = nibble | fifth bit << 4, w = d * q + m
+        const uint32_t dm = u ? r.s1 : r.s0, hb = u ? r.h1 : r.h0;
+        const float d = half_bits(dm & 0xFFFFu), m = half_bits(dm >> 16);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const uint32_t byte = ((&r.q[u].x)[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+            const uint32_t lo = (byte & 0xFu) | (((hb >> j) & 1u) << 4);
+            const uint32_t hi = (byte >> 4) | (((hb >> (j + 16)) & 1u) << 4);
+            v[j] = fmaf(d, (float)lo, m);
+            v[16 + j] = fmaf(d, (float)hi, m);
+        }
+    }
+}
+
+template <bool GATEUP, int FMT>
 __global__ void __launch_bounds__(kQ8Threads, 1)
-    q8_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const Q8GemmArgs g)
+    dq_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const Q8GemmArgs g)
 {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t fa_bar[kQ8Stages], fb_bar[kQ8Stages], empty_bar[kQ8Stages], accf_bar, acce_bar;
@@ -172,22 +258,14 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
             const int mt = tile / g.NT, nt = tile % g.NT;
             const int e = g.ptiles[mt].x;
             const int row = GATEUP ? (n < 128 ? nt * 128 + n : g.up_off + nt * 128 + (n - 128)) : nt * 256 + n;
-            const uint8_t *qrow = g.qs + (int64_t)e * g.qs_stride + (int64_t)row * g.K;
+            const uint8_t *qrow = g.qs + (int64_t)e * g.qs_stride + (int64_t)row * g.qs_row;
             const uint8_t *srow = g.sc + (int64_t)e * g.sc_stride + (int64_t)row * g.sc_row;
-            uint4 q[4];
-            uint32_t sc2;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) q[i] = __ldg(reinterpret_cast<const uint4 *>(qrow) + i);
-            sc2 = __ldg(reinterpret_cast<const uint32_t *>(srow));
+            const uint8_t *hrow = FMT == MOE_FMT_Q5_1 ? g.qh + (int64_t)e * g.qh_stride + (int64_t)row * g.qh_row : nullptr;
+            DqSlice<FMT> cur = dq_load<FMT>(qrow, srow, hrow, 0);
             for (int kt = 0; kt < KT; ++kt, ++it) {
                 const int s = it % kQ8Stages, u = it / kQ8Stages;
-                uint4 qn[4];
-                uint32_t scn = 0;
-                if (kt + 1 < KT) {  // next K slice of this row, in flight while we convert
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) qn[i] = __ldg(reinterpret_cast<const uint4 *>(qrow + (kt + 1) * 64) + i);
-                    scn = __ldg(reinterpret_cast<const uint32_t *>(srow + (kt + 1) * 4));
-                }
+                DqSlice<FMT> nxt = cur;
+                if (kt + 1 < KT) nxt = dq_load<FMT>(qrow, srow, hrow, kt + 1);  // in flight while we convert
                 if (u > 0) {
                     bool ok = true;
                     if (lane == 0) ok = mbar_wait(&empty_bar[s], (u - 1) & 1);
@@ -197,26 +275,26 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
                         break;
                     }
                 }
-                const float d0 = __half2float(__ushort_as_half((unsigned short)(sc2 & 0xFFFFu)));
-                const float d1 = __half2float(__ushort_as_half((unsigned short)(sc2 >> 16)));
                 uint8_t *b_row = smem + s * kQ8Stage + 2 * kQ8A + (n >> 3) * 1024 + (n & 7) * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {  // chunk c: 8 codes, k = 8c .. 8c+7
-                    const uint32_t w0 = (&q[c >> 1].x)[(c & 1) * 2], w1 = (&q[c >> 1].x)[(c & 1) * 2 + 1];
-                    const float d = c < 4 ? d0 : d1;
-                    uint4 o;
-                    o.x = pack_bf16x2(byte_f(w0, 0) * d, byte_f(w0, 1) * d);
-                    o.y = pack_bf16x2(byte_f(w0, 2) * d, byte_f(w0, 3) * d);
-                    o.z = pack_bf16x2(byte_f(w1, 0) * d, byte_f(w1, 1) * d);
-                    o.w = pack_bf16x2(byte_f(w1, 2) * d, byte_f(w1, 3) * d);
-                    *reinterpret_cast<uint4 *>(b_row + ((c ^ (n & 7)) << 4)) = o;
+                for (int blk = 0; blk < 2; ++blk) {
+                    float v[32];
+                    dq_block<FMT>(cur, blk, g.tab, v);
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {  // chunk c = 4 blk + cc: k = 8c .. 8c+7
+                        const int c = 4 * blk + cc;
+                        uint4 o;
+                        o.x = pack_bf16x2(v[8 * cc], v[8 * cc + 1]);
+                        o.y = pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
+                        o.z = pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
+                        o.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
+                        *reinterpret_cast<uint4 *>(b_row + ((c ^ (n & 7)) << 4)) = o;
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&fb_bar[s]);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) q[i] = qn[i];
-                sc2 = scn;
+                cur = nxt;
             }
         }
     } else {  // ---- epilogue, warps 0-7
@@ -324,20 +402,40 @@ __global__ void __launch_bounds__(256) gather_scatter_kernel(const uint16_t *x, 
     }
 }
 
+
+
+using DqKernel = void (*)(const CUtensorMap, const Q8GemmArgs);
+
+DqKernel dq_pick(bool gateup, int fmt)
+{
+    switch (fmt) {
+    case MOE_FMT_Q8_0: return gateup ? dq_grouped_gemm_kernel<true, MOE_FMT_Q8_0> : dq_grouped_gemm_kernel<false, MOE_FMT_Q8_0>;
+    case MOE_FMT_IQ4_NL:
+        return gateup ? dq_grouped_gemm_kernel<true, MOE_FMT_IQ4_NL> : dq_grouped_gemm_kernel<false, MOE_FMT_IQ4_NL>;
+    case MOE_FMT_Q5_1: return gateup ? dq_grouped_gemm_kernel<true, MOE_FMT_Q5_1> : dq_grouped_gemm_kernel<false, MOE_FMT_Q5_1>;
+    default: return nullptr;
+    }
+}
+
+bool dq_fmt(int f) { return f == MOE_FMT_Q8_0 || f == MOE_FMT_IQ4_NL || f == MOE_FMT_Q5_1; }
+
 }  // namespace
+
+bool prefill_q8_supported(int fmt_gu, int fmt_dn, int H, int I, int E, int k)
+{
+    return dq_fmt(fmt_gu) && dq_fmt(fmt_dn) && H % 256 == 0 && I % 256 == 0 && E <= 1023 && k <= 32;
+}
 
 cudaError_t prefill_q8_set_attributes()
 {
-    cudaError_t e = cudaFuncSetAttribute(q8_grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kQ8Smem);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(q8_grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kQ8Smem);
-}
-
-bool prefill_q8_supported(int H, int I, int E, int k)
-{
-    return H % 256 == 0 && I % 256 == 0 && E <= 1023 && k <= 32;
+    const int fmts[3] = {MOE_FMT_Q8_0, MOE_FMT_IQ4_NL, MOE_FMT_Q5_1};
+    for (int f : fmts)
+        for (int gu = 0; gu < 2; ++gu) {
+            const cudaError_t e =
+                cudaFuncSetAttribute(dq_pick(gu != 0, f), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQ8Smem);
+            if (e != cudaSuccess) return e;
+        }
+    return cudaSuccess;
 }
 
 cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s)
@@ -348,7 +446,7 @@ cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s)
     if ((e = cudaMemsetAsync(w.cnt, 0, sizeof(int32_t) * (E + 1), s)) != cudaSuccess) return e;
     if ((e = prefill_route(a.x, a.wr, T, H, E, k, w.logits, w.idx, w.gate, w.cnt, a.err, s)) != cudaSuccess) return e;
     if ((e = prefill_plan_launch(w, E, T, a.has_shared, a.err, s)) != cudaSuccess) return e;
-    uint16_t *xp = reinterpret_cast<uint16_t *>(w.a_q);  // bf16 slot rows, sized for the Q8_0 path
+    uint16_t *xp = reinterpret_cast<uint16_t *>(w.a_q);  // bf16 slot rows, sized for the dequantising path
     gather_scatter_kernel<<<(T + 7) / 8, 256, 0, s>>>(reinterpret_cast<const uint16_t *>(a.x), T, H, k, E,
                                                        a.has_shared, w.idx, w.gate, w.pad_off, w.fill, xp, w.perm_tok,
                                                        w.row_gate, w.slot_pos, w.max_rows);
@@ -362,9 +460,14 @@ cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s)
     g.K = H;
     g.qs = a.gu->qs;
     g.qs_stride = a.gu->qs_stride;
+    g.qs_row = a.gu->qs_row;
     g.sc = a.gu->sc;
     g.sc_stride = a.gu->sc_stride;
     g.sc_row = a.gu->sc_row;
+    g.qh = a.gu->qh;
+    g.qh_stride = a.gu->qh_stride;
+    g.qh_row = a.gu->qh_row;
+    g.tab = a.tab_gu;
     g.up_off = I;
     g.perm_tok = w.perm_tok;
     g.row_gate = w.row_gate;
@@ -373,7 +476,9 @@ cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s)
     g.out = a.out;
     g.H = H;
     g.err = a.err;
-    q8_grouped_gemm_kernel<true><<<a.num_sms, kQ8Threads, kQ8Smem, s>>>(ma, g);
+    DqKernel kgu = dq_pick(true, a.gu->fmt), kdn = dq_pick(false, a.dn->fmt);
+    if (!kgu || !kdn) return cudaErrorInvalidValue;
+    kgu<<<a.num_sms, kQ8Threads, kQ8Smem, s>>>(ma, g);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(a.out, 0, sizeof(float) * (size_t)T * H, s)) != cudaSuccess) return e;
     CUtensorMap mh;
@@ -383,11 +488,16 @@ cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s)
     d.K = I;
     d.qs = a.dn->qs;
     d.qs_stride = a.dn->qs_stride;
+    d.qs_row = a.dn->qs_row;
     d.sc = a.dn->sc;
     d.sc_stride = a.dn->sc_stride;
     d.sc_row = a.dn->sc_row;
+    d.qh = a.dn->qh;
+    d.qh_stride = a.dn->qh_stride;
+    d.qh_row = a.dn->qh_row;
+    d.tab = a.tab_dn;
     d.up_off = 0;
-    q8_grouped_gemm_kernel<false><<<a.num_sms, kQ8Threads, kQ8Smem, s>>>(mh, d);
+    kdn<<<a.num_sms, kQ8Threads, kQ8Smem, s>>>(mh, d);
     return cudaGetLastError();
 }
 

@@ -107,6 +107,9 @@ WORKLOADS = {
                               DT_BF16, 8192, zipf_s=1.1),
     "prefill_q8": Workload("prefill_q8", 2048, 512, 512, 10, False, FMT_Q8_0, FMT_Q8_0, DT_BF16,
                            8192, zipf_s=1.1),
+    # the model-shaped layer's formats (IQ4_NL gate/up, Q5_1 down, shared expert) in a prefill chunk
+    "prefill_iq4nl_q51": Workload("prefill_iq4nl_q51", 2048, 512, 512, 10, True, FMT_IQ4_NL, FMT_Q5_1,
+                                  DT_BF16, 8192, zipf_s=1.1),
 }
 
 _lib = None

@@ -89,3 +89,38 @@ def test_prefill_q8_bf16_dequant_ragged_batch():
 def test_prefill_q8_full_chunk_sampled():
     rng = np.random.default_rng(1)
     _run_q8(8192, sample=np.sort(rng.choice(8192, 16, replace=False)))
+
+
+def _run_dq(wl, T, layer=0, sample=None):
+    import block_quantized_expert_moe_b200 as bq
+    li = synth.layer_inputs(wl, layer)
+    x = synth.tokens(wl, li.router, layer, 0, T)
+    out, idx, gate, counts = gpu_layer(li, x, wl.top_k, path=bq.MOE_PATH_PREFILL)
+    tok = np.arange(T) if sample is None else np.asarray(sample)
+    # weights and h are rounded to bf16 for the tensor cores; the oracle stays exact
+    ref, ridx, rgate = oracle_layer(li, x, wl.top_k, tokens=tok)
+    assert_routing_equal(idx[tok], gate[tok], ridx, rgate)
+    if sample is None:
+        assert np.array_equal(counts, expected_counts(ridx, wl.n_experts, T, wl.has_shared))
+    err = normwise_err(out[tok], ref)
+    assert err <= PREFILL_TOL, err
+    return err
+
+
+def test_prefill_iq4nl_q51_dequant_ragged_batch():
+    """The model-shaped layer's formats through the bf16-dequantising tensor-core path (shared expert)."""
+    err = _run_dq(synth.WORKLOADS["prefill_iq4nl_q51"], 300)
+    print(f"prefill IQ4_NL/Q5_1 -> bf16 T=300: err vs exact oracle {err:.2e}")
+
+
+def test_prefill_mixed_formats_small_shapes():
+    # Q5_1 gate/up with an IQ4_NL down projection, and Q8_0 with Q5_1: 4-bit and 8-bit dequantisers
+    for gu, dn, seed in ((synth.FMT_Q5_1, synth.FMT_IQ4_NL, 41), (synth.FMT_Q8_0, synth.FMT_Q5_1, 42)):
+        wl = synth.Workload("mixed", 1024, 48, 256, 6, True, gu, dn, synth.DT_BF16, 200, zipf_s=1.1, seed=seed)
+        _run_dq(wl, 200)
+
+
+def test_prefill_iq4nl_q51_full_chunk_sampled():
+    rng = np.random.default_rng(2)
+    _run_dq(synth.WORKLOADS["prefill_iq4nl_q51"], 8192, sample=np.sort(rng.choice(8192, 16, replace=False)))
+
