@@ -1,5 +1,7 @@
-// Tensor-core prefill for Q8_0 experts: the weight blocks are dequantised to
-// bf16 in shared memory and multiplied with tcgen05.mma kind::f16.
+// Tensor-core prefill for Q8_0, IQ4_NL and Q5_1 experts: the weight blocks are
+// dequantised to bf16 in shared memory and multiplied with tcgen05.mma
+// kind::f16.  One kernel instance per format (the two projections may differ);
+// only the dequantiser warps depend on it.
 //
 // The same padded slot space as the NVFP4 prefill (every 128-row M tile
 // belongs to one expert).  A CTA tile is up to two consecutive M tiles of one
@@ -12,8 +14,10 @@
 //   warp 8       TMA producer of the activation tiles (bf16, 128-byte swizzle)
 //   warp 9       MMA issuer (one elected thread)
 //   warps 10-17  dequantisers: thread n owns weight row n of the stage; it
-//                loads the row's 64 int8 codes and two fp16 scales (the next
-//                stage's already in flight), converts q*d to bf16 and stores
+//                loads the row's two 32-weight blocks (Q8_0: 64 int8 codes and
+//                two fp16 scales; IQ4_NL: 32 code bytes looked up in the pack's
+//                table; Q5_1: 32 code bytes, fifth bits, {d, m}) with the next
+//                stage's already in flight, converts to bf16 and stores
 //                the eight 16-byte chunks at their 128-byte-swizzle positions,
 //                then makes them visible to the tensor core (fence.proxy.async)
 //
