@@ -382,6 +382,15 @@ def ours_arm(a, wl):
                      if stage_ms[4] > 0 and T == 1 else None)
     if grid_event_us is not None:
         grid_event_us["cta0_points"] = [round(float(v / nf * 1e3), 3) for v in stage_ms[24:32]]
+    elif stage_ms[0] > 0 and stage_ms[15] > 0:
+        # grouped path: the router kernel's events (first/last CTA), from its first CTA's start
+        route_names = ["last_start", "first_staged", "last_staged", "first_logits", "last_logits",
+                       "first_topk_end", "last_topk_end", "first_plan_end", "last_plan_end"]
+        grid_event_us = {"route_" + n: float(stage_ms[15 + i] / nf * 1e3) for i, n in enumerate(route_names)}
+        # the selecting / planning CTA's own clock between its steps
+        step_names = ["stage_logits", "select", "topk_rest", "ticket", "counts", "scans", "groups",
+                      "slot_order", "tail"]
+        fused_phase_us = {"route_" + n: float(stage_ms[6 + i] / nf * 1e3) for i, n in enumerate(step_names)}
     dom = max(stage_us, key=lambda s: stage_us[s])
     # one token: the streaming kernel (whole-row bulk copies) runs in place of the fused one
     kname = "stream1_kernel" if dom == "fused" and T == 1 else KERNEL_NAMES[dom]

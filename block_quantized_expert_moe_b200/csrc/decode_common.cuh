@@ -113,6 +113,25 @@ __device__ __forceinline__ float key_to_float(unsigned key)
     return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
+// Row t of the logits into shared memory with all of a lane's loads in flight
+// (a loop of dependent load/store pairs would pay one L2 round trip per
+// element of the lane).
+template <int NPL>
+__device__ __forceinline__ void stage_logits(const float *src, float *row, int E, int lane)
+{
+    float v[NPL];
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+        const int e = lane + 32 * j;
+        v[j] = e < E ? __ldcg(src + e) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E) row[e] = v[j];
+    }
+}
+
 // Best (largest key, lowest position on ties) of a lane's NPL keys, as a tree.
 template <int NPL>
 __device__ __forceinline__ void lane_best(const unsigned (&key)[NPL], unsigned &bk, int &bi)

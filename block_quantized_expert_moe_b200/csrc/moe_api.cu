@@ -590,6 +590,7 @@ moe_status moe_route_topk(const void *x, moe_dtype x_dtype, const uint16_t *rout
     a.idx = idx_out;
     a.gate = gate_out;
     a.do_plan = 0;
+    a.err = a.ticket + 1;  // word 1 of the workspace: a timed-out wait
     if (x_dtype == MOE_DT_BF16 && n_tokens > kDecodeMaxTokens) {
         // many tokens: the router as a tensor-core GEMM (word 1 of the workspace
         // records a timed-out wait), then top-k per token
@@ -779,6 +780,8 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     ra.dense = path == MOE_PATH_DENSE;
     ra.dgate = w.dgate;
     ra.n_dense_rows = w.n_dense_rows;
+    if (pbase >= 0 && pm->prof_stamps && pm->prof_nstamp < pm->prof_stamp_cap)
+        ra.stamps = pm->prof_stamps + kStampStride * (size_t)pm->prof_nstamp++;
     moe_status st = check_launch(launch_route(ra, route_grid(p->E, T, ra.rt, p->num_sms), s));
     if (st != MOE_OK) return st;
     prof_mark(pm, pbase, 1, s);

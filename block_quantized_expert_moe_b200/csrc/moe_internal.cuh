@@ -95,6 +95,13 @@ struct RouteArgs {
     int dense;
     float *dgate;           // [slots] gate of (active expert, token), 0 if not routed
     int32_t *n_dense_rows;  // active experts (incl. shared) x T
+    // profiling only (null otherwise): grid events folded into words 10..19 of
+    // a forward's stamps, as {2^62 - first, last} global-timer pairs: 0 start,
+    // 1 x and router rows staged, 2 logits written, 3 top-k done, 4 plan done; words 0..9
+    // the SM clock of the selecting / planning CTA at: top-k begin, row staged,
+    // selected, top-k done, plan begin, counts, scans, groups written, slot
+    // order written, plan done
+    long long *stamps;
 };
 
 // 16-entry code table of a 4-bit format, built on the host by build_code_table:
@@ -128,7 +135,7 @@ struct CombineArgs {
 };
 
 // launchers (return cudaGetLastError of the launch)
-size_t route_smem_bytes(int H, int rt, int E);
+size_t route_smem_bytes(int H, int rt, int E, int grid, int T);
 void init_device_attributes();  // once per device, with that device current
 int route_tokens_per_pass(int H);
 cudaError_t launch_route(const RouteArgs &a, int grid, cudaStream_t s);

@@ -159,7 +159,8 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(const float *logits, int
     if (k <= 32 && E <= 1024) {
         // the token's logits into shared memory, then the one-pass threshold selection
         float *row = topk_smem + (size_t)(threadIdx.x >> 5) * (E + 128);
-        for (int e = lane; e < E; e += 32) row[e] = __ldg(logits + (size_t)t * E + e);
+        if (E <= 512) stage_logits<16>(logits + (size_t)t * E, row, E, lane);
+        else stage_logits<32>(logits + (size_t)t * E, row, E, lane);
         __syncwarp();
         int me;
         float mg;

@@ -27,12 +27,85 @@
 
 #include "decode_common.cuh"
 #include "moe_internal.cuh"
+#include "quant_dot.cuh"
+#include "tc_common.cuh"
 
 namespace moe {
 
 namespace {
 
 constexpr int kRouteMaxBlockGroups = 14;  // per-group tickets at words 2..15 of the ticket area
+constexpr int kPlanIdxCache = 4096;       // selections the plan keeps in shared memory
+constexpr size_t kRouteWrSmem = 128 * 1024;  // router rows a CTA may stage in shared memory
+constexpr int kSmallPlanT = 64;           // token masks of one 64-bit word: the short plan
+
+__host__ __device__ inline size_t route_al16(size_t v) { return (v + 15) & ~(size_t)15; }
+
+// Shared-memory regions of the kernel, from (H, rt, E, rows per CTA); host and
+// device compute them alike.
+struct RouteSmem {
+    bool staged;     // the CTA's router rows are bulk-copied into shared memory
+    size_t wr, red;  // x rows as given (bf16 or fp32) at 0, then the router rows, partials
+    size_t gemv;     // bytes of the logit phase
+    size_t idx;      // the selections (short plan), after the top-k rows and the plan
+    size_t total;
+};
+
+__host__ __device__ inline RouteSmem route_smem(int H, int rt, int E, int rmax)
+{
+    RouteSmem m;
+    const size_t xb = (size_t)rt * H * 4;  // room for rt fp32 rows
+    m.staged = (size_t)rmax * H * 2 <= kRouteWrSmem;
+    m.wr = xb;
+    m.red = m.wr + route_al16((size_t)rmax * H * 2);
+    m.gemv = m.staged ? m.red + (size_t)(kThreads / 32) * 32 * 4 : xb;
+    const size_t topk = (size_t)(kThreads / 32) * (E + 128) * 4;
+    const size_t plan = (size_t)E * 8 + (size_t)4 * (E + 1) * 4 + 64 * 4;
+    m.idx = route_al16(topk > plan ? topk : plan);
+    size_t t = m.idx + (size_t)kPlanIdxCache * 4;
+    // the general top-k fallback (k > 32 or E > 1024): two rows per warp and flags
+    const size_t fb = (size_t)2 * (kThreads / 32) * E * 4 + (kThreads / 32) * 32 * 4;
+    if (fb > t) t = fb;
+    m.total = m.gemv > t ? m.gemv : t;
+    return m;
+}
+
+// 8 consecutive x values of token t starting at element 8c, from the raw rows
+// in shared memory, as four (even, odd) pairs.
+template <bool XBF16>
+__device__ __forceinline__ void x_chunk(const unsigned char *xs, int H, int t, int c, float2 (&x)[4])
+{
+    if constexpr (XBF16) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(xs + ((size_t)t * H + c * 8) * 2);
+        x[0] = make_float2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u));
+        x[1] = make_float2(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+        x[2] = make_float2(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u));
+        x[3] = make_float2(__uint_as_float(v.w << 16), __uint_as_float(v.w & 0xFFFF0000u));
+    } else {
+        const float4 *p = reinterpret_cast<const float4 *>(xs + ((size_t)t * H + c * 8) * 4);
+        const float4 lo = p[0], hi = p[1];
+        x[0] = make_float2(lo.x, lo.y);
+        x[1] = make_float2(lo.z, lo.w);
+        x[2] = make_float2(hi.x, hi.y);
+        x[3] = make_float2(hi.z, hi.w);
+    }
+}
+
+// Profiling only: thread 0 folds the global timer into event ev's first/last pair.
+__device__ __forceinline__ void route_event(long long *st, int ev)
+{
+    if (!st || threadIdx.x != 0) return;
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    atomicMax(st + 10 + 2 * ev, (1ll << 62) - (long long)t);
+    atomicMax(st + 11 + 2 * ev, (long long)t);
+}
+
+// Profiling only: thread 0 records its SM clock in word i of the stamps.
+__device__ __forceinline__ void route_clock(long long *st, int i, bool on)
+{
+    if (st && on && threadIdx.x == 0) st[i] = clock64();
+}
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
@@ -48,7 +121,7 @@ __device__ __forceinline__ uint4 ldg_nc16(const void *p)
 
 // In-place exclusive scan of n <= 4*kThreads ints in shared memory; returns
 // the total to every thread.  Uses `tmp` (>= 32 ints) for warp totals.
-__device__ int block_exclusive_scan(int *v, int n, int *tmp)
+__device__ __forceinline__ int block_exclusive_scan(int *v, int n, int *tmp)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int loc[4], s = 0;
@@ -90,7 +163,7 @@ __device__ int block_exclusive_scan(int *v, int n, int *tmp)
     return total;
 }
 
-__device__ void topk_phase(const RouteArgs &a, unsigned char *smem, int t_begin, int t_end)
+__device__ __forceinline__ void topk_phase(const RouteArgs &a, unsigned char *smem, int t_begin, int t_end, int *idx_s)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nw = kThreads / 32;
@@ -99,17 +172,21 @@ __device__ void topk_phase(const RouteArgs &a, unsigned char *smem, int t_begin,
         // one warp per token: the row into shared memory, then the threshold
         // selection (candidates at or above the k-th largest lane maximum)
         float *row = reinterpret_cast<float *>(smem) + (size_t)warp * (E + 128);
-        unsigned *cand = reinterpret_cast<unsigned *>(row + E);
         for (int t = t_begin + warp; t < t_end; t += nw) {
-            for (int e = lane; e < E; e += 32) row[e] = __ldcg(a.logits + (size_t)t * E + e);
+            if (E <= 512) stage_logits<16>(a.logits + (size_t)t * E, row, E, lane);
+            else stage_logits<32>(a.logits + (size_t)t * E, row, E, lane);
             __syncwarp();
+            route_clock(a.stamps, 1, t == 0);
             int me;
             float mg;
+            unsigned *cand = reinterpret_cast<unsigned *>(row + E);
             if (E <= 512) topk_threshold<16>(row, E, k, me, mg, cand);
             else topk_threshold<32>(row, E, k, me, mg, cand);
+            route_clock(a.stamps, 2, t == 0);
             if (lane < k) {
                 a.idx[(size_t)t * k + lane] = me;
                 a.gate[(size_t)t * k + lane] = mg;
+                if (idx_s) idx_s[t * k + lane] = me;
             }
             __syncwarp();
         }
@@ -146,6 +223,7 @@ __device__ void topk_phase(const RouteArgs &a, unsigned char *smem, int t_begin,
                 taken[bi >> 5] |= 1u << (bi & 31);
                 selv[j] = bv;
                 a.idx[(size_t)t * k + j] = bi;
+                if (idx_s) idx_s[t * k + j] = bi;
             }
             __syncwarp();
         }
@@ -157,7 +235,7 @@ __device__ void topk_phase(const RouteArgs &a, unsigned char *smem, int t_begin,
 // Dense-batched plan: active expert a (ascending id, the shared expert last)
 // owns slots a*T .. a*T+T-1, one per token of the batch; its gate for token t is
 // the routing gate if t selected it, else 0.
-__device__ void plan_dense(const RouteArgs &a, unsigned char *smem)
+__device__ __forceinline__ void plan_dense(const RouteArgs &a, unsigned char *smem)
 {
     const int tid = threadIdx.x;
     const int E = a.E, k = a.k, T = a.T, tt = a.tt;
@@ -205,7 +283,119 @@ __device__ void plan_dense(const RouteArgs &a, unsigned char *smem)
     }
 }
 
-__device__ void plan_phase(const RouteArgs &a, unsigned char *smem)
+// Plan for at most 64 tokens with four barriers: per-expert counts and 64-bit
+// token masks (shared-memory atomics); a block-wide scan of the counts and of
+// the group counts (thread i owns experts EPT i .. EPT i + EPT - 1, EPT = E / 256
+// rounded up; warp totals through shared memory, read back by every thread)
+// that also writes the groups; then
+// every selection's slot is its expert's offset plus the number of earlier
+// tokens in the expert's mask, so slots follow token order inside an expert.
+// `local`: the selections are already in idx_s (this CTA selected every token).
+__device__ __forceinline__ void plan_small(const RouteArgs &a, unsigned char *smem, int *idx_s, bool local)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = kThreads / 32;
+    const int E = a.E, k = a.k, T = a.T, tt = a.tt, n = T * k;
+    unsigned long long *mask = reinterpret_cast<unsigned long long *>(smem);
+    int *cnt = reinterpret_cast<int *>(mask + E);
+    int *off = cnt + (E + 1);
+    int *wsum = off + (E + 1);  // [2][nw] warp totals of counts and groups
+    if (!local)
+        for (int i0 = tid; i0 < n; i0 += 4 * kThreads) {
+            int v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) v[q] = i0 + q * kThreads < n ? __ldcg(a.idx + i0 + q * kThreads) : 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (i0 + q * kThreads < n) idx_s[i0 + q * kThreads] = v[q];
+        }
+    for (int e = tid; e < E; e += kThreads) {
+        cnt[e] = 0;
+        mask[e] = 0ull;
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += kThreads) {
+        const int e = idx_s[i];
+        atomicAdd(&cnt[e], 1);
+        atomicOr(&mask[e], 1ull << (i / k));
+    }
+    __syncthreads();
+    route_clock(a.stamps, 5, true);
+    // experts EPT tid .. EPT tid + EPT - 1 (E <= 1024 = 4 x 256: up to four each)
+    const int EPT = (E + kThreads - 1) / kThreads, eb = tid * EPT;
+    int c[4], cs = 0, gs = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        c[q] = q < EPT && eb + q < E ? cnt[eb + q] : 0;
+        cs += c[q];
+        gs += (c[q] + tt - 1) / tt;
+    }
+    int ci = cs, gi = gs;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, ci, o), w = __shfl_up_sync(0xffffffffu, gi, o);
+        if (lane >= o) {
+            ci += u;
+            gi += w;
+        }
+    }
+    if (lane == 31) {
+        wsum[warp] = ci;
+        wsum[nw + warp] = gi;
+    }
+    __syncthreads();
+    int co = ci - cs, go = gi - gs, slots = 0, routed_groups = 0;
+#pragma unroll
+    for (int w = 0; w < nw; ++w) {
+        const int a0 = wsum[w], a1 = wsum[nw + w];
+        if (w < warp) {
+            co += a0;
+            go += a1;
+        }
+        slots += a0;
+        routed_groups += a1;
+    }
+    const int shared_groups = a.has_shared ? (T + tt - 1) / tt : 0;
+    const bool bad = routed_groups + shared_groups > a.max_groups || slots != n;
+    if (bad) {
+        if (tid == 0) {
+            atomicExch(a.err, (int)MOE_ERR_DEVICE);
+            *a.n_groups = 0;
+        }
+        return;  // uniform: every thread computed the same totals
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int e = eb + q;
+        if (q < EPT && e < E) {
+            off[e] = co;
+            a.cnt[e] = c[q];
+            a.off[e] = co;
+            for (int j = 0; j * tt < c[q]; ++j) a.groups[go + j] = make_int4(e, co + j * tt, min(tt, c[q] - j * tt), 0);
+            co += c[q];
+            go += (c[q] + tt - 1) / tt;
+        }
+    }
+    for (int j = tid; j < shared_groups; j += kThreads)
+        a.groups[routed_groups + j] = make_int4(E, n + j * tt, min(tt, T - j * tt), 0);
+    if (tid == 0) {
+        a.cnt[E] = a.has_shared ? T : 0;
+        a.off[E] = n;
+        *a.n_groups = routed_groups + shared_groups;
+    }
+    __syncthreads();
+    route_clock(a.stamps, 6, true);
+    route_clock(a.stamps, 7, true);
+    for (int i = tid; i < n; i += kThreads) {
+        const int t = i / k, e = idx_s[i];
+        const int pos = off[e] + __popcll(mask[e] & ((1ull << t) - 1ull));
+        a.perm_tok[pos] = t;
+        a.slot_pos[i] = pos;
+    }
+    for (int t = tid; t < (a.has_shared ? T : 0); t += kThreads) a.perm_tok[n + t] = t;
+    route_clock(a.stamps, 8, true);
+}
+
+__device__ __forceinline__ void plan_phase(const RouteArgs &a, unsigned char *smem)
 {
     const int tid = threadIdx.x;
     const int E = a.E, k = a.k, T = a.T, tt = a.tt;
@@ -215,10 +405,25 @@ __device__ void plan_phase(const RouteArgs &a, unsigned char *smem)
     int *run = off + (E + 1);
     int *gbase = run + (E + 1);
     int *tmp = gbase + (E + 1);
+    // the selections, read three times below, into shared memory once when they
+    // fit (four loads in flight per thread), else read from L2 each time
+    int *idx_s = tmp + 64;
+    const bool cached = T * k <= kPlanIdxCache;
+    if (cached)
+        for (int i0 = tid; i0 < T * k; i0 += 4 * kThreads) {
+            int v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) v[q] = i0 + q * kThreads < T * k ? __ldcg(a.idx + i0 + q * kThreads) : 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (i0 + q * kThreads < T * k) idx_s[i0 + q * kThreads] = v[q];
+        }
+    const int *sel = cached ? idx_s : a.idx;
     for (int e = tid; e < E; e += kThreads) { cnt[e] = 0; run[e] = 0; }
     __syncthreads();
-    for (int i = tid; i < T * k; i += kThreads) atomicAdd(&cnt[__ldcg(a.idx + i)], 1);
+    for (int i = tid; i < T * k; i += kThreads) atomicAdd(&cnt[cached ? sel[i] : __ldcg(sel + i)], 1);
     __syncthreads();
+    route_clock(a.stamps, 5, true);
     for (int e = tid; e < E; e += kThreads) {
         off[e] = cnt[e];
         gbase[e] = (cnt[e] + tt - 1) / tt;
@@ -226,6 +431,7 @@ __device__ void plan_phase(const RouteArgs &a, unsigned char *smem)
     __syncthreads();
     const int slots = block_exclusive_scan(off, E, tmp);
     const int routed_groups = block_exclusive_scan(gbase, E, tmp);
+    route_clock(a.stamps, 6, true);
     const int shared_groups = a.has_shared ? (T + tt - 1) / tt : 0;
     const int total_groups = routed_groups + shared_groups;
     if (total_groups > a.max_groups || slots != T * k) {
@@ -249,6 +455,7 @@ __device__ void plan_phase(const RouteArgs &a, unsigned char *smem)
         *a.n_groups = total_groups;
     }
     for (int t = tid; t < (a.has_shared ? T : 0); t += kThreads) a.perm_tok[T * k + t] = t;
+    route_clock(a.stamps, 7, true);
     // stable slot order: within expert e, slots follow token order
     for (int c0 = 0; c0 < T; c0 += 64) {
         const int nt = min(64, T - c0);
@@ -256,13 +463,15 @@ __device__ void plan_phase(const RouteArgs &a, unsigned char *smem)
         __syncthreads();
         for (int i = tid; i < nt * k; i += kThreads) {
             int t = c0 + i / k;
-            int e = __ldcg(a.idx + (size_t)t * k + i % k);
+            const size_t at = (size_t)t * k + i % k;
+            int e = cached ? sel[at] : __ldcg(sel + at);
             atomicOr(&mask[e], 1ull << (t - c0));
         }
         __syncthreads();
         for (int i = tid; i < nt * k; i += kThreads) {
             int t = c0 + i / k, j = i % k;
-            int e = __ldcg(a.idx + (size_t)t * k + j);
+            const size_t at = (size_t)t * k + j;
+            int e = cached ? sel[at] : __ldcg(sel + at);
             unsigned long long below = (t - c0) ? (mask[e] & ((1ull << (t - c0)) - 1ull)) : 0ull;
             int pos = off[e] + run[e] + __popcll(below);
             a.perm_tok[pos] = t;
@@ -272,101 +481,227 @@ __device__ void plan_phase(const RouteArgs &a, unsigned char *smem)
         for (int e = tid; e < E; e += kThreads) run[e] += __popcll(mask[e]);
         __syncthreads();
     }
+    route_clock(a.stamps, 8, true);
+}
+
+// Sum over the warp's lanes of each of v[0..31], transposed: lane l ends with
+// the total of v[l] in v[0] (31 shuffles in five halving steps).
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[32])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int j = 0; j < o; ++j) {
+            const float send = up ? v[j] : v[j + o];
+            const float keep = up ? v[j + o] : v[j];
+            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0];
+}
+
+// Logits of the CTA's staged router rows for the nt tokens of this pass.
+// Rows go four to a warp (each x chunk read from shared memory feeds four
+// rows); lane l takes 16-byte weight chunks l, l + 32, ... of the rows, so a
+// warp's 32 chunk loads cover consecutive bytes; when the CTA has fewer row
+// quads than warps, the chunks of a quad are split over several warps and
+// their partial sums added in warp order.
+template <bool XBF16>
+__device__ __forceinline__ void gemv_staged(const RouteArgs &a, const unsigned char *smem, const RouteSmem &m, int e0,
+                                            int nrow, int t0, int nt)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = kThreads / 32;
+    const int H = a.H, E = a.E, nch = H >> 3, NI = (nch + 31) / 32;
+    const uint16_t *wrs = reinterpret_cast<const uint16_t *>(smem + m.wr);
+    float *red = reinterpret_cast<float *>(const_cast<unsigned char *>(smem) + m.red);
+    const int nq = (nrow + 3) / 4;
+    const int wpq = nq >= nw ? 1 : nw / nq, qpp = nw / wpq;  // warps per quad, quads per pass
+    const int part = warp % wpq;
+    for (int q = warp / wpq; q < nq; q += qpp) {
+        float2 acc[4][8];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int t = 0; t < 8; ++t) acc[r][t] = make_float2(0.f, 0.f);
+        for (int i = part; i < NI; i += wpq) {
+            const int c = lane + 32 * i;
+            if (c >= nch) break;
+            float2 w[4][4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const uint4 v = 4 * q + r < nrow
+                                    ? *reinterpret_cast<const uint4 *>(wrs + (size_t)(4 * q + r) * H + c * 8)
+                                    : make_uint4(0, 0, 0, 0);
+                w[r][0] = make_float2(bf16lo(v.x), bf16hi(v.x));
+                w[r][1] = make_float2(bf16lo(v.y), bf16hi(v.y));
+                w[r][2] = make_float2(bf16lo(v.z), bf16hi(v.z));
+                w[r][3] = make_float2(bf16lo(v.w), bf16hi(v.w));
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                if (t < nt) {
+                    float2 x[4];
+                    x_chunk<XBF16>(smem, H, t, c, x);
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        float2 s2 = acc[r][t];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) s2 = qd::fma2(w[r][h], x[h], s2);
+                        acc[r][t] = s2;
+                    }
+                }
+            }
+        }
+        float v[32];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int t = 0; t < 8; ++t) v[r * 8 + t] = acc[r][t].x + acc[r][t].y;
+        const float sum = warp_transpose_sum(v);  // lane = 8 r + t
+        const int r = lane >> 3, t = lane & 7;
+        if (wpq == 1) {
+            if (t < nt && 4 * q + r < nrow) a.logits[(size_t)(t0 + t) * E + e0 + 4 * q + r] = sum;
+        } else {
+            red[(q * wpq + part) * 32 + lane] = sum;
+        }
+    }
+    if (wpq > 1) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < nq * 32; i += kThreads) {
+            const int q = i >> 5, l = i & 31, r = l >> 3, t = l & 7;
+            float sum = 0.f;
+            for (int p = 0; p < wpq; ++p) sum += red[(q * wpq + p) * 32 + l];
+            if (t < nt && 4 * q + r < nrow) a.logits[(size_t)(t0 + t) * E + e0 + 4 * q + r] = sum;
+        }
+    }
+}
+
+// Logits of rows [e0, e1) for the nt tokens of this pass, router rows read from
+// global memory (CTAs whose rows do not fit the staging area), one row per warp.
+template <bool XBF16>
+__device__ __forceinline__ void gemv_global(const RouteArgs &a, const unsigned char *xs, int e0, int e1, int t0, int nt)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = kThreads / 32;
+    const int H = a.H, E = a.E, nch = H >> 3;
+    for (int e = e0 + warp; e < e1; e += nw) {
+        const uint16_t *wrow = a.wr + (size_t)e * H;
+        float2 acc[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) acc[t] = make_float2(0.f, 0.f);
+        for (int cb = 0; cb < nch; cb += 32 * 8) {
+            uint4 wv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                int c = cb + lane + 32 * i;
+                wv[i] = c < nch ? ldg_nc16(wrow + c * 8) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                int c = cb + lane + 32 * i;
+                if (c >= nch) break;
+                const float2 w[4] = {make_float2(bf16lo(wv[i].x), bf16hi(wv[i].x)),
+                                     make_float2(bf16lo(wv[i].y), bf16hi(wv[i].y)),
+                                     make_float2(bf16lo(wv[i].z), bf16hi(wv[i].z)),
+                                     make_float2(bf16lo(wv[i].w), bf16hi(wv[i].w))};
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    if (t < nt) {
+                        float2 x[4];
+                        x_chunk<XBF16>(xs, H, t, c, x);
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) acc[t] = qd::fma2(w[h], x[h], acc[t]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            float v = acc[t].x + acc[t].y;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0 && t < nt) a.logits[(size_t)(t0 + t) * E + e] = v;
+        }
+    }
+}
+
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     tc::smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+                 : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads) route_kernel(const RouteArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_last;
-    float *xs = reinterpret_cast<float *>(smem);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = kThreads / 32;
+    __shared__ __align__(8) uint64_t wr_bar, x_bar;
+    route_event(a.stamps, 0);
     const int H = a.H, E = a.E;
-    // CTA b takes token block b % ntb (rt tokens) and a slice of the expert rows,
-    // so every CTA stages its tokens once and the grid covers all SMs
-    // token blocks of rt tokens, dealt to NB block groups (more blocks than
-    // groups: a CTA handles blocks j, j + NB, ...)
+    // CTA b takes token block b % NB and a slice of the expert rows (token
+    // blocks of rt tokens dealt to NB block groups: with more blocks than
+    // groups a CTA takes blocks j, j + NB, ...), so every CTA stages its tokens
+    // once and the grid covers the SMs
     const int ntb = (a.T + a.rt - 1) / a.rt, NB = min(ntb, kRouteMaxBlockGroups), per = gridDim.x / NB;
     const int tb = blockIdx.x % NB, slice = blockIdx.x / NB;
     const int e0 = slice < per ? (int)((long long)E * slice / per) : E;
     const int e1 = slice < per ? (int)((long long)E * (slice + 1) / per) : E;
-    const int nch = H >> 3;  // 16-byte chunks of 8 bf16 in a router row
-    for (int t0 = tb * a.rt; t0 < a.T && e1 > e0; t0 += NB * a.rt) {
-        const int nt = min(a.rt, a.T - t0);
-        __syncthreads();
-        for (int i0 = threadIdx.x; i0 < nt * nch; i0 += 4 * kThreads) {
-            float4 lo[4], hi[4];  // four chunks' loads in flight before any store
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int i = i0 + q * kThreads;
-                if (i >= nt * nch) break;
-                const int t = i / nch, c = i - t * nch;
-                if (a.x_dtype == MOE_DT_BF16) {
-                    uint4 v = ldg_nc16(reinterpret_cast<const uint16_t *>(a.x) + (size_t)(t0 + t) * H + c * 8);
-                    lo[q] = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
-                    hi[q] = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
-                } else {
-                    const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(a.x) +
-                                                                       (size_t)(t0 + t) * H + c * 8);
-                    lo[q] = __ldg(p);
-                    hi[q] = __ldg(p + 1);
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int i = i0 + q * kThreads;
-                if (i >= nt * nch) break;
-                const int t = i / nch, c = i - t * nch;
-                float4 *d = reinterpret_cast<float4 *>(xs + (size_t)t * H + c * 8);
-                d[0] = lo[q];
-                d[1] = hi[q];
-            }
+    const RouteSmem m = route_smem(H, a.rt, E, (E + per - 1) / per);
+    const bool xbf16 = a.x_dtype == MOE_DT_BF16;
+    const uint32_t xrow = (uint32_t)H * (xbf16 ? 2u : 4u);
+    // bulk copies: the CTA's router rows (contiguous, once) and each pass's x
+    // rows as given, all issued by one thread and landing together
+    const bool staged = m.staged && e1 > e0;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&wr_bar, 1);
+        tc::mbar_init(&x_bar, 1);
+        tc::fence_mbar_init();
+        if (staged) {
+            const uint32_t bytes = (uint32_t)((e1 - e0) * H * 2);
+            tc::mbar_arrive_expect_tx(&wr_bar, bytes);
+            bulk_g2s(smem + m.wr, a.wr + (size_t)e0 * H, bytes, &wr_bar);
         }
-        __syncthreads();
-        for (int e = e0 + warp; e < e1; e += nw) {
-            const uint16_t *wrow = a.wr + (size_t)e * H;
-            float acc[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) acc[t] = 0.f;
-            for (int cb = 0; cb < nch; cb += 32 * 8) {
-                uint4 wv[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    int c = cb + lane + 32 * i;
-                    wv[i] = c < nch ? ldg_nc16(wrow + c * 8) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    int c = cb + lane + 32 * i;
-                    if (c >= nch) break;
-                    float w0 = bf16lo(wv[i].x), w1 = bf16hi(wv[i].x), w2 = bf16lo(wv[i].y), w3 = bf16hi(wv[i].y);
-                    float w4 = bf16lo(wv[i].z), w5 = bf16hi(wv[i].z), w6 = bf16lo(wv[i].w), w7 = bf16hi(wv[i].w);
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        if (t < nt) {
-                            const float4 *xp = reinterpret_cast<const float4 *>(xs + (size_t)t * H + c * 8);
-                            float4 x0 = xp[0], x1 = xp[1];
-                            float s = acc[t];
-                            s = fmaf(w0, x0.x, s); s = fmaf(w1, x0.y, s);
-                            s = fmaf(w2, x0.z, s); s = fmaf(w3, x0.w, s);
-                            s = fmaf(w4, x1.x, s); s = fmaf(w5, x1.y, s);
-                            s = fmaf(w6, x1.z, s); s = fmaf(w7, x1.w, s);
-                            acc[t] = s;
-                        }
-                    }
-                }
+    }
+    for (int t0 = tb * a.rt, pass = 0; t0 < a.T && e1 > e0; t0 += NB * a.rt, ++pass) {
+        const int nt = min(a.rt, a.T - t0);
+        __syncthreads();  // the previous pass's x is consumed (and the barriers initialised)
+        if (threadIdx.x == 0) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc::mbar_arrive_expect_tx(&x_bar, (uint32_t)nt * xrow);
+            for (int t = 0; t < nt; ++t)
+                bulk_g2s(smem + (size_t)t * xrow, static_cast<const unsigned char *>(a.x) + (size_t)(t0 + t) * xrow,
+                         xrow, &x_bar);
+        }
+        // bounded waits; the CTA agrees on the outcome so its barriers stay uniform
+        bool ok = tc::mbar_wait(&x_bar, pass & 1);
+        if (staged && pass == 0) ok = tc::mbar_wait(&wr_bar, 0) && ok;
+        if (__syncthreads_or(!ok)) {
+            // record the error, give the copies in flight a second bounded wait
+            // before shared memory is reused, and skip the logits
+            if (threadIdx.x == 0) {
+                if (a.err) atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
+                tc::mbar_wait(&x_bar, pass & 1);
+                if (staged) tc::mbar_wait(&wr_bar, 0);
             }
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                float v = acc[t];
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0 && t < nt) a.logits[(size_t)(t0 + t) * E + e] = v;
-            }
+            __syncthreads();
+            break;
+        }
+        if (pass == 0) route_event(a.stamps, 1);
+        if (staged) {
+            if (xbf16) gemv_staged<true>(a, smem, m, e0, e1 - e0, t0, nt);
+            else gemv_staged<false>(a, smem, m, e0, e1 - e0, t0, nt);
+        } else {
+            if (xbf16) gemv_global<true>(a, smem, e0, e1, t0, nt);
+            else gemv_global<false>(a, smem, e0, e1, t0, nt);
         }
     }
     // the last CTA of this token block selects its tokens' experts; the last
     // token block to finish builds the plan (tickets: [0] blocks, [2 + tb] CTAs)
     __syncthreads();
+    route_event(a.stamps, 2);
     if (threadIdx.x == 0) {
         __threadfence();
         const int ticket = atomicAdd(a.ticket + 2 + tb, 1);
@@ -375,23 +710,38 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const RouteArgs a)
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    for (int t0 = tb * a.rt; t0 < a.T; t0 += NB * a.rt) topk_phase(a, smem, t0, min(a.T, t0 + a.rt));
+    route_clock(a.stamps, 0, tb == 0);
+    // the short plan (<= 64 tokens) reads the selections from shared memory;
+    // with one block group this CTA selects every token and writes them there
+    const bool small = a.do_plan && !a.dense && a.T <= kSmallPlanT && a.T * a.k <= kPlanIdxCache && a.k <= 32 &&
+                       E <= 1024;
+    int *idx_s = reinterpret_cast<int *>(smem + m.idx);
+    for (int t0 = tb * a.rt; t0 < a.T; t0 += NB * a.rt)
+        topk_phase(a, smem, t0, min(a.T, t0 + a.rt), small && NB == 1 ? idx_s : nullptr);
     __syncthreads();
+    route_event(a.stamps, 3);
+    route_clock(a.stamps, 3, tb == 0);
     if (threadIdx.x == 0) {
         a.ticket[2 + tb] = 0;
-        __threadfence();
-        const int ticket = atomicAdd(a.ticket, 1);
-        s_last = ticket == NB - 1;
+        if (NB > 1) {  // one block group: this CTA is already the last
+            __threadfence();
+            const int ticket = atomicAdd(a.ticket, 1);
+            s_last = ticket == NB - 1;
+        }
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
+    if (NB > 1) __threadfence();
+    route_clock(a.stamps, 4, true);
     if (a.do_plan) {
         __syncthreads();
         if (a.dense) plan_dense(a, smem);
+        else if (small) plan_small(a, smem, idx_s, NB == 1);
         else plan_phase(a, smem);
     }
     __syncthreads();
+    route_event(a.stamps, 4);
+    route_clock(a.stamps, 9, true);
     if (threadIdx.x == 0) *a.ticket = 0;
 }
 
@@ -403,21 +753,16 @@ int route_tokens_per_pass(int H)
     return rt < 1 ? 1 : (rt > 8 ? 8 : rt);
 }
 
-size_t route_smem_bytes(int H, int rt, int E)
+size_t route_smem_bytes(int H, int rt, int E, int grid, int T)
 {
-    size_t stage = (size_t)rt * H * sizeof(float);
-    size_t topk = (size_t)2 * (kThreads / 32) * E * sizeof(float) + (kThreads / 32) * 32 * sizeof(uint32_t);
-    const size_t topk_thr = (size_t)(kThreads / 32) * (E + 128) * sizeof(float);  // row + candidates per warp
-    if (topk_thr > topk) topk = topk_thr;
-    size_t plan = (size_t)E * 8 + (size_t)4 * (E + 1) * sizeof(int) + 64 * sizeof(int);
-    size_t m = stage > topk ? stage : topk;
-    return m > plan ? m : plan;
+    const int NB = min((T + rt - 1) / rt, kRouteMaxBlockGroups), per = grid / NB;
+    return route_smem(H, rt, E, (E + per - 1) / per).total;
 }
 
 int route_grid(int E, int T, int rt, int num_sms)
 {
     const int ntb = min((T + rt - 1) / rt, kRouteMaxBlockGroups);  // block groups
-    int per = (E + (kThreads / 32) - 1) / (kThreads / 32);  // row slices: >= one warp's row each
+    int per = (E + 3) / 4;  // row slices: at least one quad of rows each
     if (per * ntb > num_sms) per = num_sms / ntb > 0 ? num_sms / ntb : 1;
     return per * ntb;
 }
@@ -429,7 +774,7 @@ cudaError_t route_set_attributes()
 
 cudaError_t launch_route(const RouteArgs &a, int grid, cudaStream_t s)
 {
-    size_t smem = route_smem_bytes(a.H, a.rt, a.E);
+    size_t smem = route_smem_bytes(a.H, a.rt, a.E, grid, a.T);
     route_kernel<<<grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();
 }

@@ -101,6 +101,7 @@ extern "C" moe_status moe_route_topk_noalloc(const void *x, moe_dtype x_dtype, c
     a.idx = idx_out;
     a.gate = gate_out;
     a.do_plan = 0;
+    a.err = a.ticket + 1;  // word 1: a timed-out wait
     if (cudaMemsetAsync(a.ticket, 0, 64, s) != cudaSuccess) return MOE_ERR_CUDA;  // the tickets (words 0, 2..)
     return launch_route(a, route_grid(n_experts, n_tokens, a.rt, sms), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -170,7 +170,7 @@ __device__ __forceinline__ void grid_event(long long *st, int ev)
 // copies the whole buffer into shared memory with one bulk copy, which every
 // thread waits for.  One poller per CTA and one copy request stream keep the
 // L2 lines of the buffer from being hammered by every warp of the grid.
-__device__ bool s1_exchange(unsigned *cnt, const void *src, void *dst, uint32_t bytes, uint64_t *bar, int32_t *err,
+__device__ __forceinline__ bool s1_exchange(unsigned *cnt, const void *src, void *dst, uint32_t bytes, uint64_t *bar, int32_t *err,
                             int *flags, int armbit)
 {
     __syncthreads();  // this CTA's part is written
@@ -311,7 +311,7 @@ __device__ __forceinline__ bool s1_wait(uint64_t *bar, int32_t *err, int *fail)
 // from shared memory, then the gate and the up dot products.  The body is
 // small and shared by every iteration, so it stays in the instruction cache.
 template <int FMT>
-__device__ void s1_gateup(const FusedArgs &a, const S1Layout &L, uint8_t *smem, const Seg *seg, int nseg,
+__device__ __forceinline__ void s1_gateup(const FusedArgs &a, const S1Layout &L, uint8_t *smem, const Seg *seg, int nseg,
                           int npairs, const float4 *xs4, const float *xsum, const int *grp_e, int *fail)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -398,7 +398,7 @@ __device__ void s1_gateup(const FusedArgs &a, const S1Layout &L, uint8_t *smem, 
 }
 
 // ---- Q5_1 down: per-unit sums of every group's h (staged, unit-swizzled) -----------
-__device__ void s1_h_sums(const S1Layout &L, uint8_t *smem, int I)
+__device__ __forceinline__ void s1_h_sums(const S1Layout &L, uint8_t *smem, int I)
 {
     const int NU = I >> 5;
     const float4 *hs4 = reinterpret_cast<const float4 *>(smem + L.h);
@@ -460,7 +460,7 @@ __device__ __forceinline__ float s1_row_dot(const FusedArgs &a, const S1Layout &
 }
 
 template <int FMT>
-__device__ void s1_down(const FusedArgs &a, const S1Layout &L, uint8_t *smem, int r0, int nd, const int *grp_e,
+__device__ __forceinline__ void s1_down(const FusedArgs &a, const S1Layout &L, uint8_t *smem, int r0, int nd, const int *grp_e,
                         const float *grp_gate, int *fail)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -668,8 +668,15 @@ __global__ void __launch_bounds__(kS1Threads, 1) stream1_kernel(const FusedArgs 
     }
     __syncthreads();
     const bool routed = flags[0] == 0;
+    // the gate/up chunks first: their bytes are needed first, and the SM's copy
+    // engine and the memory system serve requests roughly in issue order; the
+    // down rows (not read before the h hand-over) are issued after a barrier
     if (routed && lane == 0)
-        for (int it = warp; it < nseg + L.ng; it += kS1Warps)
+        for (int it = warp; it < nseg; it += kS1Warps)
+            issue_item(src, Ls, smem, seg, nseg, it, true, k, grp_e, r0, nd, flags + 1);
+    __syncthreads();
+    if (routed && lane == 0)
+        for (int it = nseg + warp; it < nseg + L.ng; it += kS1Warps)
             issue_item(src, Ls, smem, seg, nseg, it, true, k, grp_e, r0, nd, flags + 1);
     if (stamp) a.stamps[28] = clock64();
     if (stamp) a.stamps[4] = clock64();

@@ -168,8 +168,9 @@ size_t moe_route_workspace_bytes(int n_tokens, int n_experts);
  *   workspace device, moe_route_workspace_bytes(n_tokens, n_experts) bytes,
  *             owned by the caller; its contents need no initialisation
  * hidden % 8 == 0, 1 <= top_k <= n_experts <= 1024.  More than 64 bf16 tokens
- * run the router as a tensor-core GEMM; if one of its bounded waits runs out,
- * int32 word 1 of the workspace holds MOE_ERR_TIMEOUT afterwards. */
+ * run the router as a tensor-core GEMM.  If one of the kernels' bounded waits
+ * (the GEMM's pipeline, or the bulk copy of router rows into shared memory)
+ * runs out, int32 word 1 of the workspace holds MOE_ERR_TIMEOUT afterwards. */
 moe_status moe_route_topk(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
                           int n_tokens, int hidden, int n_experts, int top_k, int32_t *idx_out,
                           float *gate_out, void *workspace, size_t workspace_bytes,
