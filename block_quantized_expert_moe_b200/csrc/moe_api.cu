@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -52,6 +53,8 @@ struct moe_pack {
     int pdl = 1;                  // launch it as a programmatic dependent of the previous kernel
     int sgm = -1;                 // streamed grouped matvecs usable (-1: not yet checked)
     SgmProj sg_gu{}, sg_dn{};
+    int dtc = -1;                 // tensor-core grouped decode usable (-1: not yet checked)
+    DecodeTcMaps dtc_maps{};
     bool has_prefill = false;     // tensor-core prefill workspace present
     PrefillWorkspace pws;
 };
@@ -144,6 +147,7 @@ moe_status init_device(int dev)
     if (fused_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (stream1_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (sgm_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
+    if (decode_tc_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_nvfp4_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_q8_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
@@ -286,6 +290,38 @@ moe_status dev_alloc(moe_pack *p, size_t bytes, void **out)
     return MOE_OK;
 }
 
+float half_to_float(uint16_t h)
+{
+    const int e = (h >> 10) & 31, m = h & 1023;
+    const float mag = e == 0 ? std::ldexp((float)m, -24) : e == 31 ? INFINITY : std::ldexp((float)(1024 + m), e - 25);
+    return (h & 0x8000) ? -mag : mag;
+}
+
+// Whether every weight d q (Q8_0, IQ4_NL: |q| <= 128) or d q + m (Q5_1,
+// q <= 31) of the scale plane `sc` is an fp16 normal number or zero: the
+// tensor-core decode path expands the blocks to fp16.  NVFP4 always is (a code
+// of at most 12 halves times an E4M3 scale: at most 5376, at least 2^-10).
+bool f16_safe(int fmt, const std::vector<uint8_t> &sc, int64_t stride, int64_t used, int n_slots)
+{
+    if (fmt == MOE_FMT_NVFP4) return true;
+    for (int s = 0; s < n_slots; ++s) {
+        const uint8_t *p = sc.data() + (int64_t)s * stride;
+        if (fmt == MOE_FMT_Q5_1) {
+            for (int64_t i = 0; i + 4 <= used; i += 4) {
+                const float d = half_to_float((uint16_t)(p[i] | p[i + 1] << 8));
+                const float m = half_to_float((uint16_t)(p[i + 2] | p[i + 3] << 8));
+                if (!(std::fabs(d) * 31.f + std::fabs(m) <= 60000.f)) return false;
+            }
+        } else {
+            for (int64_t i = 0; i + 2 <= used; i += 2) {
+                const float d = std::fabs(half_to_float((uint16_t)(p[i] | p[i + 1] << 8)));
+                if (!(d == 0.f || (d >= 0x1p-14f && d * 128.f <= 60000.f))) return false;
+            }
+        }
+    }
+    return true;
+}
+
 // Build one projection's planes for all slots (routed experts + shared).
 moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, const uint8_t *blocks,
                       const uint8_t *shared_blocks, const float *ts, int n_slots, const uint8_t *perm)
@@ -321,6 +357,7 @@ moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, con
     });
     for (char c : ok)
         if (!c) return MOE_ERR_INVALID_ARG;
+    dp.f16_ok = f16_safe(fmt, hs, dp.sc_stride, (int64_t)rows * dp.sc_row, n_slots);
     void *dq, *ds, *dh = nullptr, *dt = nullptr;
     moe_status st;
     if ((st = dev_alloc(p, hq.size(), &dq)) != MOE_OK) return st;
@@ -365,7 +402,8 @@ moe_status build_workspace(moe_pack *p)
         {(void **)&w.slot_pos, T * k * 4}, {(void **)&w.groups, (int64_t)w.max_groups * 16},
         {(void **)&w.n_groups, 4}, {(void **)&w.ticket, 64}, {(void **)&w.err, 4}, {(void **)&w.bar, 8},
         {(void **)&w.h, slots * p->I * 4}, {(void **)&w.y, slots * p->H * 4},
-        {(void **)&w.dgate, slots * 4}, {(void **)&w.n_dense_rows, 4},
+        {(void **)&w.dgate, slots * 4}, {(void **)&w.n_dense_rows, 4}, {(void **)&w.slot_scale, slots * 4},
+        {(void **)&w.xg, slots * p->H * 2},
         {(void **)&w.xcnt, 16},
     };
     int64_t total = 0;
@@ -454,6 +492,7 @@ const char *moe_status_string(moe_status s)
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_TIMEOUT: return "device-side wait timed out";
     case MOE_ERR_DEVICE: return "device-side plan error";
+    case MOE_ERR_RANGE: return "value outside the fp16 range of the tensor-core decode path";
     default: return "unknown status";
     }
 }
@@ -667,9 +706,20 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
                       ? 1
                       : 0;
     }
+    if (pm->dtc < 0) {
+        const int64_t slots = std::max<int64_t>((int64_t)p->max_tokens * (p->max_top_k + 1), 1);
+        pm->dtc = decode_tc_supported(p->gu, p->dn, p->H, p->I, p->max_tokens, p->max_top_k) &&
+                          decode_tc_maps(&pm->dtc_maps, p->gu, p->dn, p->E + (p->has_shared ? 1 : 0), w.xg, w.h,
+                                         (int)slots, p->H, p->I)
+                      ? 1
+                      : 0;
+    }
+    // 2..64 tokens: the tensor-core grouped decode when the pack's weights are
+    // fp16-representable
+    const bool use_dtc = path == MOE_PATH_DECODE && T >= 2 && T <= kDecodeTcMaxN && pm->dtc == 1;
     // one token: the single-token kernels; 2..8 tokens: the fused kernel unless
-    // the streamed grouped matvecs apply
-    if (path == MOE_PATH_DECODE && T <= kFusedMaxT && k <= kFusedMaxK && (T == 1 || pm->sgm != 1)) {
+    // the streamed grouped matvecs or the tensor-core grouped decode apply
+    if (path == MOE_PATH_DECODE && T <= kFusedMaxT && k <= kFusedMaxK && (T == 1 || (pm->sgm != 1 && !use_dtc))) {
         FusedArgs fa{};
         fa.x = x;
         fa.x_dtype = x_dtype;
@@ -744,7 +794,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     // tokens per work group: 8 unless a single token, or 8 staged fp32 rows of
     // the longer reduction would not fit in shared memory
     const int kmax = std::max(p->H, p->I);
-    const int tt = (T == 1 || (size_t)8 * kmax * 4 * 33 / 32 > 200 * 1024) ? 1 : 8;
+    const int tt = use_dtc ? kDecodeTcMaxN : (T == 1 || (size_t)8 * kmax * 4 * 33 / 32 > 200 * 1024) ? 1 : 8;
     int pbase = -1;
     if (pm->prof_on && (size_t)pm->prof_used + 5 <= pm->prof_ev.size()) {
         pbase = pm->prof_used;
@@ -786,7 +836,21 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     if (st != MOE_OK) return st;
     prof_mark(pm, pbase, 1, s);
 
-    if (path == MOE_PATH_DECODE && T >= 2 && tt == 8 && pm->sgm == 1) {
+    if (use_dtc) {
+        // x into fp16 slot rows, then the two tensor-core GEMMs (y per slot);
+        // the combine below sums each token's slots
+        st = check_launch(launch_decode_tc_gather(x, x_dtype, T, p->H, k, p->has_shared, w.slot_pos, w.xg,
+                                                  w.slot_scale, s));
+        if (st != MOE_OK) return st;
+        st = check_launch(launch_decode_tc(pm->dtc_maps, true, p->gu, w.groups, w.n_groups, p->H, p->I, p->ct_gu,
+                                           w.slot_scale, w.h, w.y, w.err, p->num_sms, s));
+        if (st != MOE_OK) return st;
+        prof_mark(pm, pbase, 2, s);
+        st = check_launch(launch_decode_tc(pm->dtc_maps, false, p->dn, w.groups, w.n_groups, p->H, p->I, p->ct_dn,
+                                           w.slot_scale, w.h, w.y, w.err, p->num_sms, s));
+        if (st != MOE_OK) return st;
+        prof_mark(pm, pbase, 3, s);
+    } else if (path == MOE_PATH_DECODE && T >= 2 && tt == 8 && pm->sgm == 1) {
         st = check_launch(launch_sgm(pm->sg_gu, p->gu, w.groups, w.n_groups, w.perm_tok, x, x_dtype, w.h, p->I,
                                      p->I, true, p->ct_gu, w.err, p->num_sms, s));
         if (st != MOE_OK) return st;

@@ -41,6 +41,9 @@ struct DevProj {
     const uint8_t *sr = nullptr;
     int64_t sr_stride = 0;
     int sr_row = 0;
+    // every weight of the projection is an fp16 normal number or zero (the
+    // tensor-core decode path expands blocks to fp16)
+    bool f16_ok = false;
 };
 
 // Byte offset of E4M3 scale q (0..3) of row r in 64-wide K step s, in the
@@ -68,12 +71,22 @@ struct Workspace {
     int32_t *err = nullptr;      // sticky device error (moe_status)
     float *dgate = nullptr;      // dense-batched plan: per slot gate (0 when not routed)
     int32_t *n_dense_rows = nullptr;
-    float *h = nullptr;          // [slots x I]
+    float *h = nullptr;          // [slots x I] (tensor-core decode: fp16 h)
     float *y = nullptr;          // [slots x H]
+    uint16_t *xg = nullptr;      // [slots x H] tensor-core decode: fp16 x slot rows
+    float *slot_scale = nullptr; // [slots] tensor-core decode: power-of-two scale of the slot's x
     int max_groups = 0;
     // single-token streaming kernel: {finished-CTA ticket, logits arrivals, h
     // arrivals}; all zero between launches (the last CTA to finish resets them)
     unsigned *xcnt = nullptr;
+};
+
+// Tensor-core grouped decode (2 to kDecodeTcMaxN tokens): TMA maps of the
+// fp16 slot rows of x and of h (workspace buffers, fixed per pack).
+constexpr int kDecodeTcMaxN = 64;
+struct DecodeTcMaps {
+    CUtensorMap xg, h;
+    CUtensorMap gu[3], dn[3];  // codes, row-major scales, fifth bits of each projection
 };
 
 struct RouteArgs {
@@ -229,6 +242,17 @@ bool sgm_prepare(const DevProj &w, int n_slots, bool gateup, SgmProj *out);
 int sgm_max_groups();
 int sgm_stages(const SgmProj &p, int K);
 cudaError_t sgm_set_attributes();
+
+// Tensor-core grouped decode (decode_tc.cu)
+bool decode_tc_supported(const DevProj &gu, const DevProj &dn, int H, int I, int max_tokens, int max_top_k);
+cudaError_t decode_tc_set_attributes();
+bool decode_tc_maps(DecodeTcMaps *m, const DevProj &gu, const DevProj &dn, int n_experts, const void *xg,
+                    const void *h16, int slots, int H, int I);
+cudaError_t launch_decode_tc_gather(const void *x, int x_dtype, int T, int H, int k, int has_shared,
+                                    const int32_t *slot_pos, void *xg, float *slot_scale, cudaStream_t s);
+cudaError_t launch_decode_tc(const DecodeTcMaps &m, bool gateup, const DevProj &w, const int4 *groups,
+                             const int32_t *n_groups, int H, int I, const CodeTable &tab, const float *slot_scale,
+                             void *h16, float *y, int32_t *err, int grid, cudaStream_t s);
 cudaError_t launch_sgm(const SgmProj &p, const DevProj &w, const int4 *groups, const int32_t *n_groups,
                        const int32_t *perm_tok, const void *x, int x_dtype, float *out, int out_stride, int rows_out,
                        bool gateup, const CodeTable &tab, int32_t *err, int grid, cudaStream_t s);

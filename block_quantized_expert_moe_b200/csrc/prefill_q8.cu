@@ -33,6 +33,7 @@
 #include <cuda_runtime.h>
 
 #include "moe_internal.cuh"
+#include "dequant.cuh"
 #include "quant_dot.cuh"
 #include "tc_common.cuh"
 #include "tma_maps.cuh"
@@ -77,100 +78,6 @@ struct Q8GemmArgs {
     int H;
     int32_t *err;
 };
-
-__device__ __forceinline__ float byte_f(uint32_t w, int i)  // biased int8 -> float
-{
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(w), "r"(0x4B000000u), "r"(0x7650u + i));
-    return __uint_as_float(d) - 8388736.f;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
-{
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
-// One 64-wide K slice (two 32-weight blocks) of a weight row, as loaded.
-template <int FMT>
-struct DqSlice {
-    uint4 q[FMT == MOE_FMT_Q8_0 ? 4 : 2];  // codes
-    uint32_t s0, s1;                       // block scales (Q8_0 / IQ4_NL: fp16 d; Q5_1: {d, m})
-    uint32_t h0, h1;                       // Q5_1 fifth bits
-};
-
-template <int FMT>
-__device__ __forceinline__ DqSlice<FMT> dq_load(const uint8_t *qrow, const uint8_t *srow, const uint8_t *hrow, int kt)
-{
-    DqSlice<FMT> r;
-    r.h0 = r.h1 = 0;
-    if constexpr (FMT == MOE_FMT_Q8_0) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) r.q[i] = __ldg(reinterpret_cast<const uint4 *>(qrow + kt * 64) + i);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) r.q[i] = __ldg(reinterpret_cast<const uint4 *>(qrow + kt * 32) + i);
-    }
-    if constexpr (FMT == MOE_FMT_Q5_1) {
-        const uint2 sv = __ldg(reinterpret_cast<const uint2 *>(srow + kt * 8));
-        const uint2 hv = __ldg(reinterpret_cast<const uint2 *>(hrow + kt * 8));
-        r.s0 = sv.x;
-        r.s1 = sv.y;
-        r.h0 = hv.x;
-        r.h1 = hv.y;
-    } else {
-        const uint32_t sv = __ldg(reinterpret_cast<const uint32_t *>(srow + kt * 4));
-        r.s0 = sv & 0xFFFFu;
-        r.s1 = sv >> 16;
-    }
-    return r;
-}
-
-__device__ __forceinline__ float half_bits(uint32_t b) { return __half2float(__ushort_as_half((unsigned short)b)); }
-
-// The 32 weights of block u of the slice, in element order.
-template <int FMT>
-__device__ __forceinline__ void dq_block(const DqSlice<FMT> &r, int u, const CodeTable &ct, float (&v)[32])
-{
-    if constexpr (FMT == MOE_FMT_Q8_0) {
-        const float d = half_bits(u ? r.s1 : r.s0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t w = (&r.q[2 * u].x)[i];
-#pragma unroll
-            for (int b = 0; b < 4; ++b) v[4 * i + b] = byte_f(w, b) * d;
-        }
-    } else if constexpr (FMT == MOE_FMT_IQ4_NL) {
-        // element j < 16: low nibble of byte j; j >= 16: high nibble of byte j - 16
-        const float d = half_bits(u ? r.s1 : r.s0);
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            uint32_t o0, o1;
-            qd::lut16((&r.q[u].x)[s], ct, o0, o1);  // o0 = [lo0 hi0 lo1 hi1], o1 = [lo2 hi2 lo3 hi3] of bytes 4s..
-            const uint32_t oo[2] = {o0, o1};
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const uint32_t o = oo[b >> 1];
-                const float lo = __uint_as_float(qd::prmt(o, 0x4B000000u, 0x7650u + 2 * (b & 1))) - ct.magic;
-                const float hi = __uint_as_float(qd::prmt(o, 0x4B000000u, 0x7650u + 2 * (b & 1) + 1)) - ct.magic;
-                v[4 * s + b] = lo * d;
-                v[16 + 4 * s + b] = hi * d;
-            }
-        }
-    } else {  // Q5_1: q = nibble | fifth bit << 4, w = d * q + m
-        const uint32_t dm = u ? r.s1 : r.s0, hb = u ? r.h1 : r.h0;
-        const float d = half_bits(dm & 0xFFFFu), m = half_bits(dm >> 16);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const uint32_t byte = ((&r.q[u].x)[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-            const uint32_t lo = (byte & 0xFu) | (((hb >> j) & 1u) << 4);
-            const uint32_t hi = (byte >> 4) | (((hb >> (j + 16)) & 1u) << 4);
-            v[j] = fmaf(d, (float)lo, m);
-            v[16 + j] = fmaf(d, (float)hi, m);
-        }
-    }
-}
 
 template <bool GATEUP, int FMT>
 __global__ void __launch_bounds__(kQ8Threads, 1)
@@ -265,11 +172,16 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
             const uint8_t *qrow = g.qs + (int64_t)e * g.qs_stride + (int64_t)row * g.qs_row;
             const uint8_t *srow = g.sc + (int64_t)e * g.sc_stride + (int64_t)row * g.sc_row;
             const uint8_t *hrow = FMT == MOE_FMT_Q5_1 ? g.qh + (int64_t)e * g.qh_stride + (int64_t)row * g.qh_row : nullptr;
-            DqSlice<FMT> cur = dq_load<FMT>(qrow, srow, hrow, 0);
+            // the 64-wide K slice kt = blocks 2 kt, 2 kt + 1; the next slice's loads
+            // are in flight while this one is converted
+            dq::Blk<FMT> cur[2] = {dq::load_blk<FMT>(qrow, srow, hrow, 0), dq::load_blk<FMT>(qrow, srow, hrow, 1)};
             for (int kt = 0; kt < KT; ++kt, ++it) {
                 const int s = it % kQ8Stages, u = it / kQ8Stages;
-                DqSlice<FMT> nxt = cur;
-                if (kt + 1 < KT) nxt = dq_load<FMT>(qrow, srow, hrow, kt + 1);  // in flight while we convert
+                dq::Blk<FMT> nxt[2] = {cur[0], cur[1]};
+                if (kt + 1 < KT) {
+                    nxt[0] = dq::load_blk<FMT>(qrow, srow, hrow, 2 * kt + 2);
+                    nxt[1] = dq::load_blk<FMT>(qrow, srow, hrow, 2 * kt + 3);
+                }
                 if (u > 0) {
                     bool ok = true;
                     if (lane == 0) ok = mbar_wait(&empty_bar[s], (u - 1) & 1);
@@ -283,22 +195,23 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
 #pragma unroll
                 for (int blk = 0; blk < 2; ++blk) {
                     float v[32];
-                    dq_block<FMT>(cur, blk, g.tab, v);
+                    dq::blk_values<FMT>(cur[blk], g.tab, v);
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc) {  // chunk c = 4 blk + cc: k = 8c .. 8c+7
                         const int c = 4 * blk + cc;
                         uint4 o;
-                        o.x = pack_bf16x2(v[8 * cc], v[8 * cc + 1]);
-                        o.y = pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
-                        o.z = pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
-                        o.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
+                        o.x = dq::pack_bf16x2(v[8 * cc], v[8 * cc + 1]);
+                        o.y = dq::pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
+                        o.z = dq::pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
+                        o.w = dq::pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
                         *reinterpret_cast<uint4 *>(b_row + ((c ^ (n & 7)) << 4)) = o;
                     }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&fb_bar[s]);
-                cur = nxt;
+                cur[0] = nxt[0];
+                cur[1] = nxt[1];
             }
         }
     } else {  // ---- epilogue, warps 0-7
@@ -329,7 +242,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
                             for (int i = 0; i < 16; i += 2) {
                                 const float a0 = vg[i], a1 = vg[i + 1];
                                 // silu with the fast exponential (well inside the prefill tolerance)
-                                o[i / 2] = pack_bf16x2(a0 * __frcp_rn(1.f + __expf(-a0)) * vu[i],
+                                o[i / 2] = dq::pack_bf16x2(a0 * __frcp_rn(1.f + __expf(-a0)) * vu[i],
                                                        a1 * __frcp_rn(1.f + __expf(-a1)) * vu[i + 1]);
                             }
                             uint4 *dst = reinterpret_cast<uint4 *>(g.h + (size_t)row * g.I + nt * 128 + c);

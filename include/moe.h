@@ -48,7 +48,9 @@ typedef enum {
     MOE_ERR_OOM = 4,          /* device or host allocation failed (pack only) */
     MOE_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
     MOE_ERR_TIMEOUT = 6,      /* a bounded device-side wait ran out */
-    MOE_ERR_DEVICE = 7        /* a kernel detected an inconsistent plan */
+    MOE_ERR_DEVICE = 7,       /* a kernel detected an inconsistent plan */
+    MOE_ERR_RANGE = 8         /* an intermediate left the fp16 range of the tensor-core
+                                 decode path (|h| > 65504); run MOE_PATH_GROUPED instead */
 } moe_status;
 
 /* Block formats, each along the reduction (K) dimension of a weight row:

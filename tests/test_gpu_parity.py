@@ -158,8 +158,11 @@ def test_fused_and_grouped_decode_paths_both_match_the_oracle(name, layer, T):
         err = normwise_err(out, ref)
         assert err <= DECODE_TOL, (path, err)
         outs[path] = out
-    # same fp32 arithmetic in a different order: close, not necessarily bitwise
-    assert normwise_err(outs[bq.MOE_PATH_DECODE], outs[bq.MOE_PATH_GROUPED]) <= 1e-5
+    # one token: the same fp32 arithmetic in a different order, close but not
+    # necessarily bitwise; two or more: the decode path runs the tensor cores on
+    # fp16 operands (weights and h rounded to 11 significant bits, 2^-12
+    # relative each), the grouped path stays in fp32
+    assert normwise_err(outs[bq.MOE_PATH_DECODE], outs[bq.MOE_PATH_GROUPED]) <= (1e-5 if T == 1 else 1e-3)
 
 
 def test_fused_decode_ragged_shapes():
