@@ -37,6 +37,8 @@
 // and the CTA stops issuing work.  An h outside the fp16 range records
 // MOE_ERR_RANGE (the CUDA-core grouped path takes such layers).
 #include <cuda.h>
+
+#include <algorithm>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -54,10 +56,9 @@ using namespace tc;
 constexpr int kDtEpiWarps = 4;
 constexpr int kDtBWarp = 4, kDtMmaWarp = 5, kDtRawWarp = 6, kDtDeqWarp0 = 7, kDtDeqWarps = 8;
 constexpr int kDtThreads = 32 * (kDtDeqWarp0 + kDtDeqWarps);  // 15 warps
-constexpr int kDtMmaStages = 2, kDtRawStages = 2;
+constexpr int kDtMaxAStages = 4, kDtMaxRawStages = 4, kDtMaxBSlots = 8;
+constexpr size_t kDtSmemBudget = 225 * 1024;  // dynamic shared memory per CTA
 constexpr int kDtA = 128 * 128;                  // 128 rows x 64 fp16 of K
-constexpr int kDtB = kDecodeTcMaxN * 128;        // up to 64 token rows x 64 fp16
-constexpr int kDtMmaStage = 2 * kDtA + kDtB;     // gate and up tiles (down uses the first), B
 constexpr int kDtTmemCols = 128;                 // gate accumulator at column 0, up at 64
 
 // One raw stage holds K = 256 (four MMA slices) of every A tile's rows, as the
@@ -71,7 +72,7 @@ struct RawLayout {
     static constexpr int kScales = 128 * kScW;
     static constexpr int kQh = FMT == MOE_FMT_Q5_1 ? 128 * 32 : 0;
     static constexpr int kStage = TILES * (kCodes + kScales + kQh);
-    static constexpr size_t kSmem = (size_t)kDtRawStages * kStage + (size_t)kDtMmaStages * kDtMmaStage + 1024;
+    static constexpr int kA = TILES * kDtA;  // one A stage: the expanded fp16 tiles of a 64-wide slice
     __device__ static int codes(int t) { return t * kCodes; }
     __device__ static int scales(int t) { return TILES * kCodes + t * kScales; }
     __device__ static int qh(int t) { return TILES * (kCodes + kScales) + t * kQh; }
@@ -82,6 +83,9 @@ struct DtArgs {
     const int32_t *n_groups;
     int NB;                    // 128-row tiles per group
     int K;                     // reduction length (a multiple of 256)
+    // shared memory: nr raw stages | na A stages | nbs B slots of bslot bytes
+    // (the group's padded token rows x 64 fp16), at a_off and b_off
+    int nr, na, nbs, bslot, a_off, b_off;
     CodeTable tab;
     const float *ts;           // NVFP4 per-expert scale
     int up_off;                // gate/up: row offset of the up rows (= I)
@@ -99,6 +103,19 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N)
     return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Position in a ring of n buffers: slot s, and u = how many times the ring has
+// wrapped (the parity of an mbarrier phase); advanced without a division.
+struct Ring {
+    int s = 0, u = 0;
+    __device__ __forceinline__ void next(int n)
+    {
+        if (++s == n) {
+            s = 0;
+            ++u;
+        }
+    }
+};
+
 // Address in a raw stage of the 16-byte code chunk c (0..7) of row r in box bx
 // (128-byte rows, chunk swizzled by r % 8).
 __device__ __forceinline__ const uint8_t *raw_code(const uint8_t *box0, int bx, int r, int c)
@@ -114,12 +131,14 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     constexpr int TILES = GATEUP ? 2 : 1;
     using RL = RawLayout<FMT, TILES>;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t fa_bar[kDtMmaStages], fb_bar[kDtMmaStages], empty_bar[kDtMmaStages];
-    __shared__ __align__(8) uint64_t rf_bar[kDtRawStages], re_bar[kDtRawStages], accf_bar, acce_bar;
+    __shared__ __align__(8) uint64_t fa_bar[kDtMaxAStages], ae_bar[kDtMaxAStages], fb_bar[kDtMaxBSlots],
+        be_bar[kDtMaxBSlots];
+    __shared__ __align__(8) uint64_t rf_bar[kDtMaxRawStages], re_bar[kDtMaxRawStages], accf_bar, acce_bar;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *raw = smem, *mma = smem + kDtRawStages * RL::kStage;
+    const int NR = g.nr, NA = g.na, NBS = g.nbs;
+    uint8_t *raw = smem, *atile = smem + g.a_off, *btile = smem + g.b_off;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tasks = *g.n_groups * g.NB;
     const int KT = g.K / 64, KR = g.K / 256;  // MMA slices and raw stages per task
@@ -129,12 +148,15 @@ __global__ void __launch_bounds__(kDtThreads, 1)
         tmem_relinquish();
     }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kDtMmaStages; ++s) {
+        for (int s = 0; s < NA; ++s) {
             mbar_init(&fa_bar[s], kDtDeqWarps);
-            mbar_init(&fb_bar[s], 1);
-            mbar_init(&empty_bar[s], 1);
+            mbar_init(&ae_bar[s], 1);
         }
-        for (int s = 0; s < kDtRawStages; ++s) {
+        for (int s = 0; s < NBS; ++s) {
+            mbar_init(&fb_bar[s], 1);
+            mbar_init(&be_bar[s], 1);
+        }
+        for (int s = 0; s < NR; ++s) {
             mbar_init(&rf_bar[s], 1);
             mbar_init(&re_bar[s], kDtDeqWarps);
         }
@@ -153,12 +175,12 @@ __global__ void __launch_bounds__(kDtThreads, 1)
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmS);
             if (FMT == MOE_FMT_Q5_1) prefetch_tmap(&tmH);
-            int it = 0;
+            Ring rr;
             for (int task = blockIdx.x; task < n_tasks && !abort_flag; task += gridDim.x) {
                 const int4 gr = g.groups[task / g.NB];
                 const int b = task % g.NB;
-                for (int j = 0; j < KR; ++j, ++it) {
-                    const int s = it % kDtRawStages, u = it / kDtRawStages;
+                for (int j = 0; j < KR; ++j, rr.next(NR)) {
+                    const int s = rr.s, u = rr.u;
                     if (u > 0 && !mbar_wait(&re_bar[s], (u - 1) & 1)) {
                         abort_flag = 1;
                         break;
@@ -181,17 +203,17 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     } else if (warp == kDtBWarp) {  // ---- B tiles: the group's slot rows, 16 at a time
         if (lane == 0) {
             prefetch_tmap(&tmB);
-            int it = 0;
+            Ring rb;
             for (int task = blockIdx.x; task < n_tasks && !abort_flag; task += gridDim.x) {
                 const int4 gr = g.groups[task / g.NB];
                 const int n16 = (gr.z + 15) >> 4;
-                for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % kDtMmaStages, u = it / kDtMmaStages;
-                    if (u > 0 && !mbar_wait(&empty_bar[s], (u - 1) & 1)) {
+                for (int kt = 0; kt < KT; ++kt, rb.next(NBS)) {
+                    const int s = rb.s, u = rb.u;
+                    if (u > 0 && !mbar_wait(&be_bar[s], (u - 1) & 1)) {
                         abort_flag = 1;
                         break;
                     }
-                    uint8_t *b_s = mma + s * kDtMmaStage + 2 * kDtA;
+                    uint8_t *b_s = btile + s * g.bslot;
                     mbar_arrive_expect_tx(&fb_bar[s], (uint32_t)n16 * 2048u);
                     for (int jj = 0; jj < n16; ++jj)
                         tma_load_2d(b_s + jj * 2048, &tmB, &fb_bar[s], kt * 64, gr.y + 16 * jj);
@@ -200,7 +222,8 @@ __global__ void __launch_bounds__(kDtThreads, 1)
         }
     } else if (warp == kDtMmaWarp) {  // ---- MMA issuer
         if (lane == 0) {
-            int it = 0, tcount = 0;
+            Ring ra, rb;
+            int tcount = 0;
             for (int task = blockIdx.x; task < n_tasks && !abort_flag; task += gridDim.x, ++tcount) {
                 const int4 gr = g.groups[task / g.NB];
                 const uint32_t idesc = idesc_f16(128, (gr.z + 15) & ~15);
@@ -209,15 +232,15 @@ __global__ void __launch_bounds__(kDtThreads, 1)
                     break;
                 }
                 tc_fence_after_sync();
-                for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % kDtMmaStages, u = it / kDtMmaStages;
-                    if (!mbar_wait(&fa_bar[s], u & 1) || !mbar_wait(&fb_bar[s], u & 1)) {
+                for (int kt = 0; kt < KT; ++kt, ra.next(NA), rb.next(NBS)) {
+                    const int sa = ra.s, ua = ra.u, sb = rb.s, ub = rb.u;
+                    if (!mbar_wait(&fa_bar[sa], ua & 1) || !mbar_wait(&fb_bar[sb], ub & 1)) {
                         abort_flag = 1;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint8_t *a_s = mma + s * kDtMmaStage;
-                    const uint64_t bd = desc_kmajor_sw128(a_s + 2 * kDtA);
+                    const uint8_t *a_s = atile + sa * RL::kA;
+                    const uint64_t bd = desc_kmajor_sw128(btile + sb * g.bslot);
 #pragma unroll
                     for (int hh = 0; hh < TILES; ++hh) {
                         const uint64_t ad = desc_kmajor_sw128(a_s + hh * kDtA);
@@ -225,7 +248,8 @@ __global__ void __launch_bounds__(kDtThreads, 1)
                         for (int kk = 0; kk < 4; ++kk)
                             mma_f16(tmem + hh * 64, ad + 2 * kk, bd + 2 * kk, idesc, (kt | kk) != 0);
                     }
-                    mma_commit(&empty_bar[s]);
+                    mma_commit(&ae_bar[sa]);
+                    mma_commit(&be_bar[sb]);
                 }
                 mma_commit(&accf_bar);
             }
@@ -238,11 +262,11 @@ __global__ void __launch_bounds__(kDtThreads, 1)
         const int tile = GATEUP ? n >> 7 : 0;
         const int bsel = GATEUP ? 0 : n >> 7;
         constexpr int BPS = GATEUP ? 2 : 1;
-        int it = 0, rit = 0;
+        Ring ra, rr;
         bool ok = true;
         for (int task = blockIdx.x; task < n_tasks && ok && !abort_flag; task += gridDim.x) {
-            for (int j = 0; j < KR && ok; ++j, ++rit) {
-                const int rs = rit % kDtRawStages, ru = rit / kDtRawStages;
+            for (int j = 0; j < KR && ok; ++j, rr.next(NR)) {
+                const int rs = rr.s, ru = rr.u;
                 if (!mbar_wait(&rf_bar[rs], ru & 1)) {
                     abort_flag = 1;
                     ok = false;
@@ -251,18 +275,18 @@ __global__ void __launch_bounds__(kDtThreads, 1)
                 const uint8_t *st = raw + rs * RL::kStage;
                 const uint8_t *cq = st + RL::codes(tile), *cs = st + RL::scales(tile), *ch = st + RL::qh(tile);
 #pragma unroll 1
-                for (int d = 0; d < 4; ++d, ++it) {
-                    const int s = it % kDtMmaStages, u = it / kDtMmaStages;
+                for (int d = 0; d < 4; ++d, ra.next(NA)) {
+                    const int s = ra.s, u = ra.u;
                     if (u > 0) {
                         bool w = true;
-                        if (lane == 0) w = mbar_wait(&empty_bar[s], (u - 1) & 1);
+                        if (lane == 0) w = mbar_wait(&ae_bar[s], (u - 1) & 1);
                         if (!__shfl_sync(0xffffffffu, w, 0)) {
                             abort_flag = 1;
                             ok = false;
                             break;
                         }
                     }
-                    uint8_t *a_row = mma + s * kDtMmaStage + tile * kDtA + (r >> 3) * 1024 + (r & 7) * 128;
+                    uint8_t *a_row = atile + s * RL::kA + tile * kDtA + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
                     for (int q = 0; q < BPS; ++q) {
                         const int blk = 2 * d + q + bsel;  // block of the raw stage (0..7)
@@ -441,13 +465,36 @@ DtKernel dt_pick(int fmt)
     }
 }
 
-size_t dt_smem(bool gateup, int fmt)
+// Shared-memory plan of one launch: two A stages, two to eight B slots (B rows
+// come from L2), two to four raw stages (from HBM).  Measured on B200: four A
+// stages instead of two made the 8- and 64-token layers slower.
+struct DtLayout {
+    int nr, na, nbs, bslot;
+    size_t raw, a, total;
+};
+
+template <int FMT>
+DtLayout dt_layout_fmt(bool gateup, int nmax)
+{
+    DtLayout L;
+    L.raw = gateup ? RawLayout<FMT, 2>::kStage : RawLayout<FMT, 1>::kStage;
+    L.a = gateup ? RawLayout<FMT, 2>::kA : RawLayout<FMT, 1>::kA;
+    L.bslot = nmax * 128;
+    L.nr = L.na = L.nbs = 2;
+    auto total = [&] { return 1024 + L.nr * L.raw + L.na * L.a + (size_t)L.nbs * L.bslot; };
+    while (L.nbs < kDtMaxBSlots && total() + L.bslot <= kDtSmemBudget) ++L.nbs;
+    while (L.nr < kDtMaxRawStages && total() + L.raw <= kDtSmemBudget) ++L.nr;
+    L.total = total();
+    return L;
+}
+
+DtLayout dt_layout(bool gateup, int fmt, int nmax)
 {
     switch (fmt) {
-    case MOE_FMT_Q8_0: return gateup ? RawLayout<MOE_FMT_Q8_0, 2>::kSmem : RawLayout<MOE_FMT_Q8_0, 1>::kSmem;
-    case MOE_FMT_Q5_1: return gateup ? RawLayout<MOE_FMT_Q5_1, 2>::kSmem : RawLayout<MOE_FMT_Q5_1, 1>::kSmem;
-    case MOE_FMT_IQ4_NL: return gateup ? RawLayout<MOE_FMT_IQ4_NL, 2>::kSmem : RawLayout<MOE_FMT_IQ4_NL, 1>::kSmem;
-    default: return gateup ? RawLayout<MOE_FMT_NVFP4, 2>::kSmem : RawLayout<MOE_FMT_NVFP4, 1>::kSmem;
+    case MOE_FMT_Q8_0: return dt_layout_fmt<MOE_FMT_Q8_0>(gateup, nmax);
+    case MOE_FMT_Q5_1: return dt_layout_fmt<MOE_FMT_Q5_1>(gateup, nmax);
+    case MOE_FMT_IQ4_NL: return dt_layout_fmt<MOE_FMT_IQ4_NL>(gateup, nmax);
+    default: return dt_layout_fmt<MOE_FMT_NVFP4>(gateup, nmax);
     }
 }
 
@@ -495,7 +542,7 @@ cudaError_t decode_tc_set_attributes()
         for (int gu = 0; gu < 2; ++gu) {
             const cudaError_t e = cudaFuncSetAttribute(gu ? dt_pick<true>(f) : dt_pick<false>(f),
                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       (int)dt_smem(gu != 0, f));
+                                                       (int)kDtSmemBudget);
             if (e != cudaSuccess) return e;
         }
     return cudaSuccess;
@@ -519,9 +566,18 @@ cudaError_t launch_decode_tc_gather(const void *x, int x_dtype, int T, int H, in
 
 cudaError_t launch_decode_tc(const DecodeTcMaps &m, bool gateup, const DevProj &w, const int4 *groups,
                              const int32_t *n_groups, int H, int I, const CodeTable &tab, const float *slot_scale,
-                             void *h16, float *y, int32_t *err, int grid, cudaStream_t s)
+                             void *h16, float *y, int32_t *err, int max_tokens, int grid, cudaStream_t s)
 {
+    const int nmax = (std::min(std::max(max_tokens, 1), kDecodeTcMaxN) + 15) & ~15;
+    const DtLayout L = dt_layout(gateup, w.fmt, nmax);
+    if (L.total > kDtSmemBudget) return cudaErrorInvalidValue;
     DtArgs a{};
+    a.nr = L.nr;
+    a.na = L.na;
+    a.nbs = L.nbs;
+    a.bslot = L.bslot;
+    a.a_off = (int)(L.nr * L.raw);
+    a.b_off = (int)(L.nr * L.raw + L.na * L.a);
     a.groups = groups;
     a.n_groups = n_groups;
     a.NB = gateup ? I / 128 : H / 128;
@@ -538,7 +594,7 @@ cudaError_t launch_decode_tc(const DecodeTcMaps &m, bool gateup, const DevProj &
     DtKernel kfn = gateup ? dt_pick<true>(w.fmt) : dt_pick<false>(w.fmt);
     if (!kfn) return cudaErrorInvalidValue;
     const CUtensorMap *pm = gateup ? m.gu : m.dn;
-    kfn<<<grid, kDtThreads, dt_smem(gateup, w.fmt), s>>>(gateup ? m.xg : m.h, pm[0], pm[1], pm[2], a);
+    kfn<<<grid, kDtThreads, L.total, s>>>(gateup ? m.xg : m.h, pm[0], pm[1], pm[2], a);
     return cudaGetLastError();
 }
 

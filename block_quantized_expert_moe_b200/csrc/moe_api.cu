@@ -843,11 +843,11 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
                                                   w.slot_scale, s));
         if (st != MOE_OK) return st;
         st = check_launch(launch_decode_tc(pm->dtc_maps, true, p->gu, w.groups, w.n_groups, p->H, p->I, p->ct_gu,
-                                           w.slot_scale, w.h, w.y, w.err, p->num_sms, s));
+                                           w.slot_scale, w.h, w.y, w.err, p->max_tokens, p->num_sms, s));
         if (st != MOE_OK) return st;
         prof_mark(pm, pbase, 2, s);
         st = check_launch(launch_decode_tc(pm->dtc_maps, false, p->dn, w.groups, w.n_groups, p->H, p->I, p->ct_dn,
-                                           w.slot_scale, w.h, w.y, w.err, p->num_sms, s));
+                                           w.slot_scale, w.h, w.y, w.err, p->max_tokens, p->num_sms, s));
         if (st != MOE_OK) return st;
         prof_mark(pm, pbase, 3, s);
     } else if (path == MOE_PATH_DECODE && T >= 2 && tt == 8 && pm->sgm == 1) {

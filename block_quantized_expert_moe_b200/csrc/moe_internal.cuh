@@ -252,7 +252,7 @@ cudaError_t launch_decode_tc_gather(const void *x, int x_dtype, int T, int H, in
                                     const int32_t *slot_pos, void *xg, float *slot_scale, cudaStream_t s);
 cudaError_t launch_decode_tc(const DecodeTcMaps &m, bool gateup, const DevProj &w, const int4 *groups,
                              const int32_t *n_groups, int H, int I, const CodeTable &tab, const float *slot_scale,
-                             void *h16, float *y, int32_t *err, int grid, cudaStream_t s);
+                             void *h16, float *y, int32_t *err, int max_tokens, int grid, cudaStream_t s);
 cudaError_t launch_sgm(const SgmProj &p, const DevProj &w, const int4 *groups, const int32_t *n_groups,
                        const int32_t *perm_tok, const void *x, int x_dtype, float *out, int out_stride, int rows_out,
                        bool gateup, const CodeTable &tab, int32_t *err, int grid, cudaStream_t s);
