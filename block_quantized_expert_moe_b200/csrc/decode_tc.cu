@@ -465,9 +465,10 @@ DtKernel dt_pick(int fmt)
     }
 }
 
-// Shared-memory plan of one launch: two A stages, two to eight B slots (B rows
-// come from L2), two to four raw stages (from HBM).  Measured on B200: four A
-// stages instead of two made the 8- and 64-token layers slower.
+// Shared-memory plan of one launch: two of each ring at least, then up to four
+// A stages (each slice is a round trip between the expanding warps and the MMA
+// issuer), up to eight B slots (B rows come from L2), up to four raw stages
+// (from HBM), as far as 225 KB allow.
 struct DtLayout {
     int nr, na, nbs, bslot;
     size_t raw, a, total;
@@ -482,6 +483,7 @@ DtLayout dt_layout_fmt(bool gateup, int nmax)
     L.bslot = nmax * 128;
     L.nr = L.na = L.nbs = 2;
     auto total = [&] { return 1024 + L.nr * L.raw + L.na * L.a + (size_t)L.nbs * L.bslot; };
+    while (L.na < kDtMaxAStages && total() + L.a <= kDtSmemBudget) ++L.na;
     while (L.nbs < kDtMaxBSlots && total() + L.bslot <= kDtSmemBudget) ++L.nbs;
     while (L.nr < kDtMaxRawStages && total() + L.raw <= kDtSmemBudget) ++L.nr;
     L.total = total();

@@ -82,18 +82,22 @@ typedef enum { MOE_DT_F32 = 1, MOE_DT_BF16 = 2 } moe_dtype;
 /* Kernel path of a forward.  AUTO picks DECODE for n_tokens <= 64 (decode and
  * speculative-verify batches) and PREFILL above when the pack can run it (both
  * projections NVFP4 - native block-scaled FP4 MMA with the activations rounded
- * to NVFP4 per token - or both Q8_0 - weights dequantised to bf16 for bf16 MMA;
- * hidden and inter multiples of 256, bf16 activations, top_k <= 32; its
- * buffers are sized at pack time when max_tokens > 64), else GROUPED.  DENSE is the dense-batched
- * comparison variant (pack created with MOE_PACK_DENSE, n_tokens <= 64): every
- * active expert multiplies the whole batch, with a zero gate for the tokens not
- * routed to it. */
+ * to NVFP4 per token - or Q8_0 / IQ4_NL / Q5_1 in any mix - weights dequantised
+ * to bf16 for bf16 MMA; hidden and inter multiples of 256, bf16 activations,
+ * top_k <= 32; its buffers are sized at pack time when max_tokens > 64), else
+ * GROUPED.  DECODE: one token runs the single-token streaming kernel; 2 to 64
+ * tokens run the tensor-core grouped decode (weights expanded to fp16, fp32
+ * accumulation; hidden and inter multiples of 256 and every weight an fp16
+ * normal number or zero, checked at pack time), else the CUDA-core grouped
+ * kernels.  DENSE is the dense-batched comparison variant (pack created with
+ * MOE_PACK_DENSE, n_tokens <= 64): every active expert multiplies the whole
+ * batch, with a zero gate for the tokens not routed to it. */
 typedef enum {
     MOE_PATH_AUTO = 0,
-    MOE_PATH_DECODE = 1,   /* one fused launch for n_tokens <= 8, top_k <= 16, else GROUPED */
+    MOE_PATH_DECODE = 1,   /* see above; falls back to GROUPED where its kernels do not apply */
     MOE_PATH_PREFILL = 2,
     MOE_PATH_DENSE = 3,
-    MOE_PATH_GROUPED = 4   /* decode as separate route / gate-up / down / combine launches */
+    MOE_PATH_GROUPED = 4   /* decode as separate route / gate-up / down / combine launches, fp32 CUDA cores */
 } moe_path;
 
 /* Description of one layer's experts, all in HOST memory; moe_pack_experts
@@ -232,10 +236,13 @@ moe_status moe_read_routing(const moe_pack *pack, int n_tokens, int top_k, int32
  * whole tensor-core prefill sequence; [6..14] the fused kernel's phases as seen
  * by its first CTA (token staging, router, barrier, plan, gate/up, barrier,
  * down, barrier, combine), from its SM clock at the device's nominal rate;
- * [15..23] single-token streaming kernel only, from the global timer, relative
- * to the first CTA's start: last CTA start, first and last CTA to publish its
- * router rows, to issue its routed copies, to finish gate/up, to end;
- * [24..31] its first CTA's time at eight internal points (kernel-specific).  It
+ * [15..23] from the global timer, relative to the first CTA's start: for the
+ * single-token streaming kernel the last CTA start, first and last CTA to
+ * publish its router rows, to issue its routed copies, to finish gate/up, to
+ * end; for the router kernel of the grouped paths the last CTA start, first
+ * and last CTA with x and its router rows staged, with its logits written, and
+ * the top-k and plan completions ([6..14] then hold the selecting CTA's steps);
+ * [24..31] the streaming kernel's first CTA's time at eight internal points.  It
  * stores the
  * forward count in *n_forwards, and frees the events.  Forwards beyond
  * max_forwards are not recorded. */
