@@ -28,10 +28,10 @@
 //   warps 0-3   epilogue (tensor-memory lanes 32w .. 32w + 31 = tile rows)
 //   warp 4      TMA producer of the B tiles (16-row boxes, 128-byte swizzle)
 //   warp 5      MMA issuer (one elected thread)
-//   warps 6-13  dequantisers: gate/up thread n owns A row n (0-127 gate,
-//               128-255 up), both 32-blocks of each 64-wide K slice; down
-//               thread n owns row n % 128, block n / 128 of each slice; each
-//               keeps four slices of raw blocks in flight in registers
+//   warp 6      TMA producer of the raw weight tiles (codes, scales, fifth
+//               bits; K = 256 of every tile row per stage)
+//   warps 7-22  dequantisers: each thread expands one 32-block of one tile
+//               row per slice into the fp16 A tile
 //
 // Every mbarrier wait is bounded; a wait that runs out records MOE_ERR_TIMEOUT
 // and the CTA stops issuing work.  An h outside the fp16 range records
@@ -54,8 +54,8 @@ namespace {
 using namespace tc;
 
 constexpr int kDtEpiWarps = 4;
-constexpr int kDtBWarp = 4, kDtMmaWarp = 5, kDtRawWarp = 6, kDtDeqWarp0 = 7, kDtDeqWarps = 8;
-constexpr int kDtThreads = 32 * (kDtDeqWarp0 + kDtDeqWarps);  // 15 warps
+constexpr int kDtBWarp = 4, kDtMmaWarp = 5, kDtRawWarp = 6, kDtDeqWarp0 = 7, kDtDeqWarps = 16;
+constexpr int kDtThreads = 32 * (kDtDeqWarp0 + kDtDeqWarps);  // 23 warps
 constexpr int kDtMaxAStages = 4, kDtMaxRawStages = 4, kDtMaxBSlots = 8;
 constexpr size_t kDtSmemBudget = 225 * 1024;  // dynamic shared memory per CTA
 constexpr int kDtA = 128 * 128;                  // 128 rows x 64 fp16 of K
@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < NA; ++s) {
-            mbar_init(&fa_bar[s], kDtDeqWarps);
+            mbar_init(&fa_bar[s], GATEUP ? kDtDeqWarps : kDtDeqWarps / 2);
             mbar_init(&ae_bar[s], 1);
         }
         for (int s = 0; s < NBS; ++s) {
@@ -255,13 +255,15 @@ __global__ void __launch_bounds__(kDtThreads, 1)
             }
         }
     } else if (warp >= kDtDeqWarp0) {  // ---- dequantisers: raw blocks -> fp16 A tiles
-        // gate/up: thread n owns row n % 128 of tile n / 128 and both blocks of
-        // each 64-wide slice; down: row n % 128, block n / 128 of each slice
+        // thread n expands one 32-block of one row per slice: gate/up row n % 128
+        // of tile (n / 128) % 2, block n / 256 of every slice; down row n % 128,
+        // block (n / 128) % 2 of the slices of parity n / 256 (a slice of down is
+        // half the rows' work of gate/up)
         const int n = threadIdx.x - 32 * kDtDeqWarp0;
         const int r = n & 127;
-        const int tile = GATEUP ? n >> 7 : 0;
-        const int bsel = GATEUP ? 0 : n >> 7;
-        constexpr int BPS = GATEUP ? 2 : 1;
+        const int tile = GATEUP ? (n >> 7) & 1 : 0;
+        const int bsel = GATEUP ? n >> 8 : (n >> 7) & 1;
+        const int par = GATEUP ? -1 : n >> 8;
         Ring ra, rr;
         bool ok = true;
         for (int task = blockIdx.x; task < n_tasks && ok && !abort_flag; task += gridDim.x) {
@@ -277,6 +279,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
 #pragma unroll 1
                 for (int d = 0; d < 4; ++d, ra.next(NA)) {
                     const int s = ra.s, u = ra.u;
+                    if (!GATEUP && (d & 1) != par) continue;  // the other half of the warps' slice
                     if (u > 0) {
                         bool w = true;
                         if (lane == 0) w = mbar_wait(&ae_bar[s], (u - 1) & 1);
@@ -287,9 +290,8 @@ __global__ void __launch_bounds__(kDtThreads, 1)
                         }
                     }
                     uint8_t *a_row = atile + s * RL::kA + tile * kDtA + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-                    for (int q = 0; q < BPS; ++q) {
-                        const int blk = 2 * d + q + bsel;  // block of the raw stage (0..7)
+                    {
+                        const int blk = 2 * d + bsel;  // block of the raw stage (0..7)
                         uint32_t qw[8];
                         if constexpr (FMT == MOE_FMT_Q8_0) {
                             const uint4 a = *reinterpret_cast<const uint4 *>(raw_code(cq, blk >> 2, r, (2 * blk) & 7));
@@ -313,7 +315,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
                         dq::blk_f16<FMT>(qw, sc, hb, g.tab, o4);
 #pragma unroll
                         for (int cc = 0; cc < 4; ++cc) {  // chunk c: elements 8c .. 8c+7 of the slice
-                            const int c = 4 * (q + bsel) + cc;
+                            const int c = 4 * bsel + cc;
                             *reinterpret_cast<uint4 *>(a_row + ((c ^ (r & 7)) << 4)) = o4[cc];
                         }
                     }
