@@ -395,7 +395,11 @@ def ours_arm(a, wl):
     # one token: the streaming kernel (whole-row bulk copies) runs in place of the fused one
     kname = "stream1_kernel" if dom == "fused" and T == 1 else KERNEL_NAMES[dom]
     if a.path == "auto" and T >= 2 and dom in ("gate_up", "down"):
-        kname = f"sgm_kernel<{dom.replace('_', '/')}>"  # streamed grouped matvec (row per lane)
+        # 2-64 tokens with H and I multiples of 256 run the tensor-core grouped
+        # decode (its gate/up stage includes the x gather); else the streamed
+        # CUDA-core grouped matvec (row per lane)
+        tc = T <= 64 and H % 256 == 0 and wl.inter % 256 == 0
+        kname = f"dtc_kernel<{dom.replace('_', '/')}>" if tc else f"sgm_kernel<{dom.replace('_', '/')}>"
     hbm, peak_src = peaks()
     traffic = kernel_traffic(dom, wl.name)
     if dom == "prefill":
