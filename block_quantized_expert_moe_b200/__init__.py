@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(HERE, "libmoe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_FMT_MISMATCH = 0, 1, 2, 3
 MOE_ERR_OOM, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE, MOE_ERR_RANGE = 4, 5, 6, 7, 8
-MOE_FMT_FROM_PACK, MOE_FMT_Q8_0, MOE_FMT_Q5_1, MOE_FMT_IQ4_NL, MOE_FMT_NVFP4 = 0, 1, 2, 3, 4
+MOE_FMT_FROM_PACK, MOE_FMT_Q8_0, MOE_FMT_Q5_1, MOE_FMT_IQ4_NL, MOE_FMT_NVFP4, MOE_FMT_Q5_0 = 0, 1, 2, 3, 4, 5
 MOE_DT_F32, MOE_DT_BF16 = 1, 2
 MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_DENSE, MOE_PATH_GROUPED = 0, 1, 2, 3, 4
 

@@ -31,7 +31,8 @@ struct moe_pack {
     int device = 0;
     int num_sms = 0;
     int E = 0, H = 0, I = 0, has_shared = 0, max_tokens = 0, max_top_k = 0, flags = 0;
-    int fmt_gu = 0, fmt_dn = 0;
+    int fmt_gu = 0, fmt_dn = 0;        // device formats (a Q5_0 projection runs as Q5_1)
+    int fmt_gu_in = 0, fmt_dn_in = 0;  // the formats the caller packed
     DevProj gu, dn;
     CodeTable ct_gu{}, ct_dn{};
     uint8_t perm_gu[16], perm_dn[16];  // stored position of each 4-bit code
@@ -172,13 +173,17 @@ struct DeviceGuard {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool valid_fmt(int f) { return f >= MOE_FMT_Q8_0 && f <= MOE_FMT_NVFP4; }
+bool valid_fmt(int f) { return f >= MOE_FMT_Q8_0 && f <= MOE_FMT_Q5_0; }
+
+// The device format of a projection: Q5_0 runs as Q5_1 with m = -16 d.
+int device_fmt(int f) { return f == MOE_FMT_Q5_0 ? MOE_FMT_Q5_1 : f; }
 
 int64_t canon_row_bytes(int fmt, int64_t cols)
 {
     switch (fmt) {
     case MOE_FMT_Q8_0: return cols / 32 * 34;
     case MOE_FMT_Q5_1: return cols / 32 * 24;
+    case MOE_FMT_Q5_0: return cols / 32 * 22;
     case MOE_FMT_IQ4_NL: return cols / 32 * 18;
     case MOE_FMT_NVFP4: return cols / 16 * 9;
     default: return -1;
@@ -191,7 +196,8 @@ void plane_rows(int fmt, int cols, int &qs_row, int &sc_row, int &qh_row)
     qh_row = 0;
     switch (fmt) {
     case MOE_FMT_Q8_0: qs_row = cols; sc_row = cols / 32 * 2; break;
-    case MOE_FMT_Q5_1: qs_row = cols / 2; sc_row = cols / 32 * 4; qh_row = cols / 32 * 4; break;
+    case MOE_FMT_Q5_1:
+    case MOE_FMT_Q5_0: qs_row = cols / 2; sc_row = cols / 32 * 4; qh_row = cols / 32 * 4; break;
     case MOE_FMT_IQ4_NL: qs_row = cols / 2; sc_row = cols / 32 * 2; break;
     default: qs_row = cols / 2; sc_row = 0; break;  // NVFP4: scales in the block-scale layout
     }
@@ -206,6 +212,27 @@ int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
 // Repack one expert's projection (rows x cols canonical blocks) into planes.
 // Returns false on an invalid NVFP4 block scale.
+float half_to_float(uint16_t h)
+{
+    const int e = (h >> 10) & 31, m = h & 1023;
+    const float mag = e == 0 ? std::ldexp((float)m, -24) : e == 31 ? INFINITY : std::ldexp((float)(1024 + m), e - 25);
+    return (h & 0x8000) ? -mag : mag;
+}
+
+// fp16 bits of f, which must be exactly representable (a power-of-two multiple
+// of an fp16 number within range).
+uint16_t half_from_exact(float f)
+{
+    const uint16_t sign = std::signbit(f) ? 0x8000u : 0u;
+    const float a = std::fabs(f);
+    if (a == 0.f) return sign;
+    int e;
+    const float m = std::frexp(a, &e);  // a = m 2^e, m in [0.5, 1)
+    const int E = e - 1 + 15;
+    if (E >= 1) return (uint16_t)(sign | (E << 10) | (uint32_t)std::ldexp(2.f * m - 1.f, 10));
+    return (uint16_t)(sign | (uint32_t)std::ldexp(a, 24));  // subnormal: a = mant 2^-24
+}
+
 bool repack_expert(int fmt, const uint8_t *src, int rows, int cols, uint8_t *qs, uint8_t *sc,
                    uint8_t *qh, uint8_t *sr, const uint8_t *perm)
 {
@@ -232,6 +259,20 @@ bool repack_expert(int fmt, const uint8_t *src, int rows, int cols, uint8_t *qs,
                 std::memcpy(s + 4 * b, blk, 4);      // d, m
                 std::memcpy(h + 4 * b, blk + 4, 4);  // qh
                 std::memcpy(q + 16 * b, blk + 8, 16);
+            }
+        } else if (fmt == MOE_FMT_Q5_0) {  // as Q5_1 planes with m = -16 d (exact)
+            uint8_t *h = qh + (int64_t)r * qh_row;
+            for (int b = 0; b < cols / 32; ++b) {
+                const uint8_t *blk = row + b * 22;
+                const float d = half_to_float((uint16_t)(blk[0] | blk[1] << 8));
+                if (!(std::fabs(d) * 16.f <= 65504.f)) return false;
+                const uint16_t m = half_from_exact(-16.f * d);
+                s[4 * b] = blk[0];
+                s[4 * b + 1] = blk[1];
+                s[4 * b + 2] = (uint8_t)m;
+                s[4 * b + 3] = (uint8_t)(m >> 8);
+                std::memcpy(h + 4 * b, blk + 2, 4);  // qh
+                std::memcpy(q + 16 * b, blk + 6, 16);
             }
         } else if (fmt == MOE_FMT_IQ4_NL) {
             for (int b = 0; b < cols / 32; ++b) {
@@ -290,13 +331,6 @@ moe_status dev_alloc(moe_pack *p, size_t bytes, void **out)
     return MOE_OK;
 }
 
-float half_to_float(uint16_t h)
-{
-    const int e = (h >> 10) & 31, m = h & 1023;
-    const float mag = e == 0 ? std::ldexp((float)m, -24) : e == 31 ? INFINITY : std::ldexp((float)(1024 + m), e - 25);
-    return (h & 0x8000) ? -mag : mag;
-}
-
 // Whether every weight d q (Q8_0, IQ4_NL: |q| <= 128) or d q + m (Q5_1,
 // q <= 31) of the scale plane `sc` is an fp16 normal number or zero: the
 // tensor-core decode path expands the blocks to fp16.  NVFP4 always is (a code
@@ -326,7 +360,7 @@ bool f16_safe(int fmt, const std::vector<uint8_t> &sc, int64_t stride, int64_t u
 moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, const uint8_t *blocks,
                       const uint8_t *shared_blocks, const float *ts, int n_slots, const uint8_t *perm)
 {
-    dp.fmt = fmt;
+    dp.fmt = device_fmt(fmt);  // fmt: the canonical blocks' format
     dp.rows = rows;
     dp.cols = cols;
     plane_rows(fmt, cols, dp.qs_row, dp.sc_row, dp.qh_row);
@@ -357,7 +391,7 @@ moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, con
     });
     for (char c : ok)
         if (!c) return MOE_ERR_INVALID_ARG;
-    dp.f16_ok = f16_safe(fmt, hs, dp.sc_stride, (int64_t)rows * dp.sc_row, n_slots);
+    dp.f16_ok = f16_safe(dp.fmt, hs, dp.sc_stride, (int64_t)rows * dp.sc_row, n_slots);
     void *dq, *ds, *dh = nullptr, *dt = nullptr;
     moe_status st;
     if ((st = dev_alloc(p, hq.size(), &dq)) != MOE_OK) return st;
@@ -534,8 +568,10 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
     p->max_tokens = d->max_tokens;
     p->max_top_k = d->max_top_k;
     p->flags = d->flags;
-    p->fmt_gu = d->fmt_gate_up;
-    p->fmt_dn = d->fmt_down;
+    p->fmt_gu_in = d->fmt_gate_up;
+    p->fmt_dn_in = d->fmt_down;
+    p->fmt_gu = device_fmt(d->fmt_gate_up);
+    p->fmt_dn = device_fmt(d->fmt_down);
     p->ct_gu = build_code_table(p->fmt_gu, d->iq4nl_table, p->perm_gu);
     p->ct_dn = build_code_table(p->fmt_dn, d->iq4nl_table, p->perm_dn);
     for (auto &row : p->grid_cache) row[0] = row[1] = 0;
@@ -543,10 +579,10 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
     std::vector<float> gts, dts;
     if (p->fmt_gu == MOE_FMT_NVFP4) gts.assign(d->gate_up_tensor_scale, d->gate_up_tensor_scale + n_slots);
     if (p->fmt_dn == MOE_FMT_NVFP4) dts.assign(d->down_tensor_scale, d->down_tensor_scale + n_slots);
-    st = build_proj(p, p->gu, p->fmt_gu, 2 * p->I, p->H, static_cast<const uint8_t *>(d->gate_up_blocks),
+    st = build_proj(p, p->gu, p->fmt_gu_in, 2 * p->I, p->H, static_cast<const uint8_t *>(d->gate_up_blocks),
                     static_cast<const uint8_t *>(d->shared_gate_up_blocks), gts.data(), n_slots, p->perm_gu);
     if (st == MOE_OK)
-        st = build_proj(p, p->dn, p->fmt_dn, p->H, p->I, static_cast<const uint8_t *>(d->down_blocks),
+        st = build_proj(p, p->dn, p->fmt_dn_in, p->H, p->I, static_cast<const uint8_t *>(d->down_blocks),
                         static_cast<const uint8_t *>(d->shared_down_blocks), dts.data(), n_slots, p->perm_dn);
     if (st == MOE_OK) st = build_workspace(p);
     const bool nv = p->fmt_gu == MOE_FMT_NVFP4 && p->fmt_dn == MOE_FMT_NVFP4 &&
@@ -652,7 +688,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
     if (n_tokens < 1 || n_tokens > p->max_tokens) return MOE_ERR_INVALID_ARG;
     if (top_k < 1 || top_k > p->max_top_k) return MOE_ERR_INVALID_ARG;
-    if (fmt != MOE_FMT_FROM_PACK && fmt != p->fmt_gu) return MOE_ERR_FMT_MISMATCH;
+    if (fmt != MOE_FMT_FROM_PACK && fmt != p->fmt_gu_in) return MOE_ERR_FMT_MISMATCH;
     const bool prefill_ok = p->has_prefill && x_dtype == MOE_DT_BF16 && top_k <= 32;
     if (path == MOE_PATH_AUTO)
         path = n_tokens <= kDecodeMaxTokens ? MOE_PATH_DECODE : (prefill_ok ? MOE_PATH_PREFILL : MOE_PATH_GROUPED);

@@ -6,9 +6,12 @@
 // Here the plan is built at the end of the router launch:
 //
 //   phase 1 (all CTAs)   logits[t][e] = sum_h Wr[e][h] x[t][h], fp32 accumulate;
-//                        CTA b takes token block b % ntb (8 tokens, staged in
-//                        shared memory as fp32 once) and a slice of the expert
-//                        rows, one warp per row
+//                        CTA b takes token block b % NB (<= 8 tokens) and a
+//                        slice of the expert rows; one thread bulk-copies the
+//                        slice's router rows and the tokens' x rows into shared
+//                        memory, four rows per warp (gemv_staged; rows read
+//                        from global memory, one per warp, when the slice does
+//                        not fit)
 //   phase 2 (last CTA of each token block)  one warp per token: the threshold
 //                        top-k (candidates at or above the k-th largest lane
 //                        maximum, ranked in one pass; ties to the lower expert
@@ -19,7 +22,8 @@
 //                        token masks and popcounts, so the plan is identical
 //                        from run to run; then the list of work groups
 //                        {expert, first slot, tokens <= tt} for the grouped
-//                        matvecs, the shared expert's groups last.
+//                        kernels, the shared expert's groups last (plan_small
+//                        for <= 64 tokens: four barriers; plan_phase above).
 //
 // "Last" is decided by global tickets (atomicAdd after a fence: one per token
 // block, one over blocks); no CTA ever waits on another.

@@ -56,25 +56,31 @@ typedef enum {
 /* Block formats, each along the reduction (K) dimension of a weight row:
  *   Q8_0   32 weights in 34 B: fp16 d, int8 q[32]                 w = d*q
  *   Q5_1   32 weights in 24 B: fp16 d, fp16 m, u32 qh, qs[16]     w = d*q + m, q in [0,31]
+ *   Q5_0   32 weights in 22 B: fp16 d, u32 qh, qs[16]             w = d*(q - 16), q in [0,31]
  *   IQ4_NL 32 weights in 18 B: fp16 d, qs[16] (4-bit indices)     w = d*T[i], T from the pack desc
  *   NVFP4  16 weights in  9 B: E4M3 scale, 8 B of E2M1 codes, and one fp32
  *          scale s per matrix                                     w = s*e4m3*e2m1
  * Byte order inside a block (little endian):
  *   Q8_0   [0,2) d  [2,34) q
  *   Q5_1   [0,2) d  [2,4) m  [4,8) qh (bit j is bit 4 of element j)  [8,24) qs
+ *   Q5_0   [0,2) d  [2,6) qh  [6,22) qs (as Q5_1 without m)
  *   IQ4_NL [0,2) d  [2,18) qs
- *   for Q5_1 and IQ4_NL element j < 16 is the low nibble of qs[j] and element
+ *   for Q5_1, Q5_0 and IQ4_NL element j < 16 is the low nibble of qs[j] and element
  *   j >= 16 the high nibble of qs[j-16];
  *   NVFP4  [0] E4M3 scale  [1,9) codes: element 2i is the low, 2i+1 the high
  *   nibble of byte 1+i.
  * IQ4_NL is 4.5 bits per weight, the size the UD-IQ2_XS model card ("What was
- * changed") gives when it requantises a Q5_0 tensor (5.5 bits) to IQ4_NL. */
+ * changed") gives when it requantises a Q5_0 tensor (5.5 bits) to IQ4_NL.
+ * A Q5_0 projection is packed as Q5_1 planes with m = -16 d (exact; 16|d| must
+ * not exceed 65504, else MOE_ERR_INVALID_ARG): every kernel serves it, at two
+ * more bytes per block of HBM traffic. */
 typedef enum {
     MOE_FMT_FROM_PACK = 0, /* forward: accept the pack's formats */
     MOE_FMT_Q8_0 = 1,
     MOE_FMT_Q5_1 = 2,
     MOE_FMT_IQ4_NL = 3,
-    MOE_FMT_NVFP4 = 4
+    MOE_FMT_NVFP4 = 4,
+    MOE_FMT_Q5_0 = 5
 } moe_fmt;
 
 typedef enum { MOE_DT_F32 = 1, MOE_DT_BF16 = 2 } moe_dtype;

@@ -11,7 +11,7 @@ import numpy as np
 
 from . import build as _build
 
-Q8_0, Q5_1, IQ4_NL, NVFP4 = 1, 2, 3, 4
+Q8_0, Q5_1, IQ4_NL, NVFP4, Q5_0 = 1, 2, 3, 4, 5
 
 _lib = None
 

@@ -25,6 +25,10 @@
  * decoders below are written from the format definitions:
  *   Q8_0   32 weights: fp16 d, 32 int8 q              w = d*q
  *   Q5_1   32 weights: fp16 d, fp16 m, 32 5-bit q     w = d*q + m
+ *   Q5_0   32 weights: fp16 d, 32 5-bit q             w = d*(q - 16)  (5.5 bits
+ *                      per weight, the size the model card gives; the centred
+ *                      code is the plainest reading of a five-bit format with a
+ *                      single scale)
  *   IQ4_NL 32 weights: fp16 d, 32 4-bit indices i     w = d*T[i], T a 16-entry
  *                                                     int8 table (an input)
  *   NVFP4  16 weights: E4M3 scale b, 16 E2M1 codes n, and one fp32 scale s per
@@ -36,6 +40,7 @@
  *   Q8_0   34 B: [0,2) d, [2,34) q[32]
  *   Q5_1   24 B: [0,2) d, [2,4) m, [4,8) qh (bit j = bit 4 of element j),
  *               [8,24) qs: element j<16 low nibble of qs[j], j>=16 high nibble of qs[j-16]
+ *   Q5_0   22 B: [0,2) d, [2,6) qh, [6,22) qs, bits and nibbles as Q5_1
  *   IQ4_NL 18 B: [0,2) d, [2,18) qs, nibble order as Q5_1
  *   NVFP4   9 B: [0] E4M3 scale, [1,9) element 2i low / 2i+1 high nibble of byte i
  *
@@ -111,6 +116,7 @@ int64_t oracle_row_bytes(int fmt, int64_t cols)
     switch (fmt) {
     case ORACLE_Q8_0: return cols / 32 * 34;
     case ORACLE_Q5_1: return cols / 32 * 24;
+    case ORACLE_Q5_0: return cols / 32 * 22;
     case ORACLE_IQ4_NL: return cols / 32 * 18;
     case ORACLE_NVFP4: return cols / 16 * 9;
     default: return -1;
@@ -152,6 +158,18 @@ int oracle_decode_row(int fmt, const uint8_t *row, int64_t cols, const int8_t *t
                 int lo = j < 16 ? (qs[j] & 15) : (qs[j - 16] >> 4);
                 int q = lo | (int)(((qh >> j) & 1u) << 4);
                 o[j] = d * q + m;
+            }
+            break;
+        }
+        case ORACLE_Q5_0: {
+            const uint8_t *blk = row + b * 22;
+            double d = oracle_fp16(rd16(blk));
+            uint32_t qh = rd32(blk + 2);
+            const uint8_t *qs = blk + 6;
+            for (int j = 0; j < 32; ++j) {
+                int lo = j < 16 ? (qs[j] & 15) : (qs[j - 16] >> 4);
+                int q = lo | (int)(((qh >> j) & 1u) << 4);
+                o[j] = d * (double)(q - 16);
             }
             break;
         }

@@ -4,7 +4,7 @@
 #define MOE_ORACLE_H
 #include <stdint.h>
 
-enum { ORACLE_Q8_0 = 1, ORACLE_Q5_1 = 2, ORACLE_IQ4_NL = 3, ORACLE_NVFP4 = 4 };
+enum { ORACLE_Q8_0 = 1, ORACLE_Q5_1 = 2, ORACLE_IQ4_NL = 3, ORACLE_NVFP4 = 4, ORACLE_Q5_0 = 5 };
 
 typedef struct {
     int n_experts, hidden, inter, has_shared;

@@ -28,9 +28,10 @@ import numpy as np
 
 from . import build as _build
 
-FMT_Q8_0, FMT_Q5_1, FMT_IQ4_NL, FMT_NVFP4 = 1, 2, 3, 4
+FMT_Q8_0, FMT_Q5_1, FMT_IQ4_NL, FMT_NVFP4, FMT_Q5_0 = 1, 2, 3, 4, 5
 DT_F32, DT_BF16 = 1, 2
-FMT_NAMES = {FMT_Q8_0: "q8_0", FMT_Q5_1: "q5_1", FMT_IQ4_NL: "iq4_nl", FMT_NVFP4: "nvfp4"}
+FMT_NAMES = {FMT_Q8_0: "q8_0", FMT_Q5_1: "q5_1", FMT_IQ4_NL: "iq4_nl", FMT_NVFP4: "nvfp4",
+             FMT_Q5_0: "q5_0"}
 
 # Synthetic IQ4_NL table: the 16 Lloyd-Max levels of N(0,1) (J. Max, "Quantizing
 # for minimum distortion", IRE Trans. IT-6, 1960), scaled so the outermost level
@@ -150,7 +151,7 @@ def _p(a):
 
 def row_bytes(fmt, cols):
     return {FMT_Q8_0: cols // 32 * 34, FMT_Q5_1: cols // 32 * 24, FMT_IQ4_NL: cols // 32 * 18,
-            FMT_NVFP4: cols // 16 * 9}[fmt]
+            FMT_NVFP4: cols // 16 * 9, FMT_Q5_0: cols // 32 * 22}[fmt]
 
 
 def normal(key, n, sigma=1.0):

@@ -40,7 +40,7 @@
 
 #define GOLDEN 0x9E3779B97F4A7C15ULL
 
-enum { FMT_Q8_0 = 1, FMT_Q5_1 = 2, FMT_IQ4_NL = 3, FMT_NVFP4 = 4 };
+enum { FMT_Q8_0 = 1, FMT_Q5_1 = 2, FMT_IQ4_NL = 3, FMT_NVFP4 = 4, FMT_Q5_0 = 5 };
 enum { DT_F32 = 1, DT_BF16 = 2 };
 
 static uint64_t mix64(uint64_t z)
@@ -166,6 +166,7 @@ int64_t synth_row_bytes(int fmt, int64_t cols)
     switch (fmt) {
     case FMT_Q8_0: return cols / 32 * 34;
     case FMT_Q5_1: return cols / 32 * 24;
+    case FMT_Q5_0: return cols / 32 * 22;
     case FMT_IQ4_NL: return cols / 32 * 18;
     case FMT_NVFP4: return cols / 16 * 9;
     default: return -1;
@@ -209,6 +210,29 @@ static void enc_q5_1(const float *w, uint8_t *blk)
     }
     blk[4] = (uint8_t)qh; blk[5] = (uint8_t)(qh >> 8);
     blk[6] = (uint8_t)(qh >> 16); blk[7] = (uint8_t)(qh >> 24);
+}
+
+/* Q5_0: the element of largest magnitude v sets d = -v/16 (fp16), so it gets
+ * code 0; the others q = round(w/d) + 16, clamped to [0, 31]. */
+static void enc_q5_0(const float *w, uint8_t *blk)
+{
+    int jx = 0;
+    for (int j = 1; j < 32; ++j) if (fabs_(w[j]) > fabs_(w[jx])) jx = j;
+    uint16_t dh = f32_to_f16_rne(-w[jx] / 16.f);
+    float d = f16_to_f32(dh);
+    put16(blk, dh);
+    uint32_t qh = 0;
+    uint8_t *qs = blk + 6;
+    memset(qs, 0, 16);
+    for (int j = 0; j < 32; ++j) {
+        float q = d == 0.f ? 16.f : round_away(w[j] / d) + 16.f;
+        int qi = (int)fmin_(31.f, fmax_(0.f, q));
+        if (j < 16) qs[j] |= (uint8_t)(qi & 15);
+        else qs[j - 16] |= (uint8_t)((qi & 15) << 4);
+        qh |= (uint32_t)((qi >> 4) & 1) << j;
+    }
+    blk[2] = (uint8_t)qh; blk[3] = (uint8_t)(qh >> 8);
+    blk[4] = (uint8_t)(qh >> 16); blk[5] = (uint8_t)(qh >> 24);
 }
 
 /* nearest table entry, ties to the lower index.  The table is sorted by value
@@ -343,6 +367,7 @@ int synth_encode(int fmt, const float *w, int64_t rows, int64_t cols, const int8
             switch (fmt) {
             case FMT_Q8_0: enc_q8_0(src, dst); break;
             case FMT_Q5_1: enc_q5_1(src, dst); break;
+            case FMT_Q5_0: enc_q5_0(src, dst); break;
             case FMT_IQ4_NL: enc_iq4_nl(src, dst, table, &srt); break;
             case FMT_NVFP4: enc_nvfp4(src, dst, s_t); break;
             }

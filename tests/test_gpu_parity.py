@@ -53,7 +53,7 @@ def test_zipf_batch_nvfp4_64_tokens():
     _check(li, synth.tokens(wl, li.router, 2), wl.top_k)
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_Q8_0, synth.FMT_Q5_1, synth.FMT_IQ4_NL, synth.FMT_NVFP4])
+@pytest.mark.parametrize("fmt", [synth.FMT_Q8_0, synth.FMT_Q5_1, synth.FMT_IQ4_NL, synth.FMT_NVFP4, synth.FMT_Q5_0])
 def test_every_format_on_both_projections(fmt):
     wl = synth.Workload("fmt", 1024, 32, 256, 4, True, fmt, fmt, synth.DT_BF16, 13, seed=fmt)
     li = synth.layer_inputs(wl)
@@ -62,7 +62,7 @@ def test_every_format_on_both_projections(fmt):
 
 @pytest.mark.parametrize("fmt_gu,fmt_dn", [(synth.FMT_Q8_0, synth.FMT_Q8_0), (synth.FMT_Q5_1, synth.FMT_Q5_1),
                                            (synth.FMT_IQ4_NL, synth.FMT_IQ4_NL), (synth.FMT_NVFP4, synth.FMT_NVFP4),
-                                           (synth.FMT_NVFP4, synth.FMT_Q5_1)])
+                                           (synth.FMT_NVFP4, synth.FMT_Q5_1), (synth.FMT_IQ4_NL, synth.FMT_Q5_0)])
 def test_single_token_streaming_kernel_every_format(fmt_gu, fmt_dn):
     """One token with whole-row bulk copies (hidden and inter multiples of 256):
     fewer experts than SMs, so many CTAs own no router row and a few pairs."""

@@ -115,7 +115,9 @@ def test_prefill_iq4nl_q51_dequant_ragged_batch():
 
 def test_prefill_mixed_formats_small_shapes():
     # Q5_1 gate/up with an IQ4_NL down projection, and Q8_0 with Q5_1: 4-bit and 8-bit dequantisers
-    for gu, dn, seed in ((synth.FMT_Q5_1, synth.FMT_IQ4_NL, 41), (synth.FMT_Q8_0, synth.FMT_Q5_1, 42)):
+    # Q5_0 runs through the Q5_1 planes (m = -16 d)
+    for gu, dn, seed in ((synth.FMT_Q5_1, synth.FMT_IQ4_NL, 41), (synth.FMT_Q8_0, synth.FMT_Q5_1, 42),
+                         (synth.FMT_Q5_0, synth.FMT_IQ4_NL, 43)):
         wl = synth.Workload("mixed", 1024, 48, 256, 6, True, gu, dn, synth.DT_BF16, 200, zipf_s=1.1, seed=seed)
         _run_dq(wl, 200)
 

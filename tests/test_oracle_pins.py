@@ -115,6 +115,38 @@ def test_q5_1_closed_form_and_high_bit_walk():
         assert np.array_equal(got, want), j
 
 
+def _q5_0_block(d_bits, q):
+    # the Q5_1 block without m: d, qh, qs
+    b = _q5_1_block(d_bits, 0, q)
+    return np.concatenate([b[:2], b[4:]])
+
+
+def test_q5_0_closed_form_high_bit_walk_and_negative_scale():
+    q = np.arange(32)
+    blk = _q5_0_block(0x3C00, q)  # d = 1
+    assert blk.size == 22
+    assert np.array_equal(oracle.decode_row(oracle.Q5_0, blk, 32), q - 16.0)
+    # d = -0.5: the code is centred, then scaled (sign included)
+    assert np.array_equal(oracle.decode_row(oracle.Q5_0, _q5_0_block(0xB800, q), 32), -0.5 * (q - 16.0))
+    for j in range(32):  # one fifth bit at a time: only element j leaves -16 + low bits
+        qj = np.zeros(32, np.int64)
+        qj[j] = 16 + (j % 16)
+        got = oracle.decode_row(oracle.Q5_0, _q5_0_block(0x3C00, qj), 32)
+        want = np.full(32, -16.0)
+        want[j] = j % 16
+        assert np.array_equal(got, want), j
+
+
+def test_q5_0_equals_q5_1_with_m_minus_16d():
+    # the identity the pack uses to serve Q5_0 through the Q5_1 planes
+    rng = np.random.default_rng(3)
+    for d_bits, m_bits in ((0x3C00, 0xCC00), (0x2E66, 0xBE66), (0x0401, 0x9401)):  # d, -16 d exactly
+        q = rng.integers(0, 32, 32)
+        a = oracle.decode_row(oracle.Q5_0, _q5_0_block(d_bits, q), 32)
+        b = oracle.decode_row(oracle.Q5_1, _q5_1_block(d_bits, m_bits, q), 32)
+        assert np.array_equal(a, b), hex(d_bits)
+
+
 def _iq4_block(d_bits, idx):
     qs = np.zeros(16, np.uint8)
     for j in range(32):
@@ -163,8 +195,8 @@ def test_sizes_match_pages():
     bpw = {f: float(v) for f, v in _golden("format_sizes.txt")}
     assert oracle.lib().oracle_row_bytes(oracle.IQ4_NL, 32) * 8 / 32 == bpw["IQ4_NL"]
     # Q5_0 (d + 32 five-bit values) is 22 B per 32; Q5_1 adds the fp16 m
-    assert (22 + 2) * 8 / 32 == oracle.lib().oracle_row_bytes(oracle.Q5_1, 32) * 8 / 32
-    assert 22 * 8 / 32 == bpw["Q5_0"]
+    assert oracle.lib().oracle_row_bytes(oracle.Q5_0, 32) * 8 / 32 == bpw["Q5_0"]
+    assert oracle.lib().oracle_row_bytes(oracle.Q5_1, 32) == oracle.lib().oracle_row_bytes(oracle.Q5_0, 32) + 2
     assert oracle.lib().oracle_row_bytes(oracle.Q8_0, 32) == 34
     assert oracle.lib().oracle_row_bytes(oracle.NVFP4, 16) * 8 / 16 == 4.5
     g = {k: float(v) for k, v in _golden("expert_bytes.txt")}

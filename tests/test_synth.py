@@ -47,6 +47,23 @@ def test_q5_1_roundtrip_within_half_step():
     assert np.all(err <= d[..., None] / 2 * (1 + 1e-3) + 1e-6)
 
 
+def test_q5_0_roundtrip_within_half_step_and_extreme_exact():
+    w, deq, blocks, _ = _roundtrip(synth.FMT_Q5_0)
+    d = blocks.reshape(64, -1, 22)[..., :2].copy().view(np.float16)[..., 0].astype(np.float64)
+    err = np.abs(w - deq).reshape(64, -1, 32)
+    ad = np.abs(d[..., None])
+    # codes run -16 .. 15 around zero: an element opposite the extreme one can
+    # need +16 and is clamped to 15 (error at most one step); the rest round
+    clamped = w.reshape(64, -1, 32) / d[..., None] > 15.5
+    assert np.all(err <= ad * (1 + 1e-3) + 1e-6)
+    assert np.all(err[~clamped] <= ad[..., 0:1].repeat(32, -1)[~clamped] / 2 * (1 + 1e-3) + 1e-6)
+    # the element of largest magnitude gets code 0: it decodes to -16 d
+    wb = w.reshape(64, -1, 32)
+    jx = np.abs(wb).argmax(-1)
+    ext = np.take_along_axis(deq.reshape(64, -1, 32), jx[..., None], -1)[..., 0]
+    assert np.array_equal(ext, -16.0 * d)
+
+
 def test_iq4_nl_picks_nearest_level():
     w, deq, blocks, _ = _roundtrip(synth.FMT_IQ4_NL)
     d = blocks.reshape(64, -1, 18)[..., :2].copy().view(np.float16)[..., 0].astype(np.float64)
