@@ -206,3 +206,32 @@ def test_dense_batched_variant_matches_oracle(name, T):
     ref, ridx, rgate = oracle_layer(li, x, wl.top_k)
     assert_routing_equal(idx, gate, ridx, rgate)
     assert normwise_err(out, ref) <= DECODE_TOL
+
+
+def test_grouped_cuda_core_path_when_weights_are_not_fp16_normal():
+    """Block scales below 2^-14 make some weights fp16 subnormals: the pack turns
+    the tensor-core decode off and 2-64 tokens run the CUDA-core grouped kernels."""
+    wl = synth.Workload("tiny_scales", 2048, 64, 512, 8, True, synth.FMT_Q8_0, synth.FMT_Q8_0, synth.DT_BF16, 8,
+                        sigma_w=3e-4, seed=21)
+    li = synth.layer_inputs(wl)
+    _check(li, synth.tokens(wl, li.router), wl.top_k)
+
+
+def test_tensor_core_decode_reports_h_outside_fp16_range():
+    """Weights large enough that h = silu(G x) (U x) passes 65,504: the tensor-core
+    decode records MOE_ERR_RANGE; the fp32 grouped path computes the layer."""
+    import block_quantized_expert_moe_b200 as bq
+    wl = synth.Workload("big_h", 1024, 32, 256, 4, True, synth.FMT_Q8_0, synth.FMT_Q8_0, synth.DT_BF16, 8,
+                        sigma_w=1000.0, seed=22)
+    li = synth.layer_inputs(wl)
+    x = synth.tokens(wl, li.router)
+    pack = bq.pack_layer(li, max_tokens=8, max_top_k=wl.top_k)
+    out = torch.zeros(8, wl.hidden, device="cuda")
+    bq.moe_layer_forward(to_device(x), router_to_device(li.router), pack, bq.MOE_FMT_FROM_PACK, wl.top_k, out)
+    torch.cuda.synchronize()
+    assert bq.moe_get_device_error(pack) == bq.MOE_ERR_RANGE
+    pack.free()
+    out_g, idx, gate, _ = gpu_layer(li, x, wl.top_k, path=bq.MOE_PATH_GROUPED)
+    ref, ridx, rgate = oracle_layer(li, x, wl.top_k)
+    assert_routing_equal(idx, gate, ridx, rgate)
+    assert normwise_err(out_g, ref) <= DECODE_TOL
