@@ -368,7 +368,10 @@ def ours_arm(a, wl):
         stage_ms += m
         nf += n
     prefill_kernels = 7 if wl.fmt_gate_up == synth.FMT_NVFP4 else 6  # route GEMM, top-k, plan, gather, GEMMs (+ h quant)
-    launches_per_fwd = 1 if stage_ms[4] > 0 else (prefill_kernels if stage_ms[5] > 0 else 4)
+    # grouped decode: route, (x gather,) gate/up, down, combine; the x gather runs
+    # with the tensor-core kernels (2-64 tokens, H and I multiples of 256)
+    tc_path = a.path == "auto" and 2 <= T <= 64 and H % 256 == 0 and wl.inter % 256 == 0
+    launches_per_fwd = 1 if stage_ms[4] > 0 else (prefill_kernels if stage_ms[5] > 0 else (5 if tc_path else 4))
     stage_us = {s: float(stage_ms[i] / nf * 1e3) for i, s in enumerate(STAGES) if stage_ms[i] > 0}
     phase_names = (["stage_x", "router", "logit_poll_topk", "issue", "gate_up", "h_poll", "down", "-", "tail"]
                    if T == 1 else

@@ -235,3 +235,10 @@ def test_tensor_core_decode_reports_h_outside_fp16_range():
     ref, ridx, rgate = oracle_layer(li, x, wl.top_k)
     assert_routing_equal(idx, gate, ridx, rgate)
     assert normwise_err(out_g, ref) <= DECODE_TOL
+
+
+def test_tensor_core_decode_with_fp32_tokens():
+    """fp32 x (rounded to fp16 in the gather, 2^-12 relative) through the tensor-core decode."""
+    wl, li = _layer("tiny_q8")
+    x = synth.tokens(wl, li.router, 0, 0, 6)
+    _check(li, x, wl.top_k)
