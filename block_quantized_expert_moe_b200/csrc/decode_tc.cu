@@ -13,7 +13,7 @@
 // most 2^-12 relatively, x is exact (bf16 has 8) once scaled by a power of two
 // below 2^15 per token, h loses 2^-12.
 //
-//   gather    one warp per token: x[t] into the fp16 rows of its k routed
+//   gather    one CTA per token: x[t] into the fp16 rows of its k routed
 //             slots and of its shared-expert slot (the plan's slot order: every
 //             expert's slots contiguous), times 2^-s with s the smallest
 //             exponent that brings max |x[t]| below 2^15; the slot's 2^s beside
@@ -35,12 +35,12 @@
 //
 // Every mbarrier wait is bounded; a wait that runs out records MOE_ERR_TIMEOUT
 // and the CTA stops issuing work.  An h outside the fp16 range records
-// MOE_ERR_RANGE (the CUDA-core grouped path takes such layers).
+// MOE_ERR_RANGE (MOE_PATH_GROUPED computes such layers in fp32).
 #include <cuda.h>
-
-#include <algorithm>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "dequant.cuh"
 #include "moe_internal.cuh"

@@ -732,8 +732,9 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
         prof_mark(pm, pbase, 1, s);
         return st;
     }
-    // two or more tokens: the streamed grouped matvecs (rows per lane, TMA-fed),
-    // when the planes' rows fit their tile loads
+    // two or more tokens: the tensor-core grouped decode (below), else the
+    // streamed grouped matvecs (rows per lane, TMA-fed) when the planes' rows
+    // fit their tile loads, else the fused or plain grouped kernels
     if (pm->sgm < 0) {
         const int slots = p->E + (p->has_shared ? 1 : 0);
         pm->sgm = (w.max_groups <= sgm_max_groups() && p->I % 16 == 0 && p->H % 32 == 0 &&
