@@ -638,11 +638,12 @@ moe_status moe_route_topk(const void *x, moe_dtype x_dtype, const uint16_t *rout
                           int hidden, int n_experts, int top_k, int32_t *idx_out, float *gate_out,
                           void *workspace, size_t workspace_bytes, void *stream)
 {
+    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+    if (n_tokens < 0 || hidden < 8 || hidden % 8 || hidden > 16384) return MOE_ERR_INVALID_ARG;
+    if (n_experts < 1 || n_experts > 1024 || top_k < 1 || top_k > n_experts) return MOE_ERR_INVALID_ARG;
+    if (n_tokens == 0) return MOE_OK;  // an empty batch: nothing to enqueue
     if (!x || !router_w || !idx_out || !gate_out || !workspace) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(router_w) || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
-    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
-    if (n_tokens < 1 || hidden < 8 || hidden % 8 || hidden > 16384) return MOE_ERR_INVALID_ARG;
-    if (n_experts < 1 || n_experts > 1024 || top_k < 1 || top_k > n_experts) return MOE_ERR_INVALID_ARG;
     if (workspace_bytes < moe_route_workspace_bytes(n_tokens, n_experts)) return MOE_ERR_INVALID_ARG;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -683,10 +684,9 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
                                 const moe_pack *p, moe_fmt fmt, int n_tokens, int top_k, float *out,
                                 moe_path path, void *stream)
 {
-    if (!p || !x || !router_w || !out) return MOE_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(router_w) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    if (!p) return MOE_ERR_INVALID_ARG;
     if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
-    if (n_tokens < 1 || n_tokens > p->max_tokens) return MOE_ERR_INVALID_ARG;
+    if (n_tokens < 0 || n_tokens > p->max_tokens) return MOE_ERR_INVALID_ARG;
     if (top_k < 1 || top_k > p->max_top_k) return MOE_ERR_INVALID_ARG;
     if (fmt != MOE_FMT_FROM_PACK && fmt != p->fmt_gu_in) return MOE_ERR_FMT_MISMATCH;
     const bool prefill_ok = p->has_prefill && x_dtype == MOE_DT_BF16 && top_k <= 32;
@@ -697,6 +697,10 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
         return MOE_ERR_UNSUPPORTED;
     if (path != MOE_PATH_DECODE && path != MOE_PATH_GROUPED && path != MOE_PATH_PREFILL && path != MOE_PATH_DENSE)
         return MOE_ERR_UNSUPPORTED;
+    // an empty batch enqueues nothing and leaves the pack's routing record as it was
+    if (n_tokens == 0) return MOE_OK;
+    if (!x || !router_w || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
     DeviceGuard g(p->device);
     if (!g.ok) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

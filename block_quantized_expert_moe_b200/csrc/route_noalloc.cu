@@ -70,11 +70,12 @@ extern "C" moe_status moe_route_topk_noalloc(const void *x, moe_dtype x_dtype, c
                                               int n_tokens, int hidden, int n_experts, int top_k,
                                               int32_t *idx_out, float *gate_out, void *stream)
 {
+    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+    if (n_tokens < 0 || hidden < 8 || hidden % 8 || hidden > 16384) return MOE_ERR_INVALID_ARG;
+    if (n_experts < 1 || n_experts > 1024 || top_k < 1 || top_k > n_experts) return MOE_ERR_INVALID_ARG;
+    if (n_tokens == 0) return MOE_OK;  // an empty batch: nothing to enqueue
     if (!x || !router_w || !idx_out || !gate_out) return MOE_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(router_w)) & 15u) return MOE_ERR_INVALID_ARG;
-    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
-    if (n_tokens < 1 || hidden < 8 || hidden % 8 || hidden > 16384) return MOE_ERR_INVALID_ARG;
-    if (n_experts < 1 || n_experts > 1024 || top_k < 1 || top_k > n_experts) return MOE_ERR_INVALID_ARG;
     if ((long long)n_tokens * n_experts > kNoallocLogits) return MOE_ERR_INVALID_ARG;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;

@@ -179,7 +179,9 @@ size_t moe_route_workspace_bytes(int n_tokens, int n_experts);
  *   gate_out  device, [n_tokens x top_k] fp32 gates (sum to 1 per token)
  *   workspace device, moe_route_workspace_bytes(n_tokens, n_experts) bytes,
  *             owned by the caller; its contents need no initialisation
- * hidden % 8 == 0, 1 <= top_k <= n_experts <= 1024.  More than 64 bf16 tokens
+ * hidden % 8 == 0, 1 <= top_k <= n_experts <= 1024, n_tokens >= 0; with
+ * n_tokens == 0 the call returns MOE_OK and enqueues nothing (the pointers are
+ * not read and may be NULL).  More than 64 bf16 tokens
  * run the router as a tensor-core GEMM.  If one of the kernels' bounded waits
  * (the GEMM's pipeline, or the bulk copy of router rows into shared memory)
  * runs out, int32 word 1 of the workspace holds MOE_ERR_TIMEOUT afterwards. */
@@ -212,8 +214,11 @@ moe_status moe_route_topk_noalloc(const void *x, moe_dtype x_dtype, const uint16
  *   router_w device [n_experts x hidden] bf16 bits
  *   fmt      MOE_FMT_FROM_PACK, or the pack's gate/up format (checked)
  *   out      device [n_tokens x hidden] fp32
- * 1 <= n_tokens <= max_tokens, 1 <= top_k <= max_top_k.  Enqueues on `stream`
- * (a cudaStream_t; NULL is the legacy default stream). */
+ * 0 <= n_tokens <= max_tokens, 1 <= top_k <= max_top_k.  Enqueues on `stream`
+ * (a cudaStream_t; NULL is the legacy default stream).  An empty batch
+ * (n_tokens == 0) returns MOE_OK after the pack, format, top_k and path checks,
+ * enqueues nothing, does not read x or out (either may be NULL) and leaves the
+ * routing that moe_read_routing reports as the previous forward left it. */
 moe_status moe_layer_forward(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
                              const moe_pack *pack, moe_fmt fmt, int n_tokens, int top_k,
                              float *out, void *stream);
@@ -226,7 +231,9 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
 /* After a forward: copy its routing and plan to HOST memory (synchronises
  * `stream`).  Any pointer may be NULL.
  *   idx   [n_tokens x top_k] int32, gate [n_tokens x top_k] fp32,
- *   counts [n_experts + 1] int32 tokens per expert (last entry: shared). */
+ *   counts [n_experts + 1] int32 tokens per expert (last entry: shared).
+ * 1 <= n_tokens <= max_tokens and 1 <= top_k <= max_top_k, else
+ * MOE_ERR_INVALID_ARG; they should be the last non-empty forward's. */
 moe_status moe_read_routing(const moe_pack *pack, int n_tokens, int top_k, int32_t *idx,
                             float *gate, int32_t *counts, void *stream);
 

@@ -88,3 +88,16 @@ def test_forward_and_route_reject_null_and_misaligned_pointers():
     assert bq.lib.moe_route_topk(a, 2, a, 1, 64, 4, 5, a, a, a, 4096, None) == bq.MOE_ERR_INVALID_ARG
     assert bq.lib.moe_route_topk(a, 2, a, 1, 60, 4, 2, a, a, a, 4096, None) == bq.MOE_ERR_INVALID_ARG
     assert bq.lib.moe_route_topk(a, 2, a, 1, 64, 4, 2, a, a, a, 16, None) == bq.MOE_ERR_INVALID_ARG
+
+
+def test_empty_batch_routes_nothing_without_a_device():
+    # n_tokens == 0 is a no-op: MOE_OK before any pointer is read or any CUDA call is made
+    assert bq.lib.moe_route_topk(None, 2, None, 0, 64, 4, 2, None, None, None, 0, None) == bq.MOE_OK
+    assert bq.lib.moe_route_topk_noalloc(None, 1, None, 0, 64, 4, 2, None, None, None) == bq.MOE_OK
+    assert bq.moe_route_workspace_bytes(0, 4) == 0
+    # the other arguments are still checked, and a negative count is an error
+    assert bq.lib.moe_route_topk(None, 2, None, 0, 60, 4, 2, None, None, None, 0, None) == bq.MOE_ERR_INVALID_ARG
+    assert bq.lib.moe_route_topk(None, 2, None, 0, 64, 4, 5, None, None, None, 0, None) == bq.MOE_ERR_INVALID_ARG
+    assert bq.lib.moe_route_topk(None, 7, None, 0, 64, 4, 2, None, None, None, 0, None) == bq.MOE_ERR_INVALID_ARG
+    assert bq.lib.moe_route_topk(None, 2, None, -1, 64, 4, 2, None, None, None, 0, None) == bq.MOE_ERR_INVALID_ARG
+    assert bq.lib.moe_layer_forward(None, 2, None, None, 0, 0, 1, None, None) == bq.MOE_ERR_INVALID_ARG

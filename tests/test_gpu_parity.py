@@ -133,6 +133,32 @@ def test_fmt_argument_is_checked():
     pack.free()
 
 
+def test_empty_batch_is_a_no_op():
+    """Zero tokens: every entry point returns MOE_OK, enqueues nothing and leaves the
+    routing record of the previous forward in place."""
+    import block_quantized_expert_moe_b200 as bq
+    wl, li = _layer("tiny_q8")
+    x = synth.tokens(wl, li.router, 0, 0, 3)
+    pack = bq.pack_layer(li, max_tokens=8)
+    wr = router_to_device(li.router)
+    out = torch.empty(3, wl.hidden, device="cuda")
+    bq.moe_layer_forward(to_device(x), wr, pack, bq.MOE_FMT_FROM_PACK, wl.top_k, out)
+    before = bq.moe_read_routing(pack, 3, wl.top_k)
+    empty_x = torch.empty(0, wl.hidden, device="cuda")
+    empty_out = torch.empty(0, wl.hidden, device="cuda")
+    for path in (bq.MOE_PATH_AUTO, bq.MOE_PATH_DECODE, bq.MOE_PATH_GROUPED):
+        bq.moe_layer_forward_ex(empty_x, wr, pack, bq.MOE_FMT_FROM_PACK, wl.top_k, empty_out, path)
+    idx = torch.empty(0, wl.top_k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(0, wl.top_k, dtype=torch.float32, device="cuda")
+    ws = torch.empty(bq.moe_route_workspace_bytes(0, wl.n_experts), dtype=torch.uint8, device="cuda")
+    bq.moe_route_topk(empty_x, wr, wl.top_k, idx, gate, ws)
+    torch.cuda.synchronize()
+    after = bq.moe_read_routing(pack, 3, wl.top_k)
+    assert all(np.array_equal(a, b) for a, b in zip(before, after))
+    assert bq.moe_get_device_error(pack) == bq.MOE_OK
+    pack.free()
+
+
 def test_pack_rejects_nan_block_scale():
     import block_quantized_expert_moe_b200 as bq
     wl = synth.Workload("nan", 64, 4, 32, 2, False, synth.FMT_NVFP4, synth.FMT_NVFP4, synth.DT_BF16, 1)
@@ -242,3 +268,18 @@ def test_tensor_core_decode_with_fp32_tokens():
     wl, li = _layer("tiny_q8")
     x = synth.tokens(wl, li.router, 0, 0, 6)
     _check(li, x, wl.top_k)
+
+
+def test_tensor_core_decode_sixty_four_identical_tokens():
+    """The largest group the tensor-core decode takes: 64 copies of one token send all 64
+    to the same k experts (N = 64 per tile).  Tokens are independent, so every output row
+    must equal the first, bit for bit, and match the oracle."""
+    wl, li = _layer("model_decode", layer=1)
+    x = np.repeat(synth.tokens(wl, li.router, 1, 0, 1), 64, axis=0)
+    out, idx, gate, counts = gpu_layer(li, x, wl.top_k)
+    ref, ridx, rgate = oracle_layer(li, x[:1], wl.top_k)
+    assert_routing_equal(idx[:1], gate[:1], ridx, rgate)
+    assert (idx == idx[0]).all() and (gate == gate[0]).all()
+    assert np.array_equal(counts, expected_counts(np.repeat(ridx, 64, axis=0), wl.n_experts, 64, wl.has_shared))
+    assert (out == out[0]).all()
+    assert normwise_err(out[:1], ref) <= DECODE_TOL
