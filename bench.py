@@ -183,6 +183,15 @@ def oracle_rate(li, wl, budget_s, max_s=30.0):
     return done / spent, done, spent, oracle.threads()
 
 
+def workload_config(wl, layers, tokens, world):
+    """The workload keys both arms report in `config`."""
+    return {"workload": wl.name, "layers_per_step": layers, "tokens_per_layer": tokens,
+            "hidden": wl.hidden, "experts": wl.n_experts, "inter": wl.inter, "top_k": wl.top_k,
+            "shared_expert": wl.has_shared,
+            "formats": f"{synth.FMT_NAMES[wl.fmt_gate_up]}/{synth.FMT_NAMES[wl.fmt_down]}",
+            "parallelism": f"replicas x{world}"}
+
+
 def reference_arm(a, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -190,7 +199,7 @@ def reference_arm(a, wl):
     li = synth.layer_inputs(wl, 0)
     import oracle
     ex = oracle.Experts.from_layer(li)
-    n = max(1, wl.tokens)
+    n = max(1, a.tokens or wl.tokens)
     per_step = []
     total_tok = 0
     for s in range(a.warmup + a.steps):
@@ -208,7 +217,8 @@ def reference_arm(a, wl):
             "impl": "reference", "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
             "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "tokens_per_layer": n, "parallelism": "replicas"},
+            "config": dict(workload_config(wl, 1, n, a.gpus), path="oracle",
+                           l2="host memory: one layer per step, fp64 oracle on the host cores"),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -464,13 +474,9 @@ def ours_arm(a, wl):
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
                 "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": {"workload": wl.name, "layers_per_step": L, "tokens_per_layer": T,
-                           "hidden": H, "experts": E, "inter": I, "top_k": k,
-                           "shared_expert": wl.has_shared,
-                           "formats": f"{synth.FMT_NAMES[wl.fmt_gate_up]}/{synth.FMT_NAMES[wl.fmt_down]}",
-                           "parallelism": f"replicas x{world}", "path": a.path,
-                           "l2": f"inputs larger than L2: {L} distinct layers, "
-                                 f"{unique_bytes_step / 1e6:.0f} MB of selected expert weights per step"},
+                "config": dict(workload_config(wl, L, T, world), path=a.path,
+                               l2=f"inputs larger than L2: {L} distinct layers, "
+                                  f"{unique_bytes_step / 1e6:.0f} MB of selected expert weights per step"),
                 "expert_gbs": expert_gbs, "expert_gbs_frac": expert_gbs / hbm,
                 "unique_expert_bytes_per_step": unique_bytes_step,
                 "active_experts_per_layer": float(np.mean(n_active)),

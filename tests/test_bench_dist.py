@@ -57,3 +57,27 @@ def test_single_rank_needs_no_process_group():
     assert bench.reduce_max(None, 3.5, "cpu") == 3.5
     bench.sync_barrier(None, lambda: None)
     assert bench.job_throughput(1, 10, 48, 1, 100.0) == 4800.0
+
+
+def test_reference_arm_line_on_the_host():
+    """`bench.py --impl reference` times the oracle on the host and prints one JSON line
+    with the contract's keys and the workload keys of the GPU arm's config."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_q8", "--steps", "2", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3 and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    import bench
+    import synth
+    want = bench.workload_config(synth.WORKLOADS["tiny_q8"], 1, 1, 1)
+    assert {k: d["config"][k] for k in want} == want
