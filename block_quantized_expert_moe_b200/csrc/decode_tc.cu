@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t fa_bar[kDtMaxAStages], ae_bar[kDtMaxAStages], fb_bar[kDtMaxBSlots],
         be_bar[kDtMaxBSlots];
-    __shared__ __align__(8) uint64_t rf_bar[kDtMaxRawStages], re_bar[kDtMaxRawStages], accf_bar, acce_bar;
+    __shared__ __align__(8) uint64_t rf_bar[kDtMaxRawStages], re_bar[kDtMaxRawStages], accf_bar, acce_bar, dr_bar;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tasks = *g.n_groups * g.NB;
     const int KT = g.K / 64, KR = g.K / 256;  // MMA slices and raw stages per task
+    int raw_issued = 0, b_issued = 0;         // stages the two TMA producers armed
 
     if (warp == kDtMmaWarp) {
         tmem_alloc(&tmem_base, kDtTmemCols);
@@ -162,6 +163,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
         }
         mbar_init(&accf_bar, 1);
         mbar_init(&acce_bar, kDtEpiWarps);
+        mbar_init(&dr_bar, 1);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -199,6 +201,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
                     }
                 }
             }
+            raw_issued = rr.u * NR + rr.s;
         }
     } else if (warp == kDtBWarp) {  // ---- B tiles: the group's slot rows, 16 at a time
         if (lane == 0) {
@@ -219,6 +222,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
                         tma_load_2d(b_s + jj * 2048, &tmB, &fb_bar[s], kt * 64, gr.y + 16 * jj);
                 }
             }
+            b_issued = rb.u * NBS + rb.s;
         }
     } else if (warp == kDtMmaWarp) {  // ---- MMA issuer
         if (lane == 0) {
@@ -377,7 +381,14 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     }
     tc_fence_before_sync();
     __syncthreads();
-    if (abort_flag && threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+    if (abort_flag) {  // block-uniform after the barrier: drain what was issued, then release
+        if (lane == 0 && warp == kDtRawWarp) drain_ring(rf_bar, NR, raw_issued);
+        if (lane == 0 && warp == kDtBWarp) drain_ring(fb_bar, NBS, b_issued);
+        if (lane == 0 && warp == kDtMmaWarp) drain_mma(&dr_bar);
+        if (threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+        tc_fence_before_sync();
+        __syncthreads();
+    }
     if (warp == kDtMmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, kDtTmemCols);

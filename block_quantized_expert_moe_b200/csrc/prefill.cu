@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * BN;
     const int KT = (g.K + kBK - 1) / kBK;
+    int tma_issued = 0;  // stages the TMA producer armed
 
     if (warp == 5) {
         tmem_alloc(&tmem_base, BN);
@@ -89,6 +90,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 mbar_arrive_expect_tx(&full_bar[s], STAGE);
                 tma_load_2d(a_s, &tmA, &full_bar[s], kt * kBK, m0);
                 tma_load_2d(b_s, &tmB, &full_bar[s], kt * kBK, n0);
+                tma_issued = kt + 1;
             }
         }
     } else if (warp == 5) {
@@ -135,13 +137,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             }
-        } else if (threadIdx.x == 0) {
-            atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+        } else {
+            abort_flag = 1;
+            if (threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
         }
     }
     tc_fence_before_sync();
     __syncthreads();
-    if (abort_flag && threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+    if (abort_flag) {  // block-uniform after the barrier: drain what was issued, then release
+        if (warp == 4 && lane == 0) drain_ring(full_bar, STAGES, tma_issued);
+        if (warp == 5 && lane == 0) mbar_wait(&acc_bar, 0);  // committed after the last MMA this thread issued
+        if (threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+        tc_fence_before_sync();
+        __syncthreads();
+    }
     if (warp == 5) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, BN);
@@ -330,13 +339,14 @@ __global__ void __launch_bounds__(kNvThreads, 1)
                               const NvGemmArgs g)
 {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full_bar[kNvStages], empty_bar[kNvStages], accf_bar, acce_bar;
+    __shared__ __align__(8) uint64_t full_bar[kNvStages], empty_bar[kNvStages], accf_bar, acce_bar, dr_bar;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = *g.n_tiles * g.NT;
     const int KT = g.K / 256;  // stages per tile
+    int tma_issued = 0;        // stages the TMA producer armed
 
     if (warp == kNvMmaWarp) {
         tmem_alloc(&tmem_base, kNvTmemCols);
@@ -349,6 +359,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
         }
         mbar_init(&accf_bar, 1);
         mbar_init(&acce_bar, kNvEpiWarps);
+        mbar_init(&dr_bar, 1);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -396,6 +407,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
                     }
                 }
             }
+            tma_issued = it;
         }
     } else if (warp == kNvMmaWarp) {
         if (lane == 0) {
@@ -436,6 +448,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
             const bool ok = mbar_wait(&accf_bar, tcount & 1);
             tc_fence_after_sync();
             if (!ok || abort_flag) {
+                abort_flag = 1;
                 if (threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
                 break;
             }
@@ -489,7 +502,13 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     }
     tc_fence_before_sync();
     __syncthreads();
-    if (abort_flag && threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+    if (abort_flag) {  // block-uniform after the barrier: drain what was issued, then release
+        if (warp == kNvTmaWarp && lane == 0) drain_ring(full_bar, kNvStages, tma_issued);
+        if (warp == kNvMmaWarp && lane == 0) drain_mma(&dr_bar);
+        if (threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+        tc_fence_before_sync();
+        __syncthreads();
+    }
     if (warp == kNvMmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, kNvTmemCols);

@@ -84,13 +84,15 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     dq_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const Q8GemmArgs g)
 {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t fa_bar[kQ8Stages], fb_bar[kQ8Stages], empty_bar[kQ8Stages], accf_bar, acce_bar;
+    __shared__ __align__(8) uint64_t fa_bar[kQ8Stages], fb_bar[kQ8Stages], empty_bar[kQ8Stages], accf_bar, acce_bar,
+        dr_bar;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = *g.n_ptiles * g.NT;
     const int KT = g.K / 64;
+    int tma_issued = 0;  // stages the activation producer armed
 
     if (warp == kQ8MmaWarp) {
         tmem_alloc(&tmem_base, 512);
@@ -104,6 +106,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         }
         mbar_init(&accf_bar, 1);
         mbar_init(&acce_bar, kQ8EpiWarps);
+        mbar_init(&dr_bar, 1);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -130,6 +133,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
                     if (pt.z == 2) tma_load_2d(a_s + kQ8A, &tmA, &fa_bar[s], kt * 64, pt.y + 128);
                 }
             }
+            tma_issued = it;
         }
     } else if (warp == kQ8MmaWarp) {  // ---- MMA issuer
         if (lane == 0) {
@@ -220,6 +224,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
             const bool ok = mbar_wait(&accf_bar, tcount & 1);
             tc_fence_after_sync();
             if (!ok || abort_flag) {
+                abort_flag = 1;
                 if (threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
                 break;
             }
@@ -274,7 +279,13 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     }
     tc_fence_before_sync();
     __syncthreads();
-    if (abort_flag && threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+    if (abort_flag) {  // block-uniform after the barrier: drain what was issued, then release
+        if (warp == kQ8TmaWarp && lane == 0) drain_ring(fa_bar, kQ8Stages, tma_issued);
+        if (warp == kQ8MmaWarp && lane == 0) drain_mma(&dr_bar);
+        if (threadIdx.x == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+        tc_fence_before_sync();
+        __syncthreads();
+    }
     if (warp == kQ8MmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);

@@ -165,6 +165,32 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar)
                  : "memory");
 }
 
+// ---- draining an aborted pipeline ------------------------------------------
+// After a bounded wait has given up, copies and MMAs that were already issued
+// may still be landing in shared or tensor memory; the CTA waits for them
+// (again bounded) before it releases either.
+
+// A producer that armed `issued` stages so far, in a ring of n full barriers
+// (one expect-tx arrival each): the last min(n, issued) arms are the newest
+// phase of each barrier, so their completion covers every copy in flight.
+__device__ __forceinline__ bool drain_ring(uint64_t *full, int n, int issued)
+{
+    bool ok = true;
+    for (int i = 1; i <= n && i <= issued; ++i) {
+        const int p = issued - i;
+        ok = mbar_wait(&full[p % n], (uint32_t)(p / n) & 1u) && ok;
+    }
+    return ok;
+}
+
+// The MMA issuer: `bar` is a fresh barrier (count 1, never used); the commit
+// arrives once every tensor-core operation this thread issued has finished.
+__device__ __forceinline__ bool drain_mma(uint64_t *bar)
+{
+    mma_commit(bar);
+    return mbar_wait(bar, 0);
+}
+
 // Copy 32 rows x 16 bytes of shared memory (matrix descriptor) into tensor
 // memory at `taddr`, replicated to the four 32-lane quarters.
 __device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc)
