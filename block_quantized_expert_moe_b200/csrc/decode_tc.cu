@@ -339,7 +339,10 @@ __global__ void __launch_bounds__(kDtThreads, 1)
             tc_fence_after_sync();
             // the warp leaves together (its tensor-memory loads are warp-wide)
             if (!__all_sync(0xffffffffu, w_ok) || __any_sync(0xffffffffu, abort_flag != 0)) {
-                if (lane == 0) atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+                if (lane == 0) {
+                    abort_flag = 1;
+                    atomicExch(g.err, (int)MOE_ERR_TIMEOUT);
+                }
                 break;
             }
             const int4 gr = g.groups[task / g.NB];
