@@ -41,12 +41,13 @@ struct moe_pack {
     int64_t arena_bytes = 0, workspace_bytes = 0;
     int grid_cache[2][2];  // [gateup][tt==8]
     // kernel-stage timing (moe_profile_begin/end): per recorded forward, the
-    // first event index and its path (fused: 2 events, grouped: 5)
+    // first event index and its kind (0 grouped: 5 events around route, gate/up,
+    // down and combine; 1 single-kernel decode: 2 events; 2 prefill: 2 events)
     bool prof_on = false;
     std::vector<cudaEvent_t> prof_ev;
     std::vector<std::pair<int, int>> prof_fwd;
     int prof_used = 0;
-    long long *prof_stamps = nullptr;  // device, 16 clock64 stamps per recorded fused forward
+    long long *prof_stamps = nullptr;  // device, kStampStride stamps per recorded forward
     int prof_nstamp = 0, prof_stamp_cap = 0;
     int fused_grid[2] = {0, 0};   // [tt==8]
     int stream1 = -1;             // single-token streaming kernel usable (-1: not yet checked)
@@ -455,7 +456,7 @@ moe_status build_workspace(moe_pack *p)
     return MOE_OK;
 }
 
-// Buffers of the tensor-core prefill (NVFP4 experts, more than 64 tokens).
+// Buffers of the tensor-core prefill (packs for more than 64 tokens whose formats it takes).
 moe_status build_prefill_workspace(moe_pack *p)
 {
     const int64_t T = p->max_tokens, k = p->max_top_k, E = p->E, H = p->H, I = p->I;
