@@ -26,7 +26,11 @@
  * enqueued.  Forward and route calls only enqueue work on `stream`; they do
  * not synchronise the host and do not allocate.  A launch failure returns
  * MOE_ERR_CUDA.  Errors raised inside kernels (a bounded wait that ran out, a
- * plan overflow) set a sticky word that moe_get_device_error() returns.
+ * plan overflow) set a sticky word that moe_get_device_error() returns.  Every
+ * device-side wait gives up after one to two seconds; the kernel then waits
+ * (again bounded) for the copies and tensor-core operations it has already
+ * issued, releases its tensor memory and returns, so the context stays usable
+ * and the forward's outputs are undefined.
  * One pack runs one forward at a time: two forwards on one pack must be
  * ordered (same stream, or events); concurrent streams need separate packs.
  */
