@@ -72,6 +72,8 @@ def _load():
     L.moe_layer_forward.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, vp]
     L.moe_layer_forward_ex.restype = i32
     L.moe_layer_forward_ex.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, i32, vp]
+    L.moe_debug_fail_alloc_after.restype = i32
+    L.moe_debug_fail_alloc_after.argtypes = [i32]
     L.moe_read_routing.restype = i32
     L.moe_read_routing.argtypes = [vp, i32, i32, vp, vp, vp, vp]
     L.moe_profile_begin.restype = i32
@@ -175,6 +177,11 @@ def moe_pack_query(pack):
     info = moe_pack_info()
     _check(lib.moe_pack_query(pack.handle, ctypes.byref(info)), "moe_pack_query")
     return {f: getattr(info, f) for f, _ in moe_pack_info._fields_}
+
+
+def moe_debug_fail_alloc_after(n):
+    """Tests only: the (n+1)-th device allocation of moe_pack_experts from now fails once (-1: off)."""
+    _check(lib.moe_debug_fail_alloc_after(n), "moe_debug_fail_alloc_after")
 
 
 def moe_route_workspace_bytes(n_tokens, n_experts):

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -320,8 +321,16 @@ void free_pack_memory(moe_pack *p)
     p->allocations.clear();
 }
 
+// Allocation-failure injection (moe_debug_fail_alloc_after): device
+// allocations left before one fails; -1 = off.  The failing call turns it off.
+std::atomic<int> g_fail_alloc_after{-1};
+
 moe_status dev_alloc(moe_pack *p, size_t bytes, void **out)
 {
+    int left = g_fail_alloc_after.load();
+    while (left >= 0 && !g_fail_alloc_after.compare_exchange_weak(left, left - 1)) {
+    }
+    if (left == 0) return MOE_ERR_OOM;  // the injected failure
     void *ptr = nullptr;
     if (cudaMalloc(&ptr, bytes ? bytes : 16) != cudaSuccess) {
         cudaGetLastError();
@@ -598,6 +607,13 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
         return st;
     }
     *out = p;
+    return MOE_OK;
+}
+
+moe_status moe_debug_fail_alloc_after(int n)
+{
+    if (n < -1) return MOE_ERR_INVALID_ARG;
+    g_fail_alloc_after.store(n);
     return MOE_OK;
 }
 

@@ -266,6 +266,14 @@ moe_status moe_read_routing(const moe_pack *pack, int n_tokens, int top_k, int32
 moe_status moe_profile_begin(moe_pack *pack, int max_forwards);
 moe_status moe_profile_end(moe_pack *pack, double *ms, int *n_forwards);
 
+/* Fault injection for tests of the pack's error path: after n (>= 0) more
+ * device allocations by moe_pack_experts succeed, the next one fails, once:
+ * moe_pack_experts then frees what it had allocated and returns MOE_ERR_OOM
+ * with *out NULL.  n = -1 turns the injection off (the failing allocation
+ * also turns it off); n < -1 is MOE_ERR_INVALID_ARG.  Process-wide; no device
+ * is touched by this call. */
+moe_status moe_debug_fail_alloc_after(int n);
+
 /* Sticky device-side error of the pack (synchronises its device), then clears it. */
 moe_status moe_get_device_error(const moe_pack *pack);
 
