@@ -72,6 +72,8 @@ def _load():
     L.moe_layer_forward.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, vp]
     L.moe_layer_forward_ex.restype = i32
     L.moe_layer_forward_ex.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, i32, vp]
+    L.moe_debug_wait_timeout.restype = i32
+    L.moe_debug_wait_timeout.argtypes = [vp, vp]
     L.moe_debug_fail_alloc_after.restype = i32
     L.moe_debug_fail_alloc_after.argtypes = [i32]
     L.moe_read_routing.restype = i32
@@ -177,6 +179,11 @@ def moe_pack_query(pack):
     info = moe_pack_info()
     _check(lib.moe_pack_query(pack.handle, ctypes.byref(info)), "moe_pack_query")
     return {f: getattr(info, f) for f, _ in moe_pack_info._fields_}
+
+
+def moe_debug_wait_timeout(pack, stream=None):
+    """Tests only: a kernel's bounded wait runs out (~1 s) and records MOE_ERR_TIMEOUT in the pack."""
+    _check(lib.moe_debug_wait_timeout(pack.handle, _stream_ptr(stream)), "moe_debug_wait_timeout")
 
 
 def moe_debug_fail_alloc_after(n):

@@ -1092,6 +1092,14 @@ moe_status moe_profile_end(moe_pack *p, double *ms, int *n_forwards)
     return st;
 }
 
+moe_status moe_debug_wait_timeout(const moe_pack *p, void *stream)
+{
+    if (!p) return MOE_ERR_INVALID_ARG;
+    DeviceGuard g(p->device);
+    if (!g.ok) return MOE_ERR_CUDA;
+    return check_launch(launch_wait_probe(p->ws.err, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_get_device_error(const moe_pack *p)
 {
     if (!p) return MOE_ERR_INVALID_ARG;

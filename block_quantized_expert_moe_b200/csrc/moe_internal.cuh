@@ -223,6 +223,9 @@ cudaError_t prefill_set_attributes();
 cudaError_t prefill_nvfp4_set_attributes();
 bool prefill_nvfp4_supported(int H, int I, int E, int k);
 cudaError_t prefill_nvfp4_forward(const PrefillNvArgs &a, cudaStream_t s);
+// One-thread kernel that waits (bounded) on an mbarrier nothing arrives on and
+// records MOE_ERR_TIMEOUT in *err: the failure-path diagnostic.
+cudaError_t launch_wait_probe(int32_t *err, cudaStream_t s);
 cudaError_t prefill_plan_launch(const PrefillWorkspace &w, int E, int T, int has_shared, int32_t *err, cudaStream_t s);
 cudaError_t prefill_q8_set_attributes();
 bool prefill_q8_supported(int fmt_gu, int fmt_dn, int H, int I, int E, int k);  // Q8_0 / IQ4_NL / Q5_1

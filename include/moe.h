@@ -274,6 +274,14 @@ moe_status moe_profile_end(moe_pack *pack, double *ms, int *n_forwards);
  * is touched by this call. */
 moe_status moe_debug_fail_alloc_after(int n);
 
+/* Diagnostic for tests of the failure path: enqueues on `stream` one
+ * single-thread kernel that waits on an mbarrier nothing arrives on, with the
+ * bounded wait every pipeline of the library uses; after about a second it
+ * gives up and records MOE_ERR_TIMEOUT in the pack's error word, which
+ * moe_get_device_error then returns.  The context stays usable.  Argument and
+ * launch errors as the forward. */
+moe_status moe_debug_wait_timeout(const moe_pack *pack, void *stream);
+
 /* Sticky device-side error of the pack (synchronises its device), then clears it. */
 moe_status moe_get_device_error(const moe_pack *pack);
 

@@ -103,7 +103,7 @@ def test_empty_batch_routes_nothing_without_a_device():
     assert bq.lib.moe_layer_forward(None, 2, None, None, 0, 0, 1, None, None) == bq.MOE_ERR_INVALID_ARG
 
 
-def test_alloc_failure_hook_arguments_without_a_device():
+def test_fault_injection_entry_points_check_arguments_without_a_device():
     assert bq.lib.moe_debug_fail_alloc_after(-2) == bq.MOE_ERR_INVALID_ARG
     assert bq.lib.moe_debug_fail_alloc_after(3) == bq.MOE_OK
     assert bq.lib.moe_debug_fail_alloc_after(-1) == bq.MOE_OK
@@ -112,3 +112,4 @@ def test_alloc_failure_hook_arguments_without_a_device():
     h = ctypes.c_void_p()
     assert bq.lib.moe_pack_experts(None, 0, ctypes.byref(h)) == bq.MOE_ERR_INVALID_ARG
     bq.moe_debug_fail_alloc_after(-1)
+    assert bq.lib.moe_debug_wait_timeout(None, None) == bq.MOE_ERR_INVALID_ARG

@@ -1,9 +1,16 @@
-"""Host-side fault injection: a device allocation inside moe_pack_experts fails
-(moe_debug_fail_alloc_after).  Every allocation point must return MOE_ERR_OOM
-with no pack, free what it had allocated, and leave the library able to pack
-and run a layer that matches the oracle.  The failure is made on the host: no
-kernel runs while it is armed."""
-import numpy as np
+"""Failure paths, made without faulting the GPU.
+
+* A device allocation inside moe_pack_experts fails (moe_debug_fail_alloc_after,
+  made on the host): every allocation point returns MOE_ERR_OOM with no pack and
+  frees what it had, and the library still packs and runs a layer that matches
+  the oracle.
+* A device-side bounded wait runs out (moe_debug_wait_timeout: an mbarrier that
+  nothing arrives on): the kernel gives up after about a second, the pack's
+  error word reads MOE_ERR_TIMEOUT once, and the same pack then runs a forward
+  that matches the oracle.
+"""
+import time
+
 import pytest
 
 import synth
@@ -46,3 +53,26 @@ def test_pack_reports_each_injected_allocation_failure_and_recovers():
     ref, ridx, rgate = oracle_layer(li, x, wl.top_k)
     assert_routing_equal(idx, gate, ridx, rgate)
     assert normwise_err(out, ref) <= DECODE_TOL
+
+
+def test_bounded_wait_runs_out_records_timeout_and_the_context_stays_usable():
+    import block_quantized_expert_moe_b200 as bq
+    wl = synth.WORKLOADS["tiny_q8"]
+    li = synth.layer_inputs(wl)
+    pack = bq.pack_layer(li, max_tokens=4)
+    try:
+        assert bq.moe_get_device_error(pack) == bq.MOE_OK
+        t0 = time.perf_counter()
+        bq.moe_debug_wait_timeout(pack)
+        torch.cuda.synchronize()
+        waited = time.perf_counter() - t0
+        assert bq.moe_get_device_error(pack) == bq.MOE_ERR_TIMEOUT
+        assert bq.moe_get_device_error(pack) == bq.MOE_OK  # reading clears the word
+        assert 0.2 < waited < 10.0, waited  # 2^31 SM clocks: about a second
+        x = synth.tokens(wl, li.router, 0, 1, 4)
+        out, idx, gate, _ = gpu_layer(li, x, wl.top_k, pack=pack)
+        ref, ridx, rgate = oracle_layer(li, x, wl.top_k)
+        assert_routing_equal(idx, gate, ridx, rgate)
+        assert normwise_err(out, ref) <= DECODE_TOL
+    finally:
+        pack.free()
