@@ -81,3 +81,20 @@ def test_reference_arm_line_on_the_host():
     import synth
     want = bench.workload_config(synth.WORKLOADS["tiny_q8"], 1, 1, 1)
     assert {k: d["config"][k] for k in want} == want
+
+
+def test_traffic_is_reported_only_for_the_captured_kernel_source(monkeypatch):
+    """The roofline's `traffic` comes from profiles/traffic.json only while the kernel
+    sources hash to the sha the ncu capture was taken on; otherwise it is null."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    key, entry = next(iter(rec.items()))
+    stage, wl_name = key.split(":")
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: entry["source_sha"])
+    assert bench.kernel_traffic(stage, wl_name) == entry["bytes_per_launch"]
+    assert entry["bytes_per_launch"] == entry["dram_read"] + entry["dram_write"]
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "0" * 16)
+    assert bench.kernel_traffic(stage, wl_name) is None
+    assert bench.kernel_traffic(stage, "no_such_workload") is None
