@@ -112,6 +112,13 @@ def _stream_ptr(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _shape2(t, name):
+    shape = tuple(getattr(t, "shape", ()))
+    if len(shape) != 2:
+        raise ValueError(f"{name} must be 2-D, not of shape {shape}")
+    return shape
+
+
 def _dtype_code(t):
     import torch
     if t.dtype == torch.float32:
@@ -121,11 +128,50 @@ def _dtype_code(t):
     raise TypeError(f"activations must be float32 or bfloat16, not {t.dtype}")
 
 
+def _check_tensor(t, name, dtypes, shape):
+    """What the C ABI cannot check from a pointer: type, dtype, shape, contiguity."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor, not {type(t).__name__}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must be {' or '.join(str(d) for d in dtypes)}, not {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _device_ptrs(named, device):
+    """Device pointers of already checked tensors, all in CUDA memory on `device`
+    (default: the first tensor's); raises before any library call."""
+    ptrs = []
+    for name, t in named:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor: the library reads and writes device memory")
+        if device is None:
+            device = t.device.index
+        if t.device.index != device:
+            raise ValueError(f"{name} is on cuda:{t.device.index}, expected cuda:{device}")
+        ptrs.append(t.data_ptr())
+    return ptrs
+
+
+def _act_dtypes():
+    import torch
+    return (torch.float32, torch.bfloat16)
+
+
+def _bf16_bits_dtypes():
+    import torch
+    return (torch.bfloat16, torch.int16, torch.uint16)
+
+
 class Pack:
     """An uploaded expert pack (owns device memory until free())."""
 
-    def __init__(self, handle, desc):
+    def __init__(self, handle, desc, device=0):
         self.handle = handle
+        self.device = device
         self.n_experts = desc.n_experts
         self.hidden = desc.hidden
         self.inter = desc.inter
@@ -168,7 +214,7 @@ def moe_pack_experts(n_experts, hidden, inter, fmt_gate_up, fmt_down, gate_up_bl
                       _np_ptr(sgu), _np_ptr(sdn), flags)
     h = ctypes.c_void_p()
     _check(lib.moe_pack_experts(ctypes.byref(d), device, ctypes.byref(h)), "moe_pack_experts")
-    return Pack(h, d)
+    return Pack(h, d, device)
 
 
 def moe_pack_free(pack):
@@ -199,37 +245,57 @@ def moe_route_topk(x, router_w, top_k, idx_out, gate_out, workspace, stream=None
     """x: CUDA [T, H] float32/bfloat16; router_w: CUDA [E, H] bf16 bits (bfloat16,
     int16 or uint16 tensor); idx_out int32 [T, k]; gate_out float32 [T, k];
     workspace: CUDA uint8 tensor of moe_route_workspace_bytes(T, E) bytes."""
-    T, H = x.shape
-    E = router_w.shape[0]
-    _check(lib.moe_route_topk(x.data_ptr(), _dtype_code(x), router_w.data_ptr(), T, H, E, top_k,
-                              idx_out.data_ptr(), gate_out.data_ptr(), workspace.data_ptr(),
-                              workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
-           "moe_route_topk")
+    T, H, E, named = _route_tensors(x, router_w, top_k, idx_out, gate_out)
+    _check_tensor(workspace, "workspace", (workspace.dtype,), tuple(getattr(workspace, "shape", ())))
+    px, pw, pi, pg, pws = _device_ptrs(named + [("workspace", workspace)], None)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.moe_route_topk(px, _dtype_code(x), pw, T, H, E, top_k, pi, pg, pws, ws_bytes,
+                              _stream_ptr(stream)), "moe_route_topk")
 
 
 def moe_route_topk_noalloc(x, router_w, top_k, idx_out, gate_out, stream=None):
     """moe_route_topk for callers that cannot allocate: the scratch is a fixed
     array inside the library (n_tokens * n_experts <= 65536; calls that overlap
     on the GPU race; the first call on a device must precede any capture)."""
-    T, H = x.shape
-    E = router_w.shape[0]
-    _check(lib.moe_route_topk_noalloc(x.data_ptr(), _dtype_code(x), router_w.data_ptr(), T, H, E, top_k,
-                                      idx_out.data_ptr(), gate_out.data_ptr(), _stream_ptr(stream)),
+    T, H, E, named = _route_tensors(x, router_w, top_k, idx_out, gate_out)
+    px, pw, pi, pg = _device_ptrs(named, None)
+    _check(lib.moe_route_topk_noalloc(px, _dtype_code(x), pw, T, H, E, top_k, pi, pg, _stream_ptr(stream)),
            "moe_route_topk_noalloc")
+
+
+def _route_tensors(x, router_w, top_k, idx_out, gate_out):
+    import torch
+    T, H = _shape2(x, "x")
+    E = _shape2(router_w, "router_w")[0]
+    _check_tensor(x, "x", _act_dtypes(), (T, H))
+    _check_tensor(router_w, "router_w", _bf16_bits_dtypes(), (E, H))
+    _check_tensor(idx_out, "idx_out", (torch.int32,), (T, top_k))
+    _check_tensor(gate_out, "gate_out", (torch.float32,), (T, top_k))
+    return T, H, E, [("x", x), ("router_w", router_w), ("idx_out", idx_out), ("gate_out", gate_out)]
+
+
+def _forward_ptrs(x, router_w, pack, out):
+    import torch
+    T = _shape2(x, "x")[0]
+    H, E = pack.hidden, pack.n_experts
+    _check_tensor(x, "x", _act_dtypes(), (T, H))
+    _check_tensor(router_w, "router_w", _bf16_bits_dtypes(), (E, H))
+    _check_tensor(out, "out", (torch.float32,), (T, H))
+    px, pw, po = _device_ptrs([("x", x), ("router_w", router_w), ("out", out)], pack.device)
+    return T, px, pw, po
 
 
 def moe_layer_forward(x, router_w, pack, fmt, top_k, out, stream=None):
     """out[T, H] (float32 CUDA) = the MoE layer on x[T, H] (float32/bfloat16 CUDA)."""
-    _check(lib.moe_layer_forward(x.data_ptr(), _dtype_code(x), router_w.data_ptr(), pack.handle,
-                                 fmt, x.shape[0], top_k, out.data_ptr(), _stream_ptr(stream)),
+    T, px, pw, po = _forward_ptrs(x, router_w, pack, out)
+    _check(lib.moe_layer_forward(px, _dtype_code(x), pw, pack.handle, fmt, T, top_k, po, _stream_ptr(stream)),
            "moe_layer_forward")
 
 
 def moe_layer_forward_ex(x, router_w, pack, fmt, top_k, out, path, stream=None):
-    _check(lib.moe_layer_forward_ex(x.data_ptr(), _dtype_code(x), router_w.data_ptr(), pack.handle,
-                                    fmt, x.shape[0], top_k, out.data_ptr(), path,
-                                    _stream_ptr(stream)),
-           "moe_layer_forward_ex")
+    T, px, pw, po = _forward_ptrs(x, router_w, pack, out)
+    _check(lib.moe_layer_forward_ex(px, _dtype_code(x), pw, pack.handle, fmt, T, top_k, po, path,
+                                    _stream_ptr(stream)), "moe_layer_forward_ex")
 
 
 def moe_read_routing(pack, n_tokens, top_k, stream=None):

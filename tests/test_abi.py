@@ -113,3 +113,36 @@ def test_fault_injection_entry_points_check_arguments_without_a_device():
     assert bq.lib.moe_pack_experts(None, 0, ctypes.byref(h)) == bq.MOE_ERR_INVALID_ARG
     bq.moe_debug_fail_alloc_after(-1)
     assert bq.lib.moe_debug_wait_timeout(None, None) == bq.MOE_ERR_INVALID_ARG
+
+
+def test_binding_rejects_bad_tensors_before_calling_the_library():
+    """The C ABI sees only pointers; the binding checks what a pointer cannot carry."""
+    import torch
+    d = _desc(n_experts=4, hidden=64, inter=32)
+    pack = bq.Pack(None, d, 0)  # never reaches the library: every call below fails its checks first
+    x = torch.zeros(2, 64)
+    wr = torch.zeros(4, 64, dtype=torch.int16)
+    out = torch.zeros(2, 64)
+    with pytest.raises(ValueError, match="CUDA"):  # host memory would reach a kernel
+        bq.moe_layer_forward(x, wr, pack, 0, 2, out)
+    with pytest.raises(TypeError, match="x must be"):
+        bq.moe_layer_forward(x.double(), wr, pack, 0, 2, out)
+    with pytest.raises(ValueError, match="router_w must have shape"):
+        bq.moe_layer_forward(x, torch.zeros(5, 64, dtype=torch.int16), pack, 0, 2, out)
+    with pytest.raises(ValueError, match="x must have shape"):
+        bq.moe_layer_forward(torch.zeros(2, 32), wr, pack, 0, 2, out)
+    with pytest.raises(ValueError, match="out must have shape"):
+        bq.moe_layer_forward(x, wr, pack, 0, 2, torch.zeros(3, 64))
+    with pytest.raises(TypeError, match="out must be"):
+        bq.moe_layer_forward(x, wr, pack, 0, 2, out.to(torch.bfloat16))
+    with pytest.raises(ValueError, match="contiguous"):
+        bq.moe_layer_forward_ex(torch.zeros(64, 2).t(), wr, pack, 0, 2, out, bq.MOE_PATH_AUTO)
+    with pytest.raises(ValueError, match="2-D"):
+        bq.moe_layer_forward(torch.zeros(64), wr, pack, 0, 2, out)
+    idx, gate = torch.zeros(2, 2, dtype=torch.int32), torch.zeros(2, 2)
+    with pytest.raises(ValueError, match="CUDA"):
+        bq.moe_route_topk(x, wr, 2, idx, gate, torch.zeros(4096, dtype=torch.uint8))
+    with pytest.raises(TypeError, match="idx_out must be"):
+        bq.moe_route_topk_noalloc(x, wr, 2, idx.long(), gate)
+    with pytest.raises(ValueError, match="gate_out must have shape"):
+        bq.moe_route_topk_noalloc(x, wr, 2, idx, torch.zeros(2, 3))
