@@ -277,6 +277,31 @@ def _small_layer(fmt_gu=oracle.Q8_0, fmt_dn=oracle.Q8_0, shared=True, E=12, H=64
     return wl, synth.layer_inputs(wl)
 
 
+def test_expert_of_every_format_is_the_ffn_of_its_decoded_matrices():
+    """The expert FFN assembled from the pinned block decoders, for every format pair and the
+    shared expert's slot: gate rows first then up rows, SwiGLU, down, each projection with its
+    own NVFP4 tensor scale and the layer's IQ4_NL table.  A swapped gate/up half, a wrong
+    scale index or a transposed down matrix in any format's path fails here."""
+    rng = np.random.default_rng(11)
+    pairs = ((oracle.Q8_0, oracle.Q8_0), (oracle.Q5_1, oracle.Q5_1), (oracle.Q5_0, oracle.Q5_0),
+             (oracle.IQ4_NL, oracle.IQ4_NL), (oracle.NVFP4, oracle.NVFP4), (oracle.IQ4_NL, oracle.Q5_1),
+             (oracle.Q5_0, oracle.IQ4_NL), (oracle.NVFP4, oracle.Q8_0))
+    for fgu, fdn in pairs:
+        wl, li = _small_layer(fgu, fdn, E=3, seed=10 * fgu + fdn)
+        ex = oracle.Experts.from_layer(li)
+        H, I = wl.hidden, wl.inter
+        for e in range(wl.n_experts + 1):  # slot n_experts holds the shared expert
+            gs = 1.0 if li.gate_up_scale is None else float(li.gate_up_scale[e])
+            ds = 1.0 if li.down_scale is None else float(li.down_scale[e])
+            GU = oracle.decode_matrix(fgu, li.gate_up[e], 2 * I, H, li.table, gs)
+            D = oracle.decode_matrix(fdn, li.down[e], H, I, li.table, ds)
+            x = rng.normal(0, 1, H)
+            a, b = GU[:I] @ x, GU[I:] @ x
+            want = D @ (a / (1 + np.exp(-a)) * b)
+            got = ex.expert(e, x)
+            assert np.allclose(got, want, rtol=1e-12, atol=1e-13 * np.abs(want).max()), (fgu, fdn, e)
+
+
 def test_dense_sum_identity_when_k_equals_E_and_uniform_gates():
     for fmts in ((oracle.Q8_0, oracle.Q8_0), (oracle.IQ4_NL, oracle.Q5_1), (oracle.NVFP4, oracle.NVFP4)):
         wl, li = _small_layer(*fmts)
