@@ -302,6 +302,29 @@ def test_expert_of_every_format_is_the_ffn_of_its_decoded_matrices():
             assert np.allclose(got, want, rtol=1e-12, atol=1e-13 * np.abs(want).max()), (fgu, fdn, e)
 
 
+def test_layer_is_the_gate_weighted_sum_of_its_selected_experts():
+    """The layer restated in numpy from its definition: bf16 router logits, the k largest
+    (lower index on ties), softmax renormalised over the selection, each selected expert
+    weighted by its own gate, plus the shared expert with gate 1.  Gates differ from
+    one another here, so a combine that pairs an expert with another selection's gate fails."""
+    for fmts in ((oracle.Q8_0, oracle.Q8_0), (oracle.IQ4_NL, oracle.Q5_1), (oracle.NVFP4, oracle.NVFP4)):
+        wl, li = _small_layer(*fmts, k=4)
+        ex = oracle.Experts.from_layer(li)
+        x = synth.tokens_f64(wl, synth.tokens(wl, li.router))
+        out, idx, gate = ex.layer(x, li.router, wl.top_k)
+        wf = synth.bf16_to_f32(li.router).astype(np.float64)
+        for t in range(x.shape[0]):
+            lt = [sum(float(wf[e, h]) * float(x[t, h]) for h in range(wl.hidden)) for e in range(wl.n_experts)]
+            sel = sorted(range(wl.n_experts), key=lambda e: (-lt[e], e))[:wl.top_k]
+            w = [math.exp(lt[e] - lt[sel[0]]) for e in sel]
+            g = [v / sum(w) for v in w]
+            assert max(g) - min(g) > 1e-3  # distinct gates: the pairing matters
+            want = sum(gj * ex.expert(e, x[t]) for gj, e in zip(g, sel)) + ex.expert(wl.n_experts, x[t])
+            assert list(idx[t]) == sel
+            assert np.allclose(gate[t], g, rtol=1e-12, atol=0)
+            assert np.allclose(out[t], want, rtol=1e-11, atol=1e-13 * np.abs(want).max())
+
+
 def test_dense_sum_identity_when_k_equals_E_and_uniform_gates():
     for fmts in ((oracle.Q8_0, oracle.Q8_0), (oracle.IQ4_NL, oracle.Q5_1), (oracle.NVFP4, oracle.NVFP4)):
         wl, li = _small_layer(*fmts)
