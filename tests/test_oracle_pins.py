@@ -412,3 +412,22 @@ def test_act_quant_nvfp4_exact_values_and_ties():
     got = oracle.act_quant_nvfp4(v)
     assert got[0] == 6 * 448 * s
     assert list(got[1:8] / 448) == [0.0, 1.0, 1.0, 2.0, 4.0, 4.0, 2.0]
+
+
+def test_act_quant_nvfp4_block_scale_ties_and_subnormals():
+    """Block scales on exact E4M3 ties, worked by hand.  v[0] = 6 * 448 makes the
+    per-vector scale exactly 1, so a block scale is (block max) / 6 rounded to E4M3:
+      block 1: max 63 -> 10.5, halfway between 10 and 11 -> 10 (even mantissa);
+               63 / 10 = 6.3 -> E2M1 6 -> 60;  -35 / 10 = -3.5, halfway -> -4 -> -40
+      block 2: max 21 * 2^-9 -> 3.5 * 2^-9, halfway between the subnormal steps
+               3 and 4 * 2^-9 -> 4 * 2^-9 = 2^-7;  21 * 2^-9 / 2^-7 = 5.25 -> 6 -> 0.046875"""
+    v = np.zeros(48)
+    v[0] = 6 * 448
+    v[16], v[17] = 63.0, -35.0
+    v[32] = 21 * 2.0 ** -9
+    got = oracle.act_quant_nvfp4(v)
+    want = np.zeros(48)
+    want[0] = 6 * 448
+    want[16], want[17] = 60.0, -40.0
+    want[32] = 0.046875
+    assert np.array_equal(got, want), got[np.nonzero(got != want)]
