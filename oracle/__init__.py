@@ -21,8 +21,7 @@ class _Desc(ctypes.Structure):
                 ("has_shared", ctypes.c_int), ("fmt_gate_up", ctypes.c_int),
                 ("fmt_down", ctypes.c_int), ("gate_up", ctypes.c_void_p),
                 ("down", ctypes.c_void_p), ("gate_up_scale", ctypes.c_void_p),
-                ("down_scale", ctypes.c_void_p), ("table", ctypes.c_void_p),
-                ("expert_map", ctypes.c_void_p)]
+                ("down_scale", ctypes.c_void_p), ("table", ctypes.c_void_p)]
 
 
 def lib():
@@ -112,34 +111,28 @@ def act_quant_nvfp4(v):
 
 
 class Experts:
-    """Expert blocks handed to the oracle.  `slots` maps expert id -> row of the
-    block arrays (None: row e holds expert e, shared expert at row n_experts)."""
+    """Expert blocks handed to the oracle: row e of the block arrays holds expert e,
+    row n_experts the shared expert (when there is one)."""
 
     def __init__(self, n_experts, hidden, inter, has_shared, fmt_gate_up, fmt_down, gate_up, down,
-                 gate_up_scale=None, down_scale=None, table=None, slots=None):
+                 gate_up_scale=None, down_scale=None, table=None):
         self.keep = [np.ascontiguousarray(gate_up, np.uint8), np.ascontiguousarray(down, np.uint8)]
         gs = None if gate_up_scale is None else np.ascontiguousarray(gate_up_scale, np.float64)
         ds = None if down_scale is None else np.ascontiguousarray(down_scale, np.float64)
         tab = None if table is None else np.ascontiguousarray(table, np.int8)
-        emap = None
-        if slots is not None:
-            emap = np.full(n_experts + 1, -1, np.int32)
-            for e, s in slots.items():
-                emap[e] = s
-        self.keep += [gs, ds, tab, emap]
+        self.keep += [gs, ds, tab]
         self.desc = _Desc(n_experts, hidden, inter, 1 if has_shared else 0, fmt_gate_up, fmt_down,
-                          _p(self.keep[0]), _p(self.keep[1]), _p(gs), _p(ds), _p(tab), _p(emap))
+                          _p(self.keep[0]), _p(self.keep[1]), _p(gs), _p(ds), _p(tab))
         self.hidden = hidden
         self.n_experts = n_experts
 
     @classmethod
-    def from_layer(cls, li, slots=None, gate_up=None, down=None, gate_up_scale=None,
-                   down_scale=None):
+    def from_layer(cls, li, gate_up=None, down=None, gate_up_scale=None, down_scale=None):
         wl = li.wl
         return cls(wl.n_experts, wl.hidden, wl.inter, wl.has_shared, wl.fmt_gate_up, wl.fmt_down,
                    li.gate_up if gate_up is None else gate_up, li.down if down is None else down,
                    li.gate_up_scale if gate_up_scale is None else gate_up_scale,
-                   li.down_scale if down_scale is None else down_scale, li.table, slots)
+                   li.down_scale if down_scale is None else down_scale, li.table)
 
     def expert(self, e, x, act_quant=0):
         x = np.ascontiguousarray(x, np.float64)

@@ -281,24 +281,22 @@ void oracle_act_quant_nvfp4(const double *in, int64_t n, double *out)
 
 /* ---- experts and the layer --------------------------------------------- */
 
-static const uint8_t *expert_ptr(const oracle_desc *d, int proj, int e, int *slot_out)
+/* Blocks of expert e (e = n_experts: the shared expert) of one projection. */
+static const uint8_t *expert_ptr(const oracle_desc *d, int proj, int e)
 {
-    int slot = d->expert_map ? d->expert_map[e] : e;
-    if (slot < 0) return NULL;
-    *slot_out = slot;
-    if (proj == 0) return d->gate_up + (int64_t)slot * oracle_row_bytes(d->fmt_gate_up, d->hidden) * 2 * d->inter;
-    return d->down + (int64_t)slot * oracle_row_bytes(d->fmt_down, d->inter) * d->hidden;
+    if (e < 0 || e > d->n_experts || (e == d->n_experts && !d->has_shared)) return NULL;
+    if (proj == 0) return d->gate_up + (int64_t)e * oracle_row_bytes(d->fmt_gate_up, d->hidden) * 2 * d->inter;
+    return d->down + (int64_t)e * oracle_row_bytes(d->fmt_down, d->inter) * d->hidden;
 }
 
 /* One expert's SwiGLU FFN on one token: y = D (silu(G x) * (U x)). */
 int oracle_expert(const oracle_desc *d, int e, const double *x, double *y, int act_quant)
 {
-    int H = d->hidden, I = d->inter, slot;
-    const uint8_t *gu = expert_ptr(d, 0, e, &slot);
-    if (!gu) return -4;
-    double gts = d->gate_up_scale ? d->gate_up_scale[slot] : 1.0;
-    const uint8_t *dn = expert_ptr(d, 1, e, &slot);
-    double dts = d->down_scale ? d->down_scale[slot] : 1.0;
+    int H = d->hidden, I = d->inter;
+    const uint8_t *gu = expert_ptr(d, 0, e), *dn = expert_ptr(d, 1, e);
+    if (!gu || !dn) return -4;
+    double gts = d->gate_up_scale ? d->gate_up_scale[e] : 1.0;
+    double dts = d->down_scale ? d->down_scale[e] : 1.0;
     int64_t gub = oracle_row_bytes(d->fmt_gate_up, H), dnb = oracle_row_bytes(d->fmt_down, I);
     double *row = (double *)malloc(sizeof(double) * (size_t)(H > I ? H : I));
     double *hv = (double *)malloc(sizeof(double) * (size_t)I);

@@ -11,10 +11,9 @@ typedef struct {
     int fmt_gate_up, fmt_down;
     const uint8_t *gate_up;        /* canonical blocks, per expert [2I rows x H] */
     const uint8_t *down;           /* canonical blocks, per expert [H rows x I]  */
-    const double *gate_up_scale;   /* NVFP4 matrix scales per expert slot, else NULL */
+    const double *gate_up_scale;   /* NVFP4 matrix scales per expert (shared last), else NULL */
     const double *down_scale;
     const int8_t *table;           /* IQ4_NL 16-entry table, else NULL */
-    const int32_t *expert_map;     /* expert id (0..E, E = shared) -> slot, -1 absent; NULL = identity */
 } oracle_desc;
 
 double oracle_fp16(uint16_t u);
