@@ -98,3 +98,20 @@ def test_traffic_is_reported_only_for_the_captured_kernel_source(monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_sha", lambda: "0" * 16)
     assert bench.kernel_traffic(stage, wl_name) is None
     assert bench.kernel_traffic(stage, "no_such_workload") is None
+
+
+def test_reference_arm_under_torchrun_prints_once_from_rank_0():
+    """Launched like the scaling run (two ranks, 127.0.0.1): rank 0 alone times the oracle
+    and prints the line; the other rank exits 0 without work."""
+    import json
+    import subprocess
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--workload", "tiny_q8", "--steps", "1", "--warmup", "3"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
