@@ -8,6 +8,8 @@
   nothing arrives on): the kernel gives up after about a second, the pack's
   error word reads MOE_ERR_TIMEOUT once, and the same pack then runs a forward
   that matches the oracle.
+The file sorts after the parity tests: it arms process-wide fault injection and
+spends about a second in a deliberately exhausted wait.
 """
 import time
 

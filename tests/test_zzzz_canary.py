@@ -2,7 +2,8 @@
 (and the router exactly the T rows of idx / gate) that the call names.  The
 buffers handed to the library are row slices of larger tensors whose first and
 last rows hold a sentinel that must survive the call; the rows in between must
-be finite (NaN-filled before the call, so an unwritten row shows up too)."""
+be finite (NaN-filled before the call, so an unwritten row shows up too).
+The file sorts last: it repeats paths the parity tests cover, with offset buffers."""
 import numpy as np
 import pytest
 
