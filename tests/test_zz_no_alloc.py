@@ -4,8 +4,8 @@ workspace one (moe_route_topk), through the C ABI, on two calls in a row.
 moe_route_topk_noalloc serves callers that cannot allocate device memory
 (an open global-mode stream capture, or a framework that forbids cudaMalloc
 after start-up); its scratch is a fixed array inside the library.  This file is
-collected last so a run that stops at the first failure has run every other
-test before it."""
+collected after the parity tests so a run that stops at the first failure has
+run them first."""
 import numpy as np
 import pytest
 
