@@ -146,3 +146,32 @@ def test_binding_rejects_bad_tensors_before_calling_the_library():
         bq.moe_route_topk_noalloc(x, wr, 2, idx.long(), gate)
     with pytest.raises(ValueError, match="gate_out must have shape"):
         bq.moe_route_topk_noalloc(x, wr, 2, idx, torch.zeros(2, 3))
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include "moe.h"
+int main(void)
+{
+    moe_pack *p = NULL;
+    moe_status empty = moe_route_topk(NULL, MOE_DT_BF16, NULL, 0, 64, 4, 2, NULL, NULL, NULL, 0, NULL);
+    moe_status bad = moe_pack_experts(NULL, 0, &p);
+    printf("%s|%zu|%d|%d|%d\n", moe_status_string(MOE_ERR_INVALID_ARG), moe_route_workspace_bytes(8, 512),
+           (int)empty, (int)bad, p == NULL);
+    return 0;
+}
+"""
+
+
+def test_header_compiles_as_c99_and_the_library_links_from_c(tmp_path):
+    """The boundary is a C ABI: a C99 program (warnings as errors) includes include/moe.h,
+    links libmoe.so and calls it; the calls used need no device."""
+    src = tmp_path / "client.c"
+    exe = tmp_path / "client"
+    src.write_text(C_CLIENT)
+    libdir = os.path.dirname(bq.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lmoe", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.strip()
+    assert out == f"invalid argument|{256 + 8 * 512 * 4}|{bq.MOE_OK}|{bq.MOE_ERR_INVALID_ARG}|1"
