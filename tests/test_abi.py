@@ -175,3 +175,14 @@ def test_header_compiles_as_c99_and_the_library_links_from_c(tmp_path):
                    check=True, capture_output=True, text=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.strip()
     assert out == f"invalid argument|{256 + 8 * 512 * 4}|{bq.MOE_OK}|{bq.MOE_ERR_INVALID_ARG}|1"
+
+
+def test_python_constants_equal_the_header():
+    """Every MOE_* enumerator and flag of include/moe.h has the same value in the binding."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    consts = {n: int(v) for n, v in re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(\d+)", src)}
+    consts.update({n: int(v) for n, v in re.findall(r"#define\s+(MOE_[A-Z0-9_]+)\s+(\d+)", src)})
+    assert len(consts) >= 23, consts  # 9 statuses, 6 formats, 2 dtypes, 5 paths, 1 flag
+    for name, value in consts.items():
+        assert getattr(bq, name) == value, name
