@@ -186,3 +186,27 @@ def test_python_constants_equal_the_header():
     assert len(consts) >= 23, consts  # 9 statuses, 6 formats, 2 dtypes, 5 paths, 1 flag
     for name, value in consts.items():
         assert getattr(bq, name) == value, name
+
+
+def test_ctypes_structures_match_the_header_layout(tmp_path):
+    """moe_pack_desc and moe_pack_info: every field at the C compiler's offset, same sizes."""
+    structs = {"moe_pack_desc": bq.moe_pack_desc, "moe_pack_info": bq.moe_pack_info}
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "moe.h"', "int main(void)", "{"]
+    for cname, py in structs.items():
+        lines.append(f'    printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in py._fields_:
+            lines.append(f'    printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    lines += ["    return 0;", "}"]
+    src = tmp_path / "layout.c"
+    exe = tmp_path / "layout"
+    src.write_text("\n".join(lines) + "\n")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                    str(exe)], check=True, capture_output=True, text=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        cname, field, value = line.split()
+        got[(cname, field)] = int(value)
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for field, _ in py._fields_:
+            assert got[(cname, field)] == getattr(py, field).offset, (cname, field)

@@ -431,3 +431,26 @@ def test_act_quant_nvfp4_block_scale_ties_and_subnormals():
     want[16], want[17] = 60.0, -40.0
     want[32] = 0.046875
     assert np.array_equal(got, want), got[np.nonzero(got != want)]
+
+
+def test_oracle_ctypes_descriptor_matches_its_header(tmp_path):
+    """The oracle's ctypes descriptor puts every field where the C compiler does, so the
+    oracle reads the blocks, scales and table it is handed."""
+    import ctypes
+    import subprocess
+    desc = oracle._Desc
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "oracle.h"', "int main(void)", "{",
+             '    printf("size %zu\\n", sizeof(oracle_desc));']
+    for field, _ in desc._fields_:
+        lines.append(f'    printf("{field} %zu\\n", offsetof(oracle_desc, {field}));')
+    lines += ["    return 0;", "}"]
+    src, exe = tmp_path / "odesc.c", tmp_path / "odesc"
+    src.write_text("\n".join(lines) + "\n")
+    here = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(here, "oracle"), str(src), "-o",
+                    str(exe)], check=True, capture_output=True, text=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], check=True, capture_output=True,
+                                                        text=True).stdout.splitlines())
+    assert int(got["size"]) == ctypes.sizeof(desc)
+    for field, _ in desc._fields_:
+        assert int(got[field]) == getattr(desc, field).offset, field
