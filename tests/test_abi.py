@@ -163,11 +163,11 @@ int main(void)
 """
 
 
-def test_header_compiles_as_c99_and_the_library_links_from_c(tmp_path):
+def test_header_compiles_as_c99_and_the_library_links_from_c(repo_tmp):
     """The boundary is a C ABI: a C99 program (warnings as errors) includes include/moe.h,
     links libmoe.so and calls it; the calls used need no device."""
-    src = tmp_path / "client.c"
-    exe = tmp_path / "client"
+    src = repo_tmp / "client.c"
+    exe = repo_tmp / "client"
     src.write_text(C_CLIENT)
     libdir = os.path.dirname(bq.LIB_PATH)
     subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
@@ -188,7 +188,7 @@ def test_python_constants_equal_the_header():
         assert getattr(bq, name) == value, name
 
 
-def test_ctypes_structures_match_the_header_layout(tmp_path):
+def test_ctypes_structures_match_the_header_layout(repo_tmp):
     """moe_pack_desc and moe_pack_info: every field at the C compiler's offset, same sizes."""
     structs = {"moe_pack_desc": bq.moe_pack_desc, "moe_pack_info": bq.moe_pack_info}
     lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "moe.h"', "int main(void)", "{"]
@@ -197,8 +197,8 @@ def test_ctypes_structures_match_the_header_layout(tmp_path):
         for field, _ in py._fields_:
             lines.append(f'    printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
     lines += ["    return 0;", "}"]
-    src = tmp_path / "layout.c"
-    exe = tmp_path / "layout"
+    src = repo_tmp / "layout.c"
+    exe = repo_tmp / "layout"
     src.write_text("\n".join(lines) + "\n")
     subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o",
                     str(exe)], check=True, capture_output=True, text=True)

@@ -100,7 +100,7 @@ def test_traffic_is_reported_only_for_the_captured_kernel_source(monkeypatch):
     assert bench.kernel_traffic(stage, "no_such_workload") is None
 
 
-def test_reference_arm_under_torchrun_prints_once_from_rank_0():
+def test_reference_arm_under_torchrun_prints_once_from_rank_0(repo_tmp):
     """Launched like the scaling run (two ranks, 127.0.0.1): rank 0 alone times the oracle
     and prints the line; the other rank exits 0 without work."""
     import json
@@ -109,7 +109,8 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_0():
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
            "--impl", "reference", "--gpus", "2", "--workload", "tiny_q8", "--steps", "1", "--warmup", "3"]
-    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    env = dict(os.environ, TMPDIR=str(repo_tmp))  # torchrun's log directory stays in the repository
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1, r.stdout

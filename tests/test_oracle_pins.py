@@ -433,7 +433,7 @@ def test_act_quant_nvfp4_block_scale_ties_and_subnormals():
     assert np.array_equal(got, want), got[np.nonzero(got != want)]
 
 
-def test_oracle_ctypes_descriptor_matches_its_header(tmp_path):
+def test_oracle_ctypes_descriptor_matches_its_header(repo_tmp):
     """The oracle's ctypes descriptor puts every field where the C compiler does, so the
     oracle reads the blocks, scales and table it is handed."""
     import ctypes
@@ -444,7 +444,7 @@ def test_oracle_ctypes_descriptor_matches_its_header(tmp_path):
     for field, _ in desc._fields_:
         lines.append(f'    printf("{field} %zu\\n", offsetof(oracle_desc, {field}));')
     lines += ["    return 0;", "}"]
-    src, exe = tmp_path / "odesc.c", tmp_path / "odesc"
+    src, exe = repo_tmp / "odesc.c", repo_tmp / "odesc"
     src.write_text("\n".join(lines) + "\n")
     here = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(here, "oracle"), str(src), "-o",
