@@ -151,6 +151,22 @@ def kernel_traffic(stage, wl_name):
     return rec.get("bytes_per_launch")
 
 
+def traffic_source(stage, wl_name):
+    """Where roofline.traffic comes from, or why it is null."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path)).get(f"{stage}:{wl_name}")
+    except Exception:
+        rec = None
+    cur = kernel_source_sha()
+    if not rec:
+        return {"status": f"no ncu capture recorded for {stage}:{wl_name}", "kernel_source_sha": cur}
+    same = rec.get("source_sha") == cur
+    return {"status": "captured on this kernel source" if same
+            else "kernel source changed since the capture: null until it is retaken",
+            "captured_sha": rec.get("source_sha"), "kernel_source_sha": cur, "command": rec.get("command")}
+
+
 def kernel_source_sha():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_quantized_expert_moe_b200", "csrc")
@@ -431,6 +447,7 @@ def ours_arm(a, wl):
                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                     else "fallback 6650 GB/s",
                     "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": stage_us[dom]}
+    roofline["traffic_source"] = traffic_source(dom, wl.name)
     del gp
 
     # ---- end to end: pinned host input -> forward -> host output, every layer, every step

@@ -95,9 +95,14 @@ def test_traffic_is_reported_only_for_the_captured_kernel_source(monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_sha", lambda: entry["source_sha"])
     assert bench.kernel_traffic(stage, wl_name) == entry["bytes_per_launch"]
     assert entry["bytes_per_launch"] == entry["dram_read"] + entry["dram_write"]
+    assert bench.traffic_source(stage, wl_name)["status"] == "captured on this kernel source"
     monkeypatch.setattr(bench, "kernel_source_sha", lambda: "0" * 16)
     assert bench.kernel_traffic(stage, wl_name) is None
+    src = bench.traffic_source(stage, wl_name)
+    assert src["captured_sha"] == entry["source_sha"] and src["kernel_source_sha"] == "0" * 16
+    assert "changed" in src["status"] and src["command"] == entry["command"]
     assert bench.kernel_traffic(stage, "no_such_workload") is None
+    assert "no ncu capture" in bench.traffic_source(stage, "no_such_workload")["status"]
 
 
 def test_reference_arm_under_torchrun_prints_once_from_rank_0(repo_tmp):
