@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="headline only (default: also the 8-token stack and both prefill chunks)")
     ap.add_argument("--quick", action="store_true", help="for profiler runs: few steps, no baselines")
     ap.add_argument("--path", choices=["auto", "grouped", "dense"], default="auto",
                     help="decode kernel path (dense: the dense-batched comparison variant)")
@@ -280,46 +282,18 @@ def _to_dev_x(x_np):
     return torch.from_numpy(np.ascontiguousarray(x_np)).cuda()
 
 
-def ours_arm(a, wl):
-    import torch
-    import block_quantized_expert_moe_b200 as bq
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    dev = torch.cuda.current_device()
-    T = a.tokens or wl.tokens
-    L = a.layers
+def measure(a, bq, torch, wl, layers, T, dist, world, dev, e2e=True):
+    """Time K replays of one CUDA graph holding a forward of every layer (T tokens
+    each, drawn for workload `wl`), then the same work with an event around each
+    kernel.  Returns the measurement as a dict (max over ranks)."""
+    L = len(layers)
     k = wl.top_k
-    H, E = wl.hidden, wl.n_experts
+    H, E, I = wl.hidden, wl.n_experts, wl.inter
     xbytes = 2 if wl.x_dtype == synth.DT_BF16 else 4
-
-    t0 = time.time()
-    layers = []
-    li0 = None
-    for l in range(L):
-        li = synth.layer_inputs(wl, l)
-        x = synth.tokens(wl, li.router, l, 0, T)
-        pack = bq.pack_layer(li, max_tokens=T, max_top_k=k, device=dev,
-                             flags=bq.MOE_PACK_DENSE if a.path == "dense" else 0)
-        layers.append({"pack": pack, "x": _to_dev_x(x), "xh": x,
-                       "wr": torch.from_numpy(li.router.view(np.int16)).cuda(),
-                       "out": torch.empty(T, H, device="cuda")})
-        if l == 0:
-            li0 = li
-        del li
-    gen_s = time.time() - t0
-    log(f"[bench] rank {rank}: built {L} layers of {wl.name} in {gen_s:.1f} s")
+    for l, ly in enumerate(layers):
+        x = synth.tokens(wl, ly["router_np"], l, 0, T)
+        ly.update(x=_to_dev_x(x), xh=x, out=torch.empty(T, H, device="cuda"))
     info = layers[0]["pack"].info()
-
     path = {"auto": bq.MOE_PATH_AUTO, "grouped": bq.MOE_PATH_GROUPED, "dense": bq.MOE_PATH_DENSE}[a.path]
 
     def fwd(ly):
@@ -335,18 +309,16 @@ def ours_arm(a, wl):
     torch.cuda.synchronize()
     gu_b, dn_b = info["gate_up_bytes_per_expert"], info["down_bytes_per_expert"]
     exp_b = info["expert_bytes"]
-    I = wl.inter
     stage_bytes = {
         "route_plan": [E * H * 2 + T * H * xbytes + 2 * T * E * 4 for _ in layers],
         "gate_up": [na * gu_b + T * H * xbytes + s * I * 4 for na, s in zip(n_active, slots)],
         "down": [na * dn_b + s * I * 4 + s * H * 4 for na, s in zip(n_active, slots)],
         "combine": [s * H * 4 + T * H * 4 for s in slots],
     }
-    # the fused kernel reads the router, every active expert's blocks and x,
-    # writes and re-reads h, and writes out
+    # the one-launch kernels read the router, every active expert's blocks and x,
+    # write and re-read h, and write out
     stage_bytes["fused"] = [E * H * 2 + na * exp_b + T * H * xbytes + 2 * s * I * 4 + T * H * 4
                             for na, s in zip(n_active, slots)]
-    # prefill: tensor work of the router and both expert GEMMs
     prefill_flops = [2.0 * T * H * E + 2.0 * s * H * 2 * I + 2.0 * s * I * H for s in slots]
     unique_bytes_step = sum(na * exp_b + E * H * 2 for na in n_active)
 
@@ -375,6 +347,7 @@ def ours_arm(a, wl):
     barrier()
     value = job_throughput(world, a.steps, L, T, ms)
     expert_gbs = world * a.steps * unique_bytes_step / (ms / 1e3) / 1e9
+    layer_us = ms / a.steps / L * 1e3  # timed graph: one layer's forward
 
     # ---- kernel-stage durations: the same work with event records around each kernel
     kp = max(1, min(a.steps, 10))
@@ -393,10 +366,11 @@ def ours_arm(a, wl):
         m, n = bq.moe_profile_end(ly["pack"])
         stage_ms += m
         nf += n
+    del gp
     prefill_kernels = 7 if wl.fmt_gate_up == synth.FMT_NVFP4 else 6  # route GEMM, top-k, plan, gather, GEMMs (+ h quant)
     # grouped decode: route, (x gather,) gate/up, down, combine; the x gather runs
     # with the tensor-core kernels (2-64 tokens, H and I multiples of 256)
-    tc_path = a.path == "auto" and 2 <= T <= 64 and H % 256 == 0 and wl.inter % 256 == 0
+    tc_path = a.path == "auto" and 2 <= T <= 64 and H % 256 == 0 and I % 256 == 0
     launches_per_fwd = 1 if stage_ms[4] > 0 else (prefill_kernels if stage_ms[5] > 0 else (5 if tc_path else 4))
     stage_us = {s: float(stage_ms[i] / nf * 1e3) for i, s in enumerate(STAGES) if stage_ms[i] > 0}
     phase_names = (["stage_x", "router", "logit_poll_topk", "issue", "gate_up", "h_poll", "down", "-", "tail"]
@@ -404,55 +378,57 @@ def ours_arm(a, wl):
                    ["stage_x", "router", "barrier1", "plan", "gate_up", "barrier2", "down", "barrier3", "combine"])
     fused_phase_us = ({n: float(stage_ms[6 + i] / nf * 1e3) for i, n in enumerate(phase_names) if n != "-"}
                       if stage_ms[4] > 0 else None)
-    # streaming kernel: first/last CTA reaching each grid event, from the first CTA's start
     grid_names = ["last_start", "first_router", "last_router", "first_issue", "last_issue",
                   "first_gate_up", "last_gate_up", "first_end", "last_end"]
     grid_event_us = ({n: float(stage_ms[15 + i] / nf * 1e3) for i, n in enumerate(grid_names)}
-                     if stage_ms[4] > 0 and T == 1 else None)
+                     if stage_ms[4] > 0 and stage_ms[15] > 0 else None)
     if grid_event_us is not None:
         grid_event_us["cta0_points"] = [round(float(v / nf * 1e3), 3) for v in stage_ms[24:32]]
     elif stage_ms[0] > 0 and stage_ms[15] > 0:
-        # grouped path: the router kernel's events (first/last CTA), from its first CTA's start
         route_names = ["last_start", "first_staged", "last_staged", "first_logits", "last_logits",
                        "first_topk_end", "last_topk_end", "first_plan_end", "last_plan_end"]
         grid_event_us = {"route_" + n: float(stage_ms[15 + i] / nf * 1e3) for i, n in enumerate(route_names)}
-        # the selecting / planning CTA's own clock between its steps
         step_names = ["stage_logits", "select", "topk_rest", "ticket", "counts", "scans", "groups",
                       "slot_order", "tail"]
         fused_phase_us = {"route_" + n: float(stage_ms[6 + i] / nf * 1e3) for i, n in enumerate(step_names)}
     dom = max(stage_us, key=lambda s: stage_us[s])
-    # one token: the streaming kernel (whole-row bulk copies) runs in place of the fused one
-    kname = "stream1_kernel" if dom == "fused" and T == 1 else KERNEL_NAMES[dom]
+    kname = KERNEL_NAMES[dom]
+    if dom == "fused":
+        kname = "stream1_kernel" if T == 1 else ("tail_kernel" if tc_path else "fused_decode_kernel")
     if a.path == "auto" and T >= 2 and dom in ("gate_up", "down"):
-        # 2-64 tokens with H and I multiples of 256 run the tensor-core grouped
-        # decode (its gate/up stage includes the x gather); else the streamed
-        # CUDA-core grouped matvec (row per lane)
-        tc = T <= 64 and H % 256 == 0 and wl.inter % 256 == 0
-        kname = f"dtc_kernel<{dom.replace('_', '/')}>" if tc else f"sgm_kernel<{dom.replace('_', '/')}>"
+        kname = f"dtc_kernel<{dom.replace('_', '/')}>" if tc_path else f"sgm_kernel<{dom.replace('_', '/')}>"
     hbm, peak_src = peaks()
     traffic = kernel_traffic(dom, wl.name)
+    if launches_per_fwd == 1:
+        # one launch per layer: its duration inside the timed region is the
+        # timed graph's time per layer
+        launch_us, launch_src = layer_us, "timed graph: ms_per_step / layers (one launch per layer)"
+    else:
+        launch_us, launch_src = stage_us[dom], ("event-bracketed replay of the same graph (kernel times of a "
+                                                "multi-launch forward; their sum is profiled_layer_us)")
     if dom == "prefill":
         kind = "fp4" if wl.fmt_gate_up == synth.FMT_NVFP4 else "bf16"
         tpk, tsrc = tensor_peak(kind)
         fl = float(np.mean(prefill_flops))
-        achieved = fl / (stage_us[dom] * 1e-6) / 1e12
+        achieved = fl / (layer_us * 1e-6) / 1e12
         roofline = {"bound": "tensor", "achieved": achieved, "peak": tpk, "unit": "TFLOP/s",
                     "frac": achieved / tpk, "traffic": traffic, "kernel": KERNEL_NAMES[dom],
-                    "peak_source": tsrc, "algorithmic_flops_per_launch": fl, "avg_launch_us": stage_us[dom]}
+                    "peak_source": tsrc, "algorithmic_flops_per_launch": fl, "avg_launch_us": layer_us,
+                    "launch_time_source": "timed graph: ms_per_step / layers (the whole prefill sequence)"}
     else:
         dom_bytes = float(np.mean(stage_bytes[dom]))
-        achieved = dom_bytes / (stage_us[dom] * 1e-6) / 1e9
+        achieved = dom_bytes / (launch_us * 1e-6) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                     "frac": achieved / hbm, "traffic": traffic, "kernel": kname,
                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                     else "fallback 6650 GB/s",
-                    "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": stage_us[dom]}
+                    "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": launch_us,
+                    "launch_time_source": launch_src}
     roofline["traffic_source"] = traffic_source(dom, wl.name)
-    del gp
 
     # ---- end to end: pinned host input -> forward -> host output, every layer, every step
-    e2e = None
-    if not a.no_e2e:
+    e2e_rec = None
+    if e2e and not a.no_e2e:
         xh = [torch.from_numpy(ly["xh"].view(np.int16) if ly["xh"].dtype == np.uint16 else ly["xh"]).pin_memory()
               for ly in layers]
         oh = [torch.empty(T, H, dtype=torch.float32).pin_memory() for _ in layers]
@@ -472,35 +448,112 @@ def ours_arm(a, wl):
         en.synchronize()
         ems = max_over_ranks(st.elapsed_time(en))
         barrier()
-        e2e = {"value": world * a.steps * L * T / (ems / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": L * T * H * xbytes, "d2h_bytes_per_step": L * T * H * 4,
-               "ms_per_step": ems / a.steps}
+        e2e_rec = {"value": world * a.steps * L * T / (ems / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": L * T * H * xbytes, "d2h_bytes_per_step": L * T * H * 4,
+                   "ms_per_step": ems / a.steps}
         del ge
+    del g
+    return {"value": value, "ms_per_step": ms / a.steps, "layer_us": layer_us,
+            "config": workload_config(wl, L, T, world),
+            "l2": f"inputs larger than L2: {L} distinct layers, "
+                  f"{unique_bytes_step / 1e6:.0f} MB of selected expert weights per step",
+            "expert_gbs": expert_gbs, "expert_gbs_frac": expert_gbs / hbm,
+            "unique_expert_bytes_per_step": unique_bytes_step,
+            "active_experts_per_layer": float(np.mean(n_active)),
+            "stage_us": stage_us, "profiled_layer_us": float(sum(stage_us.values())),
+            "fused_phase_us": fused_phase_us, "grid_event_us": grid_event_us, "roofline": roofline,
+            "clocks": clk.summary(), "e2e": e2e_rec, "gpu_launches": launches_per_fwd * L * a.steps,
+            "launches_per_layer": launches_per_fwd}
+
+
+def build_layers(bq, torch, wl, L, max_tokens, dev, flags=0):
+    layers = []
+    for l in range(L):
+        li = synth.layer_inputs(wl, l)
+        pack = bq.pack_layer(li, max_tokens=max_tokens, max_top_k=wl.top_k, device=dev, flags=flags)
+        layers.append({"pack": pack, "router_np": li.router,
+                       "wr": torch.from_numpy(li.router.view(np.int16)).cuda(), "li": li if l == 0 else None})
+        del li
+    return layers
+
+
+def free_layers(layers):
+    for ly in layers:
+        ly["pack"].free()
+
+
+# configurations measured beside the headline in the default run: the 48-layer
+# speculative-verify stack on the headline's own layers (same weights: the
+# generator keys them by layer), and the prefill chunk with NVFP4 and Q8_0 weights
+EXTRA_PREFILL = ("prefill_nvfp4", "prefill_q8")
+
+
+def ours_arm(a, wl):
+    import torch
+    import block_quantized_expert_moe_b200 as bq
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.cuda.current_device()
+    T = a.tokens or wl.tokens
+    L = a.layers
+    extras = not a.no_extra and wl.name == "model_decode" and not a.tokens
+    sv = synth.WORKLOADS["spec_verify"]
+    t0 = time.time()
+    layers = build_layers(bq, torch, wl, L, max(T, sv.tokens) if extras else T, dev,
+                          bq.MOE_PACK_DENSE if a.path == "dense" else 0)
+    gen_s = time.time() - t0
+    log(f"[bench] rank {rank}: built {L} layers of {wl.name} in {gen_s:.1f} s")
+    li0 = layers[0]["li"]
+    head = measure(a, bq, torch, wl, layers, T, dist, world, dev)
+    extra = {}
+    if extras:
+        extra["spec_verify"] = measure(a, bq, torch, sv, layers, sv.tokens, dist, world, dev, e2e=False)
+    free_layers(layers)
+    del layers
+    if extras:
+        for name in EXTRA_PREFILL:
+            pw = synth.WORKLOADS[name]
+            pl = build_layers(bq, torch, pw, 2, pw.tokens, dev)
+            extra[name] = measure(a, bq, torch, pw, pl, pw.tokens, dist, world, dev, e2e=False)
+            free_layers(pl)
+            del pl
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline and not a.quick:
+        import oracle
         v, n, secs, cores = oracle_rate(li0, wl, a.cpu_seconds)
+        oracle.set_threads(1)
+        v1, n1, secs1, _ = oracle_rate(li0, wl, a.cpu_seconds / 2)
+        oracle.set_threads(cores)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{n} tokens of layer 0 ({wl.name}) in {secs:.1f} s, fp64 oracle, "
-                         f"OpenMP over tokens"}
+                         f"OpenMP over tokens",
+               "value_1core": v1, "sample_1core": f"{n1} tokens of layer 0 in {secs1:.1f} s on one thread"}
 
-    del g
-    for ly in layers:
-        ly["pack"].free()
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
-                "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
+        line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": dict(workload_config(wl, L, T, world), path=a.path,
-                               l2=f"inputs larger than L2: {L} distinct layers, "
-                                  f"{unique_bytes_step / 1e6:.0f} MB of selected expert weights per step"),
-                "expert_gbs": expert_gbs, "expert_gbs_frac": expert_gbs / hbm,
-                "unique_expert_bytes_per_step": unique_bytes_step,
-                "active_experts_per_layer": float(np.mean(n_active)),
-                "stage_us": stage_us, "fused_phase_us": fused_phase_us, "grid_event_us": grid_event_us, "roofline": roofline,
-                "clocks": clk.summary(),
-                "e2e": e2e, "gpu_launches": launches_per_fwd * L * a.steps, "cpu_baseline": cpu,
-                "gen_seconds": gen_s}
+                "config": dict(head["config"], path=a.path, l2=head["l2"])}
+        for key in ("expert_gbs", "expert_gbs_frac", "unique_expert_bytes_per_step", "active_experts_per_layer",
+                    "layer_us", "stage_us", "profiled_layer_us", "fused_phase_us", "grid_event_us", "roofline",
+                    "clocks", "e2e", "gpu_launches", "launches_per_layer"):
+            line[key] = head[key]
+        line["cpu_baseline"] = cpu
+        line["gen_seconds"] = gen_s
+        if extra:
+            line["workloads"] = {n: {kk: vv for kk, vv in m.items() if kk not in ("e2e", "l2")}
+                                 for n, m in extra.items()}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
@@ -513,6 +566,7 @@ def main():
     if a.quick:
         a.no_e2e = True
         a.no_cpu_baseline = True
+        a.no_extra = True
     if a.impl == "reference":
         reference_arm(a, wl)
     else:

@@ -46,7 +46,7 @@ class moe_pack_info(ctypes.Structure):
     _fields_ = [("gate_up_bytes_per_expert", ctypes.c_int64),
                 ("down_bytes_per_expert", ctypes.c_int64), ("expert_bytes", ctypes.c_int64),
                 ("arena_bytes", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64),
-                ("device", ctypes.c_int)]
+                ("device", ctypes.c_int), ("code_table_masked", ctypes.c_int)]
 
 
 def _load():
@@ -68,12 +68,18 @@ def _load():
     L.moe_route_topk.argtypes = [vp, i32, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
     L.moe_route_topk_noalloc.restype = i32
     L.moe_route_topk_noalloc.argtypes = [vp, i32, vp, i32, i32, i32, i32, vp, vp, vp]
+    L.moe_route_noalloc_status.restype = i32
+    L.moe_route_noalloc_status.argtypes = []
+    L.moe_debug_noalloc_wait_timeout.restype = i32
+    L.moe_debug_noalloc_wait_timeout.argtypes = [vp]
     L.moe_layer_forward.restype = i32
     L.moe_layer_forward.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, vp]
     L.moe_layer_forward_ex.restype = i32
     L.moe_layer_forward_ex.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, i32, vp]
     L.moe_debug_wait_timeout.restype = i32
     L.moe_debug_wait_timeout.argtypes = [vp, vp]
+    L.moe_debug_act_quant_nvfp4.restype = i32
+    L.moe_debug_act_quant_nvfp4.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
     L.moe_debug_fail_alloc_after.restype = i32
     L.moe_debug_fail_alloc_after.argtypes = [i32]
     L.moe_read_routing.restype = i32
@@ -237,6 +243,24 @@ def moe_debug_fail_alloc_after(n):
     _check(lib.moe_debug_fail_alloc_after(n), "moe_debug_fail_alloc_after")
 
 
+def moe_debug_act_quant_nvfp4(x, stream=None):
+    """Tests only: the NVFP4 prefill's activation quantiser on the rows of x (CUDA
+    [rows, cols]; bf16: the gate/up activations' quantiser, float32: the down
+    activations').  Returns CUDA tensors (codes uint8 [rows, cols/2], E4M3 scales
+    uint8 [rows, cols/16], row scales float32 [rows])."""
+    import torch
+    rows, cols = _shape2(x, "x")
+    _check_tensor(x, "x", _act_dtypes(), (rows, cols))
+    dev = x.device
+    codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(rows, max(cols // 16, 1), dtype=torch.uint8, device=dev)
+    row_scale = torch.empty(rows, dtype=torch.float32, device=dev)
+    px, pc, ps, pr = _device_ptrs([("x", x), ("codes", codes), ("scales", scales), ("row_scale", row_scale)], None)
+    _check(lib.moe_debug_act_quant_nvfp4(px, _dtype_code(x), rows, cols, pc, ps, pr, _stream_ptr(stream)),
+           "moe_debug_act_quant_nvfp4")
+    return codes, scales, row_scale
+
+
 def moe_route_workspace_bytes(n_tokens, n_experts):
     return lib.moe_route_workspace_bytes(n_tokens, n_experts)
 
@@ -261,6 +285,18 @@ def moe_route_topk_noalloc(x, router_w, top_k, idx_out, gate_out, stream=None):
     px, pw, pi, pg = _device_ptrs(named, None)
     _check(lib.moe_route_topk_noalloc(px, _dtype_code(x), pw, T, H, E, top_k, pi, pg, _stream_ptr(stream)),
            "moe_route_topk_noalloc")
+
+
+def moe_route_noalloc_status():
+    """Status of the last moe_route_topk_noalloc call on the current device (MOE_OK
+    or MOE_ERR_TIMEOUT); synchronises the device and clears it."""
+    return lib.moe_route_noalloc_status()
+
+
+def moe_debug_noalloc_wait_timeout(stream=None):
+    """Tests only: a bounded wait runs out (~1 s) and records MOE_ERR_TIMEOUT in the
+    allocation-free router's error word."""
+    _check(lib.moe_debug_noalloc_wait_timeout(_stream_ptr(stream)), "moe_debug_noalloc_wait_timeout")
 
 
 def _route_tensors(x, router_w, top_k, idx_out, gate_out):

@@ -18,6 +18,8 @@
 namespace moe {
 cudaError_t route_set_attributes();
 cudaError_t matvec_set_attributes();
+cudaError_t debug_act_quant(const void *x, bool bf16, int rows, int cols, uint8_t *codes, uint8_t *sf_atoms,
+                            float *row_scale, int32_t *scratch, cudaStream_t s);
 }  // namespace moe
 
 // kernel-stage slots of the profiling API (moe_profile_end's ms[])
@@ -642,6 +644,10 @@ moe_status moe_pack_query(const moe_pack *p, moe_pack_info *info)
     info->arena_bytes = p->arena_bytes;
     info->workspace_bytes = p->workspace_bytes;
     info->device = p->device;
+    const auto masked = [](int fmt, const CodeTable &t) {
+        return (fmt == MOE_FMT_IQ4_NL || fmt == MOE_FMT_NVFP4) && !t.xor_mode;
+    };
+    info->code_table_masked = (masked(p->fmt_gu, p->ct_gu) ? 1 : 0) | (masked(p->fmt_dn, p->ct_dn) ? 2 : 0);
     return MOE_OK;
 }
 
@@ -809,6 +815,9 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
                 probe.k = p->max_top_k;
                 pm->stream1 = stream1_supported(probe, p->num_sms, 226 * 1024) ? 1 : 0;
                 pm->stream1_smem = pm->stream1 ? stream1_smem_bytes(probe, p->num_sms) : 0;
+                // its grid hand-overs need every CTA resident at once: one CTA
+                // per SM must fit (grid = SMs), checked once per pack
+                if (pm->stream1 && stream1_blocks_per_sm(probe, pm->stream1_smem) < 1) pm->stream1 = 0;
             }
             if (pm->stream1 && p->max_top_k <= kFusedMaxK) {
                 int pbase = -1;
@@ -1098,6 +1107,40 @@ moe_status moe_debug_wait_timeout(const moe_pack *p, void *stream)
     DeviceGuard g(p->device);
     if (!g.ok) return MOE_ERR_CUDA;
     return check_launch(launch_wait_probe(p->ws.err, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_debug_act_quant_nvfp4(const void *x, moe_dtype x_dtype, int rows, int cols, uint8_t *codes,
+                                     uint8_t *scales, float *row_scale, void *stream)
+{
+    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+    if (rows < 1 || rows > 65536 || cols < 64 || cols > 16384 || cols % 64) return MOE_ERR_INVALID_ARG;
+    if (!x || !codes || !scales || !row_scale || !aligned16(x) || !aligned16(codes)) return MOE_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    moe_status st = init_device(dev);
+    if (st != MOE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int ks = cols / 64, blocks128 = (rows + 127) / 128;
+    const size_t atom_bytes = (size_t)blocks128 * ks * 512, scratch_bytes = (size_t)(7 * rows + 8) * 4;
+    void *atoms = nullptr, *scratch = nullptr;
+    std::vector<uint8_t> h_atoms(atom_bytes), h_sc((size_t)rows * (cols / 16));
+    st = MOE_ERR_CUDA;
+    if (cudaMalloc(&atoms, atom_bytes) == cudaSuccess && cudaMalloc(&scratch, scratch_bytes) == cudaSuccess &&
+        cudaMemsetAsync(atoms, 0, atom_bytes, s) == cudaSuccess &&
+        cudaMemsetAsync(scratch, 0, scratch_bytes, s) == cudaSuccess &&
+        debug_act_quant(x, x_dtype == MOE_DT_BF16, rows, cols, codes, static_cast<uint8_t *>(atoms), row_scale,
+                        static_cast<int32_t *>(scratch), s) == cudaSuccess &&
+        cudaMemcpyAsync(h_atoms.data(), atoms, atom_bytes, cudaMemcpyDeviceToHost, s) == cudaSuccess &&
+        cudaStreamSynchronize(s) == cudaSuccess) {
+        for (int r = 0; r < rows; ++r)
+            for (int b = 0; b < cols / 16; ++b)
+                h_sc[(size_t)r * (cols / 16) + b] = h_atoms[(size_t)sf_offset(r, b >> 2, b & 3, ks)];
+        if (cudaMemcpy(scales, h_sc.data(), h_sc.size(), cudaMemcpyHostToDevice) == cudaSuccess) st = MOE_OK;
+    }
+    cudaGetLastError();
+    if (atoms) cudaFree(atoms);
+    if (scratch) cudaFree(scratch);
+    return st;
 }
 
 moe_status moe_get_device_error(const moe_pack *p)

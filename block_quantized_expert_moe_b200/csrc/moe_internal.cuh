@@ -265,6 +265,7 @@ cudaError_t launch_sgm(const SgmProj &p, const DevProj &w, const int4 *groups, c
 // shared memory as soon as it is known.
 size_t stream1_smem_bytes(const FusedArgs &a, int grid);
 bool stream1_supported(const FusedArgs &a, int grid, size_t smem_limit);
+int stream1_blocks_per_sm(const FusedArgs &a, size_t smem);
 cudaError_t stream1_set_attributes();
 cudaError_t launch_stream1(const FusedArgs &a, int grid, size_t smem, int pdl, cudaStream_t s);
 

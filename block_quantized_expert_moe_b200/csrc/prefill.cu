@@ -783,7 +783,48 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const float *h, int row
     }
 }
 
+// Diagnostic: the prefill's activation quantisers on plain rows.  x_bf16 rows
+// go through quant_scatter_kernel (the gate/up activations: row t routed to a
+// one-token "expert" t, so it lands at padded row t), fp32 rows through
+// quant_rows_kernel (the down activations); codes come out row-major, scales
+// in the block-scale layout (sf_offset) of rows rounded up to 128.
+__global__ void debug_iota_kernel(int32_t *idx, int32_t *pad_off, int32_t *fill, int32_t *perm_tok, int32_t *n_rows,
+                                  int rows)
+{
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= rows; i += gridDim.x * blockDim.x) {
+        if (i < rows) {
+            idx[i] = i;
+            perm_tok[i] = i;
+        }
+        pad_off[i] = i;
+        fill[i] = 0;
+        if (i == 0) *n_rows = rows;
+    }
+}
+
 }  // namespace
+
+cudaError_t debug_act_quant(const void *x, bool bf16, int rows, int cols, uint8_t *codes, uint8_t *sf_atoms,
+                            float *row_scale, int32_t *scratch, cudaStream_t s)
+{
+    // scratch: idx, pad_off, fill, perm_tok [rows + 1 each], gate, row_gate,
+    // slot_pos [rows each], n_rows and an unused error word
+    int32_t *idx = scratch, *pad_off = idx + rows + 1, *fill = pad_off + rows + 1, *perm_tok = fill + rows + 1;
+    float *gate = reinterpret_cast<float *>(perm_tok + rows + 1), *row_gate = gate + rows;
+    int32_t *slot_pos = reinterpret_cast<int32_t *>(row_gate + rows), *n_rows = slot_pos + rows;
+    debug_iota_kernel<<<(rows + 256) / 256, 256, 0, s>>>(idx, pad_off, fill, perm_tok, n_rows, rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (bf16) {
+        quant_scatter_kernel<<<(rows + 7) / 8, 256, 0, s>>>(static_cast<const uint16_t *>(x), rows, cols, 1, rows, 0,
+                                                             idx, gate, pad_off, fill, codes, sf_atoms, cols / 64,
+                                                             row_scale, perm_tok, row_gate, slot_pos, rows);
+    } else {
+        quant_rows_kernel<<<(rows + 7) / 8, 256, 0, s>>>(static_cast<const float *>(x), rows, n_rows, cols, perm_tok,
+                                                          codes, sf_atoms, cols / 64, row_scale);
+    }
+    return cudaGetLastError();
+}
 
 cudaError_t prefill_plan_launch(const PrefillWorkspace &w, int E, int T, int has_shared, int32_t *err, cudaStream_t s)
 {

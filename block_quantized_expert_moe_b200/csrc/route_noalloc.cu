@@ -20,9 +20,14 @@
 //     caller's stream) and overwrites every logit it reads, but two calls that
 //     overlap on the GPU (different streams with no ordering between them)
 //     race on the array and give wrong results;
-//   * the first call on a device looks up the array's device address (once per
-//     device, with that device current); make that first call before any
-//     stream capture begins.
+//   * the first call on a device looks up the array's device address and sets
+//     the router kernel's shared-memory limit (once per device, with that
+//     device current; a failed set-up is retried by the next call); make that
+//     first call before any stream capture begins;
+//   * every call runs the CUDA-core router kernel (route_kernel), also for more
+//     than 64 bf16 tokens, where moe_route_topk uses the tensor-core GEMM;
+//   * a time-out of the kernel's bounded wait is recorded in word 1 of the
+//     array (each call clears it first); moe_route_noalloc_status reads it.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -42,9 +47,18 @@ static __device__ __align__(256) unsigned char g_route_scratch[kNoallocHeader + 
 
 std::mutex g_noalloc_mutex;
 void *g_noalloc_ptr[64];
+bool g_noalloc_attr[64];  // the router kernel's shared-memory limit is set on this device
 
-// Device address of the scratch on `dev` (the current device), looked up
-// once per device.
+}  // namespace
+
+cudaError_t route_set_attributes();
+cudaError_t launch_wait_probe(int32_t *err, cudaStream_t s);
+
+namespace {
+
+// Device address of the scratch on `dev` (the current device), looked up once
+// per device, and the router kernel's attributes, set once per device; only
+// successes are remembered, so a failed set-up is retried by the next call.
 cudaError_t noalloc_scratch(int dev, unsigned char **out)
 {
     std::lock_guard<std::mutex> lk(g_noalloc_mutex);
@@ -54,13 +68,16 @@ cudaError_t noalloc_scratch(int dev, unsigned char **out)
         if (e != cudaSuccess) return e;
         g_noalloc_ptr[dev] = p;
     }
+    if (!g_noalloc_attr[dev]) {
+        cudaError_t e = route_set_attributes();
+        if (e != cudaSuccess) return e;
+        g_noalloc_attr[dev] = true;
+    }
     *out = static_cast<unsigned char *>(g_noalloc_ptr[dev]);
     return cudaSuccess;
 }
 
 }  // namespace
-
-cudaError_t route_set_attributes();
 
 }  // namespace moe
 
@@ -81,10 +98,6 @@ extern "C" moe_status moe_route_topk_noalloc(const void *x, moe_dtype x_dtype, c
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
     unsigned char *scratch = nullptr;
     if (noalloc_scratch(dev, &scratch) != cudaSuccess) return MOE_ERR_CUDA;
-    static std::once_flag attr_once[64];
-    cudaError_t attr_rc = cudaSuccess;
-    std::call_once(attr_once[dev], [&] { attr_rc = route_set_attributes(); });
-    if (attr_rc != cudaSuccess) return MOE_ERR_CUDA;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -105,4 +118,29 @@ extern "C" moe_status moe_route_topk_noalloc(const void *x, moe_dtype x_dtype, c
     a.err = a.ticket + 1;  // word 1: a timed-out wait
     if (cudaMemsetAsync(a.ticket, 0, 64, s) != cudaSuccess) return MOE_ERR_CUDA;  // the tickets (words 0, 2..)
     return launch_route(a, route_grid(n_experts, n_tokens, a.rt, sms), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" moe_status moe_route_noalloc_status(void)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    unsigned char *scratch = nullptr;
+    if (noalloc_scratch(dev, &scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    int32_t e = 0;
+    if (cudaMemcpy(&e, scratch + 4, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (e && cudaMemset(scratch + 4, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+    return static_cast<moe_status>(e);
+}
+
+extern "C" moe_status moe_debug_noalloc_wait_timeout(void *stream)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    unsigned char *scratch = nullptr;
+    if (noalloc_scratch(dev, &scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    return launch_wait_probe(reinterpret_cast<int32_t *>(scratch + 4), static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
 }

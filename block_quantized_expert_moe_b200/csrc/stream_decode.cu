@@ -766,6 +766,20 @@ bool stream1_supported(const FusedArgs &a, int grid, size_t smem_limit)
     return L.total <= smem_limit && L.total <= (size_t)kS1SmemLimit;
 }
 
+// CTAs of this kernel that fit on one SM at once with `smem` bytes of dynamic
+// shared memory (0 when the query fails).  Its CTAs hand data to one another,
+// so the forward uses it only when one CTA per SM fits: grid = SMs.
+int stream1_blocks_per_sm(const FusedArgs &a, size_t smem)
+{
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, s1_pick(a.gu.fmt, a.dn.fmt), kS1Threads, smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
 cudaError_t stream1_set_attributes()
 {
     const int fmts[4] = {MOE_FMT_Q8_0, MOE_FMT_Q5_1, MOE_FMT_IQ4_NL, MOE_FMT_NVFP4};

@@ -33,6 +33,12 @@
  * and the forward's outputs are undefined.
  * One pack runs one forward at a time: two forwards on one pack must be
  * ordered (same stream, or events); concurrent streams need separate packs.
+ * The one-launch decode kernels (one token, and the device-planned tail of
+ * 2-64 tokens) run one CTA per SM whose CTAs hand data to one another, so all
+ * of them must be resident at once: a forward that long-running kernels of
+ * another stream on the same GPU keep from some SMs waits for them, and if
+ * that lasts beyond its bounded waits it records MOE_ERR_TIMEOUT (outputs
+ * undefined) instead of hanging.
  */
 #ifndef MOE_H
 #define MOE_H
@@ -158,6 +164,11 @@ typedef struct {
     int64_t arena_bytes;          /* all experts incl. shared */
     int64_t workspace_bytes;
     int device;
+    /* 4-bit code lookups of the decode kernels: bit 0 set when the gate/up
+     * projection's table needs the masked lookup (its entries cannot be paired
+     * for the XOR-combined one), bit 1 the same for down; 0 otherwise and for
+     * formats without a table */
+    int code_table_masked;
 } moe_pack_info;
 
 /* Validate `desc`, repack every expert's blocks into the device layout (scales
@@ -206,12 +217,30 @@ moe_status moe_route_topk(const void *x, moe_dtype x_dtype, const uint16_t *rout
  *   by each call;
  *   all calls on a device share the scratch: calls that overlap on the GPU
  *   (unordered streams) race and give wrong results;
- *   the first call on a device looks up the scratch address - make it before
- *   any stream capture starts.
+ *   the first call on a device looks up the scratch address and sets the
+ *   router kernel's shared-memory limit - make it before any stream capture
+ *   starts (a set-up that failed is retried by the next call);
+ *   every call runs the CUDA-core router kernel, also for more than 64 bf16
+ *   tokens (where moe_route_topk uses its tensor-core GEMM); its outputs are
+ *   the same;
+ *   a bounded wait that ran out leaves idx_out and gate_out undefined and is
+ *   reported by moe_route_noalloc_status().
  * Other arguments, layouts and outputs as moe_route_topk. */
 moe_status moe_route_topk_noalloc(const void *x, moe_dtype x_dtype, const uint16_t *router_w,
                                   int n_tokens, int hidden, int n_experts, int top_k,
                                   int32_t *idx_out, float *gate_out, void *stream);
+
+/* Status of the last moe_route_topk_noalloc call on the current device:
+ * MOE_OK, or MOE_ERR_TIMEOUT when one of its kernel's bounded waits ran out
+ * (its outputs are then undefined).  Synchronises the device, allocates
+ * nothing, and clears the recorded error. */
+moe_status moe_route_noalloc_status(void);
+
+/* Diagnostic for tests of that status: enqueues on `stream` the one-thread
+ * bounded wait of moe_debug_wait_timeout with the allocation-free router's
+ * error word as its target; about a second later moe_route_noalloc_status()
+ * returns MOE_ERR_TIMEOUT once. */
+moe_status moe_debug_noalloc_wait_timeout(void *stream);
 
 /* The whole layer: route, plan, grouped gate/up + SwiGLU, down, combine.
  *   x        device [n_tokens x hidden] fp32 or bf16
@@ -281,6 +310,25 @@ moe_status moe_debug_fail_alloc_after(int n);
  * moe_get_device_error then returns.  The context stays usable.  Argument and
  * launch errors as the forward. */
 moe_status moe_debug_wait_timeout(const moe_pack *pack, void *stream);
+
+/* Diagnostic for tests of the NVFP4 tensor-core prefill's activation rounding
+ * (its reading of the block-scaled FP4 MMA, which needs both operands in NVFP4):
+ * runs the prefill's own quantiser on `rows` plain rows and writes what it
+ * produces.  bf16 x goes through the quantiser of the gate/up activations (the
+ * layer input), fp32 x through the one of the down activations (h).  Per row:
+ *   row_scale[r] = max_i |x[r,i]| / (6 * 448)                (fp32)
+ *   scales[r,b]  = E4M3 (round to nearest even, saturating) of
+ *                  max over block b of |x| / (6 * row_scale[r])
+ *   codes        = E2M1 of x / (row_scale * e4m3(scale)), nearest even,
+ *                  saturating; 0 for a block whose scale is 0; element 2i in
+ *                  the low nibble of byte i of the row
+ *   x         device [rows x cols] bf16 or fp32
+ *   codes     device [rows x cols/2] bytes, scales device [rows x cols/16]
+ *             E4M3 bytes (row-major), row_scale device [rows] fp32
+ * 1 <= rows <= 65536, 64 <= cols <= 16384 and cols % 64 == 0.  Allocates
+ * temporaries and synchronises `stream` (tests only, not for a hot path). */
+moe_status moe_debug_act_quant_nvfp4(const void *x, moe_dtype x_dtype, int rows, int cols, uint8_t *codes,
+                                     uint8_t *scales, float *row_scale, void *stream);
 
 /* Sticky device-side error of the pack (synchronises its device), then clears it. */
 moe_status moe_get_device_error(const moe_pack *pack);

@@ -46,6 +46,7 @@ def lib():
         L.oracle_layer.restype = i32
         L.oracle_layer.argtypes = [ctypes.POINTER(_Desc), vp, vp, i32, i32, vp, vp, vp, i32]
         L.oracle_threads.restype = i32
+        L.oracle_set_threads.argtypes = [i32]
         _lib = L
     return _lib
 
@@ -72,6 +73,11 @@ def e2m1(c):
 
 def threads():
     return lib().oracle_threads()
+
+
+def set_threads(n):
+    """OpenMP threads of later layer calls (timing on one core: 1)."""
+    lib().oracle_set_threads(int(n))
 
 
 def decode_row(fmt, row, cols, table=None, tensor_scale=1.0):

@@ -32,4 +32,5 @@ int oracle_expert(const oracle_desc *d, int e, const double *x, double *y, int a
 int oracle_layer(const oracle_desc *d, const double *x, const uint16_t *wr, int T, int k,
                  double *out, int32_t *idx_out, double *gate_out, int act_quant);
 int oracle_threads(void);
+void oracle_set_threads(int n);
 #endif
