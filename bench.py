@@ -51,8 +51,10 @@ def parse():
     ap.add_argument("--no-extra", action="store_true",
                     help="headline only (default: also the 8-token stack and both prefill chunks)")
     ap.add_argument("--quick", action="store_true", help="for profiler runs: few steps, no baselines")
-    ap.add_argument("--path", choices=["auto", "grouped", "dense"], default="auto",
-                    help="decode kernel path (dense: the dense-batched comparison variant)")
+    ap.add_argument("--path", choices=["auto", "grouped", "dense", "tail", "staged", "prefill_bf16"], default="auto",
+                    help="kernel path (dense: the dense-batched comparison variant; tail: the one-launch tail, "
+                         "also at one token; staged: its tensor-core work as separate launches; prefill_bf16: "
+                         "the bf16-dequantising prefill for every format)")
     return ap.parse_args()
 
 
@@ -91,7 +93,7 @@ class ClockSampler:
                 self.samples.append((mhz, rs))
             except Exception:
                 pass
-            time.sleep(0.005)
+            time.sleep(0.001)
 
     def __enter__(self):
         if self.ok:
@@ -294,7 +296,9 @@ def measure(a, bq, torch, wl, layers, T, dist, world, dev, e2e=True):
         x = synth.tokens(wl, ly["router_np"], l, 0, T)
         ly.update(x=_to_dev_x(x), xh=x, out=torch.empty(T, H, device="cuda"))
     info = layers[0]["pack"].info()
-    path = {"auto": bq.MOE_PATH_AUTO, "grouped": bq.MOE_PATH_GROUPED, "dense": bq.MOE_PATH_DENSE}[a.path]
+    path = {"auto": bq.MOE_PATH_AUTO, "grouped": bq.MOE_PATH_GROUPED, "dense": bq.MOE_PATH_DENSE,
+            "tail": bq.MOE_PATH_TAIL, "staged": bq.MOE_PATH_DECODE_STAGED,
+            "prefill_bf16": bq.MOE_PATH_PREFILL_BF16}[a.path]
 
     def fwd(ly):
         bq.moe_layer_forward_ex(ly["x"], ly["wr"], ly["pack"], bq.MOE_FMT_FROM_PACK, k, ly["out"], path)
@@ -370,16 +374,24 @@ def measure(a, bq, torch, wl, layers, T, dist, world, dev, e2e=True):
     prefill_kernels = 7 if wl.fmt_gate_up == synth.FMT_NVFP4 else 6  # route GEMM, top-k, plan, gather, GEMMs (+ h quant)
     # grouped decode: route, (x gather,) gate/up, down, combine; the x gather runs
     # with the tensor-core kernels (2-64 tokens, H and I multiples of 256)
-    tc_path = a.path == "auto" and 2 <= T <= 64 and H % 256 == 0 and I % 256 == 0
+    tc_path = a.path in ("auto", "staged", "tail") and 2 <= T <= 64 and H % 256 == 0 and I % 256 == 0
     launches_per_fwd = 1 if stage_ms[4] > 0 else (prefill_kernels if stage_ms[5] > 0 else (5 if tc_path else 4))
     stage_us = {s: float(stage_ms[i] / nf * 1e3) for i, s in enumerate(STAGES) if stage_ms[i] > 0}
-    phase_names = (["stage_x", "router", "logit_poll_topk", "issue", "gate_up", "h_poll", "down", "-", "tail"]
-                   if T == 1 else
-                   ["stage_x", "router", "barrier1", "plan", "gate_up", "barrier2", "down", "barrier3", "combine"])
-    fused_phase_us = ({n: float(stage_ms[6 + i] / nf * 1e3) for i, n in enumerate(phase_names) if n != "-"}
-                      if stage_ms[4] > 0 else None)
-    grid_names = ["last_start", "first_router", "last_router", "first_issue", "last_issue",
-                  "first_gate_up", "last_gate_up", "first_end", "last_end"]
+    phase_names = ["stage_x", "router", "logit_poll_topk", "issue", "gate_up", "h_poll", "down", "-", "tail"]
+    one_launch_tail = stage_ms[4] > 0 and (a.path == "tail" or (a.path == "auto" and tc_path))
+    if one_launch_tail:
+        # CTA 0's steps in the one-launch tail
+        fused_phase_us = {n: float(stage_ms[6 + i] / nf * 1e3) for i, n in enumerate(
+            ["wait_route", "barrier", "topk", "plan", "x_rows", "units", "combine"])}
+    elif stage_ms[4] > 0 and T == 1:
+        fused_phase_us = {n: float(stage_ms[6 + i] / nf * 1e3) for i, n in enumerate(phase_names) if n != "-"}
+    else:
+        fused_phase_us = None
+    grid_names = (["last_start", "first_router", "last_router", "first_issue", "last_issue",
+                   "first_gate_up", "last_gate_up", "first_end", "last_end"] if T == 1 and a.path != "tail" else
+                  # the one-launch tail: routed (grid barrier reached), planned, units done, combined
+                  ["last_start", "first_routed", "last_routed", "first_planned", "last_planned",
+                   "first_units_done", "last_units_done", "first_end", "last_end"])
     grid_event_us = ({n: float(stage_ms[15 + i] / nf * 1e3) for i, n in enumerate(grid_names)}
                      if stage_ms[4] > 0 and stage_ms[15] > 0 else None)
     if grid_event_us is not None:
@@ -394,8 +406,9 @@ def measure(a, bq, torch, wl, layers, T, dist, world, dev, e2e=True):
     dom = max(stage_us, key=lambda s: stage_us[s])
     kname = KERNEL_NAMES[dom]
     if dom == "fused":
-        kname = "stream1_kernel" if T == 1 else ("tail_kernel" if tc_path else "fused_decode_kernel")
-    if a.path == "auto" and T >= 2 and dom in ("gate_up", "down"):
+        kname = ("tail_kernel" if a.path == "tail" or (tc_path and a.path == "auto")
+                 else "stream1_kernel" if T == 1 else "fused_decode_kernel")
+    if a.path in ("auto", "staged") and T >= 2 and dom in ("gate_up", "down"):
         kname = f"dtc_kernel<{dom.replace('_', '/')}>" if tc_path else f"sgm_kernel<{dom.replace('_', '/')}>"
     hbm, peak_src = peaks()
     traffic = kernel_traffic(dom, wl.name)

@@ -20,6 +20,7 @@ MOE_ERR_OOM, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE, MOE_ERR_RANGE = 4, 5
 MOE_FMT_FROM_PACK, MOE_FMT_Q8_0, MOE_FMT_Q5_1, MOE_FMT_IQ4_NL, MOE_FMT_NVFP4, MOE_FMT_Q5_0 = 0, 1, 2, 3, 4, 5
 MOE_DT_F32, MOE_DT_BF16 = 1, 2
 MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_DENSE, MOE_PATH_GROUPED = 0, 1, 2, 3, 4
+MOE_PATH_DECODE_STAGED, MOE_PATH_TAIL, MOE_PATH_PREFILL_BF16 = 5, 6, 7
 
 
 class MoeError(RuntimeError):
@@ -36,7 +37,8 @@ class moe_pack_desc(ctypes.Structure):
                 ("down_blocks", ctypes.c_void_p), ("gate_up_tensor_scale", ctypes.c_void_p),
                 ("down_tensor_scale", ctypes.c_void_p), ("iq4nl_table", ctypes.c_void_p),
                 ("shared_gate_up_blocks", ctypes.c_void_p),
-                ("shared_down_blocks", ctypes.c_void_p), ("flags", ctypes.c_int)]
+                ("shared_down_blocks", ctypes.c_void_p), ("flags", ctypes.c_int),
+                ("expert_begin", ctypes.c_int), ("expert_end", ctypes.c_int)]
 
 
 MOE_PACK_DENSE = 1
@@ -205,9 +207,11 @@ class Pack:
 def moe_pack_experts(n_experts, hidden, inter, fmt_gate_up, fmt_down, gate_up_blocks, down_blocks,
                      gate_up_tensor_scale=None, down_tensor_scale=None, iq4nl_table=None,
                      shared_gate_up_blocks=None, shared_down_blocks=None, max_tokens=64,
-                     max_top_k=None, device=0, flags=0):
+                     max_top_k=None, device=0, flags=0, expert_window=None):
     """Upload a layer's experts.  Blocks are host uint8 arrays in the canonical
-    layout of include/moe.h (expert-major); NVFP4 scales float32 [E(+1)]."""
+    layout of include/moe.h (expert-major); NVFP4 scales float32 [E(+1)].
+    expert_window=(begin, end): the blocks hold only those routed experts (expert
+    parallelism: the forward computes that window's share of the layer)."""
     keep = [np.ascontiguousarray(gate_up_blocks, np.uint8), np.ascontiguousarray(down_blocks, np.uint8)]
     opt = lambda a, dt: None if a is None else np.ascontiguousarray(a, dt)
     gts, dts = opt(gate_up_tensor_scale, np.float32), opt(down_tensor_scale, np.float32)
@@ -217,7 +221,8 @@ def moe_pack_experts(n_experts, hidden, inter, fmt_gate_up, fmt_down, gate_up_bl
     d = moe_pack_desc(n_experts, hidden, inter, 1 if sgu is not None else 0, max_tokens,
                       max_top_k if max_top_k is not None else n_experts, fmt_gate_up, fmt_down,
                       _np_ptr(keep[0]), _np_ptr(keep[1]), _np_ptr(gts), _np_ptr(dts), _np_ptr(tab),
-                      _np_ptr(sgu), _np_ptr(sdn), flags)
+                      _np_ptr(sgu), _np_ptr(sdn), flags,
+                      *((0, 0) if expert_window is None else expert_window))
     h = ctypes.c_void_p()
     _check(lib.moe_pack_experts(ctypes.byref(d), device, ctypes.byref(h)), "moe_pack_experts")
     return Pack(h, d, device)
@@ -362,14 +367,20 @@ def moe_get_device_error(pack):
     return lib.moe_get_device_error(pack.handle)
 
 
-def pack_layer(li, max_tokens=64, max_top_k=None, device=0, flags=0):
-    """Pack a synth.LayerInputs-like object (router, gate_up, down, scales, table)."""
+def pack_layer(li, max_tokens=64, max_top_k=None, device=0, flags=0, expert_window=None, shared=True):
+    """Pack a synth.LayerInputs-like object (router, gate_up, down, scales, table).
+    expert_window=(begin, end) packs only those routed experts (and the shared
+    expert if the layer has one and `shared`)."""
     wl = li.wl
     E = wl.n_experts
-    gs = li.gate_up_scale
-    ds = li.down_scale
-    return moe_pack_experts(E, wl.hidden, wl.inter, wl.fmt_gate_up, wl.fmt_down, li.gate_up[:E],
-                            li.down[:E], gs, ds, li.table,
-                            li.gate_up[E] if wl.has_shared else None,
-                            li.down[E] if wl.has_shared else None, max_tokens,
-                            max_top_k if max_top_k is not None else wl.top_k, device, flags)
+    b, e = (0, E) if expert_window is None else expert_window
+    has_sh = wl.has_shared and shared
+    idx = list(range(b, e)) + ([E] if has_sh else [])
+    gs = None if li.gate_up_scale is None else li.gate_up_scale[idx]
+    ds = None if li.down_scale is None else li.down_scale[idx]
+    return moe_pack_experts(E, wl.hidden, wl.inter, wl.fmt_gate_up, wl.fmt_down, li.gate_up[b:e],
+                            li.down[b:e], gs, ds, li.table,
+                            li.gate_up[E] if has_sh else None,
+                            li.down[E] if has_sh else None, max_tokens,
+                            max_top_k if max_top_k is not None else wl.top_k, device, flags,
+                            None if expert_window is None else (b, e))

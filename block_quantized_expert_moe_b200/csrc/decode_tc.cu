@@ -548,7 +548,7 @@ bool decode_tc_supported(const DevProj &gu, const DevProj &dn, int H, int I, int
 {
     if (!gu.f16_ok || !dn.f16_ok || !gu.sr || !dn.sr) return false;
     if (H % 256 || I % 256) return false;  // 128-row tiles; K in raw stages of 256
-    if (max_tokens < 2 || H > 16384) return false;
+    if (max_tokens < 1 || H > 16384) return false;  // (the staged launches run 2-64 tokens, the tail 1-64)
     // the slot rows the B maps cover must fit 32-bit TMA coordinates
     return (int64_t)max_tokens * (max_top_k + 1) < (1ll << 30);
 }

@@ -34,6 +34,8 @@ struct moe_pack {
     int device = 0;
     int num_sms = 0;
     int E = 0, H = 0, I = 0, has_shared = 0, max_tokens = 0, max_top_k = 0, flags = 0;
+    int eb = 0, ee = 0;  // routed experts [eb, ee) are in this pack (expert parallelism)
+    int n_local = 0;     // ee - eb; pack slot of expert e is e - eb, the shared expert's n_local
     int fmt_gu = 0, fmt_dn = 0;        // device formats (a Q5_0 projection runs as Q5_1)
     int fmt_gu_in = 0, fmt_dn_in = 0;  // the formats the caller packed
     DevProj gu, dn;
@@ -60,6 +62,8 @@ struct moe_pack {
     SgmProj sg_gu{}, sg_dn{};
     int dtc = -1;                 // tensor-core grouped decode usable (-1: not yet checked)
     DecodeTcMaps dtc_maps{};
+    int tail_ok[kDecodeTcMaxN + 1][2];  // one-launch tail usable for T tokens, x dtype (-1: not yet checked)
+    TailLaunch tail_launch[kDecodeTcMaxN + 1][2];
     bool has_prefill = false;     // tensor-core prefill workspace present
     PrefillWorkspace pws;
 };
@@ -156,6 +160,7 @@ moe_status init_device(int dev)
     if (prefill_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_nvfp4_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     if (prefill_q8_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
+    if (tail_set_attributes() != cudaSuccess) return MOE_ERR_CUDA;
     g_dev_ready[dev] = true;
     return MOE_OK;
 }
@@ -395,7 +400,7 @@ moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, con
     }
     std::vector<char> ok((size_t)n_slots, 1);
     parallel_for(n_slots, [&](int s) {
-        const uint8_t *src = s < p->E ? blocks + (int64_t)s * canon : shared_blocks;
+        const uint8_t *src = s < p->n_local ? blocks + (int64_t)s * canon : shared_blocks;
         ok[s] = repack_expert(fmt, src, rows, cols, hq.data() + (int64_t)s * dp.qs_stride,
                               hs.data() + (int64_t)s * dp.sc_stride,
                               dp.qh_row ? hh.data() + (int64_t)s * dp.qh_stride : nullptr,
@@ -451,6 +456,9 @@ moe_status build_workspace(moe_pack *p)
         {(void **)&w.dgate, slots * 4}, {(void **)&w.n_dense_rows, 4}, {(void **)&w.slot_scale, slots * 4},
         {(void **)&w.xg, slots * p->H * 2},
         {(void **)&w.xcnt, 16},
+        {(void **)&w.tail_ctr, T <= kDecodeMaxTokens ? (int64_t)tail_counter_words(p->E, p->H, p->I) * 4 : 0},
+        {(void **)&w.tail_part,
+         T <= kDecodeMaxTokens ? (int64_t)tail_part_floats(p->num_sms, (int)T) * 4 : 0},
     };
     int64_t total = 0;
     for (auto &it : items) total += round_up(it.bytes, 256);
@@ -485,7 +493,7 @@ moe_status build_prefill_workspace(moe_pack *p)
         {(void **)&w.ptiles, rows / 128 * 16 + 64}, {(void **)&w.n_ptiles, 4},
         {(void **)&w.n_tiles, 4}, {(void **)&w.total_rows, 4}, {(void **)&w.perm_tok, rows * 4},
         {(void **)&w.row_gate, rows * 4}, {(void **)&w.row_scale_x, rows * 4}, {(void **)&w.row_scale_h, rows * 4},
-        {(void **)&w.a_q, p->fmt_gu != MOE_FMT_NVFP4 ? rows * H * 2 : rows * H / 2},
+        {(void **)&w.a_q, rows * H * 2},  // bf16 slot rows (the NVFP4 path's codes fit in them)
         {(void **)&w.sfa, rows / 128 * (H / 64) * 512},
         {(void **)&w.h, rows * I * 4}, {(void **)&w.h_q, rows * I / 2}, {(void **)&w.sfh, rows / 128 * (I / 64) * 512},
     };
@@ -559,6 +567,9 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
     if (d->fmt_gate_up == MOE_FMT_NVFP4 && !d->gate_up_tensor_scale) return MOE_ERR_INVALID_ARG;
     if (d->fmt_down == MOE_FMT_NVFP4 && !d->down_tensor_scale) return MOE_ERR_INVALID_ARG;
     if (d->has_shared && (!d->shared_gate_up_blocks || !d->shared_down_blocks)) return MOE_ERR_INVALID_ARG;
+    const bool whole = (d->expert_begin == 0 && d->expert_end == 0);
+    if (!whole && (d->expert_begin < 0 || d->expert_end <= d->expert_begin || d->expert_end > d->n_experts))
+        return MOE_ERR_INVALID_ARG;
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess) {
         cudaGetLastError();
@@ -574,6 +585,9 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
     p->device = device;
     cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, device);
     p->E = d->n_experts;
+    p->eb = whole ? 0 : d->expert_begin;
+    p->ee = whole ? d->n_experts : d->expert_end;
+    p->n_local = p->ee - p->eb;
     p->H = d->hidden;
     p->I = d->inter;
     p->has_shared = d->has_shared ? 1 : 0;
@@ -587,7 +601,8 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
     p->ct_gu = build_code_table(p->fmt_gu, d->iq4nl_table, p->perm_gu);
     p->ct_dn = build_code_table(p->fmt_dn, d->iq4nl_table, p->perm_dn);
     for (auto &row : p->grid_cache) row[0] = row[1] = 0;
-    const int n_slots = p->E + p->has_shared;
+    for (auto &row : p->tail_ok) row[0] = row[1] = -1;
+    const int n_slots = p->n_local + p->has_shared;
     std::vector<float> gts, dts;
     if (p->fmt_gu == MOE_FMT_NVFP4) gts.assign(d->gate_up_tensor_scale, d->gate_up_tensor_scale + n_slots);
     if (p->fmt_dn == MOE_FMT_NVFP4) dts.assign(d->down_tensor_scale, d->down_tensor_scale + n_slots);
@@ -600,7 +615,7 @@ moe_status moe_pack_experts(const moe_pack_desc *d, int device, moe_pack **out)
     const bool nv = p->fmt_gu == MOE_FMT_NVFP4 && p->fmt_dn == MOE_FMT_NVFP4 &&
                     prefill_nvfp4_supported(p->H, p->I, p->E, p->max_top_k);
     // bf16-dequantising tensor-core prefill: Q8_0, IQ4_NL and Q5_1, in any mix
-    const bool q8 = prefill_q8_supported(p->fmt_gu, p->fmt_dn, p->H, p->I, p->E, p->max_top_k);
+    const bool q8 = prefill_q8_supported(p->fmt_gu, p->fmt_dn, p->H, p->I, p->E, p->max_top_k, true);
     if (st == MOE_OK && p->max_tokens > kDecodeMaxTokens && (nv || q8)) st = build_prefill_workspace(p);
     if (st == MOE_OK && cudaDeviceSynchronize() != cudaSuccess) st = MOE_ERR_CUDA;
     if (st != MOE_OK) {
@@ -713,13 +728,25 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     if (top_k < 1 || top_k > p->max_top_k) return MOE_ERR_INVALID_ARG;
     if (fmt != MOE_FMT_FROM_PACK && fmt != p->fmt_gu_in) return MOE_ERR_FMT_MISMATCH;
     const bool prefill_ok = p->has_prefill && x_dtype == MOE_DT_BF16 && top_k <= 32;
+    if (path == MOE_PATH_PREFILL_BF16 &&
+        (!prefill_ok || !prefill_q8_supported(p->fmt_gu, p->fmt_dn, p->H, p->I, p->E, top_k, true)))
+        return MOE_ERR_UNSUPPORTED;
     if (path == MOE_PATH_AUTO)
         path = n_tokens <= kDecodeMaxTokens ? MOE_PATH_DECODE : (prefill_ok ? MOE_PATH_PREFILL : MOE_PATH_GROUPED);
     if (path == MOE_PATH_PREFILL && !prefill_ok) return MOE_ERR_UNSUPPORTED;
     if (path == MOE_PATH_DENSE && (!(p->flags & MOE_PACK_DENSE) || n_tokens > kDecodeMaxTokens))
         return MOE_ERR_UNSUPPORTED;
-    if (path != MOE_PATH_DECODE && path != MOE_PATH_GROUPED && path != MOE_PATH_PREFILL && path != MOE_PATH_DENSE)
+    if (path != MOE_PATH_DECODE && path != MOE_PATH_GROUPED && path != MOE_PATH_PREFILL && path != MOE_PATH_DENSE &&
+        path != MOE_PATH_DECODE_STAGED && path != MOE_PATH_TAIL && path != MOE_PATH_PREFILL_BF16)
         return MOE_ERR_UNSUPPORTED;
+    if ((path == MOE_PATH_DECODE_STAGED || path == MOE_PATH_TAIL) && n_tokens > kDecodeTcMaxN) return MOE_ERR_UNSUPPORTED;
+    // a pack holding an expert window runs only the one-launch tail (its plan
+    // skips the other packs' experts)
+    const bool windowed = p->n_local < p->E;
+    if (windowed) {
+        if ((path != MOE_PATH_DECODE && path != MOE_PATH_TAIL) || n_tokens > kDecodeTcMaxN) return MOE_ERR_UNSUPPORTED;
+        path = MOE_PATH_TAIL;
+    }
     // an empty batch enqueues nothing and leaves the pack's routing record as it was
     if (n_tokens == 0) return MOE_OK;
     if (!x || !router_w || !out) return MOE_ERR_INVALID_ARG;
@@ -730,7 +757,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     moe_pack *pm = const_cast<moe_pack *>(p);
     const Workspace &w = p->ws;
     const int T = n_tokens, k = top_k;
-    if (path == MOE_PATH_PREFILL) {
+    if (path == MOE_PATH_PREFILL || path == MOE_PATH_PREFILL_BF16) {
         PrefillNvArgs pa{};
         pa.x = x;
         pa.wr = router_w;
@@ -755,7 +782,8 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
             pm->prof_fwd.push_back({pbase, 2});
         }
         prof_mark(pm, pbase, 0, s);
-        moe_status st = check_launch(p->fmt_gu == MOE_FMT_NVFP4 ? prefill_nvfp4_forward(pa, s) : prefill_q8_forward(pa, s));
+        const bool native = p->fmt_gu == MOE_FMT_NVFP4 && p->fmt_dn == MOE_FMT_NVFP4 && path == MOE_PATH_PREFILL;
+        moe_status st = check_launch(native ? prefill_nvfp4_forward(pa, s) : prefill_q8_forward(pa, s));
         prof_mark(pm, pbase, 1, s);
         return st;
     }
@@ -763,7 +791,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     // streamed grouped matvecs (rows per lane, TMA-fed) when the planes' rows
     // fit their tile loads, else the fused or plain grouped kernels
     if (pm->sgm < 0) {
-        const int slots = p->E + (p->has_shared ? 1 : 0);
+        const int slots = p->n_local + (p->has_shared ? 1 : 0);
         pm->sgm = (w.max_groups <= sgm_max_groups() && p->I % 16 == 0 && p->H % 32 == 0 &&
                    sgm_prepare(p->gu, slots, true, &pm->sg_gu) && sgm_prepare(p->dn, slots, false, &pm->sg_dn) &&
                    sgm_stages(pm->sg_gu, p->H) >= 2 && sgm_stages(pm->sg_dn, p->I) >= 2)
@@ -773,14 +801,66 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     if (pm->dtc < 0) {
         const int64_t slots = std::max<int64_t>((int64_t)p->max_tokens * (p->max_top_k + 1), 1);
         pm->dtc = decode_tc_supported(p->gu, p->dn, p->H, p->I, p->max_tokens, p->max_top_k) &&
-                          decode_tc_maps(&pm->dtc_maps, p->gu, p->dn, p->E + (p->has_shared ? 1 : 0), w.xg, w.h,
+                          decode_tc_maps(&pm->dtc_maps, p->gu, p->dn, p->n_local + (p->has_shared ? 1 : 0), w.xg, w.h,
                                          (int)slots, p->H, p->I)
                       ? 1
                       : 0;
     }
-    // 2..64 tokens: the tensor-core grouped decode when the pack's weights are
+    // 2..64 tokens: the one-launch tail when it fits, else the tensor-core
+    // grouped decode in separate launches, when the pack's weights are
     // fp16-representable
-    const bool use_dtc = path == MOE_PATH_DECODE && T >= 2 && T <= kDecodeTcMaxN && pm->dtc == 1;
+    bool use_tail = false;
+    if ((path == MOE_PATH_DECODE && T >= 2) || path == MOE_PATH_TAIL) {
+        const int xb = x_dtype == MOE_DT_BF16 ? 1 : 0;
+        int &ok = pm->tail_ok[T][xb];
+        if (ok < 0) {
+            TailPlanIn in{T, p->max_tokens, p->H, p->E, p->I, p->max_top_k, x_dtype, p->fmt_gu, p->fmt_dn, p->num_sms};
+            TailLaunch &L = pm->tail_launch[T][xb];
+            ok = pm->dtc == 1 && p->max_tokens <= kDecodeMaxTokens && tail_plan(in, &L) &&
+                         tail_blocks_per_sm(p->fmt_gu, p->fmt_dn, L.smem) >= 1
+                     ? 1
+                     : 0;
+        }
+        use_tail = ok == 1;
+        if (path == MOE_PATH_TAIL && !use_tail) return MOE_ERR_UNSUPPORTED;
+    }
+    if (use_tail) {
+        TailCall tc{};
+        tc.x = x;
+        tc.x_dtype = x_dtype;
+        tc.wr = router_w;
+        tc.T = T;
+        tc.H = p->H;
+        tc.E = p->E;
+        tc.eb = p->eb;
+        tc.ee = p->ee;
+        tc.I = p->I;
+        tc.k = k;
+        tc.has_shared = p->has_shared;
+        tc.gu = &p->gu;
+        tc.dn = &p->dn;
+        tc.tab_gu = p->ct_gu;
+        tc.tab_dn = p->ct_dn;
+        tc.ws = &p->ws;
+        tc.maps = &pm->dtc_maps;
+        tc.out = out;
+        int pbase = -1;
+        if (pm->prof_on && (size_t)pm->prof_used + 2 <= pm->prof_ev.size()) {
+            pbase = pm->prof_used;
+            pm->prof_used += 2;
+            pm->prof_fwd.push_back({pbase, 1});
+            if (pm->prof_stamps && pm->prof_nstamp < pm->prof_stamp_cap)
+                tc.stamps = pm->prof_stamps + kStampStride * (size_t)pm->prof_nstamp++;
+        }
+        prof_mark(pm, pbase, 0, s);
+        moe_status st = check_launch(launch_tail(tc, pm->tail_launch[T][x_dtype == MOE_DT_BF16 ? 1 : 0], p->num_sms,
+                                                 pm->pdl && pbase < 0, s));
+        prof_mark(pm, pbase, 1, s);
+        return st;
+    }
+    const bool use_dtc =
+        (path == MOE_PATH_DECODE || path == MOE_PATH_DECODE_STAGED) && T >= 2 && T <= kDecodeTcMaxN && pm->dtc == 1;
+    if (path == MOE_PATH_DECODE_STAGED && !use_dtc) return MOE_ERR_UNSUPPORTED;
     // one token: the single-token kernels; 2..8 tokens: the fused kernel unless
     // the streamed grouped matvecs or the tensor-core grouped decode apply
     if (path == MOE_PATH_DECODE && T <= kFusedMaxT && k <= kFusedMaxK && (T == 1 || (pm->sgm != 1 && !use_dtc))) {

@@ -79,6 +79,10 @@ struct Workspace {
     // single-token streaming kernel: {finished-CTA ticket, logits arrivals, h
     // arrivals}; all zero between launches (the last CTA to finish resets them)
     unsigned *xcnt = nullptr;
+    // one-launch tail (tail_decode.cu): its counters (zero between launches)
+    // and the fp32 pieces of tiles whose units span two CTAs
+    unsigned *tail_ctr = nullptr;
+    float *tail_part = nullptr;
 };
 
 // Tensor-core grouped decode (2 to kDecodeTcMaxN tokens): TMA maps of the
@@ -228,7 +232,8 @@ cudaError_t prefill_nvfp4_forward(const PrefillNvArgs &a, cudaStream_t s);
 cudaError_t launch_wait_probe(int32_t *err, cudaStream_t s);
 cudaError_t prefill_plan_launch(const PrefillWorkspace &w, int E, int T, int has_shared, int32_t *err, cudaStream_t s);
 cudaError_t prefill_q8_set_attributes();
-bool prefill_q8_supported(int fmt_gu, int fmt_dn, int H, int I, int E, int k);  // Q8_0 / IQ4_NL / Q5_1
+// Q8_0 / IQ4_NL / Q5_1 in any mix, and NVFP4 when `nvfp4` (the exact-weight variant beside the native FP4 GEMM)
+bool prefill_q8_supported(int fmt_gu, int fmt_dn, int H, int I, int E, int k, bool nvfp4);
 cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s);
 cudaError_t prefill_route(const void *x_bf16, const uint16_t *wr, int T, int H, int E, int k, float *logits,
                           int32_t *idx, float *gate, int32_t *cnt, int32_t *err, cudaStream_t s);
@@ -268,6 +273,34 @@ bool stream1_supported(const FusedArgs &a, int grid, size_t smem_limit);
 int stream1_blocks_per_sm(const FusedArgs &a, size_t smem);
 cudaError_t stream1_set_attributes();
 cudaError_t launch_stream1(const FusedArgs &a, int grid, size_t smem, int pdl, cudaStream_t s);
+
+// The one-launch device-planned tail of 1-64 tokens (tail_decode.cu).
+struct TailPlanIn {
+    int T, max_tokens, H, E, I, k, x_dtype, fmt_gu, fmt_dn, grid;
+};
+struct TailLaunch {
+    int nr, na, nb, raw_stride, bslot, n16max, rings;
+    size_t smem;
+};
+struct TailCall {
+    const void *x;
+    int x_dtype;
+    const uint16_t *wr;
+    int T, H, E, I, k, has_shared;
+    int eb, ee;  // the pack's routed experts [eb, ee) (all: 0, E)
+    const DevProj *gu, *dn;
+    CodeTable tab_gu, tab_dn;
+    const Workspace *ws;
+    const DecodeTcMaps *maps;
+    float *out;
+    long long *stamps;
+};
+int tail_counter_words(int E, int H, int I);
+size_t tail_part_floats(int grid, int max_tokens);
+bool tail_plan(const TailPlanIn &in, TailLaunch *out);  // false: the shape or the shared memory does not fit
+cudaError_t tail_set_attributes();
+int tail_blocks_per_sm(int fmt_gu, int fmt_dn, size_t smem);
+cudaError_t launch_tail(const TailCall &t, const TailLaunch &L, int grid, int pdl, cudaStream_t s);
 
 size_t fused_smem_bytes(const FusedArgs &a, int tt, int rowsplit);
 cudaError_t fused_set_attributes();

@@ -1,4 +1,4 @@
-// Tensor-core prefill for Q8_0, IQ4_NL and Q5_1 experts: the weight blocks are
+// Tensor-core prefill for Q8_0, IQ4_NL, Q5_1 (and NVFP4) experts: the weight blocks are
 // dequantised to bf16 in shared memory and multiplied with tcgen05.mma
 // kind::f16.  One kernel instance per format (the two projections may differ);
 // only the dequantiser warps depend on it.
@@ -62,13 +62,14 @@ struct Q8GemmArgs {
     const uint8_t *qs;         // codes plane: Q8_0 K bytes per row (stored +128), 4-bit K/2
     int64_t qs_stride;
     int qs_row;
-    const uint8_t *sc;         // scale plane: fp16 d per 32 (Q5_1: {d, m})
+    const uint8_t *sc;         // row-major scales: fp16 d per 32 (Q5_1: {d, m}; NVFP4: two E4M3)
     int64_t sc_stride;
     int sc_row;
     const uint8_t *qh;         // Q5_1 fifth bits, u32 per 32
     int64_t qh_stride;
     int qh_row;
-    CodeTable tab;             // IQ4_NL table (biased bytes; the pack's code positions)
+    CodeTable tab;             // IQ4_NL / NVFP4 table (biased bytes; the pack's code positions)
+    const float *ts;           // NVFP4: per-expert matrix scale (the table holds twice E2M1)
     int up_off;                // gate/up: row offset of U (= I); down: 0
     const int32_t *perm_tok;
     const float *row_gate;
@@ -231,6 +232,9 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
             const int mt = tile / g.NT, nt = tile % g.NT;
             const int4 pt = g.ptiles[mt];
             const int quarter = warp & 3, part = warp >> 2;
+            // NVFP4 codes were expanded as twice their E2M1 value; the expert's fp32
+            // scale and the 1/2 apply to its accumulators
+            const float hts = FMT == MOE_FMT_NVFP4 ? 0.5f * __ldg(g.ts + pt.x) : 1.f;
             for (int hh = 0; hh < pt.z; ++hh) {
                 const int row = pt.y + hh * 128 + quarter * 32 + lane;
                 const int tok = g.perm_tok[row];
@@ -245,10 +249,10 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
                             uint32_t o[8];
 #pragma unroll
                             for (int i = 0; i < 16; i += 2) {
-                                const float a0 = vg[i], a1 = vg[i + 1];
+                                const float a0 = vg[i] * hts, a1 = vg[i + 1] * hts;
                                 // silu with the fast exponential (well inside the prefill tolerance)
-                                o[i / 2] = dq::pack_bf16x2(a0 * __frcp_rn(1.f + __expf(-a0)) * vu[i],
-                                                       a1 * __frcp_rn(1.f + __expf(-a1)) * vu[i + 1]);
+                                o[i / 2] = dq::pack_bf16x2(a0 * __frcp_rn(1.f + __expf(-a0)) * (vu[i] * hts),
+                                                       a1 * __frcp_rn(1.f + __expf(-a1)) * (vu[i + 1] * hts));
                             }
                             uint4 *dst = reinterpret_cast<uint4 *>(g.h + (size_t)row * g.I + nt * 128 + c);
                             dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -256,7 +260,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
                         }
                     }
                 } else {
-                    const float gt = tok >= 0 ? g.row_gate[row] : 0.f;
+                    const float gt = tok >= 0 ? g.row_gate[row] * hts : 0.f;
 #pragma unroll 1
                     for (int c = part * 128; c < part * 128 + 128; c += 16) {
                         float v[16];
@@ -341,22 +345,27 @@ DqKernel dq_pick(bool gateup, int fmt)
     case MOE_FMT_IQ4_NL:
         return gateup ? dq_grouped_gemm_kernel<true, MOE_FMT_IQ4_NL> : dq_grouped_gemm_kernel<false, MOE_FMT_IQ4_NL>;
     case MOE_FMT_Q5_1: return gateup ? dq_grouped_gemm_kernel<true, MOE_FMT_Q5_1> : dq_grouped_gemm_kernel<false, MOE_FMT_Q5_1>;
+    case MOE_FMT_NVFP4:
+        return gateup ? dq_grouped_gemm_kernel<true, MOE_FMT_NVFP4> : dq_grouped_gemm_kernel<false, MOE_FMT_NVFP4>;
     default: return nullptr;
     }
 }
 
-bool dq_fmt(int f) { return f == MOE_FMT_Q8_0 || f == MOE_FMT_IQ4_NL || f == MOE_FMT_Q5_1; }
+bool dq_fmt(int f, bool nvfp4)
+{
+    return f == MOE_FMT_Q8_0 || f == MOE_FMT_IQ4_NL || f == MOE_FMT_Q5_1 || (nvfp4 && f == MOE_FMT_NVFP4);
+}
 
 }  // namespace
 
-bool prefill_q8_supported(int fmt_gu, int fmt_dn, int H, int I, int E, int k)
+bool prefill_q8_supported(int fmt_gu, int fmt_dn, int H, int I, int E, int k, bool nvfp4)
 {
-    return dq_fmt(fmt_gu) && dq_fmt(fmt_dn) && H % 256 == 0 && I % 256 == 0 && E <= 1023 && k <= 32;
+    return dq_fmt(fmt_gu, nvfp4) && dq_fmt(fmt_dn, nvfp4) && H % 256 == 0 && I % 256 == 0 && E <= 1023 && k <= 32;
 }
 
 cudaError_t prefill_q8_set_attributes()
 {
-    const int fmts[3] = {MOE_FMT_Q8_0, MOE_FMT_IQ4_NL, MOE_FMT_Q5_1};
+    const int fmts[4] = {MOE_FMT_Q8_0, MOE_FMT_IQ4_NL, MOE_FMT_Q5_1, MOE_FMT_NVFP4};
     for (int f : fmts)
         for (int gu = 0; gu < 2; ++gu) {
             const cudaError_t e =
@@ -389,9 +398,10 @@ cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s)
     g.qs = a.gu->qs;
     g.qs_stride = a.gu->qs_stride;
     g.qs_row = a.gu->qs_row;
-    g.sc = a.gu->sc;
-    g.sc_stride = a.gu->sc_stride;
-    g.sc_row = a.gu->sc_row;
+    g.sc = a.gu->sr;  // scales row by row (for NVFP4 its row-major copy)
+    g.sc_stride = a.gu->sr_stride;
+    g.sc_row = a.gu->sr_row;
+    g.ts = a.gu->ts;
     g.qh = a.gu->qh;
     g.qh_stride = a.gu->qh_stride;
     g.qh_row = a.gu->qh_row;
@@ -417,9 +427,10 @@ cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s)
     d.qs = a.dn->qs;
     d.qs_stride = a.dn->qs_stride;
     d.qs_row = a.dn->qs_row;
-    d.sc = a.dn->sc;
-    d.sc_stride = a.dn->sc_stride;
-    d.sc_row = a.dn->sc_row;
+    d.sc = a.dn->sr;
+    d.sc_stride = a.dn->sr_stride;
+    d.sc_row = a.dn->sr_row;
+    d.ts = a.dn->ts;
     d.qh = a.dn->qh;
     d.qh_stride = a.dn->qh_stride;
     d.qh_row = a.dn->qh_row;

@@ -1,0 +1,1239 @@
+// The device-planned MoE tail of 1 to 64 tokens in one launch.
+//
+// The "Qwen3.8-Flash-Next UD-IQ2_XS (L4 fix) for Basalt" model card ("What was
+// changed") names the fast decode path a device-planned MoE tail with grouped
+// kernels: the per-expert token lists are planned on the GPU, without a host
+// round trip, and each selected expert's weights are read once for all of its
+// tokens.  Here the whole tail is one persistent kernel, one CTA per SM:
+//
+//   route     CTA c takes a block of router rows and a block of tokens: logits
+//             = Wr x (fp32), its router rows bulk-copied into shared memory
+//             before the kernel waits on the previous one of the stream
+//             (programmatic dependent launch); the first CTA of each token
+//             block also picks each token's power-of-two fp16 scale; then a
+//             grid-wide counter barrier
+//   plan      every CTA selects the top-k of every token (one warp per token)
+//             and builds the same plan in its shared memory: active experts in
+//             ascending order (the groups; the shared expert last), each
+//             group's tokens in ascending order (its slots), slot of each
+//             (token, choice); then writes its share of the fp16 slot rows of
+//             x and counts it on each group's readiness counter
+//   gate/up   stream-K: the units {group, 128 row pairs, 256 of K} (gate and
+//             up rows: two 128-row tensor-core tiles) are cut into equal
+//             contiguous ranges, one per CTA; a tile whose units span CTAs is
+//             summed from their fp32 pieces, in CTA order, by the last CTA to
+//             finish its piece; then h = silu(g) * u (fp16, slot rows) and a
+//             count on the group's h counter
+//   down      the same over {group, 256 output rows, 256 of K}, each unit's B
+//             operand the group's h rows once its counter is full; y per slot
+//             (fp32); the last tile of each 256-row output block makes its CTA
+//             combine those rows: out[t] = sum_j gate_tj y[slot(t, j)] (+ the
+//             shared expert's y), in the layer's order
+//
+// The tensor-core tile is M = 128 weight rows, N = the group's tokens (padded
+// to 16), K = 64 per shared-memory stage, fp16 x fp16 -> fp32 in tensor memory:
+// the weights are expanded from their blocks to fp16 in shared memory once per
+// unit (one rounding each, exact for the 4-bit codes), the slot rows of x are
+// exact fp16 after the token's power-of-two scale, h is rounded to fp16.
+//
+//   warps 0-3   epilogue: tensor-memory lanes 32w .. 32w + 31 (tile rows)
+//   warp 4      B producer (TMA, 16-row boxes of the group's slot rows)
+//   warp 5      MMA issuer (one elected thread)
+//   warp 6      raw producer (TMA boxes of codes, scales, fifth bits)
+//   warps 7-22  expanders: each thread one 32-block of one row per slice
+//
+// Every wait is bounded (~1 s): a wait that runs out records MOE_ERR_TIMEOUT,
+// raises the CTA's abort flag and the CTA drains what it issued before it
+// frees tensor memory and returns.  Counters live in the workspace, zero
+// between launches: the last CTA to finish clears the ones the launch used.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "decode_common.cuh"
+#include "dequant.cuh"
+#include "moe_internal.cuh"
+#include "tc_common.cuh"
+#include "tma_maps.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kTlEpiWarps = 4, kTlBWarp = 4, kTlMmaWarp = 5, kTlRawWarp = 6, kTlDeqWarp0 = 7, kTlDeqWarps = 16;
+constexpr int kTlWarps = kTlDeqWarp0 + kTlDeqWarps;  // 23
+constexpr int kTlThreads = 32 * kTlWarps;
+constexpr int kTlMaxRaw = 4, kTlMaxA = 4, kTlMaxB = 8;
+constexpr int kTlA = 128 * 128;           // one 128-row tile x 64 fp16 of K
+constexpr int kTlAStage = 2 * kTlA;       // a unit's two tiles
+constexpr int kTlTmemCols = 256;          // two accumulator buffers of 128 columns
+constexpr int kTlMaxWon = 64;             // 256-row output blocks (hidden <= 16384)
+constexpr long long kTlSpin = 1ll << 31;  // clocks
+
+__host__ __device__ inline int tl_cdiv(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ inline int tl_al16(int v) { return (v + 15) & ~15; }
+
+// One raw stage: the unit's 256 rows (two 128-row tiles) x K = 256 as the TMA
+// boxes land: codes (128-byte rows, 128-byte swizzle; Q8_0 two boxes), scales
+// (16 bytes a row; Q5_1 32 with a 32-byte swizzle) and Q5_1 fifth bits (32).
+template <int FMT>
+struct TlRaw {
+    static constexpr int kCodeBoxes = FMT == MOE_FMT_Q8_0 ? 2 : 1;
+    static constexpr int kCodes = kCodeBoxes * 128 * 128;
+    static constexpr int kScW = FMT == MOE_FMT_Q5_1 ? 32 : 16;
+    static constexpr int kScales = 128 * kScW;
+    static constexpr int kQh = FMT == MOE_FMT_Q5_1 ? 128 * 32 : 0;
+    static constexpr int kStage = 2 * (kCodes + kScales + kQh);
+    __device__ static int codes(int t) { return t * kCodes; }
+    __device__ static int scales(int t) { return 2 * kCodes + t * kScales; }
+    __device__ static int qh(int t) { return 2 * (kCodes + kScales) + t * kQh; }
+};
+
+__host__ __device__ inline int tl_raw_bytes(int fmt)
+{
+    switch (fmt) {
+    case MOE_FMT_Q8_0: return TlRaw<MOE_FMT_Q8_0>::kStage;
+    case MOE_FMT_Q5_1: return TlRaw<MOE_FMT_Q5_1>::kStage;
+    case MOE_FMT_IQ4_NL: return TlRaw<MOE_FMT_IQ4_NL>::kStage;
+    default: return TlRaw<MOE_FMT_NVFP4>::kStage;
+    }
+}
+
+// Word offsets of the workspace counters (unsigned, zero between launches).
+struct TlCtr {
+    int bar, ticket, gu_tile, dn_tile, grp_x, grp_h, rb, total;
+};
+__host__ __device__ inline TlCtr tl_ctr(int E, int H, int I)
+{
+    TlCtr c;
+    c.bar = 0;
+    c.ticket = 1;
+    c.gu_tile = 4;
+    c.dn_tile = c.gu_tile + (E + 1) * (I / 128);
+    c.grp_x = c.dn_tile + (E + 1) * (H / 256);
+    c.grp_h = c.grp_x + (E + 1);
+    c.rb = c.grp_h + (E + 1);
+    c.total = c.rb + H / 256;
+    return c;
+}
+
+// The launch's plan in shared memory (after the rings), the same in every CTA.
+struct TlPlanLayout {
+    int xscale, sel_e, sel_g, slot_of, grp_e, grp_n, grp_off, slot_tok, won, total;
+};
+__host__ __device__ inline TlPlanLayout tl_plan_layout(int T, int k, int E)
+{
+    TlPlanLayout L;
+    const int tk = T * k, ng = E + 1, slots = T * (k + 1);
+    int o = 0;
+    L.xscale = o;   o = tl_al16(o + 4 * T);
+    L.sel_e = o;    o = tl_al16(o + 2 * tk);
+    L.sel_g = o;    o = tl_al16(o + 4 * tk);
+    L.slot_of = o;  o = tl_al16(o + 2 * tk);
+    L.grp_e = o;    o = tl_al16(o + 2 * ng);
+    L.grp_n = o;    o = tl_al16(o + 2 * ng);
+    L.grp_off = o;  o = tl_al16(o + 4 * ng);
+    L.slot_tok = o; o = tl_al16(o + 2 * slots);
+    L.won = o;      o = tl_al16(o + 4 * (kTlMaxWon + 1));
+    L.total = o;
+    return L;
+}
+
+// Routing geometry: token blocks of at most rt tokens, row blocks over the rest
+// of the grid.
+struct TlRoute {
+    int rt, ntb, nrb;
+};
+__host__ __device__ inline TlRoute tl_route(int T, int E, int G, int xbytes)
+{
+    TlRoute r;
+    r.rt = min(T, xbytes == 2 ? 16 : 8);
+    r.ntb = tl_cdiv(T, r.rt);
+    r.nrb = max(1, min(E, G / r.ntb));
+    return r;
+}
+
+// Bytes of the routing and planning scratch (overlaid on the rings).
+__host__ __device__ inline int tl_scratch_bytes(int T, int H, int E, int G, int xbytes)
+{
+    const TlRoute r = tl_route(T, E, G, xbytes);
+    const int rows = tl_cdiv(E, r.nrb);
+    const int gemv = tl_al16(rows * H * 2) + r.rt * H * 4;
+    const int nsw = min(kTlWarps, T);
+    const int sel = nsw * (E * 4 + 512);
+    const int plan = tl_al16((E + 1) * 4) + E * 8 + E * 4;  // counts, token masks, own {flag, tokens}
+    return max(gemv, max(sel, plan));
+}
+
+struct TailArgs {
+    const void *x;
+    int x_dtype;
+    const uint16_t *wr;
+    int T, H, E, I, k, has_shared;
+    int eb, ee;                  // routed experts [eb, ee) are in the pack, at slots e - eb
+    CodeTable tab_gu, tab_dn;
+    const float *ts_gu, *ts_dn;  // NVFP4 per-pack-slot matrix scales
+    float *logits;               // [T x E]
+    float *xscale;               // [T] 2^s, x scaled by 2^-s into fp16
+    __half *xg;                  // [slots x H] fp16 slot rows of x
+    __half *h;                   // [slots x I]
+    float *y;                    // [slots x H]
+    float *part;                 // [2 phases][G][2 pieces][n16max x 256] fp32 partial tiles
+    unsigned *ctr;               // counters (TlCtr)
+    int32_t *err;
+    float *out;                  // [T x H]
+    int32_t *idx_out;            // routing readback, written by CTA 0
+    float *gate_out;
+    int32_t *cnt_out;
+    int nr, na, nb;              // ring depths
+    int raw_stride, bslot, n16max;
+    int rings;                   // bytes of the rings (the plan follows)
+    long long *stamps;           // profiling only: grid events {2^62 - first, last} at words 10..19
+};
+
+struct Ring {
+    int s = 0, u = 0;
+    __device__ __forceinline__ void next(int n)
+    {
+        if (++s == n) {
+            s = 0;
+            ++u;
+        }
+    }
+};
+
+__device__ __forceinline__ const uint8_t *raw_code(const uint8_t *box0, int bx, int r, int c)
+{
+    return box0 + bx * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void grid_event(long long *st, int ev)
+{
+    if (!st || threadIdx.x != 0) return;
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    atomicMax(st + 10 + 2 * ev, (1ll << 62) - (long long)t);
+    atomicMax(st + 11 + 2 * ev, (long long)t);
+}
+
+// Profiling only: CTA 0's SM clock at step i (words 0..9 of the forward's stamps).
+__device__ __forceinline__ void cta0_clock(long long *st, int i)
+{
+    if (st && blockIdx.x == 0 && threadIdx.x == 0) st[i] = clock64();
+}
+
+__device__ __forceinline__ unsigned ld_acq(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Spin (bounded) until *p >= target; false if the wait ran out.
+__device__ __forceinline__ bool wait_count(const unsigned *p, unsigned target)
+{
+    if (ld_acq(p) >= target) return true;
+    const long long t0 = clock64();
+    while (ld_acq(p) < target) {
+        if (clock64() - t0 > kTlSpin) return false;
+        __nanosleep(32);
+    }
+    return true;
+}
+
+// Named barrier of the four epilogue warps.
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// The CTA whose contiguous range [U c / G, U (c + 1) / G) holds unit u.
+__device__ __forceinline__ int cta_of(int u, int U, int G) { return (int)(((long long)G * (u + 1) - 1) / U); }
+__device__ __forceinline__ int range_lo(int U, int c, int G) { return (int)((long long)U * c / G); }
+
+// Number of CTAs whose ranges hold any of units [u0, u0 + n) (ranges are
+// contiguous and ascending; CTAs with empty ranges hold none).
+__device__ __forceinline__ int owners(int u0, int n, int U, int G)
+{
+    int cnt = 0, prev = -1;
+    for (int u = u0; u < u0 + n; ++u) {
+        const int cu = cta_of(u, U, G);
+        cnt += cu != prev;
+        prev = cu;
+    }
+    return cnt;
+}
+
+// Exclusive scan of n ints in shared memory v (n <= 2 * blockDim), in place;
+// returns the total.  tmp: 32 ints of scratch.
+__device__ int block_scan(int *v, int n, int *tmp)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const int i0 = 2 * tid;
+    const int a = i0 < n ? v[i0] : 0, b = i0 + 1 < n ? v[i0 + 1] : 0;
+    int s = a + b, incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) tmp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? tmp[lane] : 0, wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < nw) tmp[lane] = wi - w;
+        if (lane == 31) tmp[31] = wi;
+    }
+    __syncthreads();
+    const int base = tmp[warp] + incl - s;
+    if (i0 < n) v[i0] = base;
+    if (i0 + 1 < n) v[i0 + 1] = base + a;
+    const int total = tmp[31];
+    __syncthreads();
+    return total;
+}
+
+// A unit of one phase (0 gate/up, 1 down) and the segment of this CTA it is in.
+struct Unit {
+    int g, b, kc;        // group, tile within the group, K chunk
+    int tile;            // tile index within the phase
+    bool first, last;    // first / last unit of this CTA's piece of the tile
+};
+
+struct Geo {
+    int KC[2], NB[2], U[2], lo[2], hi[2];
+};
+
+__device__ __forceinline__ Unit unit_at(const Geo &q, int p, int u)
+{
+    Unit x;
+    x.tile = u / q.KC[p];
+    x.kc = u - x.tile * q.KC[p];
+    x.g = x.tile / q.NB[p];
+    x.b = x.tile - x.g * q.NB[p];
+    const int t0 = x.tile * q.KC[p];
+    x.first = u == max(q.lo[p], t0);
+    x.last = u + 1 == min(q.hi[p], t0 + q.KC[p]);
+    return x;
+}
+
+// The piece CTA c wrote for tile t of phase p: 0 if t is the tile its range
+// starts in, else 1 (the range's last tile).
+__device__ __forceinline__ float *piece(const TailArgs &a, const Geo &q, int p, int c, int t, int G)
+{
+    const int first_tile = range_lo(q.U[p], c, G) / q.KC[p];
+    const int which = first_tile == t ? 0 : 1;
+    return a.part + (((size_t)p * G + c) * 2 + which) * (size_t)a.n16max * 256;
+}
+
+template <int FMT>
+__device__ __forceinline__ void raw_load(uint8_t *st, const CUtensorMap *mq, const CUtensorMap *ms,
+                                         const CUtensorMap *mh, uint64_t *bar, int kc, int row0, int row1, int ex)
+{
+    using RL = TlRaw<FMT>;
+    mbar_arrive_expect_tx(bar, (uint32_t)RL::kStage);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int row = t ? row1 : row0;
+#pragma unroll
+        for (int bx = 0; bx < RL::kCodeBoxes; ++bx)
+            tma_load_3d(st + RL::codes(t) + bx * 16384, mq, bar, (kc * RL::kCodeBoxes + bx) * 128, row, ex);
+        tma_load_3d(st + RL::scales(t), ms, bar, kc * RL::kScW, row, ex);
+        if (FMT == MOE_FMT_Q5_1) tma_load_3d(st + RL::qh(t), mh, bar, kc * 32, row, ex);
+    }
+}
+
+// Thread n of the expanders: block bsel of slice d of row r of tile `tile`.
+template <int FMT>
+__device__ __forceinline__ void expand(const uint8_t *st, uint8_t *a_stage, int r, int tile, int bsel, int d,
+                                       const CodeTable &tab)
+{
+    using RL = TlRaw<FMT>;
+    const uint8_t *cq = st + RL::codes(tile), *cs = st + RL::scales(tile), *ch = st + RL::qh(tile);
+    const int blk = 2 * d + bsel;
+    uint32_t qw[8];
+    if constexpr (FMT == MOE_FMT_Q8_0) {
+        const uint4 x0 = *reinterpret_cast<const uint4 *>(raw_code(cq, blk >> 2, r, (2 * blk) & 7));
+        const uint4 x1 = *reinterpret_cast<const uint4 *>(raw_code(cq, blk >> 2, r, ((2 * blk) & 7) + 1));
+        qw[0] = x0.x; qw[1] = x0.y; qw[2] = x0.z; qw[3] = x0.w;
+        qw[4] = x1.x; qw[5] = x1.y; qw[6] = x1.z; qw[7] = x1.w;
+    } else {
+        const uint4 x0 = *reinterpret_cast<const uint4 *>(raw_code(cq, 0, r, blk));
+        qw[0] = x0.x; qw[1] = x0.y; qw[2] = x0.z; qw[3] = x0.w;
+    }
+    uint32_t sc, hb = 0;
+    if constexpr (FMT == MOE_FMT_Q5_1) {
+        const int gsw = (r >> 2) & 1;  // 32-byte swizzle: 16-byte chunk ^ ((r / 4) % 2)
+        const int o = r * 32 + ((((blk * 4) >> 4) ^ gsw) << 4) + ((blk * 4) & 15);
+        sc = *reinterpret_cast<const uint32_t *>(cs + o);
+        hb = *reinterpret_cast<const uint32_t *>(ch + o);
+    } else {
+        sc = *reinterpret_cast<const uint16_t *>(cs + r * 16 + blk * 2);
+    }
+    uint4 o4[4];
+    dq::blk_f16<FMT>(qw, sc, hb, tab, o4);
+    uint8_t *a_row = a_stage + tile * kTlA + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * bsel + cc;
+        *reinterpret_cast<uint4 *>(a_row + ((c ^ (r & 7)) << 4)) = o4[cc];
+    }
+}
+
+__host__ __device__ constexpr uint32_t tl_idesc(int N)
+{
+    // kind::f16: f16 x f16 -> f32, both K-major, M = 128
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+template <int FG, int FD>
+__global__ void __launch_bounds__(kTlThreads, 1)
+    tail_kernel(const __grid_constant__ CUtensorMap mGuQ, const __grid_constant__ CUtensorMap mGuS,
+                const __grid_constant__ CUtensorMap mGuH, const __grid_constant__ CUtensorMap mDnQ,
+                const __grid_constant__ CUtensorMap mDnS, const __grid_constant__ CUtensorMap mDnH,
+                const __grid_constant__ CUtensorMap mXg, const __grid_constant__ CUtensorMap mH, const TailArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t rf_bar[kTlMaxRaw], re_bar[kTlMaxRaw], fa_bar[kTlMaxA], ae_bar[kTlMaxA],
+        fb_bar[kTlMaxB], be_bar[kTlMaxB], accf_bar[2], acce_bar[2], dr_bar, wr_bar;
+    __shared__ uint32_t tmem_base;
+    __shared__ volatile int abort_flag;
+    __shared__ volatile int s_epi_abort;  // the four epilogue warps leave together
+    __shared__ int s_misc[8];  // [0] groups, [1] slots, [2] won row blocks, [3] epilogue: last arrival
+    __shared__ int s_tmp[32];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int T = a.T, H = a.H, E = a.E, I = a.I, k = a.k;
+    const TlCtr C = tl_ctr(E, H, I);
+    const TlPlanLayout PL = tl_plan_layout(T, k, E);
+    uint8_t *plan = smem + a.rings;
+    float *p_xscale = reinterpret_cast<float *>(plan + PL.xscale);
+    int16_t *p_sel_e = reinterpret_cast<int16_t *>(plan + PL.sel_e);
+    float *p_sel_g = reinterpret_cast<float *>(plan + PL.sel_g);
+    int16_t *p_slot_of = reinterpret_cast<int16_t *>(plan + PL.slot_of);
+    int16_t *p_grp_e = reinterpret_cast<int16_t *>(plan + PL.grp_e);
+    int16_t *p_grp_n = reinterpret_cast<int16_t *>(plan + PL.grp_n);
+    int *p_grp_off = reinterpret_cast<int *>(plan + PL.grp_off);
+    int16_t *p_slot_tok = reinterpret_cast<int16_t *>(plan + PL.slot_tok);
+    int *p_won = reinterpret_cast<int *>(plan + PL.won);
+    const int xbytes = a.x_dtype == MOE_DT_BF16 ? 2 : 4;
+    const TlRoute R = tl_route(T, E, G, xbytes);
+    const int tb = c % R.ntb, rb = c / R.ntb;
+    const bool router_cta = rb < R.nrb;
+    const int t0 = tb * R.rt, tn = min(R.rt, T - t0);
+    const int e0 = router_cta ? E * rb / R.nrb : 0, e1 = router_cta ? E * (rb + 1) / R.nrb : 0;
+    const int rows_max = tl_cdiv(E, R.nrb);
+    uint16_t *sWr = reinterpret_cast<uint16_t *>(smem);
+    float *sX = reinterpret_cast<float *>(smem + tl_al16(rows_max * H * 2));
+
+    if (warp == kTlMmaWarp) {
+        tmem_alloc(&tmem_base, kTlTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int s = 0; s < a.na; ++s) {
+            mbar_init(&fa_bar[s], kTlDeqWarps);
+            mbar_init(&ae_bar[s], 1);
+        }
+        for (int s = 0; s < a.nb; ++s) {
+            mbar_init(&fb_bar[s], 1);
+            mbar_init(&be_bar[s], 1);
+        }
+        for (int s = 0; s < a.nr; ++s) {
+            mbar_init(&rf_bar[s], 1);
+            mbar_init(&re_bar[s], kTlDeqWarps);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&accf_bar[s], 1);
+            mbar_init(&acce_bar[s], kTlEpiWarps);
+        }
+        mbar_init(&dr_bar, 1);
+        mbar_init(&wr_bar, 1);
+        abort_flag = 0;
+        s_epi_abort = 0;
+        s_misc[0] = s_misc[1] = s_misc[2] = s_misc[3] = 0;
+        fence_mbar_init();
+        // router rows: independent of the previous kernel, requested before waiting on it
+        if (router_cta && e1 > e0) {
+            mbar_arrive_expect_tx(&wr_bar, (uint32_t)((e1 - e0) * H * 2));
+            bulk_g2s(sWr, a.wr + (size_t)e0 * H, (uint32_t)((e1 - e0) * H * 2), &wr_bar);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = tmem_base;
+    grid_event(a.stamps, 0);
+    cta0_clock(a.stamps, 0);
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // x, out and the workspace are ours from here
+
+    // ---- route: logits of rows [e0, e1) for tokens [t0, t0 + tn) ------------------------
+    if (router_cta) {
+        // x as fp32 in shared memory
+        const int nch = tn * (H / 8);
+        for (int i = tid; i < nch; i += kTlThreads) {
+            const int t = i / (H / 8), ch = i - t * (H / 8);
+            float v[8];
+            if (a.x_dtype == MOE_DT_BF16) {
+                const uint4 q = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(a.x) +
+                                                                      (size_t)(t0 + t) * H) + ch);
+                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    v[2 * j] = __uint_as_float(w[j] << 16);
+                    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+                }
+            } else {
+                const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) +
+                                                                   (size_t)(t0 + t) * H) + 2 * ch;
+                const float4 x0 = __ldg(p), x1 = __ldg(p + 1);
+                v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+                v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+            }
+            float4 *d = reinterpret_cast<float4 *>(sX + (size_t)t * H + ch * 8);
+            d[0] = make_float4(v[0], v[1], v[2], v[3]);
+            d[1] = make_float4(v[4], v[5], v[6], v[7]);
+        }
+        __syncthreads();
+        bool ok = e1 <= e0 || mbar_wait(&wr_bar, 0);
+        if (!ok && lane == 0) {
+            abort_flag = 1;
+            atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
+        }
+        // one warp per router row, eight tokens at a time; lane l takes 8
+        // consecutive weights of each 256
+        for (int e = e0 + warp; ok && e < e1; e += kTlWarps) {
+            const uint16_t *wrow = sWr + (size_t)(e - e0) * H;
+            for (int tq = 0; tq < tn; tq += 8) {
+                float acc[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+                for (int k0 = lane * 8; k0 < H; k0 += 256) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(wrow + k0);
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                    float wf[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        wf[2 * j] = __uint_as_float(ww[j] << 16);
+                        wf[2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
+                    }
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        if (tq + t < tn) {
+                            const float *xr = sX + (size_t)(tq + t) * H + k0;
+                            const float4 x0 = *reinterpret_cast<const float4 *>(xr);
+                            const float4 x1 = *reinterpret_cast<const float4 *>(xr + 4);
+                            float s = acc[t];
+                            s = fmaf(wf[0], x0.x, s); s = fmaf(wf[1], x0.y, s);
+                            s = fmaf(wf[2], x0.z, s); s = fmaf(wf[3], x0.w, s);
+                            s = fmaf(wf[4], x1.x, s); s = fmaf(wf[5], x1.y, s);
+                            s = fmaf(wf[6], x1.z, s); s = fmaf(wf[7], x1.w, s);
+                            acc[t] = s;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    if (tq + t < tn) {
+                        float s = acc[t];
+#pragma unroll
+                        for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                        if (lane == 0) a.logits[(size_t)(t0 + tq + t) * E + e] = s;
+                    }
+                }
+            }
+        }
+        if (rb == 0) {
+            // each token's power-of-two scale: max |x| brought below 2^15 (fp16 keeps x exact)
+            for (int t = warp; t < tn; t += kTlWarps) {
+                unsigned mx = 0u;
+                for (int i = lane; i < H; i += 32) mx = max(mx, __float_as_uint(fabsf(sX[(size_t)t * H + i])));
+                mx = __reduce_max_sync(0xffffffffu, mx);
+                const int ex = (int)((mx >> 23) & 0xFFu) - 127;
+                const int sh = (ex >= 15 && ex < 128) ? ex - 14 : 0;
+                if (lane == 0) a.xscale[t0 + t] = __uint_as_float((uint32_t)(127 + sh) << 23);
+            }
+        }
+    }
+    // ---- grid barrier: every logit and token scale written ------------------------------
+    __syncthreads();
+    grid_event(a.stamps, 1);
+    cta0_clock(a.stamps, 1);
+    if (tid == 0) {
+        __threadfence();
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(a.ctr + C.bar) : "memory");
+        if (!wait_count(a.ctr + C.bar, (unsigned)G)) {
+            abort_flag = 1;
+            atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
+        }
+    }
+    __syncthreads();
+    const bool run = !abort_flag;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    cta0_clock(a.stamps, 2);
+
+    // ---- plan: top-k of every token, then groups and slots --------------------------------
+    if (run) {
+        const int nsw = min(kTlWarps, T);
+        if (warp < nsw) {
+            float *row = reinterpret_cast<float *>(smem) + (size_t)warp * E;
+            unsigned *cand = reinterpret_cast<unsigned *>(smem + (size_t)nsw * E * 4) + warp * 128;
+            for (int t = warp; t < T; t += nsw) {
+                for (int e = lane; e < E; e += 32) row[e] = __ldcg(a.logits + (size_t)t * E + e);
+                __syncwarp();
+                int my_e;
+                float my_g;
+                if (E <= 512) topk_threshold<16>(row, E, k, my_e, my_g, cand);
+                else topk_threshold<32>(row, E, k, my_e, my_g, cand);
+                if (lane < k) {
+                    p_sel_e[t * k + lane] = (int16_t)my_e;
+                    p_sel_g[t * k + lane] = my_g;
+                    if (c == 0) {
+                        a.idx_out[t * k + lane] = my_e;
+                        a.gate_out[t * k + lane] = my_g;
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        for (int t = tid; t < T; t += kTlThreads) p_xscale[t] = __ldcg(a.xscale + t);
+        __syncthreads();
+        cta0_clock(a.stamps, 3);
+        // counts and 64-bit token masks per expert
+        int *cnt = reinterpret_cast<int *>(smem);
+        unsigned *mask = reinterpret_cast<unsigned *>(smem + tl_al16((E + 1) * 4));
+        for (int e = tid; e <= E; e += kTlThreads) cnt[e] = 0;
+        for (int e = tid; e < 2 * E; e += kTlThreads) mask[e] = 0u;
+        __syncthreads();
+        for (int i = tid; i < T * k; i += kTlThreads) {
+            const int e = p_sel_e[i], t = i / k;
+            if (e < a.eb || e >= a.ee) continue;  // another pack's expert (expert parallelism)
+            atomicAdd(&cnt[e], 1);
+            atomicOr(&mask[2 * e + (t >> 5)], 1u << (t & 31));
+        }
+        __syncthreads();
+        // groups: active experts in ascending order; packed scan of {flag, tokens}
+        for (int e = tid; e < E; e += kTlThreads) {
+            const int n = cnt[e];
+            if (c == 0) a.cnt_out[e] = n;
+            cnt[e] = n ? (1 << 16) | n : 0;
+        }
+        if (c == 0 && tid == 0) a.cnt_out[E] = a.has_shared ? T : 0;
+        __syncthreads();
+        // entries hold {flag, tokens} of expert e; after the scan, the groups and
+        // slots before it
+        {
+            // save each expert's own {flag, tokens} before the in-place scan overwrites it
+            int *own = reinterpret_cast<int *>(smem + tl_al16((E + 1) * 4) + E * 8);
+            for (int e = tid; e < E; e += kTlThreads) own[e] = cnt[e];
+            __syncthreads();
+            const int total = block_scan(cnt, E, s_tmp);
+            const int n_routed = total >> 16, routed_slots = total & 0xFFFF;
+            for (int e = tid; e < E; e += kTlThreads) {
+                const int v = own[e];
+                if (v) {
+                    const int g = cnt[e] >> 16;
+                    p_grp_e[g] = (int16_t)(e - a.eb);  // the expert's slot in the pack
+                    p_grp_n[g] = (int16_t)(v & 0xFFFF);
+                    p_grp_off[g] = cnt[e] & 0xFFFF;
+                }
+            }
+            if (tid == 0) {
+                int ng = n_routed;
+                if (a.has_shared) {
+                    p_grp_e[ng] = (int16_t)(a.ee - a.eb);
+                    p_grp_n[ng] = (int16_t)T;
+                    p_grp_off[ng] = routed_slots;
+                    ++ng;
+                }
+                s_misc[0] = ng;
+                s_misc[1] = routed_slots + (a.has_shared ? T : 0);
+            }
+            __syncthreads();
+            // slot of each (token, choice): the expert's first slot + earlier tokens of it
+            for (int i = tid; i < T * k; i += kTlThreads) {
+                const int e = p_sel_e[i], t = i / k;
+                if (e < a.eb || e >= a.ee) {
+                    p_slot_of[i] = -1;  // not this pack's: no slot, no share of the output
+                    continue;
+                }
+                const unsigned long long m =
+                    (unsigned long long)mask[2 * e] | ((unsigned long long)mask[2 * e + 1] << 32);
+                const int slot = (cnt[e] & 0xFFFF) + __popcll(m & ((1ull << t) - 1ull));
+                p_slot_of[i] = (int16_t)slot;
+                p_slot_tok[slot] = (int16_t)t;
+            }
+            if (a.has_shared)
+                for (int t = tid; t < T; t += kTlThreads) p_slot_tok[routed_slots + t] = (int16_t)t;
+        }
+        __syncthreads();
+        cta0_clock(a.stamps, 4);
+        // this CTA's share of the fp16 slot rows of x, then one count per group touched
+        const int S = s_misc[1], ng = s_misc[0];
+        const int s0 = (int)((long long)S * c / G), s1 = (int)((long long)S * (c + 1) / G);
+        const int cpr = H / 8;
+        for (int i = tid; i < (s1 - s0) * cpr; i += kTlThreads) {
+            const int s = s0 + i / cpr, ch = i - (i / cpr) * cpr;
+            const int t = p_slot_tok[s];
+            const float down = 1.f / p_xscale[t];  // an exact power of two
+            float v[8];
+            if (a.x_dtype == MOE_DT_BF16) {
+                const uint4 q = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(a.x) +
+                                                                      (size_t)t * H) + ch);
+                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    v[2 * j] = __uint_as_float(w[j] << 16);
+                    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+                }
+            } else {
+                const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + (size_t)t * H) +
+                                  2 * ch;
+                const float4 x0 = __ldg(p), x1 = __ldg(p + 1);
+                v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+                v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+            }
+            uint4 o;
+            o.x = dq::pack_f16x2(v[0] * down, v[1] * down);
+            o.y = dq::pack_f16x2(v[2] * down, v[3] * down);
+            o.z = dq::pack_f16x2(v[4] * down, v[5] * down);
+            o.w = dq::pack_f16x2(v[6] * down, v[7] * down);
+            reinterpret_cast<uint4 *>(a.xg + (size_t)s * H)[ch] = o;
+        }
+        __syncthreads();
+        if (tid == 0 && s1 > s0) {
+            __threadfence();
+            // groups whose slot range meets [s0, s1): the slot ranges are ascending
+            for (int g = 0; g < ng; ++g) {
+                const int o = p_grp_off[g], n = p_grp_n[g];
+                if (o < s1 && o + n > s0) atomicAdd(a.ctr + C.grp_x + g, 1u);
+            }
+        }
+    }
+    __syncthreads();
+    grid_event(a.stamps, 2);
+    cta0_clock(a.stamps, 5);
+
+    // ---- gate/up and down units -------------------------------------------------------
+    const int ng = s_misc[0];
+    Geo q;
+    q.KC[0] = H / 256;
+    q.NB[0] = I / 128;
+    q.KC[1] = I / 256;
+    q.NB[1] = H / 256;
+    for (int p = 0; p < 2; ++p) {
+        q.U[p] = ng * q.NB[p] * q.KC[p];
+        q.lo[p] = range_lo(q.U[p], c, G);
+        q.hi[p] = range_lo(q.U[p], c + 1, G);
+    }
+    uint8_t *raw = smem, *atile = smem + a.nr * a.raw_stride, *btile = atile + a.na * kTlAStage;
+    int raw_issued = 0, b_issued = 0;
+
+    if (run && warp == kTlRawWarp) {
+        if (lane == 0) {
+            prefetch_tmap(&mGuQ);
+            prefetch_tmap(&mDnQ);
+            Ring rr;
+            for (int p = 0; p < 2 && !abort_flag; ++p)
+                for (int u = q.lo[p]; u < q.hi[p] && !abort_flag; ++u, rr.next(a.nr)) {
+                    const Unit x = unit_at(q, p, u);
+                    if (rr.u > 0 && !mbar_wait(&re_bar[rr.s], (rr.u - 1) & 1)) {
+                        abort_flag = 1;
+                        break;
+                    }
+                    uint8_t *st = raw + rr.s * a.raw_stride;
+                    const int ex = p_grp_e[x.g];
+                    if (p == 0)
+                        raw_load<FG>(st, &mGuQ, &mGuS, &mGuH, &rf_bar[rr.s], x.kc, x.b * 128, I + x.b * 128, ex);
+                    else
+                        raw_load<FD>(st, &mDnQ, &mDnS, &mDnH, &rf_bar[rr.s], x.kc, x.b * 256, x.b * 256 + 128, ex);
+                }
+            raw_issued = rr.u * a.nr + rr.s;
+        }
+    } else if (run && warp == kTlBWarp) {
+        if (lane == 0) {
+            prefetch_tmap(&mXg);
+            prefetch_tmap(&mH);
+            Ring rb_;
+            int ready_g = -1, ready_p = -1;
+            for (int p = 0; p < 2 && !abort_flag; ++p)
+                for (int u = q.lo[p]; u < q.hi[p] && !abort_flag; ++u) {
+                    const Unit x = unit_at(q, p, u);
+                    const int n = p_grp_n[x.g], off = p_grp_off[x.g], n16 = (n + 15) >> 4;
+                    if (x.g != ready_g || p != ready_p) {
+                        // gate/up: the group's x slot rows written by their CTAs; down: all
+                        // of the group's h tiles finished
+                        unsigned target;
+                        const unsigned *cp;
+                        if (p == 0) {
+                            target = (unsigned)owners(off, n, s_misc[1], G);
+                            cp = a.ctr + C.grp_x + x.g;
+                        } else {
+                            target = (unsigned)q.NB[0];
+                            cp = a.ctr + C.grp_h + x.g;
+                        }
+                        if (!wait_count(cp, target)) {
+                            abort_flag = 1;
+                            atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
+                            break;
+                        }
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        ready_g = x.g;
+                        ready_p = p;
+                    }
+                    for (int sl = 0; sl < 4; ++sl, rb_.next(a.nb)) {
+                        if (rb_.u > 0 && !mbar_wait(&be_bar[rb_.s], (rb_.u - 1) & 1)) {
+                            abort_flag = 1;
+                            break;
+                        }
+                        uint8_t *b_s = btile + rb_.s * a.bslot;
+                        mbar_arrive_expect_tx(&fb_bar[rb_.s], (uint32_t)n16 * 2048u);
+                        for (int jj = 0; jj < n16; ++jj)
+                            tma_load_2d(b_s + jj * 2048, p == 0 ? &mXg : &mH, &fb_bar[rb_.s], x.kc * 256 + sl * 64,
+                                        off + 16 * jj);
+                    }
+                }
+            b_issued = rb_.u * a.nb + rb_.s;
+        }
+    } else if (run && warp == kTlMmaWarp) {
+        if (lane == 0) {
+            Ring ra, rbm;
+            int seg = 0;
+            for (int p = 0; p < 2 && !abort_flag; ++p)
+                for (int u = q.lo[p]; u < q.hi[p] && !abort_flag; ++u) {
+                    const Unit x = unit_at(q, p, u);
+                    const int ab = seg & 1;
+                    if (x.first && seg >= 2 && !mbar_wait(&acce_bar[ab], ((seg >> 1) - 1) & 1)) {
+                        abort_flag = 1;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t idesc = tl_idesc((p_grp_n[x.g] + 15) & ~15);
+                    for (int sl = 0; sl < 4; ++sl, ra.next(a.na), rbm.next(a.nb)) {
+                        if (!mbar_wait(&fa_bar[ra.s], ra.u & 1) || !mbar_wait(&fb_bar[rbm.s], rbm.u & 1)) {
+                            abort_flag = 1;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        const uint8_t *a_s = atile + ra.s * kTlAStage;
+                        const uint64_t bd = desc_kmajor_sw128(btile + rbm.s * a.bslot);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint64_t ad = desc_kmajor_sw128(a_s + hh * kTlA);
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_f16(tmem + ab * 128 + hh * 64, ad + 2 * kk, bd + 2 * kk, idesc,
+                                        !(x.first && sl == 0 && kk == 0));
+                        }
+                        mma_commit(&ae_bar[ra.s]);
+                        mma_commit(&be_bar[rbm.s]);
+                    }
+                    if (x.last) {
+                        mma_commit(&accf_bar[ab]);
+                        ++seg;
+                    }
+                }
+        }
+    } else if (run && warp >= kTlDeqWarp0) {
+        const int n = tid - 32 * kTlDeqWarp0;
+        const int r = n & 127, tile = (n >> 7) & 1, bsel = n >> 8;
+        Ring ra, rr;
+        bool ok = true;
+        for (int p = 0; p < 2 && ok && !abort_flag; ++p)
+            for (int u = q.lo[p]; u < q.hi[p] && ok && !abort_flag; ++u, rr.next(a.nr)) {
+                if (!mbar_wait(&rf_bar[rr.s], rr.u & 1)) {
+                    abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                const uint8_t *st = raw + rr.s * a.raw_stride;
+#pragma unroll 1
+                for (int d = 0; d < 4; ++d, ra.next(a.na)) {
+                    if (ra.u > 0) {
+                        bool w = true;
+                        if (lane == 0) w = mbar_wait(&ae_bar[ra.s], (ra.u - 1) & 1);
+                        if (!__shfl_sync(0xffffffffu, w, 0)) {
+                            abort_flag = 1;
+                            ok = false;
+                            break;
+                        }
+                    }
+                    uint8_t *a_s = atile + ra.s * kTlAStage;
+                    if (p == 0) expand<FG>(st, a_s, r, tile, bsel, d, a.tab_gu);
+                    else expand<FD>(st, a_s, r, tile, bsel, d, a.tab_dn);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&fa_bar[ra.s]);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&re_bar[rr.s]);
+            }
+    } else if (run && warp < kTlEpiWarps) {
+        // ---- epilogue: one tensor-memory lane (tile row) per thread --------------------
+        const int r = warp * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+        int seg = 0;
+        bool range_ok = true;
+        for (int p = 0; p < 2; ++p)
+            for (int u = q.lo[p]; u < q.hi[p]; ++u) {
+                const Unit x = unit_at(q, p, u);
+                if (!x.last) continue;
+                const int ab = seg & 1;
+                const bool w_ok = mbar_wait(&accf_bar[ab], (seg >> 1) & 1);
+                tc_fence_after_sync();
+                // one decision for all four warps (they share named barriers): each
+                // raises the vote before the barrier, all read it after; every later
+                // iteration passes a barrier before the next vote is raised
+                if (!__all_sync(0xffffffffu, w_ok) || __any_sync(0xffffffffu, abort_flag != 0)) s_epi_abort = 1;
+                epi_sync();
+                if (s_epi_abort) {
+                    if (r == 0) {
+                        abort_flag = 1;
+                        atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
+                    }
+                    p = 2;
+                    break;
+                }
+                ++seg;
+                const int n = p_grp_n[x.g], off = p_grp_off[x.g], n16 = (n + 15) >> 4;
+                const int t0u = x.tile * q.KC[p];
+                // the whole tile in this CTA: straight from tensor memory; else this
+                // CTA's piece goes out and the CTA that finishes the tile's last piece
+                // sums them in CTA order
+                const bool whole = t0u >= q.lo[p] && t0u + q.KC[p] <= q.hi[p];
+                const uint32_t tb0 = tl + ab * 128;
+                float *pc = whole ? nullptr : piece(a, q, p, c, x.tile, G);
+                bool finalize = whole;
+                if (!whole) {
+                    for (int c0 = 0; c0 < n16; ++c0) {
+                        float v0[16], v1[16];
+                        tmem_ld16(tb0 + c0 * 16, v0);
+                        tmem_ld16(tb0 + 64 + c0 * 16, v1);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (c0 * 16 + j < n) {
+                                pc[(size_t)(c0 * 16 + j) * 256 + r] = v0[j];
+                                pc[(size_t)(c0 * 16 + j) * 256 + 128 + r] = v1[j];
+                            }
+                    }
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acce_bar[ab]);
+                    __threadfence();
+                    epi_sync();
+                    if (r == 0) {
+                        const unsigned prev = atomicAdd(a.ctr + (p == 0 ? C.gu_tile : C.dn_tile) + x.tile, 1u);
+                        s_misc[3] = prev + 1 == (unsigned)owners(t0u, q.KC[p], q.U[p], G);
+                        __threadfence();
+                    }
+                    epi_sync();
+                    finalize = s_misc[3] != 0;
+                    epi_sync();
+                    if (!finalize) continue;
+                }
+                const int e = p_grp_e[x.g];
+                const float hts = (p == 0 ? FG : FD) == MOE_FMT_NVFP4 ? 0.5f * __ldg((p == 0 ? a.ts_gu : a.ts_dn) + e)
+                                                                        : 1.f;
+                for (int c0 = 0; c0 < n16; ++c0) {
+                    float v0[16], v1[16];
+                    if (whole) {
+                        tmem_ld16(tb0 + c0 * 16, v0);
+                        tmem_ld16(tb0 + 64 + c0 * 16, v1);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) v0[j] = v1[j] = 0.f;
+                        int prev = -1;
+                        for (int uu = t0u; uu < t0u + q.KC[p]; ++uu) {
+                            const int cu = cta_of(uu, q.U[p], G);
+                            if (cu == prev) continue;
+                            prev = cu;
+                            const float *ps = piece(a, q, p, cu, x.tile, G);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                if (c0 * 16 + j < n) {
+                                    v0[j] += __ldcg(ps + (size_t)(c0 * 16 + j) * 256 + r);
+                                    v1[j] += __ldcg(ps + (size_t)(c0 * 16 + j) * 256 + 128 + r);
+                                }
+                        }
+                    }
+                    if (p == 0) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int jj = c0 * 16 + j;
+                            if (jj < n) {
+                                const int slot = off + jj;
+                                const float sc = p_xscale[p_slot_tok[slot]] * hts;
+                                const float gv = v0[j] * sc, uv = v1[j] * sc;
+                                const float hv = gv / (1.f + expf(-gv)) * uv;
+                                range_ok = range_ok && fabsf(hv) <= 65504.f;
+                                a.h[(size_t)slot * I + x.b * 128 + r] = __float2half_rn(hv);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int jj = c0 * 16 + j;
+                            if (jj < n) {
+                                float *yr = a.y + (size_t)(off + jj) * H + x.b * 256 + r;
+                                yr[0] = v0[j] * hts;
+                                yr[128] = v1[j] * hts;
+                            }
+                        }
+                    }
+                }
+                if (whole) {
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acce_bar[ab]);
+                }
+                __threadfence();
+                epi_sync();
+                if (r == 0) {
+                    if (p == 0) {
+                        atomicAdd(a.ctr + C.grp_h + x.g, 1u);
+                    } else {
+                        const unsigned prev = atomicAdd(a.ctr + C.rb + x.b, 1u);
+                        if (prev + 1 == (unsigned)ng) {
+                            __threadfence();
+                            p_won[s_misc[2]++] = x.b;
+                        }
+                    }
+                }
+            }
+        if (!__all_sync(0xffffffffu, range_ok) && lane == 0) atomicExch(a.err, (int)MOE_ERR_RANGE);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (abort_flag) {  // block-uniform after the barrier: drain what was issued, then release
+        if (tid == 0 && router_cta && e1 > e0) mbar_wait(&wr_bar, 0);  // the router rows' bulk copy
+        if (lane == 0 && warp == kTlRawWarp) drain_ring(rf_bar, a.nr, raw_issued);
+        if (lane == 0 && warp == kTlBWarp) drain_ring(fb_bar, a.nb, b_issued);
+        if (lane == 0 && warp == kTlMmaWarp) drain_mma(&dr_bar);
+        if (tid == 0) atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
+        tc_fence_before_sync();
+        __syncthreads();
+    }
+    grid_event(a.stamps, 3);
+    cta0_clock(a.stamps, 6);
+    // ---- combine the 256-row output blocks this CTA finished last ----------------------
+    if (!abort_flag) {
+        const int nwon = s_misc[2];
+        const int has = a.has_shared, routed_slots = s_misc[1] - (has ? T : 0);
+        if (ng == 0)  // no expert of this pack was selected and it has no shared expert: a zero share
+            for (size_t i = (size_t)c * kTlThreads + tid; i < (size_t)T * H; i += (size_t)G * kTlThreads) a.out[i] = 0.f;
+        for (int w = 0; w < nwon; ++w) {
+            const int b = p_won[w];
+            for (int i = tid; i < T * 256; i += kTlThreads) {
+                const int t = i >> 8, row = b * 256 + (i & 255);
+                float o = 0.f;
+                for (int j = 0; j < k; ++j) {
+                    const int sl = p_slot_of[t * k + j];
+                    if (sl >= 0) o += p_sel_g[t * k + j] * __ldcg(a.y + (size_t)sl * H + row);
+                }
+                if (has) o += __ldcg(a.y + (size_t)(routed_slots + t) * H + row);
+                a.out[(size_t)t * H + row] = o;
+            }
+        }
+    }
+    __syncthreads();
+    grid_event(a.stamps, 4);
+    cta0_clock(a.stamps, 7);
+    // ---- the last CTA to finish clears the counters this launch used --------------------
+    if (tid == 0) {
+        __threadfence();
+        s_tmp[0] = atomicAdd(a.ctr + C.ticket, 1u) == (unsigned)G - 1u;
+    }
+    __syncthreads();
+    if (s_tmp[0]) {
+        __threadfence();
+        if (__ldcg(a.err) != 0) {
+            // a CTA gave up somewhere: every counter, whatever the plan reached
+            for (int i = tid; i < C.total; i += kTlThreads)
+                if (i != C.ticket) a.ctr[i] = 0u;
+        } else {
+            for (int i = tid; i < ng * q.NB[0]; i += kTlThreads) a.ctr[C.gu_tile + i] = 0u;
+            for (int i = tid; i < ng * q.NB[1]; i += kTlThreads) a.ctr[C.dn_tile + i] = 0u;
+            for (int i = tid; i < ng; i += kTlThreads) {
+                a.ctr[C.grp_x + i] = 0u;
+                a.ctr[C.grp_h + i] = 0u;
+            }
+            for (int i = tid; i < H / 256; i += kTlThreads) a.ctr[C.rb + i] = 0u;
+            if (tid == 0) a.ctr[C.bar] = 0u;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            a.ctr[C.ticket] = 0u;
+        }
+    }
+    if (warp == kTlMmaWarp) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTlTmemCols);
+    }
+}
+
+using TlKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                          const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const TailArgs);
+
+template <int FG>
+TlKernel tl_pick_dn(int fd)
+{
+    switch (fd) {
+    case MOE_FMT_Q8_0: return tail_kernel<FG, MOE_FMT_Q8_0>;
+    case MOE_FMT_Q5_1: return tail_kernel<FG, MOE_FMT_Q5_1>;
+    case MOE_FMT_IQ4_NL: return tail_kernel<FG, MOE_FMT_IQ4_NL>;
+    default: return tail_kernel<FG, MOE_FMT_NVFP4>;
+    }
+}
+
+TlKernel tl_pick(int fg, int fd)
+{
+    switch (fg) {
+    case MOE_FMT_Q8_0: return tl_pick_dn<MOE_FMT_Q8_0>(fd);
+    case MOE_FMT_Q5_1: return tl_pick_dn<MOE_FMT_Q5_1>(fd);
+    case MOE_FMT_IQ4_NL: return tl_pick_dn<MOE_FMT_IQ4_NL>(fd);
+    default: return tl_pick_dn<MOE_FMT_NVFP4>(fd);
+    }
+}
+
+constexpr int kTlSmemMax = 225 * 1024;  // dynamic shared memory per CTA (the static part comes on top)
+
+}  // namespace
+
+int tail_counter_words(int E, int H, int I) { return tl_ctr(E, H, I).total; }
+
+size_t tail_part_floats(int grid, int max_tokens) { return (size_t)2 * grid * 2 * 256 * ((std::min(max_tokens, 64) + 15) & ~15); }
+
+bool tail_plan(const TailPlanIn &in, TailLaunch *out)
+{
+    if (in.T < 1 || in.T > kDecodeTcMaxN || in.max_tokens < in.T || in.k > 16 || in.E > 1024) return false;
+    if (in.H % 256 || in.I % 256 || in.H > 16384 || in.I > 16384) return false;
+    const int xbytes = in.x_dtype == MOE_DT_BF16 ? 2 : 4;
+    const int n16max = (std::min(in.max_tokens, 64) + 15) & ~15;
+    const TlPlanLayout PL = tl_plan_layout(in.T, in.k, in.E);
+    const int raw = std::max(tl_raw_bytes(in.fmt_gu), tl_raw_bytes(in.fmt_dn));
+    const int bslot = n16max * 128;
+    const int budget = kTlSmemMax - 1024 - PL.total;
+    // two of each ring at least; then A stages (a round trip to the MMA issuer
+    // each slice), raw stages (HBM latency) and B slots (L2) while they fit
+    int nr = 2, na = 2, nb = 2;
+    auto rings = [&] { return nr * raw + na * kTlAStage + nb * bslot; };
+    if (rings() > budget) return false;
+    bool grown = true;
+    while (grown) {
+        grown = false;
+        if (nr < kTlMaxRaw && rings() + raw <= budget) { ++nr; grown = true; }
+        if (nb < kTlMaxB && rings() + bslot <= budget) { ++nb; grown = true; }
+        if (na < 3 && rings() + kTlAStage <= budget) { ++na; grown = true; }
+    }
+    const int scratch = tl_scratch_bytes(in.T, in.H, in.E, in.grid, xbytes);
+    if (scratch > rings()) return false;
+    out->nr = nr;
+    out->na = na;
+    out->nb = nb;
+    out->raw_stride = raw;
+    out->bslot = bslot;
+    out->n16max = n16max;
+    out->rings = rings();
+    out->smem = (size_t)1024 + rings() + PL.total;
+    return true;
+}
+
+cudaError_t tail_set_attributes()
+{
+    const int fmts[4] = {MOE_FMT_Q8_0, MOE_FMT_Q5_1, MOE_FMT_IQ4_NL, MOE_FMT_NVFP4};
+    for (int fg : fmts)
+        for (int fd : fmts) {
+            const cudaError_t e =
+                cudaFuncSetAttribute(tl_pick(fg, fd), cudaFuncAttributeMaxDynamicSharedMemorySize, kTlSmemMax);
+            if (e != cudaSuccess) return e;
+        }
+    return cudaSuccess;
+}
+
+int tail_blocks_per_sm(int fmt_gu, int fmt_dn, size_t smem)
+{
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, tl_pick(fmt_gu, fmt_dn), kTlThreads, smem) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+cudaError_t launch_tail(const TailCall &t, const TailLaunch &L, int grid, int pdl, cudaStream_t s)
+{
+    TailArgs a{};
+    a.x = t.x;
+    a.x_dtype = t.x_dtype;
+    a.wr = t.wr;
+    a.T = t.T;
+    a.H = t.H;
+    a.E = t.E;
+    a.I = t.I;
+    a.k = t.k;
+    a.has_shared = t.has_shared;
+    a.eb = t.eb;
+    a.ee = t.ee;
+    a.tab_gu = t.tab_gu;
+    a.tab_dn = t.tab_dn;
+    a.ts_gu = t.gu->ts;
+    a.ts_dn = t.dn->ts;
+    a.logits = t.ws->logits;
+    a.xscale = t.ws->slot_scale;
+    a.xg = reinterpret_cast<__half *>(t.ws->xg);
+    a.h = reinterpret_cast<__half *>(t.ws->h);
+    a.y = t.ws->y;
+    a.part = t.ws->tail_part;
+    a.ctr = t.ws->tail_ctr;
+    a.err = t.ws->err;
+    a.out = t.out;
+    a.idx_out = t.ws->idx;
+    a.gate_out = t.ws->gate;
+    a.cnt_out = t.ws->cnt;
+    a.nr = L.nr;
+    a.na = L.na;
+    a.nb = L.nb;
+    a.raw_stride = L.raw_stride;
+    a.bslot = L.bslot;
+    a.n16max = L.n16max;
+    a.rings = L.rings;
+    a.stamps = t.stamps;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kTlThreads);
+    cfg.dynamicSmemBytes = L.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    if (pdl) {
+        // CTAs wait on one another (grid barrier, counters): one CTA per SM and
+        // grid = SMs, all resident once the previous kernel's CTAs have left
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    } else {
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const DecodeTcMaps &m = *t.maps;
+    return cudaLaunchKernelEx(&cfg, tl_pick(t.gu->fmt, t.dn->fmt), m.gu[0], m.gu[1], m.gu[2], m.dn[0], m.dn[1],
+                              m.dn[2], m.xg, m.h, a);
+}
+
+}  // namespace moe

@@ -102,10 +102,12 @@ typedef enum { MOE_DT_F32 = 1, MOE_DT_BF16 = 2 } moe_dtype;
  * to bf16 for bf16 MMA; hidden and inter multiples of 256, bf16 activations,
  * top_k <= 32; its buffers are sized at pack time when max_tokens > 64), else
  * GROUPED.  DECODE: one token runs the single-token streaming kernel; 2 to 64
- * tokens run the tensor-core grouped decode (weights expanded to fp16, fp32
- * accumulation; hidden and inter multiples of 256 and every weight an fp16
- * normal number or zero, checked at pack time), else the CUDA-core grouped
- * kernels.  DENSE is the dense-batched comparison variant (pack created with
+ * tokens run the device-planned tail in one launch: routing, the plan, the
+ * tensor-core grouped gate/up and down (weights expanded to fp16, fp32
+ * accumulation; hidden and inter multiples of 256, top_k <= 16 and every weight
+ * an fp16 normal number or zero, checked at pack time) and the combine; where
+ * that launch does not fit, the same tensor-core work in separate launches,
+ * else the CUDA-core grouped kernels.  DENSE is the dense-batched comparison variant (pack created with
  * MOE_PACK_DENSE, n_tokens <= 64): every active expert multiplies the whole
  * batch, with a zero gate for the tokens not routed to it. */
 typedef enum {
@@ -113,7 +115,15 @@ typedef enum {
     MOE_PATH_DECODE = 1,   /* see above; falls back to GROUPED where its kernels do not apply */
     MOE_PATH_PREFILL = 2,
     MOE_PATH_DENSE = 3,
-    MOE_PATH_GROUPED = 4   /* decode as separate route / gate-up / down / combine launches, fp32 CUDA cores */
+    MOE_PATH_GROUPED = 4,  /* decode as separate route / gate-up / down / combine launches, fp32 CUDA cores */
+    MOE_PATH_DECODE_STAGED = 5, /* 2-64 tokens: the tensor-core grouped decode as separate launches (route and
+                                   plan, x gather, gate/up, down, combine); MOE_ERR_UNSUPPORTED where it does
+                                   not apply */
+    MOE_PATH_TAIL = 6,     /* 1-64 tokens: the one-launch tail (what DECODE runs for 2-64 tokens when it fits);
+                              MOE_ERR_UNSUPPORTED where it does not apply */
+    MOE_PATH_PREFILL_BF16 = 7 /* the prefill with every format's weights dequantised to bf16 in shared memory
+                                 and bf16 MMA, NVFP4 included (its weights are exact in bf16: x is not rounded
+                                 to NVFP4, h is rounded to bf16); same conditions as PREFILL */
 } moe_path;
 
 /* Description of one layer's experts, all in HOST memory; moe_pack_experts
@@ -148,6 +158,19 @@ typedef struct {
     const void *shared_gate_up_blocks;
     const void *shared_down_blocks;
     int flags;            /* MOE_PACK_* bits, 0 for none */
+    /* Expert parallelism: the pack holds only routed experts [expert_begin,
+     * expert_end) of the layer's n_experts.  The block arrays (and NVFP4 scales)
+     * then hold those experts, in order, followed by the shared expert when
+     * has_shared.  Routing still covers all n_experts (pass the whole router);
+     * a forward computes the partial layer
+     *   out_t = sum_{e in S, expert_begin <= e < expert_end} g_e y_e (+ y_shared)
+     * so the outputs of packs whose windows partition [0, n_experts), with the
+     * shared expert in exactly one of them, sum to the layer.  0 and 0 (or 0
+     * and n_experts) = every expert.  A windowed pack runs the one-launch tail
+     * (1-64 tokens: AUTO, DECODE or TAIL); other paths return
+     * MOE_ERR_UNSUPPORTED. */
+    int expert_begin;
+    int expert_end;
 } moe_pack_desc;
 
 /* moe_pack_desc.flags: size the workspace for MOE_PATH_DENSE as well (every
@@ -264,7 +287,8 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
 /* After a forward: copy its routing and plan to HOST memory (synchronises
  * `stream`).  Any pointer may be NULL.
  *   idx   [n_tokens x top_k] int32, gate [n_tokens x top_k] fp32,
- *   counts [n_experts + 1] int32 tokens per expert (last entry: shared).
+ *   counts [n_experts + 1] int32 tokens per expert (last entry: shared); a
+ *   windowed pack counts only its own experts (0 for the others).
  * 1 <= n_tokens <= max_tokens and 1 <= top_k <= max_top_k, else
  * MOE_ERR_INVALID_ARG; they should be the last non-empty forward's. */
 moe_status moe_read_routing(const moe_pack *pack, int n_tokens, int top_k, int32_t *idx,

@@ -44,11 +44,32 @@ def _bitwise(li, x, path=None, max_tokens=None, h_max=2048):
 @pytest.mark.parametrize("fmt_gu,fmt_dn", PAIRS)
 @pytest.mark.parametrize("T", [1, 5, 64])
 def test_decode_default_path_is_bitwise_exact(fmt_gu, fmt_dn, T):
-    """One token: the single-token streaming kernel; 2-64: the tensor-core grouped decode."""
+    """One token: the single-token streaming kernel; 2-64: the one-launch tail."""
     li = exact_layer(fmt_gu, fmt_dn, seed=10 * fmt_gu + fmt_dn)
     info = _bitwise(li, exact_tokens(li, T, seed=T))
     if synth.FMT_IQ4_NL in (fmt_gu, fmt_dn):
         assert info["code_table_masked"] == ((fmt_gu == synth.FMT_IQ4_NL) | 2 * (fmt_dn == synth.FMT_IQ4_NL))
+
+
+@pytest.mark.parametrize("fmt_gu,fmt_dn", PAIRS)
+@pytest.mark.parametrize("T,path", [(1, "tail"), (13, "tail"), (3, "staged"), (40, "staged")])
+def test_tail_and_staged_tensor_core_decode_are_bitwise_exact(fmt_gu, fmt_dn, T, path):
+    """The one-launch tail also at one token, and the same tensor-core work as
+    separate launches (route and plan, x gather, gate/up, down, combine)."""
+    import block_quantized_expert_moe_b200 as bq
+    li = exact_layer(fmt_gu, fmt_dn, seed=10 * fmt_gu + fmt_dn + 3)
+    p = {"tail": bq.MOE_PATH_TAIL, "staged": bq.MOE_PATH_DECODE_STAGED}[path]
+    _bitwise(li, exact_tokens(li, T, seed=T + 100), path=p)
+
+
+def test_tail_on_many_experts_and_every_sm_partition():
+    """64 experts, top-1, 64 tokens: about 60 groups, so the units of a tile meet
+    ranges of several CTAs and most tiles are summed from pieces; then 3 tokens,
+    where fewer units than SMs leave some CTAs without work."""
+    import block_quantized_expert_moe_b200 as bq
+    li = exact_layer(synth.FMT_IQ4_NL, synth.FMT_Q5_1, n_experts=64, seed=77)
+    for T in (64, 3):
+        _bitwise(li, exact_tokens(li, T, seed=T + 7), path=bq.MOE_PATH_TAIL, max_tokens=64)
 
 
 @pytest.mark.parametrize("fmt_gu,fmt_dn", PAIRS)
@@ -86,11 +107,13 @@ def test_small_ragged_shapes_are_bitwise_exact():
 
 
 @pytest.mark.parametrize("fmt_gu,fmt_dn", [(synth.FMT_Q8_0, synth.FMT_Q8_0), (synth.FMT_IQ4_NL, synth.FMT_Q5_1),
-                                           (synth.FMT_Q5_1, synth.FMT_IQ4_NL)])
+                                           (synth.FMT_Q5_1, synth.FMT_IQ4_NL), (synth.FMT_NVFP4, synth.FMT_NVFP4),
+                                           (synth.FMT_NVFP4, synth.FMT_Q5_1)])
 def test_bf16_dequant_prefill_is_bitwise_exact(fmt_gu, fmt_dn):
-    """More than 64 tokens: the bf16-dequantising tensor-core prefill.  bf16 keeps 8
-    significant bits, so h stays below 256 here (one +-1 per up row)."""
+    """More than 64 tokens: the bf16-dequantising tensor-core prefill (NVFP4 included:
+    its weights are exact in bf16).  bf16 keeps 8 significant bits, so h stays below
+    256 here (one +-1 per up row)."""
     import block_quantized_expert_moe_b200 as bq
     li = exact_layer(fmt_gu, fmt_dn, n_gate=40, n_up=1, seed=10 * fmt_gu + fmt_dn + 5)
     x = exact_tokens(li, 200, seed=11)
-    _bitwise(li, x, path=bq.MOE_PATH_PREFILL, h_max=256)
+    _bitwise(li, x, path=bq.MOE_PATH_PREFILL_BF16, h_max=256)

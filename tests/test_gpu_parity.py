@@ -56,6 +56,29 @@ def test_zipf_batch_nvfp4_64_tokens():
     print(f"zipf_batch (64 tokens, NVFP4, tensor-core decode): normwise err {err:.3e} of {DECODE_TOL:.0e}")
 
 
+@pytest.mark.parametrize("name,layer,T", [("spec_verify", 3, 8), ("zipf_batch", 4, 64), ("model_decode", 2, 1),
+                                          ("tiny_q8", 1, 17)])
+def test_one_launch_tail_matches_oracle_and_staged_path(name, layer, T):
+    """The device-planned tail in one launch (route, plan, tensor-core gate/up and down,
+    combine) against the oracle, and against the same tensor-core work run as separate
+    launches: both round weights, x and h to fp16 the same way, only the order of the
+    fp32 sums differs."""
+    import block_quantized_expert_moe_b200 as bq
+    wl, li = _layer(name, layer)
+    x = synth.tokens(wl, li.router, layer, 5, T)
+    ref, ridx, rgate = oracle_layer(li, x, wl.top_k)
+    out_t, idx, gate, counts = gpu_layer(li, x, wl.top_k, path=bq.MOE_PATH_TAIL)
+    assert_routing_equal(idx, gate, ridx, rgate)
+    assert np.array_equal(counts, expected_counts(ridx, wl.n_experts, T, wl.has_shared))
+    err = normwise_err(out_t, ref)
+    assert err <= DECODE_TOL, err
+    print(f"{name} ({T} tokens, one-launch tail): normwise err {err:.3e} of {DECODE_TOL:.0e}")
+    if T >= 2:
+        out_s, _, _, _ = gpu_layer(li, x, wl.top_k, path=bq.MOE_PATH_DECODE_STAGED)
+        assert normwise_err(out_s, ref) <= DECODE_TOL
+        assert normwise_err(out_t, out_s) <= 1e-4
+
+
 @pytest.mark.parametrize("name,T", [("model_decode", 100), ("tiny_q8", 150)])
 def test_grouped_path_above_64_tokens_matches_oracle(name, T):
     """MOE_PATH_GROUPED (fp32 CUDA-core matvecs) is not limited to decode batches:

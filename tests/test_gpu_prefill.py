@@ -126,3 +126,27 @@ def test_prefill_iq4nl_q51_full_chunk_sampled():
     rng = np.random.default_rng(2)
     _run_dq(synth.WORKLOADS["prefill_iq4nl_q51"], 8192, sample=np.sort(rng.choice(8192, 16, replace=False)))
 
+
+
+def test_prefill_nvfp4_through_bf16_dequant_against_the_exact_oracle():
+    """NVFP4 weights dequantised to bf16 in shared memory (exact), x left in bf16, bf16
+    MMA: the variant of the NVFP4 prefill that the exact oracle (no activation
+    quantisation) checks, beside the native FP4 GEMM that rounds x and h to NVFP4."""
+    import block_quantized_expert_moe_b200 as bq
+    wl = synth.WORKLOADS["prefill_nvfp4"]
+    li = synth.layer_inputs(wl, 2)
+    x = synth.tokens(wl, li.router, 2, 0, 300)
+    out, idx, gate, counts = gpu_layer(li, x, wl.top_k, path=bq.MOE_PATH_PREFILL_BF16)
+    ref, ridx, rgate = oracle_layer(li, x, wl.top_k)
+    assert_routing_equal(idx, gate, ridx, rgate)
+    assert np.array_equal(counts, expected_counts(ridx, wl.n_experts, 300, wl.has_shared))
+    err = normwise_err(out, ref)
+    assert err <= PREFILL_TOL, err
+    print(f"prefill NVFP4 -> bf16 T=300: err vs exact oracle {err:.2e}")
+    # the full 8192-token chunk, 16 sampled tokens
+    x = synth.tokens(wl, li.router, 2, 0, 8192)
+    out, idx, gate, _ = gpu_layer(li, x, wl.top_k, path=bq.MOE_PATH_PREFILL_BF16)
+    tok = np.sort(np.random.default_rng(3).choice(8192, 16, replace=False))
+    ref, ridx, rgate = oracle_layer(li, x, wl.top_k, tokens=tok)
+    assert_routing_equal(idx[tok], gate[tok], ridx, rgate)
+    assert normwise_err(out[tok], ref) <= PREFILL_TOL
