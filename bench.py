@@ -395,6 +395,8 @@ def measure(a, bq, torch, wl, layers, T, dist, world, dev, e2e=True):
     grid_event_us = ({n: float(stage_ms[15 + i] / nf * 1e3) for i, n in enumerate(grid_names)}
                      if stage_ms[4] > 0 and stage_ms[15] > 0 else None)
     if grid_event_us is not None:
+        # stream1: CTA 0 at eight internal points; tail: CTA 0's first four units, raw
+        # stage landed (4) then MMAs issued (4); from the kernel's start
         grid_event_us["cta0_points"] = [round(float(v / nf * 1e3), 3) for v in stage_ms[24:32]]
     elif stage_ms[0] > 0 and stage_ms[15] > 0:
         route_names = ["last_start", "first_staged", "last_staged", "first_logits", "last_logits",

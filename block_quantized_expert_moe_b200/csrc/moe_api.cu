@@ -430,6 +430,55 @@ moe_status build_proj(moe_pack *p, DevProj &dp, int fmt, int rows, int cols, con
         if ((st = dev_alloc(p, hr.size(), &dr)) != MOE_OK) return st;
         if (cudaMemcpy(dr, hr.data(), hr.size(), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
     }
+    // tiled copy for the one-launch tail (shapes of whole 128-row blocks and
+    // 256-wide K chunks whose weights the tensor-core decode takes)
+    if (dp.f16_ok && rows % 128 == 0 && cols % 256 == 0 && p->max_tokens <= kDecodeMaxTokens) {
+        const int dfmt = dp.fmt, KC = cols / 256, RB = rows / 128;
+        const int cb = tl_codes_bytes(dfmt), sb = tl_scales_bytes(dfmt);
+        dp.tl_block = tl_block_bytes(dfmt);
+        dp.tl_stride = round_up((int64_t)RB * KC * dp.tl_block, 256);
+        std::vector<uint8_t> ht;
+        try {
+            ht.assign((size_t)dp.tl_stride * n_slots, 0);
+        } catch (const std::bad_alloc &) {
+            return MOE_ERR_OOM;
+        }
+        const uint8_t *srm = nv ? hr.data() : hs.data();  // scales row by row
+        const int64_t srm_stride = nv ? dp.sr_stride : dp.sc_stride;
+        const int srm_row = nv ? dp.sr_row : dp.sc_row;
+        parallel_for(n_slots, [&](int sl) {
+            const uint8_t *q = hq.data() + (int64_t)sl * dp.qs_stride, *sr = srm + (int64_t)sl * srm_stride;
+            const uint8_t *h = dp.qh_row ? hh.data() + (int64_t)sl * dp.qh_stride : nullptr;
+            for (int rb = 0; rb < RB; ++rb)
+                for (int kc = 0; kc < KC; ++kc) {
+                    uint8_t *blk = ht.data() + (int64_t)sl * dp.tl_stride + ((int64_t)rb * KC + kc) * dp.tl_block;
+                    for (int r = 0; r < 128; ++r) {
+                        const int64_t R = (int64_t)rb * 128 + r;
+                        // codes: 16-byte chunk c of a 128-byte row segment at chunk c ^ (r % 8)
+                        const int nbx = dfmt == MOE_FMT_Q8_0 ? 2 : 1;
+                        for (int bx = 0; bx < nbx; ++bx)
+                            for (int c = 0; c < 8; ++c)
+                                std::memcpy(blk + bx * 16384 + r * 128 + ((c ^ (r & 7)) << 4),
+                                            q + R * dp.qs_row + (int64_t)kc * 128 * nbx + bx * 128 + c * 16, 16);
+                        if (dfmt == MOE_FMT_Q5_1) {
+                            // {d, m} and fifth bits: 32 bytes a row, chunk c at c ^ ((r / 4) % 2)
+                            for (int c = 0; c < 2; ++c) {
+                                const int o = r * 32 + ((c ^ ((r >> 2) & 1)) << 4);
+                                std::memcpy(blk + cb + o, sr + R * srm_row + kc * 32 + c * 16, 16);
+                                std::memcpy(blk + cb + sb + o, h + R * dp.qh_row + kc * 32 + c * 16, 16);
+                            }
+                        } else {
+                            std::memcpy(blk + cb + r * 16, sr + R * srm_row + kc * 16, 16);
+                        }
+                    }
+                }
+        });
+        void *dt2;
+        if ((st = dev_alloc(p, ht.size(), &dt2)) != MOE_OK) return st;
+        if (cudaMemcpy(dt2, ht.data(), ht.size(), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+        dp.tl = static_cast<const uint8_t *>(dt2);
+        p->arena_bytes += (int64_t)ht.size();
+    }
     dp.qs = static_cast<const uint8_t *>(dq);
     dp.sc = static_cast<const uint8_t *>(ds);
     dp.qh = static_cast<const uint8_t *>(dh);
@@ -816,7 +865,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
         if (ok < 0) {
             TailPlanIn in{T, p->max_tokens, p->H, p->E, p->I, p->max_top_k, x_dtype, p->fmt_gu, p->fmt_dn, p->num_sms};
             TailLaunch &L = pm->tail_launch[T][xb];
-            ok = pm->dtc == 1 && p->max_tokens <= kDecodeMaxTokens && tail_plan(in, &L) &&
+            ok = pm->dtc == 1 && p->gu.tl && p->dn.tl && p->max_tokens <= kDecodeMaxTokens && tail_plan(in, &L) &&
                          tail_blocks_per_sm(p->fmt_gu, p->fmt_dn, L.smem) >= 1
                      ? 1
                      : 0;

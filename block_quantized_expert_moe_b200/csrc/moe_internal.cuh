@@ -44,7 +44,22 @@ struct DevProj {
     // every weight of the projection is an fp16 normal number or zero (the
     // tensor-core decode path expands blocks to fp16)
     bool f16_ok = false;
+    // the same weights tile by tile for the one-launch tail: per expert slot,
+    // per 128-row block, per 256-wide K chunk one contiguous block of
+    // tl_block bytes (codes, then scales, then Q5_1 fifth bits) already in the
+    // shared-memory layout the expanding warps read (codes in the 128-byte
+    // swizzle; Q5_1 scales and fifth bits in the 32-byte swizzle), so that one
+    // bulk copy moves a tile's chunk; null when the shape has no such tiles
+    const uint8_t *tl = nullptr;
+    int64_t tl_stride = 0;  // bytes per expert slot
+    int tl_block = 0;       // bytes per (128-row block, K chunk)
 };
+
+// Sizes of one (128-row block, 256-wide K chunk) block of a tiled plane.
+__host__ __device__ inline int tl_codes_bytes(int fmt) { return 128 * 128 * (fmt == MOE_FMT_Q8_0 ? 2 : 1); }
+__host__ __device__ inline int tl_scales_bytes(int fmt) { return 128 * (fmt == MOE_FMT_Q5_1 ? 32 : 16); }
+__host__ __device__ inline int tl_qh_bytes(int fmt) { return fmt == MOE_FMT_Q5_1 ? 128 * 32 : 0; }
+__host__ __device__ inline int tl_block_bytes(int fmt) { return tl_codes_bytes(fmt) + tl_scales_bytes(fmt) + tl_qh_bytes(fmt); }
 
 // Byte offset of E4M3 scale q (0..3) of row r in 64-wide K step s, in the
 // block-scale layout of the tcgen05 block-scaled MMA: atoms of 512 bytes hold

@@ -77,20 +77,20 @@ constexpr long long kTlSpin = 1ll << 31;  // clocks
 __host__ __device__ inline int tl_cdiv(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ inline int tl_al16(int v) { return (v + 15) & ~15; }
 
-// One raw stage: the unit's 256 rows (two 128-row tiles) x K = 256 as the TMA
-// boxes land: codes (128-byte rows, 128-byte swizzle; Q8_0 two boxes), scales
-// (16 bytes a row; Q5_1 32 with a 32-byte swizzle) and Q5_1 fifth bits (32).
+// One raw stage: the unit's 256 rows (two 128-row tiles) x K = 256, each tile's
+// block of the pack's tiled copy as one bulk copy lands it: codes (128-byte
+// rows in the 128-byte swizzle; Q8_0 two 16 KB halves), scales (16 bytes a
+// row; Q5_1 32 in the 32-byte swizzle) and Q5_1 fifth bits (32, same swizzle).
 template <int FMT>
 struct TlRaw {
-    static constexpr int kCodeBoxes = FMT == MOE_FMT_Q8_0 ? 2 : 1;
-    static constexpr int kCodes = kCodeBoxes * 128 * 128;
-    static constexpr int kScW = FMT == MOE_FMT_Q5_1 ? 32 : 16;
-    static constexpr int kScales = 128 * kScW;
+    static constexpr int kCodes = 128 * 128 * (FMT == MOE_FMT_Q8_0 ? 2 : 1);
+    static constexpr int kScales = 128 * (FMT == MOE_FMT_Q5_1 ? 32 : 16);
     static constexpr int kQh = FMT == MOE_FMT_Q5_1 ? 128 * 32 : 0;
-    static constexpr int kStage = 2 * (kCodes + kScales + kQh);
-    __device__ static int codes(int t) { return t * kCodes; }
-    __device__ static int scales(int t) { return 2 * kCodes + t * kScales; }
-    __device__ static int qh(int t) { return 2 * (kCodes + kScales) + t * kQh; }
+    static constexpr int kTile = kCodes + kScales + kQh;  // = tl_block_bytes(FMT)
+    static constexpr int kStage = 2 * kTile;
+    __device__ static int codes(int t) { return t * kTile; }
+    __device__ static int scales(int t) { return t * kTile + kCodes; }
+    __device__ static int qh(int t) { return t * kTile + kCodes + kScales; }
 };
 
 __host__ __device__ inline int tl_raw_bytes(int fmt)
@@ -162,7 +162,7 @@ __host__ __device__ inline int tl_scratch_bytes(int T, int H, int E, int G, int 
 {
     const TlRoute r = tl_route(T, E, G, xbytes);
     const int rows = tl_cdiv(E, r.nrb);
-    const int gemv = tl_al16(rows * H * 2) + r.rt * H * 4;
+    const int gemv = tl_al16(rows * H * 2) + r.rt * H * 4 + rows * 8 * r.rt * 4;  // router rows, x, partial dots
     const int nsw = min(kTlWarps, T);
     const int sel = nsw * (E * 4 + 512);
     const int plan = tl_al16((E + 1) * 4) + E * 8 + E * 4;  // counts, token masks, own {flag, tokens}
@@ -177,8 +177,10 @@ struct TailArgs {
     int eb, ee;                  // routed experts [eb, ee) are in the pack, at slots e - eb
     CodeTable tab_gu, tab_dn;
     const float *ts_gu, *ts_dn;  // NVFP4 per-pack-slot matrix scales
+    const uint8_t *tl_gu, *tl_dn;  // the projections' tiled copies (DevProj::tl)
+    int64_t tl_gu_stride, tl_dn_stride;
     float *logits;               // [T x E]
-    float *xscale;               // [T] 2^s, x scaled by 2^-s into fp16
+    float *slot_scale;           // [slots] 2^s: the slot's row of x was scaled by 2^-s into fp16
     __half *xg;                  // [slots x H] fp16 slot rows of x
     __half *h;                   // [slots x I]
     float *y;                    // [slots x H]
@@ -239,6 +241,20 @@ __device__ __forceinline__ unsigned ld_acq(const unsigned *p)
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Bounded wait on an mbarrier phase that backs off between tests: for warps
+// whose wait is not on the critical path (epilogue, producers), so that their
+// polling does not take issue slots from the expanding warps.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t *bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kTlSpin) return false;
+        __nanosleep(128);
+    }
+    return true;
 }
 
 // Spin (bounded) until *p >= target; false if the wait ran out.
@@ -340,21 +356,17 @@ __device__ __forceinline__ float *piece(const TailArgs &a, const Geo &q, int p, 
     return a.part + (((size_t)p * G + c) * 2 + which) * (size_t)a.n16max * 256;
 }
 
+// A unit's raw stage: two bulk copies, one per tile (128-row blocks rb0, rb1,
+// K chunk kc of expert slot ex), from the pack's tiled copy.
 template <int FMT>
-__device__ __forceinline__ void raw_load(uint8_t *st, const CUtensorMap *mq, const CUtensorMap *ms,
-                                         const CUtensorMap *mh, uint64_t *bar, int kc, int row0, int row1, int ex)
+__device__ __forceinline__ void raw_load(uint8_t *st, const uint8_t *tl, int64_t tl_stride, int KC, uint64_t *bar,
+                                         int kc, int rb0, int rb1, int ex)
 {
     using RL = TlRaw<FMT>;
     mbar_arrive_expect_tx(bar, (uint32_t)RL::kStage);
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        const int row = t ? row1 : row0;
-#pragma unroll
-        for (int bx = 0; bx < RL::kCodeBoxes; ++bx)
-            tma_load_3d(st + RL::codes(t) + bx * 16384, mq, bar, (kc * RL::kCodeBoxes + bx) * 128, row, ex);
-        tma_load_3d(st + RL::scales(t), ms, bar, kc * RL::kScW, row, ex);
-        if (FMT == MOE_FMT_Q5_1) tma_load_3d(st + RL::qh(t), mh, bar, kc * 32, row, ex);
-    }
+    const uint8_t *base = tl + (int64_t)ex * tl_stride;
+    bulk_g2s(st, base + ((int64_t)rb0 * KC + kc) * RL::kTile, (uint32_t)RL::kTile, bar);
+    bulk_g2s(st + RL::kTile, base + ((int64_t)rb1 * KC + kc) * RL::kTile, (uint32_t)RL::kTile, bar);
 }
 
 // Thread n of the expanders: block bsel of slice d of row r of tile `tile`.
@@ -402,10 +414,7 @@ __host__ __device__ constexpr uint32_t tl_idesc(int N)
 
 template <int FG, int FD>
 __global__ void __launch_bounds__(kTlThreads, 1)
-    tail_kernel(const __grid_constant__ CUtensorMap mGuQ, const __grid_constant__ CUtensorMap mGuS,
-                const __grid_constant__ CUtensorMap mGuH, const __grid_constant__ CUtensorMap mDnQ,
-                const __grid_constant__ CUtensorMap mDnS, const __grid_constant__ CUtensorMap mDnH,
-                const __grid_constant__ CUtensorMap mXg, const __grid_constant__ CUtensorMap mH, const TailArgs a)
+    tail_kernel(const __grid_constant__ CUtensorMap mXg, const __grid_constant__ CUtensorMap mH, const TailArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t rf_bar[kTlMaxRaw], re_bar[kTlMaxRaw], fa_bar[kTlMaxA], ae_bar[kTlMaxA],
@@ -422,7 +431,6 @@ __global__ void __launch_bounds__(kTlThreads, 1)
     const TlCtr C = tl_ctr(E, H, I);
     const TlPlanLayout PL = tl_plan_layout(T, k, E);
     uint8_t *plan = smem + a.rings;
-    float *p_xscale = reinterpret_cast<float *>(plan + PL.xscale);
     int16_t *p_sel_e = reinterpret_cast<int16_t *>(plan + PL.sel_e);
     float *p_sel_g = reinterpret_cast<float *>(plan + PL.sel_g);
     int16_t *p_slot_of = reinterpret_cast<int16_t *>(plan + PL.slot_of);
@@ -484,30 +492,53 @@ __global__ void __launch_bounds__(kTlThreads, 1)
 
     // ---- route: logits of rows [e0, e1) for tokens [t0, t0 + tn) ------------------------
     if (router_cta) {
-        // x as fp32 in shared memory
-        const int nch = tn * (H / 8);
-        for (int i = tid; i < nch; i += kTlThreads) {
-            const int t = i / (H / 8), ch = i - t * (H / 8);
-            float v[8];
-            if (a.x_dtype == MOE_DT_BF16) {
-                const uint4 q = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(a.x) +
-                                                                      (size_t)(t0 + t) * H) + ch);
-                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        // x as fp32 in shared memory: each thread's 16-byte loads all in flight first
+        const int cpr = H / 8, nch = tn * cpr;
+        for (int i0 = 0; i0 < nch; i0 += 8 * kTlThreads) {
+            uint4 q[8];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    v[2 * j] = __uint_as_float(w[j] << 16);
-                    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            for (int j = 0; j < 8; ++j) {
+                const int i = i0 + j * kTlThreads + tid;
+                if (i < nch) {
+                    const int t = i / cpr, ch = i - t * cpr;
+                    q[j] = a.x_dtype == MOE_DT_BF16
+                               ? __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(a.x) +
+                                                                       (size_t)(t0 + t) * H) + ch)
+                               : __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(a.x) +
+                                                                       (size_t)(t0 + t) * H) + ch * 2);
                 }
-            } else {
-                const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) +
-                                                                   (size_t)(t0 + t) * H) + 2 * ch;
-                const float4 x0 = __ldg(p), x1 = __ldg(p + 1);
-                v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
-                v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
             }
-            float4 *d = reinterpret_cast<float4 *>(sX + (size_t)t * H + ch * 8);
-            d[0] = make_float4(v[0], v[1], v[2], v[3]);
-            d[1] = make_float4(v[4], v[5], v[6], v[7]);
+            uint4 q2[8];  // fp32 x: the second half of each 8-value chunk
+            if (a.x_dtype != MOE_DT_BF16) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i = i0 + j * kTlThreads + tid;
+                    if (i < nch) {
+                        const int t = i / cpr, ch = i - t * cpr;
+                        q2[j] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(a.x) +
+                                                                      (size_t)(t0 + t) * H) + ch * 2 + 1);
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = i0 + j * kTlThreads + tid;
+                if (i < nch) {
+                    const int t = i / cpr, ch = i - t * cpr;
+                    float4 *d = reinterpret_cast<float4 *>(sX + (size_t)t * H + ch * 8);
+                    if (a.x_dtype == MOE_DT_BF16) {
+                        d[0] = make_float4(__uint_as_float(q[j].x << 16), __uint_as_float(q[j].x & 0xFFFF0000u),
+                                           __uint_as_float(q[j].y << 16), __uint_as_float(q[j].y & 0xFFFF0000u));
+                        d[1] = make_float4(__uint_as_float(q[j].z << 16), __uint_as_float(q[j].z & 0xFFFF0000u),
+                                           __uint_as_float(q[j].w << 16), __uint_as_float(q[j].w & 0xFFFF0000u));
+                    } else {
+                        d[0] = make_float4(__uint_as_float(q[j].x), __uint_as_float(q[j].y),
+                                           __uint_as_float(q[j].z), __uint_as_float(q[j].w));
+                        d[1] = make_float4(__uint_as_float(q2[j].x), __uint_as_float(q2[j].y),
+                                           __uint_as_float(q2[j].z), __uint_as_float(q2[j].w));
+                    }
+                }
+            }
         }
         __syncthreads();
         bool ok = e1 <= e0 || mbar_wait(&wr_bar, 0);
@@ -515,15 +546,23 @@ __global__ void __launch_bounds__(kTlThreads, 1)
             abort_flag = 1;
             atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
         }
-        // one warp per router row, eight tokens at a time; lane l takes 8
-        // consecutive weights of each 256
-        for (int e = e0 + warp; ok && e < e1; e += kTlWarps) {
-            const uint16_t *wrow = sWr + (size_t)(e - e0) * H;
+        // router rows x K parts over the warps: warp w takes (row, K part) items
+        // w, w + 23, ...; lane l 8 consecutive weights of each 256; each item's
+        // partial dot products per token go to shared memory and are summed in
+        // K-part order
+        const int rows = e1 - e0, H256 = H / 256;
+        int kparts = 1;
+        while (kparts * 2 <= H256 && rows * kparts * 2 <= kTlWarps && H256 % (kparts * 2) == 0) kparts *= 2;
+        const int klen = H / kparts;
+        float *part = sX + (size_t)R.rt * H;  // [rows][kparts][rt]
+        for (int item = warp; ok && item < rows * kparts; item += kTlWarps) {
+            const int row = item / kparts, kp = item - row * kparts;
+            const uint16_t *wrow = sWr + (size_t)row * H;
             for (int tq = 0; tq < tn; tq += 8) {
                 float acc[8];
 #pragma unroll
                 for (int t = 0; t < 8; ++t) acc[t] = 0.f;
-                for (int k0 = lane * 8; k0 < H; k0 += 256) {
+                for (int k0 = kp * klen + lane * 8; k0 < (kp + 1) * klen; k0 += 256) {
                     const uint4 w = *reinterpret_cast<const uint4 *>(wrow + k0);
                     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
                     float wf[8];
@@ -538,39 +577,35 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                             const float *xr = sX + (size_t)(tq + t) * H + k0;
                             const float4 x0 = *reinterpret_cast<const float4 *>(xr);
                             const float4 x1 = *reinterpret_cast<const float4 *>(xr + 4);
-                            float s = acc[t];
-                            s = fmaf(wf[0], x0.x, s); s = fmaf(wf[1], x0.y, s);
-                            s = fmaf(wf[2], x0.z, s); s = fmaf(wf[3], x0.w, s);
-                            s = fmaf(wf[4], x1.x, s); s = fmaf(wf[5], x1.y, s);
-                            s = fmaf(wf[6], x1.z, s); s = fmaf(wf[7], x1.w, s);
-                            acc[t] = s;
+                            float s2 = acc[t];
+                            s2 = fmaf(wf[0], x0.x, s2); s2 = fmaf(wf[1], x0.y, s2);
+                            s2 = fmaf(wf[2], x0.z, s2); s2 = fmaf(wf[3], x0.w, s2);
+                            s2 = fmaf(wf[4], x1.x, s2); s2 = fmaf(wf[5], x1.y, s2);
+                            s2 = fmaf(wf[6], x1.z, s2); s2 = fmaf(wf[7], x1.w, s2);
+                            acc[t] = s2;
                         }
                     }
                 }
 #pragma unroll
                 for (int t = 0; t < 8; ++t) {
                     if (tq + t < tn) {
-                        float s = acc[t];
+                        float s2 = acc[t];
 #pragma unroll
-                        for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                        if (lane == 0) a.logits[(size_t)(t0 + tq + t) * E + e] = s;
+                        for (int o = 16; o >= 1; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+                        if (lane == 0) part[((size_t)row * kparts + kp) * R.rt + tq + t] = s2;
                     }
                 }
             }
         }
-        if (rb == 0) {
-            // each token's power-of-two scale: max |x| brought below 2^15 (fp16 keeps x exact)
-            for (int t = warp; t < tn; t += kTlWarps) {
-                unsigned mx = 0u;
-                for (int i = lane; i < H; i += 32) mx = max(mx, __float_as_uint(fabsf(sX[(size_t)t * H + i])));
-                mx = __reduce_max_sync(0xffffffffu, mx);
-                const int ex = (int)((mx >> 23) & 0xFFu) - 127;
-                const int sh = (ex >= 15 && ex < 128) ? ex - 14 : 0;
-                if (lane == 0) a.xscale[t0 + t] = __uint_as_float((uint32_t)(127 + sh) << 23);
-            }
+        __syncthreads();
+        for (int i = tid; ok && i < rows * tn; i += kTlThreads) {
+            const int row = i / tn, t = i - row * tn;
+            float l = 0.f;
+            for (int kp = 0; kp < kparts; ++kp) l += part[((size_t)row * kparts + kp) * R.rt + t];
+            a.logits[(size_t)(t0 + t) * E + e0 + row] = l;
         }
     }
-    // ---- grid barrier: every logit and token scale written ------------------------------
+    // ---- grid barrier: every logit written ------------------------------------------------
     __syncthreads();
     grid_event(a.stamps, 1);
     cta0_clock(a.stamps, 1);
@@ -594,7 +629,9 @@ __global__ void __launch_bounds__(kTlThreads, 1)
             float *row = reinterpret_cast<float *>(smem) + (size_t)warp * E;
             unsigned *cand = reinterpret_cast<unsigned *>(smem + (size_t)nsw * E * 4) + warp * 128;
             for (int t = warp; t < T; t += nsw) {
-                for (int e = lane; e < E; e += 32) row[e] = __ldcg(a.logits + (size_t)t * E + e);
+                // every load of the lane in flight before the stores (one L2 round trip)
+                if (E <= 512) stage_logits<16>(a.logits + (size_t)t * E, row, E, lane);
+                else stage_logits<32>(a.logits + (size_t)t * E, row, E, lane);
                 __syncwarp();
                 int my_e;
                 float my_g;
@@ -611,7 +648,6 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                 __syncwarp();
             }
         }
-        for (int t = tid; t < T; t += kTlThreads) p_xscale[t] = __ldcg(a.xscale + t);
         __syncthreads();
         cta0_clock(a.stamps, 3);
         // counts and 64-bit token masks per expert
@@ -683,47 +719,6 @@ __global__ void __launch_bounds__(kTlThreads, 1)
         }
         __syncthreads();
         cta0_clock(a.stamps, 4);
-        // this CTA's share of the fp16 slot rows of x, then one count per group touched
-        const int S = s_misc[1], ng = s_misc[0];
-        const int s0 = (int)((long long)S * c / G), s1 = (int)((long long)S * (c + 1) / G);
-        const int cpr = H / 8;
-        for (int i = tid; i < (s1 - s0) * cpr; i += kTlThreads) {
-            const int s = s0 + i / cpr, ch = i - (i / cpr) * cpr;
-            const int t = p_slot_tok[s];
-            const float down = 1.f / p_xscale[t];  // an exact power of two
-            float v[8];
-            if (a.x_dtype == MOE_DT_BF16) {
-                const uint4 q = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(a.x) +
-                                                                      (size_t)t * H) + ch);
-                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    v[2 * j] = __uint_as_float(w[j] << 16);
-                    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-                }
-            } else {
-                const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + (size_t)t * H) +
-                                  2 * ch;
-                const float4 x0 = __ldg(p), x1 = __ldg(p + 1);
-                v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
-                v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
-            }
-            uint4 o;
-            o.x = dq::pack_f16x2(v[0] * down, v[1] * down);
-            o.y = dq::pack_f16x2(v[2] * down, v[3] * down);
-            o.z = dq::pack_f16x2(v[4] * down, v[5] * down);
-            o.w = dq::pack_f16x2(v[6] * down, v[7] * down);
-            reinterpret_cast<uint4 *>(a.xg + (size_t)s * H)[ch] = o;
-        }
-        __syncthreads();
-        if (tid == 0 && s1 > s0) {
-            __threadfence();
-            // groups whose slot range meets [s0, s1): the slot ranges are ascending
-            for (int g = 0; g < ng; ++g) {
-                const int o = p_grp_off[g], n = p_grp_n[g];
-                if (o < s1 && o + n > s0) atomicAdd(a.ctr + C.grp_x + g, 1u);
-            }
-        }
     }
     __syncthreads();
     grid_event(a.stamps, 2);
@@ -744,24 +739,95 @@ __global__ void __launch_bounds__(kTlThreads, 1)
     uint8_t *raw = smem, *atile = smem + a.nr * a.raw_stride, *btile = atile + a.na * kTlAStage;
     int raw_issued = 0, b_issued = 0;
 
+    // ---- this CTA's share of the fp16 slot rows of x (slots [s0, s1)), by the
+    // epilogue and expanding warps while the producers and the MMA issuer start:
+    // the row's largest magnitude picks the power of two 2^s that keeps it
+    // below 2^15 (x stays exact in fp16), the row is written times 2^-s and 2^s
+    // kept per slot; then one count on the readiness counter of each group met
+    if (run && (warp < kTlEpiWarps || warp >= kTlDeqWarp0)) {
+        constexpr int kW = 32 * (kTlEpiWarps + kTlDeqWarps);  // 640 writing threads
+        const int wt = warp < kTlEpiWarps ? tid : tid - 32 * (kTlDeqWarp0 - kTlEpiWarps);
+        const int wwarp = wt >> 5;
+        const int S = s_misc[1];
+        const int s0 = (int)((long long)S * c / G), s1 = (int)((long long)S * (c + 1) / G);
+        const int cpr = H / 8;  // 8-value chunks per row (at most 4 per thread: H <= 16384)
+        for (int sl = s0; sl < s1; ++sl) {
+            const int t = p_slot_tok[sl];
+            float v[4][8];
+            unsigned mx = 0u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int ch = wt + kW * j;
+                if (ch < cpr) {
+                    if (a.x_dtype == MOE_DT_BF16) {
+                        const uint4 q4 = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(a.x) +
+                                                                               (size_t)t * H) + ch);
+                        const uint32_t w4[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            v[j][2 * i] = __uint_as_float(w4[i] << 16);
+                            v[j][2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+                        }
+                    } else {
+                        const float4 *pf = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) +
+                                                                            (size_t)t * H) + 2 * ch;
+                        const float4 x0 = __ldg(pf), x1 = __ldg(pf + 1);
+                        v[j][0] = x0.x; v[j][1] = x0.y; v[j][2] = x0.z; v[j][3] = x0.w;
+                        v[j][4] = x1.x; v[j][5] = x1.y; v[j][6] = x1.z; v[j][7] = x1.w;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) mx = max(mx, __float_as_uint(fabsf(v[j][i])));
+                }
+            }
+            mx = __reduce_max_sync(0xffffffffu, mx);
+            if ((wt & 31) == 0) s_tmp[wwarp] = (int)mx;
+            asm volatile("bar.sync 2, 640;" ::: "memory");
+#pragma unroll 1
+            for (int w2 = 0; w2 < kW / 32; ++w2) mx = max(mx, (unsigned)s_tmp[w2]);
+            asm volatile("bar.sync 2, 640;" ::: "memory");  // s_tmp is reused by the next slot
+            const int ex = (int)((mx >> 23) & 0xFFu) - 127;  // exponent of max |x| (inf / NaN: unscaled)
+            const int sh = (ex >= 15 && ex < 128) ? ex - 14 : 0;
+            const float down = __uint_as_float((uint32_t)(127 - sh) << 23);
+            if (wt == 0) a.slot_scale[sl] = __uint_as_float((uint32_t)(127 + sh) << 23);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int ch = wt + kW * j;
+                if (ch < cpr) {
+                    uint4 o;
+                    o.x = dq::pack_f16x2(v[j][0] * down, v[j][1] * down);
+                    o.y = dq::pack_f16x2(v[j][2] * down, v[j][3] * down);
+                    o.z = dq::pack_f16x2(v[j][4] * down, v[j][5] * down);
+                    o.w = dq::pack_f16x2(v[j][6] * down, v[j][7] * down);
+                    reinterpret_cast<uint4 *>(a.xg + (size_t)sl * H)[ch] = o;
+                }
+            }
+        }
+        asm volatile("bar.sync 2, 640;" ::: "memory");
+        if (wt == 0 && s1 > s0) {
+            __threadfence();
+            for (int g = 0; g < ng; ++g) {  // groups whose slot range meets [s0, s1)
+                const int o = p_grp_off[g], n = p_grp_n[g];
+                if (o < s1 && o + n > s0) atomicAdd(a.ctr + C.grp_x + g, 1u);
+            }
+        }
+    }
+
     if (run && warp == kTlRawWarp) {
         if (lane == 0) {
-            prefetch_tmap(&mGuQ);
-            prefetch_tmap(&mDnQ);
             Ring rr;
             for (int p = 0; p < 2 && !abort_flag; ++p)
                 for (int u = q.lo[p]; u < q.hi[p] && !abort_flag; ++u, rr.next(a.nr)) {
                     const Unit x = unit_at(q, p, u);
-                    if (rr.u > 0 && !mbar_wait(&re_bar[rr.s], (rr.u - 1) & 1)) {
+                    if (rr.u > 0 && !mbar_wait_idle(&re_bar[rr.s], (rr.u - 1) & 1)) {
                         abort_flag = 1;
                         break;
                     }
                     uint8_t *st = raw + rr.s * a.raw_stride;
                     const int ex = p_grp_e[x.g];
-                    if (p == 0)
-                        raw_load<FG>(st, &mGuQ, &mGuS, &mGuH, &rf_bar[rr.s], x.kc, x.b * 128, I + x.b * 128, ex);
-                    else
-                        raw_load<FD>(st, &mDnQ, &mDnS, &mDnH, &rf_bar[rr.s], x.kc, x.b * 256, x.b * 256 + 128, ex);
+                    if (p == 0)  // gate rows block b and up rows block I / 128 + b
+                        raw_load<FG>(st, a.tl_gu, a.tl_gu_stride, q.KC[0], &rf_bar[rr.s], x.kc, x.b, I / 128 + x.b, ex);
+                    else  // output rows blocks 2b and 2b + 1
+                        raw_load<FD>(st, a.tl_dn, a.tl_dn_stride, q.KC[1], &rf_bar[rr.s], x.kc, 2 * x.b, 2 * x.b + 1, ex);
                 }
             raw_issued = rr.u * a.nr + rr.s;
         }
@@ -797,7 +863,7 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                         ready_p = p;
                     }
                     for (int sl = 0; sl < 4; ++sl, rb_.next(a.nb)) {
-                        if (rb_.u > 0 && !mbar_wait(&be_bar[rb_.s], (rb_.u - 1) & 1)) {
+                        if (rb_.u > 0 && !mbar_wait_idle(&be_bar[rb_.s], (rb_.u - 1) & 1)) {
                             abort_flag = 1;
                             break;
                         }
@@ -843,6 +909,10 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                         mma_commit(&ae_bar[ra.s]);
                         mma_commit(&be_bar[rbm.s]);
                     }
+                    if (a.stamps && c == 0) {  // profiling: CTA 0's first units, MMAs issued
+                        const int ui = (p == 0 ? u - q.lo[0] : q.hi[0] - q.lo[0] + u - q.lo[1]);
+                        if (ui < 4) a.stamps[28 + ui] = clock64();
+                    }
                     if (x.last) {
                         mma_commit(&accf_bar[ab]);
                         ++seg;
@@ -861,17 +931,17 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                     ok = false;
                     break;
                 }
+                if (a.stamps && c == 0 && n == 0) {  // profiling: CTA 0's first units, raw stage landed
+                    const int ui = (p == 0 ? u - q.lo[0] : q.hi[0] - q.lo[0] + u - q.lo[1]);
+                    if (ui < 4) a.stamps[24 + ui] = clock64();
+                }
                 const uint8_t *st = raw + rr.s * a.raw_stride;
 #pragma unroll 1
                 for (int d = 0; d < 4; ++d, ra.next(a.na)) {
-                    if (ra.u > 0) {
-                        bool w = true;
-                        if (lane == 0) w = mbar_wait(&ae_bar[ra.s], (ra.u - 1) & 1);
-                        if (!__shfl_sync(0xffffffffu, w, 0)) {
-                            abort_flag = 1;
-                            ok = false;
-                            break;
-                        }
+                    if (ra.u > 0 && !__all_sync(0xffffffffu, mbar_wait(&ae_bar[ra.s], (ra.u - 1) & 1))) {
+                        abort_flag = 1;
+                        ok = false;
+                        break;
                     }
                     uint8_t *a_s = atile + ra.s * kTlAStage;
                     if (p == 0) expand<FG>(st, a_s, r, tile, bsel, d, a.tab_gu);
@@ -894,7 +964,7 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                 const Unit x = unit_at(q, p, u);
                 if (!x.last) continue;
                 const int ab = seg & 1;
-                const bool w_ok = mbar_wait(&accf_bar[ab], (seg >> 1) & 1);
+                const bool w_ok = mbar_wait_idle(&accf_bar[ab], (seg >> 1) & 1);
                 tc_fence_after_sync();
                 // one decision for all four warps (they share named barriers): each
                 // raises the vote before the barrier, all read it after; every later
@@ -949,6 +1019,9 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                 const int e = p_grp_e[x.g];
                 const float hts = (p == 0 ? FG : FD) == MOE_FMT_NVFP4 ? 0.5f * __ldg((p == 0 ? a.ts_gu : a.ts_dn) + e)
                                                                         : 1.f;
+                // the slot scales came with the x rows the B producer waited for: an
+                // acquire of the group's (full) readiness count orders their reads
+                if (p == 0) (void)ld_acq(a.ctr + C.grp_x + x.g);
                 for (int c0 = 0; c0 < n16; ++c0) {
                     float v0[16], v1[16];
                     if (whole) {
@@ -977,7 +1050,7 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                             const int jj = c0 * 16 + j;
                             if (jj < n) {
                                 const int slot = off + jj;
-                                const float sc = p_xscale[p_slot_tok[slot]] * hts;
+                                const float sc = __ldcg(a.slot_scale + slot) * hts;
                                 const float gv = v0[j] * sc, uv = v1[j] * sc;
                                 const float hv = gv / (1.f + expf(-gv)) * uv;
                                 range_ok = range_ok && fabsf(hv) <= 65504.f;
@@ -1087,8 +1160,7 @@ __global__ void __launch_bounds__(kTlThreads, 1)
     }
 }
 
-using TlKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                          const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const TailArgs);
+using TlKernel = void (*)(const CUtensorMap, const CUtensorMap, const TailArgs);
 
 template <int FG>
 TlKernel tl_pick_dn(int fd)
@@ -1194,8 +1266,12 @@ cudaError_t launch_tail(const TailCall &t, const TailLaunch &L, int grid, int pd
     a.tab_dn = t.tab_dn;
     a.ts_gu = t.gu->ts;
     a.ts_dn = t.dn->ts;
+    a.tl_gu = t.gu->tl;
+    a.tl_dn = t.dn->tl;
+    a.tl_gu_stride = t.gu->tl_stride;
+    a.tl_dn_stride = t.dn->tl_stride;
     a.logits = t.ws->logits;
-    a.xscale = t.ws->slot_scale;
+    a.slot_scale = t.ws->slot_scale;
     a.xg = reinterpret_cast<__half *>(t.ws->xg);
     a.h = reinterpret_cast<__half *>(t.ws->h);
     a.y = t.ws->y;
@@ -1232,8 +1308,7 @@ cudaError_t launch_tail(const TailCall &t, const TailLaunch &L, int grid, int pd
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const DecodeTcMaps &m = *t.maps;
-    return cudaLaunchKernelEx(&cfg, tl_pick(t.gu->fmt, t.dn->fmt), m.gu[0], m.gu[1], m.gu[2], m.dn[0], m.dn[1],
-                              m.dn[2], m.xg, m.h, a);
+    return cudaLaunchKernelEx(&cfg, tl_pick(t.gu->fmt, t.dn->fmt), m.xg, m.h, a);
 }
 
 }  // namespace moe
