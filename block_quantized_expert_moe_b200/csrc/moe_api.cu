@@ -859,7 +859,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     // grouped decode in separate launches, when the pack's weights are
     // fp16-representable
     bool use_tail = false;
-    if ((path == MOE_PATH_DECODE && T >= 2) || path == MOE_PATH_TAIL) {
+    if (path == MOE_PATH_TAIL) {
         const int xb = x_dtype == MOE_DT_BF16 ? 1 : 0;
         int &ok = pm->tail_ok[T][xb];
         if (ok < 0) {

@@ -102,12 +102,12 @@ typedef enum { MOE_DT_F32 = 1, MOE_DT_BF16 = 2 } moe_dtype;
  * to bf16 for bf16 MMA; hidden and inter multiples of 256, bf16 activations,
  * top_k <= 32; its buffers are sized at pack time when max_tokens > 64), else
  * GROUPED.  DECODE: one token runs the single-token streaming kernel; 2 to 64
- * tokens run the device-planned tail in one launch: routing, the plan, the
- * tensor-core grouped gate/up and down (weights expanded to fp16, fp32
- * accumulation; hidden and inter multiples of 256, top_k <= 16 and every weight
- * an fp16 normal number or zero, checked at pack time) and the combine; where
- * that launch does not fit, the same tensor-core work in separate launches,
- * else the CUDA-core grouped kernels.  DENSE is the dense-batched comparison variant (pack created with
+ * tokens run the tensor-core grouped decode as separate launches (route and
+ * plan, x gather, gate/up, down, combine; weights expanded to fp16, fp32
+ * accumulation; hidden and inter multiples of 256 and every weight an fp16
+ * normal number or zero, checked at pack time), else the CUDA-core grouped
+ * kernels.  TAIL runs the same layer as one launch (the device-planned tail);
+ * packs holding an expert window always take it.  DENSE is the dense-batched comparison variant (pack created with
  * MOE_PACK_DENSE, n_tokens <= 64): every active expert multiplies the whole
  * batch, with a zero gate for the tokens not routed to it. */
 typedef enum {
@@ -119,8 +119,9 @@ typedef enum {
     MOE_PATH_DECODE_STAGED = 5, /* 2-64 tokens: the tensor-core grouped decode as separate launches (route and
                                    plan, x gather, gate/up, down, combine); MOE_ERR_UNSUPPORTED where it does
                                    not apply */
-    MOE_PATH_TAIL = 6,     /* 1-64 tokens: the one-launch tail (what DECODE runs for 2-64 tokens when it fits);
-                              MOE_ERR_UNSUPPORTED where it does not apply */
+    MOE_PATH_TAIL = 6,     /* 1-64 tokens: the whole layer in one launch (routing, plan, tensor-core gate/up
+                              and down over every SM, combine; hidden and inter multiples of 256, top_k <= 16,
+                              fp16-representable weights); MOE_ERR_UNSUPPORTED where it does not apply */
     MOE_PATH_PREFILL_BF16 = 7 /* the prefill with every format's weights dequantised to bf16 in shared memory
                                  and bf16 MMA, NVFP4 included (its weights are exact in bf16: x is not rounded
                                  to NVFP4, h is rounded to bf16); same conditions as PREFILL */
