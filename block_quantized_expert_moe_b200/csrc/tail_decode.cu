@@ -26,9 +26,11 @@
 //             count on the group's h counter
 //   down      the same over {group, 256 output rows, 256 of K}, each unit's B
 //             operand the group's h rows once its counter is full; y per slot
-//             (fp32); the last tile of each 256-row output block makes its CTA
-//             combine those rows: out[t] = sum_j gate_tj y[slot(t, j)] (+ the
-//             shared expert's y), in the layer's order
+//             (fp32) and a count on the 256-row block's counter
+//   combine   CTA c owns output rows [H c / G, H (c + 1) / G) of every token:
+//             once every group's y rows of their blocks are in,
+//             out[t] = sum_j gate_tj y[slot(t, j)] (+ the shared expert's y),
+//             in the layer's order
 //
 // The tensor-core tile is M = 128 weight rows, N = the group's tokens (padded
 // to 16), K = 64 per shared-memory stage, fp16 x fp16 -> fp32 in tensor memory:
@@ -37,10 +39,13 @@
 // exact fp16 after the token's power-of-two scale, h is rounded to fp16.
 //
 //   warps 0-3   epilogue: tensor-memory lanes 32w .. 32w + 31 (tile rows)
-//   warp 4      B producer (TMA, 16-row boxes of the group's slot rows)
-//   warp 5      MMA issuer (one elected thread)
-//   warp 6      raw producer (TMA boxes of codes, scales, fifth bits)
-//   warps 7-22  expanders: each thread one 32-block of one row per slice
+//   warp 4      MMA issuer (one elected thread)
+//   warp 5      raw producer (two bulk copies a unit from the tiled planes)
+//   warps 6-13  expanders: each thread both 32-blocks of one row per slice,
+//               and up to two 16-byte chunks of the slice's B rows (the
+//               group's slot rows of x or h, read from L2 once the group's
+//               readiness counter is full), stored beside the A tiles of the
+//               same operand stage: the MMA issuer waits on one barrier a slice
 //
 // Every wait is bounded (~1 s): a wait that runs out records MOE_ERR_TIMEOUT,
 // raises the CTA's abort flag and the CTA drains what it issued before it
@@ -56,7 +61,6 @@
 #include "dequant.cuh"
 #include "moe_internal.cuh"
 #include "tc_common.cuh"
-#include "tma_maps.cuh"
 
 namespace moe {
 
@@ -64,14 +68,15 @@ namespace {
 
 using namespace tc;
 
-constexpr int kTlEpiWarps = 4, kTlBWarp = 4, kTlMmaWarp = 5, kTlRawWarp = 6, kTlDeqWarp0 = 7, kTlDeqWarps = 16;
-constexpr int kTlWarps = kTlDeqWarp0 + kTlDeqWarps;  // 23
+constexpr int kTlEpiWarps = 4, kTlMmaWarp = 4, kTlRawWarp = 5, kTlDeqWarp0 = 6, kTlDeqWarps = 8;
+constexpr int kTlWarps = kTlDeqWarp0 + kTlDeqWarps;  // 14
 constexpr int kTlThreads = 32 * kTlWarps;
-constexpr int kTlMaxRaw = 4, kTlMaxA = 4, kTlMaxB = 8;
+constexpr int kTlDeqThreads = 32 * kTlDeqWarps;      // 256: one per row of the unit's two tiles
+constexpr int kTlWriters = 32 * (kTlEpiWarps + kTlDeqWarps);  // the warps that write the x slot rows
+constexpr int kTlMaxRaw = 4, kTlMaxA = 4;
 constexpr int kTlA = 128 * 128;           // one 128-row tile x 64 fp16 of K
-constexpr int kTlAStage = 2 * kTlA;       // a unit's two tiles
+constexpr int kTlAStage = 2 * kTlA;       // a unit's two tiles (the slice's B rows follow in the stage)
 constexpr int kTlTmemCols = 256;          // two accumulator buffers of 128 columns
-constexpr int kTlMaxWon = 64;             // 256-row output blocks (hidden <= 16384)
 constexpr long long kTlSpin = 1ll << 31;  // clocks
 
 __host__ __device__ inline int tl_cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -123,7 +128,7 @@ __host__ __device__ inline TlCtr tl_ctr(int E, int H, int I)
 
 // The launch's plan in shared memory (after the rings), the same in every CTA.
 struct TlPlanLayout {
-    int xscale, sel_e, sel_g, slot_of, grp_e, grp_n, grp_off, slot_tok, won, total;
+    int xscale, sel_e, sel_g, slot_of, grp_e, grp_n, grp_off, slot_tok, total;
 };
 __host__ __device__ inline TlPlanLayout tl_plan_layout(int T, int k, int E)
 {
@@ -138,7 +143,6 @@ __host__ __device__ inline TlPlanLayout tl_plan_layout(int T, int k, int E)
     L.grp_n = o;    o = tl_al16(o + 2 * ng);
     L.grp_off = o;  o = tl_al16(o + 4 * ng);
     L.slot_tok = o; o = tl_al16(o + 2 * slots);
-    L.won = o;      o = tl_al16(o + 4 * (kTlMaxWon + 1));
     L.total = o;
     return L;
 }
@@ -191,8 +195,8 @@ struct TailArgs {
     int32_t *idx_out;            // routing readback, written by CTA 0
     float *gate_out;
     int32_t *cnt_out;
-    int nr, na, nb;              // ring depths
-    int raw_stride, bslot, n16max;
+    int nr, na;                  // ring depths
+    int raw_stride, bslot, n16max;  // B slots (na + 2 of them, after the A stages): n16max rows of 128 bytes
     int rings;                   // bytes of the rings (the plan follows)
     long long *stamps;           // profiling only: grid events {2^62 - first, last} at words 10..19
 };
@@ -220,6 +224,15 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
                  "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
+
+// 16-byte asynchronous copy global -> shared (L2 only), in the thread's current group.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void grid_event(long long *st, int ev)
 {
@@ -289,14 +302,19 @@ __device__ __forceinline__ int owners(int u0, int n, int U, int G)
     return cnt;
 }
 
-// Exclusive scan of n ints in shared memory v (n <= 2 * blockDim), in place;
+// Exclusive scan of n ints in shared memory v (n <= 4 * blockDim), in place;
 // returns the total.  tmp: 32 ints of scratch.
 __device__ int block_scan(int *v, int n, int *tmp)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    const int i0 = 2 * tid;
-    const int a = i0 < n ? v[i0] : 0, b = i0 + 1 < n ? v[i0 + 1] : 0;
-    int s = a + b, incl = s;
+    const int i0 = 4 * tid;
+    int e[4], s = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        e[j] = i0 + j < n ? v[i0 + j] : 0;
+        s += e[j];
+    }
+    int incl = s;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -315,9 +333,12 @@ __device__ int block_scan(int *v, int n, int *tmp)
         if (lane == 31) tmp[31] = wi;
     }
     __syncthreads();
-    const int base = tmp[warp] + incl - s;
-    if (i0 < n) v[i0] = base;
-    if (i0 + 1 < n) v[i0 + 1] = base + a;
+    int base = tmp[warp] + incl - s;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (i0 + j < n) v[i0 + j] = base;
+        base += e[j];
+    }
     const int total = tmp[31];
     __syncthreads();
     return total;
@@ -369,41 +390,183 @@ __device__ __forceinline__ void raw_load(uint8_t *st, const uint8_t *tl, int64_t
     bulk_g2s(st + RL::kTile, base + ((int64_t)rb1 * KC + kc) * RL::kTile, (uint32_t)RL::kTile, bar);
 }
 
-// Thread n of the expanders: block bsel of slice d of row r of tile `tile`.
+// The raw bytes of one slice of one row for one expanding thread: both 32-blocks
+// (codes, scale word, Q5_1 fifth bits), loaded from the raw stage a slice
+// ahead of their expansion.
 template <int FMT>
-__device__ __forceinline__ void expand(const uint8_t *st, uint8_t *a_stage, int r, int tile, int bsel, int d,
-                                       const CodeTable &tab)
+struct SliceRaw {
+    uint32_t q[2][FMT == MOE_FMT_Q8_0 ? 8 : 4];
+    uint32_t s[2], h[2];
+};
+
+template <int FMT>
+__device__ __forceinline__ void load_slice(const uint8_t *st, int r, int tile, int d, SliceRaw<FMT> &R)
 {
     using RL = TlRaw<FMT>;
     const uint8_t *cq = st + RL::codes(tile), *cs = st + RL::scales(tile), *ch = st + RL::qh(tile);
-    const int blk = 2 * d + bsel;
-    uint32_t qw[8];
-    if constexpr (FMT == MOE_FMT_Q8_0) {
-        const uint4 x0 = *reinterpret_cast<const uint4 *>(raw_code(cq, blk >> 2, r, (2 * blk) & 7));
-        const uint4 x1 = *reinterpret_cast<const uint4 *>(raw_code(cq, blk >> 2, r, ((2 * blk) & 7) + 1));
-        qw[0] = x0.x; qw[1] = x0.y; qw[2] = x0.z; qw[3] = x0.w;
-        qw[4] = x1.x; qw[5] = x1.y; qw[6] = x1.z; qw[7] = x1.w;
-    } else {
-        const uint4 x0 = *reinterpret_cast<const uint4 *>(raw_code(cq, 0, r, blk));
-        qw[0] = x0.x; qw[1] = x0.y; qw[2] = x0.z; qw[3] = x0.w;
+#pragma unroll
+    for (int bsel = 0; bsel < 2; ++bsel) {
+        const int blk = 2 * d + bsel;
+        if constexpr (FMT == MOE_FMT_Q8_0) {
+            const uint4 x0 = *reinterpret_cast<const uint4 *>(raw_code(cq, blk >> 2, r, (2 * blk) & 7));
+            const uint4 x1 = *reinterpret_cast<const uint4 *>(raw_code(cq, blk >> 2, r, ((2 * blk) & 7) + 1));
+            R.q[bsel][0] = x0.x; R.q[bsel][1] = x0.y; R.q[bsel][2] = x0.z; R.q[bsel][3] = x0.w;
+            R.q[bsel][4] = x1.x; R.q[bsel][5] = x1.y; R.q[bsel][6] = x1.z; R.q[bsel][7] = x1.w;
+        } else {
+            const uint4 x0 = *reinterpret_cast<const uint4 *>(raw_code(cq, 0, r, blk));
+            R.q[bsel][0] = x0.x; R.q[bsel][1] = x0.y; R.q[bsel][2] = x0.z; R.q[bsel][3] = x0.w;
+        }
+        if constexpr (FMT == MOE_FMT_Q5_1) {
+            const int gsw = (r >> 2) & 1;  // 32-byte swizzle: 16-byte chunk ^ ((r / 4) % 2)
+            const int o = r * 32 + ((((blk * 4) >> 4) ^ gsw) << 4) + ((blk * 4) & 15);
+            R.s[bsel] = *reinterpret_cast<const uint32_t *>(cs + o);
+            R.h[bsel] = *reinterpret_cast<const uint32_t *>(ch + o);
+        } else {
+            R.s[bsel] = *reinterpret_cast<const uint16_t *>(cs + r * 16 + blk * 2);
+            R.h[bsel] = 0;
+        }
     }
-    uint32_t sc, hb = 0;
-    if constexpr (FMT == MOE_FMT_Q5_1) {
-        const int gsw = (r >> 2) & 1;  // 32-byte swizzle: 16-byte chunk ^ ((r / 4) % 2)
-        const int o = r * 32 + ((((blk * 4) >> 4) ^ gsw) << 4) + ((blk * 4) & 15);
-        sc = *reinterpret_cast<const uint32_t *>(cs + o);
-        hb = *reinterpret_cast<const uint32_t *>(ch + o);
-    } else {
-        sc = *reinterpret_cast<const uint16_t *>(cs + r * 16 + blk * 2);
-    }
-    uint4 o4[4];
-    dq::blk_f16<FMT>(qw, sc, hb, tab, o4);
+}
+
+// fp16 of both blocks into row r of tile `tile` of the operand stage (128-byte
+// swizzle, K-major): 16-byte chunk c of the slice's 64 values at c ^ (r % 8).
+template <int FMT>
+__device__ __forceinline__ void store_slice(const SliceRaw<FMT> &R, uint8_t *a_stage, int r, int tile,
+                                            const CodeTable &tab)
+{
     uint8_t *a_row = a_stage + tile * kTlA + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-        const int c = 4 * bsel + cc;
-        *reinterpret_cast<uint4 *>(a_row + ((c ^ (r & 7)) << 4)) = o4[cc];
+    for (int bsel = 0; bsel < 2; ++bsel) {
+        uint4 o4[4];
+        dq::blk_f16<FMT>(R.q[bsel], R.s[bsel], R.h[bsel], tab, o4);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            const int c = 4 * bsel + cc;
+            *reinterpret_cast<uint4 *>(a_row + ((c ^ (r & 7)) << 4)) = o4[cc];
+        }
     }
+}
+
+// The expanding warps' walk over their rings, kept across the two phases.
+struct ExpState {
+    Ring ra, rr;     // operand stages, raw stages
+    int bs = 0;      // B slot of the current slice (slices in order, na + 2 slots)
+    bool pre = false;  // the current slice's B was issued during the previous slice
+    int ready_g = -1;
+};
+
+// Everything the expanding warps read of the kernel's state.
+struct ExpCtx {
+    const TailArgs *a;
+    const Geo *q;
+    const TlCtr *C;
+    const int16_t *grp_n;
+    const int *grp_off;
+    const uint8_t *raw;
+    uint8_t *atile, *bring;
+    uint64_t *rf, *re, *fa, *ae;
+    volatile int *abort_flag;
+    int G, c, n, lane, slots;
+};
+
+// One phase (0 gate/up, FMT = the gate/up format; 1 down) of the expanding
+// warps; false when a wait ran out or the CTA aborted.  Thread n (0 .. 255)
+// expands row n % 128 of tile n / 128, and copies B chunks n and n + 256 of
+// each slice: B row j (slot off + j of the group) holds K values kc * 256 +
+// 64 d .. + 63 of x (gate/up) or h (down), 8 chunks of 16 bytes, chunk
+// 8 j + cc at the 128-byte swizzled place of row j in its B slot.  A slice's B
+// is issued one slice ahead, before the wait on the operand stage, when the
+// MMAs up to slice - 1 - na are known complete: na + 2 slots keep it clear of
+// any slice still read.
+template <int FMT>
+__device__ bool expand_phase(const ExpCtx &x, int p, ExpState &es, const CodeTable &tab)
+{
+    const TailArgs &a = *x.a;
+    const Geo &q = *x.q;
+    const int n = x.n, r = n & 127, tile = n >> 7, nbs = a.na + 2;
+    const int bld = p == 0 ? a.H : a.I;
+    const __half *bbase = p == 0 ? a.xg : a.h;
+    // this thread's B chunks: destination in a slot, source from a row's start
+    int bdst[2], bsrc[2], bch[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int ch = n + kTlDeqThreads * i, j = ch >> 3, cc = ch & 7;
+        bch[i] = ch;
+        bdst[i] = (j >> 3) * 1024 + (j & 7) * 128 + ((cc ^ (j & 7)) << 4);
+        bsrc[i] = j * bld + cc * 8;
+    }
+    auto issue_b = [&](const __half *src, int nch, int slot) {
+        uint8_t *b_s = x.bring + slot * a.bslot;
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+            if (bch[i] < nch) cp_async16(b_s + bdst[i], src + bsrc[i]);
+    };
+    for (int u = q.lo[p]; u < q.hi[p]; ++u, es.rr.next(a.nr)) {
+        if (*x.abort_flag) return false;
+        const Unit un = unit_at(q, p, u);
+        const int gn = x.grp_n[un.g], goff = x.grp_off[un.g], nch = gn * 8;
+        if (un.g != es.ready_g) {
+            // the group's B rows: gate/up, its x slot rows written by the CTAs
+            // that own them; down, all of its h tiles finished.  Lane 0 waits,
+            // then every lane takes its own acquire of the (full) count
+            const unsigned *cp = a.ctr + (p == 0 ? x.C->grp_x : x.C->grp_h) + un.g;
+            bool w_ok = true;
+            if (x.lane == 0)
+                w_ok = wait_count(cp, p == 0 ? (unsigned)owners(goff, gn, x.slots, x.G) : (unsigned)q.NB[0]);
+            w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+            if (!w_ok) {
+                if (x.lane == 0) atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
+                *x.abort_flag = 1;
+                return false;
+            }
+            (void)ld_acq(cp);
+            es.ready_g = un.g;
+        }
+        const __half *bsrc_u = bbase + (size_t)goff * bld + un.kc * 256;
+        const __half *bsrc_n = nullptr;  // the next unit's B, when its rows are the same group's
+        if (u + 1 < q.hi[p]) {
+            const Unit nx = unit_at(q, p, u + 1);
+            if (nx.g == un.g) bsrc_n = bbase + (size_t)goff * bld + nx.kc * 256;
+        }
+        if (!mbar_wait(&x.rf[es.rr.s], es.rr.u & 1)) {
+            *x.abort_flag = 1;
+            return false;
+        }
+        if (a.stamps && x.c == 0 && n == 0) {  // profiling: CTA 0's first units, raw stage landed
+            const int ui = (p == 0 ? u - q.lo[0] : q.hi[0] - q.lo[0] + u - q.lo[1]);
+            if (ui < 4) a.stamps[24 + ui] = clock64();
+        }
+        const uint8_t *st = x.raw + es.rr.s * a.raw_stride;
+        SliceRaw<FMT> R;
+        load_slice<FMT>(st, r, tile, 0, R);
+#pragma unroll 1
+        for (int d = 0; d < 4; ++d, es.ra.next(a.na)) {
+            const int bn = es.bs + 1 == nbs ? 0 : es.bs + 1;
+            if (!es.pre) {
+                issue_b(bsrc_u + d * 64, nch, es.bs);
+                cp_async_commit();
+            }
+            es.pre = d < 3 || bsrc_n != nullptr;
+            if (es.pre) issue_b(d < 3 ? bsrc_u + (d + 1) * 64 : bsrc_n, nch, bn);
+            cp_async_commit();
+            SliceRaw<FMT> Rn;
+            if (d < 3) load_slice<FMT>(st, r, tile, d + 1, Rn);
+            if (es.ra.u > 0 && !__all_sync(0xffffffffu, mbar_wait(&x.ae[es.ra.s], (es.ra.u - 1) & 1))) {
+                *x.abort_flag = 1;
+                return false;
+            }
+            store_slice<FMT>(R, x.atile + es.ra.s * kTlAStage, r, tile, tab);
+            cp_async_wait_prev();  // this slice's B has landed (the next one may be in flight)
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (x.lane == 0) mbar_arrive(&x.fa[es.ra.s]);
+            if (d < 3) R = Rn;
+            es.bs = bn;
+        }
+        __syncwarp();
+        if (x.lane == 0) mbar_arrive(&x.re[es.rr.s]);
+    }
+    return true;
 }
 
 __host__ __device__ constexpr uint32_t tl_idesc(int N)
@@ -414,15 +577,15 @@ __host__ __device__ constexpr uint32_t tl_idesc(int N)
 
 template <int FG, int FD>
 __global__ void __launch_bounds__(kTlThreads, 1)
-    tail_kernel(const __grid_constant__ CUtensorMap mXg, const __grid_constant__ CUtensorMap mH, const TailArgs a)
+    tail_kernel(const __grid_constant__ TailArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t rf_bar[kTlMaxRaw], re_bar[kTlMaxRaw], fa_bar[kTlMaxA], ae_bar[kTlMaxA],
-        fb_bar[kTlMaxB], be_bar[kTlMaxB], accf_bar[2], acce_bar[2], dr_bar, wr_bar;
+        accf_bar[2], acce_bar[2], dr_bar, wr_bar;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
     __shared__ volatile int s_epi_abort;  // the four epilogue warps leave together
-    __shared__ int s_misc[8];  // [0] groups, [1] slots, [2] won row blocks, [3] epilogue: last arrival
+    __shared__ int s_misc[8];  // [0] groups, [1] slots, [3] epilogue: last arrival
     __shared__ int s_tmp[32];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -438,7 +601,6 @@ __global__ void __launch_bounds__(kTlThreads, 1)
     int16_t *p_grp_n = reinterpret_cast<int16_t *>(plan + PL.grp_n);
     int *p_grp_off = reinterpret_cast<int *>(plan + PL.grp_off);
     int16_t *p_slot_tok = reinterpret_cast<int16_t *>(plan + PL.slot_tok);
-    int *p_won = reinterpret_cast<int *>(plan + PL.won);
     const int xbytes = a.x_dtype == MOE_DT_BF16 ? 2 : 4;
     const TlRoute R = tl_route(T, E, G, xbytes);
     const int tb = c % R.ntb, rb = c / R.ntb;
@@ -457,10 +619,6 @@ __global__ void __launch_bounds__(kTlThreads, 1)
         for (int s = 0; s < a.na; ++s) {
             mbar_init(&fa_bar[s], kTlDeqWarps);
             mbar_init(&ae_bar[s], 1);
-        }
-        for (int s = 0; s < a.nb; ++s) {
-            mbar_init(&fb_bar[s], 1);
-            mbar_init(&be_bar[s], 1);
         }
         for (int s = 0; s < a.nr; ++s) {
             mbar_init(&rf_bar[s], 1);
@@ -736,73 +894,70 @@ __global__ void __launch_bounds__(kTlThreads, 1)
         q.lo[p] = range_lo(q.U[p], c, G);
         q.hi[p] = range_lo(q.U[p], c + 1, G);
     }
-    uint8_t *raw = smem, *atile = smem + a.nr * a.raw_stride, *btile = atile + a.na * kTlAStage;
-    int raw_issued = 0, b_issued = 0;
+    uint8_t *raw = smem, *atile = smem + a.nr * a.raw_stride;
+    int raw_issued = 0;
 
     // ---- this CTA's share of the fp16 slot rows of x (slots [s0, s1)), by the
-    // epilogue and expanding warps while the producers and the MMA issuer start:
-    // the row's largest magnitude picks the power of two 2^s that keeps it
-    // below 2^15 (x stays exact in fp16), the row is written times 2^-s and 2^s
-    // kept per slot; then one count on the readiness counter of each group met
+    // epilogue and expanding warps while the raw producer and the MMA issuer
+    // start: the row's largest magnitude picks the power of two 2^s that keeps
+    // it below 2^15 (x stays exact in fp16), the row is written times 2^-s and
+    // 2^s kept per slot; then one count on the readiness counter of each group
+    // met
     if (run && (warp < kTlEpiWarps || warp >= kTlDeqWarp0)) {
-        constexpr int kW = 32 * (kTlEpiWarps + kTlDeqWarps);  // 640 writing threads
         const int wt = warp < kTlEpiWarps ? tid : tid - 32 * (kTlDeqWarp0 - kTlEpiWarps);
         const int wwarp = wt >> 5;
         const int S = s_misc[1];
         const int s0 = (int)((long long)S * c / G), s1 = (int)((long long)S * (c + 1) / G);
-        const int cpr = H / 8;  // 8-value chunks per row (at most 4 per thread: H <= 16384)
+        const int cpr = H / 8;  // 8-value chunks per row
+        auto load8 = [&](int t, int ch, float *v) {
+            if (a.x_dtype == MOE_DT_BF16) {
+                const uint4 q4 =
+                    __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(a.x) + (size_t)t * H) + ch);
+                const uint32_t w4[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    v[2 * i] = __uint_as_float(w4[i] << 16);
+                    v[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+                }
+            } else {
+                const float4 *pf = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + (size_t)t * H) +
+                                   2 * ch;
+                const float4 x0 = __ldg(pf), x1 = __ldg(pf + 1);
+                v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+                v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+            }
+        };
         for (int sl = s0; sl < s1; ++sl) {
             const int t = p_slot_tok[sl];
-            float v[4][8];
             unsigned mx = 0u;
+            for (int ch = wt; ch < cpr; ch += kTlWriters) {
+                float v[8];
+                load8(t, ch, v);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int ch = wt + kW * j;
-                if (ch < cpr) {
-                    if (a.x_dtype == MOE_DT_BF16) {
-                        const uint4 q4 = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(a.x) +
-                                                                               (size_t)t * H) + ch);
-                        const uint32_t w4[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            v[j][2 * i] = __uint_as_float(w4[i] << 16);
-                            v[j][2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
-                        }
-                    } else {
-                        const float4 *pf = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) +
-                                                                            (size_t)t * H) + 2 * ch;
-                        const float4 x0 = __ldg(pf), x1 = __ldg(pf + 1);
-                        v[j][0] = x0.x; v[j][1] = x0.y; v[j][2] = x0.z; v[j][3] = x0.w;
-                        v[j][4] = x1.x; v[j][5] = x1.y; v[j][6] = x1.z; v[j][7] = x1.w;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) mx = max(mx, __float_as_uint(fabsf(v[j][i])));
-                }
+                for (int i = 0; i < 8; ++i) mx = max(mx, __float_as_uint(fabsf(v[i])));
             }
             mx = __reduce_max_sync(0xffffffffu, mx);
             if ((wt & 31) == 0) s_tmp[wwarp] = (int)mx;
-            asm volatile("bar.sync 2, 640;" ::: "memory");
+            asm volatile("bar.sync 2, %0;" ::"n"(kTlWriters) : "memory");
 #pragma unroll 1
-            for (int w2 = 0; w2 < kW / 32; ++w2) mx = max(mx, (unsigned)s_tmp[w2]);
-            asm volatile("bar.sync 2, 640;" ::: "memory");  // s_tmp is reused by the next slot
+            for (int w2 = 0; w2 < kTlWriters / 32; ++w2) mx = max(mx, (unsigned)s_tmp[w2]);
+            asm volatile("bar.sync 2, %0;" ::"n"(kTlWriters) : "memory");  // s_tmp is reused by the next slot
             const int ex = (int)((mx >> 23) & 0xFFu) - 127;  // exponent of max |x| (inf / NaN: unscaled)
             const int sh = (ex >= 15 && ex < 128) ? ex - 14 : 0;
             const float down = __uint_as_float((uint32_t)(127 - sh) << 23);
             if (wt == 0) a.slot_scale[sl] = __uint_as_float((uint32_t)(127 + sh) << 23);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int ch = wt + kW * j;
-                if (ch < cpr) {
-                    uint4 o;
-                    o.x = dq::pack_f16x2(v[j][0] * down, v[j][1] * down);
-                    o.y = dq::pack_f16x2(v[j][2] * down, v[j][3] * down);
-                    o.z = dq::pack_f16x2(v[j][4] * down, v[j][5] * down);
-                    o.w = dq::pack_f16x2(v[j][6] * down, v[j][7] * down);
-                    reinterpret_cast<uint4 *>(a.xg + (size_t)sl * H)[ch] = o;
-                }
+            for (int ch = wt; ch < cpr; ch += kTlWriters) {  // second pass: the row again, from L1 / L2
+                float v[8];
+                load8(t, ch, v);
+                uint4 o;
+                o.x = dq::pack_f16x2(v[0] * down, v[1] * down);
+                o.y = dq::pack_f16x2(v[2] * down, v[3] * down);
+                o.z = dq::pack_f16x2(v[4] * down, v[5] * down);
+                o.w = dq::pack_f16x2(v[6] * down, v[7] * down);
+                reinterpret_cast<uint4 *>(a.xg + (size_t)sl * H)[ch] = o;
             }
         }
-        asm volatile("bar.sync 2, 640;" ::: "memory");
+        asm volatile("bar.sync 2, %0;" ::"n"(kTlWriters) : "memory");
         if (wt == 0 && s1 > s0) {
             __threadfence();
             for (int g = 0; g < ng; ++g) {  // groups whose slot range meets [s0, s1)
@@ -831,55 +986,11 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                 }
             raw_issued = rr.u * a.nr + rr.s;
         }
-    } else if (run && warp == kTlBWarp) {
-        if (lane == 0) {
-            prefetch_tmap(&mXg);
-            prefetch_tmap(&mH);
-            Ring rb_;
-            int ready_g = -1, ready_p = -1;
-            for (int p = 0; p < 2 && !abort_flag; ++p)
-                for (int u = q.lo[p]; u < q.hi[p] && !abort_flag; ++u) {
-                    const Unit x = unit_at(q, p, u);
-                    const int n = p_grp_n[x.g], off = p_grp_off[x.g], n16 = (n + 15) >> 4;
-                    if (x.g != ready_g || p != ready_p) {
-                        // gate/up: the group's x slot rows written by their CTAs; down: all
-                        // of the group's h tiles finished
-                        unsigned target;
-                        const unsigned *cp;
-                        if (p == 0) {
-                            target = (unsigned)owners(off, n, s_misc[1], G);
-                            cp = a.ctr + C.grp_x + x.g;
-                        } else {
-                            target = (unsigned)q.NB[0];
-                            cp = a.ctr + C.grp_h + x.g;
-                        }
-                        if (!wait_count(cp, target)) {
-                            abort_flag = 1;
-                            atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
-                            break;
-                        }
-                        asm volatile("fence.proxy.async.global;" ::: "memory");
-                        ready_g = x.g;
-                        ready_p = p;
-                    }
-                    for (int sl = 0; sl < 4; ++sl, rb_.next(a.nb)) {
-                        if (rb_.u > 0 && !mbar_wait_idle(&be_bar[rb_.s], (rb_.u - 1) & 1)) {
-                            abort_flag = 1;
-                            break;
-                        }
-                        uint8_t *b_s = btile + rb_.s * a.bslot;
-                        mbar_arrive_expect_tx(&fb_bar[rb_.s], (uint32_t)n16 * 2048u);
-                        for (int jj = 0; jj < n16; ++jj)
-                            tma_load_2d(b_s + jj * 2048, p == 0 ? &mXg : &mH, &fb_bar[rb_.s], x.kc * 256 + sl * 64,
-                                        off + 16 * jj);
-                    }
-                }
-            b_issued = rb_.u * a.nb + rb_.s;
-        }
     } else if (run && warp == kTlMmaWarp) {
         if (lane == 0) {
-            Ring ra, rbm;
-            int seg = 0;
+            Ring ra;
+            int seg = 0, gs = 0;
+            const uint8_t *bring = atile + a.na * kTlAStage;
             for (int p = 0; p < 2 && !abort_flag; ++p)
                 for (int u = q.lo[p]; u < q.hi[p] && !abort_flag; ++u) {
                     const Unit x = unit_at(q, p, u);
@@ -890,14 +1001,14 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                     }
                     tc_fence_after_sync();
                     const uint32_t idesc = tl_idesc((p_grp_n[x.g] + 15) & ~15);
-                    for (int sl = 0; sl < 4; ++sl, ra.next(a.na), rbm.next(a.nb)) {
-                        if (!mbar_wait(&fa_bar[ra.s], ra.u & 1) || !mbar_wait(&fb_bar[rbm.s], rbm.u & 1)) {
+                    for (int sl = 0; sl < 4; ++sl, ra.next(a.na), ++gs) {
+                        if (!mbar_wait(&fa_bar[ra.s], ra.u & 1)) {
                             abort_flag = 1;
                             break;
                         }
                         tc_fence_after_sync();
                         const uint8_t *a_s = atile + ra.s * kTlAStage;
-                        const uint64_t bd = desc_kmajor_sw128(btile + rbm.s * a.bslot);
+                        const uint64_t bd = desc_kmajor_sw128(bring + (gs % (a.na + 2)) * a.bslot);
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const uint64_t ad = desc_kmajor_sw128(a_s + hh * kTlA);
@@ -907,7 +1018,6 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                                         !(x.first && sl == 0 && kk == 0));
                         }
                         mma_commit(&ae_bar[ra.s]);
-                        mma_commit(&be_bar[rbm.s]);
                     }
                     if (a.stamps && c == 0) {  // profiling: CTA 0's first units, MMAs issued
                         const int ui = (p == 0 ? u - q.lo[0] : q.hi[0] - q.lo[0] + u - q.lo[1]);
@@ -920,39 +1030,31 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                 }
         }
     } else if (run && warp >= kTlDeqWarp0) {
-        const int n = tid - 32 * kTlDeqWarp0;
-        const int r = n & 127, tile = (n >> 7) & 1, bsel = n >> 8;
-        Ring ra, rr;
-        bool ok = true;
-        for (int p = 0; p < 2 && ok && !abort_flag; ++p)
-            for (int u = q.lo[p]; u < q.hi[p] && ok && !abort_flag; ++u, rr.next(a.nr)) {
-                if (!mbar_wait(&rf_bar[rr.s], rr.u & 1)) {
-                    abort_flag = 1;
-                    ok = false;
-                    break;
-                }
-                if (a.stamps && c == 0 && n == 0) {  // profiling: CTA 0's first units, raw stage landed
-                    const int ui = (p == 0 ? u - q.lo[0] : q.hi[0] - q.lo[0] + u - q.lo[1]);
-                    if (ui < 4) a.stamps[24 + ui] = clock64();
-                }
-                const uint8_t *st = raw + rr.s * a.raw_stride;
-#pragma unroll 1
-                for (int d = 0; d < 4; ++d, ra.next(a.na)) {
-                    if (ra.u > 0 && !__all_sync(0xffffffffu, mbar_wait(&ae_bar[ra.s], (ra.u - 1) & 1))) {
-                        abort_flag = 1;
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *a_s = atile + ra.s * kTlAStage;
-                    if (p == 0) expand<FG>(st, a_s, r, tile, bsel, d, a.tab_gu);
-                    else expand<FD>(st, a_s, r, tile, bsel, d, a.tab_dn);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&fa_bar[ra.s]);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&re_bar[rr.s]);
-            }
+        ExpCtx xc;
+        xc.a = &a;
+        xc.q = &q;
+        xc.C = &C;
+        xc.grp_n = p_grp_n;
+        xc.grp_off = p_grp_off;
+        xc.raw = raw;
+        xc.atile = atile;
+        xc.bring = atile + a.na * kTlAStage;
+        xc.rf = rf_bar;
+        xc.re = re_bar;
+        xc.fa = fa_bar;
+        xc.ae = ae_bar;
+        xc.abort_flag = &abort_flag;
+        xc.G = G;
+        xc.c = c;
+        xc.n = tid - 32 * kTlDeqWarp0;
+        xc.lane = lane;
+        xc.slots = s_misc[1];
+        ExpState es;
+        if (expand_phase<FG>(xc, 0, es, a.tab_gu)) {
+            es.ready_g = -1;  // the down phase waits on the groups' h counters
+            expand_phase<FD>(xc, 1, es, a.tab_dn);
+        }
+        cp_async_wait_all();  // no copy into shared memory outlives the loop (abort included)
     } else if (run && warp < kTlEpiWarps) {
         // ---- epilogue: one tensor-memory lane (tile row) per thread --------------------
         const int r = warp * 32 + lane;
@@ -1080,11 +1182,7 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                     if (p == 0) {
                         atomicAdd(a.ctr + C.grp_h + x.g, 1u);
                     } else {
-                        const unsigned prev = atomicAdd(a.ctr + C.rb + x.b, 1u);
-                        if (prev + 1 == (unsigned)ng) {
-                            __threadfence();
-                            p_won[s_misc[2]++] = x.b;
-                        }
+                        atomicAdd(a.ctr + C.rb + x.b, 1u);  // one more group's y rows of this block are in
                     }
                 }
             }
@@ -1095,7 +1193,6 @@ __global__ void __launch_bounds__(kTlThreads, 1)
     if (abort_flag) {  // block-uniform after the barrier: drain what was issued, then release
         if (tid == 0 && router_cta && e1 > e0) mbar_wait(&wr_bar, 0);  // the router rows' bulk copy
         if (lane == 0 && warp == kTlRawWarp) drain_ring(rf_bar, a.nr, raw_issued);
-        if (lane == 0 && warp == kTlBWarp) drain_ring(fb_bar, a.nb, b_issued);
         if (lane == 0 && warp == kTlMmaWarp) drain_mma(&dr_bar);
         if (tid == 0) atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
         tc_fence_before_sync();
@@ -1103,22 +1200,38 @@ __global__ void __launch_bounds__(kTlThreads, 1)
     }
     grid_event(a.stamps, 3);
     cta0_clock(a.stamps, 6);
-    // ---- combine the 256-row output blocks this CTA finished last ----------------------
+    // ---- combine: rows [H c / G, H (c + 1) / G) of every token, once every group's
+    // y rows of their 256-row blocks are in: out[t] = sum_j gate_tj y[slot(t, j)]
+    // (+ the shared expert's y), in the layer's order ------------------------------------
     if (!abort_flag) {
-        const int nwon = s_misc[2];
         const int has = a.has_shared, routed_slots = s_misc[1] - (has ? T : 0);
-        if (ng == 0)  // no expert of this pack was selected and it has no shared expert: a zero share
-            for (size_t i = (size_t)c * kTlThreads + tid; i < (size_t)T * H; i += (size_t)G * kTlThreads) a.out[i] = 0.f;
-        for (int w = 0; w < nwon; ++w) {
-            const int b = p_won[w];
-            for (int i = tid; i < T * 256; i += kTlThreads) {
-                const int t = i >> 8, row = b * 256 + (i & 255);
-                float o = 0.f;
-                for (int j = 0; j < k; ++j) {
-                    const int sl = p_slot_of[t * k + j];
-                    if (sl >= 0) o += p_sel_g[t * k + j] * __ldcg(a.y + (size_t)sl * H + row);
+        const int r0 = (int)((long long)H * c / G), r1 = (int)((long long)H * (c + 1) / G), nrow = r1 - r0;
+        if (ng > 0 && nrow > 0 && tid == 0) {
+            for (int b = r0 / 256; b <= (r1 - 1) / 256; ++b)
+                if (!wait_count(a.ctr + C.rb + b, (unsigned)ng)) {
+                    abort_flag = 1;
+                    atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
+                    break;
                 }
-                if (has) o += __ldcg(a.y + (size_t)(routed_slots + t) * H + row);
+        }
+        __syncthreads();
+        if (!abort_flag && nrow > 0) {
+            for (int i = tid; i < T * nrow; i += kTlThreads) {
+                const int t = i / nrow, row = r0 + (i - t * nrow);
+                float o = 0.f;
+                if (ng > 0) {  // else no expert of this pack was selected and it has no shared expert: a zero share
+                    float yv[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {  // every gather in flight before the sum
+                        const int sl = j < k ? p_slot_of[t * k + j] : -1;
+                        yv[j] = sl >= 0 ? __ldcg(a.y + (size_t)sl * H + row) : 0.f;
+                    }
+                    const float ys = has ? __ldcg(a.y + (size_t)(routed_slots + t) * H + row) : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (j < k && p_slot_of[t * k + j] >= 0) o += p_sel_g[t * k + j] * yv[j];
+                    if (has) o += ys;
+                }
                 a.out[(size_t)t * H + row] = o;
             }
         }
@@ -1160,7 +1273,7 @@ __global__ void __launch_bounds__(kTlThreads, 1)
     }
 }
 
-using TlKernel = void (*)(const CUtensorMap, const CUtensorMap, const TailArgs);
+using TlKernel = void (*)(const TailArgs);
 
 template <int FG>
 TlKernel tl_pick_dn(int fd)
@@ -1193,36 +1306,36 @@ size_t tail_part_floats(int grid, int max_tokens) { return (size_t)2 * grid * 2 
 
 bool tail_plan(const TailPlanIn &in, TailLaunch *out)
 {
-    if (in.T < 1 || in.T > kDecodeTcMaxN || in.max_tokens < in.T || in.k > 16 || in.E > 1024) return false;
+    if (in.T < 1 || in.T > kDecodeTcMaxN || in.max_tokens < in.T || in.k > 16 || in.E > 1024 || in.E > 4 * kTlThreads) return false;
     if (in.H % 256 || in.I % 256 || in.H > 16384 || in.I > 16384) return false;
     const int xbytes = in.x_dtype == MOE_DT_BF16 ? 2 : 4;
     const int n16max = (std::min(in.max_tokens, 64) + 15) & ~15;
     const TlPlanLayout PL = tl_plan_layout(in.T, in.k, in.E);
     const int raw = std::max(tl_raw_bytes(in.fmt_gu), tl_raw_bytes(in.fmt_dn));
-    const int bslot = n16max * 128;
+    const int bslot = n16max * 128;  // a multiple of 2048
     const int budget = kTlSmemMax - 1024 - PL.total;
-    // two of each ring at least; then A stages (a round trip to the MMA issuer
-    // each slice), raw stages (HBM latency) and B slots (L2) while they fit
-    int nr = 2, na = 2, nb = 2;
-    auto rings = [&] { return nr * raw + na * kTlAStage + nb * bslot; };
+    // two of each ring at least; then raw stages (HBM latency) and operand
+    // stages (a round trip to the MMA issuer each slice), in turn, while they
+    // fit; na + 2 B slots
+    int nr = 2, na = 2;
+    auto rings = [&] { return nr * raw + na * kTlAStage + (na + 2) * bslot; };
     if (rings() > budget) return false;
     bool grown = true;
     while (grown) {
         grown = false;
         if (nr < kTlMaxRaw && rings() + raw <= budget) { ++nr; grown = true; }
-        if (nb < kTlMaxB && rings() + bslot <= budget) { ++nb; grown = true; }
-        if (na < 3 && rings() + kTlAStage <= budget) { ++na; grown = true; }
+        if (na < kTlMaxA && rings() + kTlAStage + bslot <= budget) { ++na; grown = true; }
     }
-    const int scratch = tl_scratch_bytes(in.T, in.H, in.E, in.grid, xbytes);
-    if (scratch > rings()) return false;
+    // the routing and planning scratch is overlaid on the rings: the region is the larger of the two
+    const int region = std::max(rings(), tl_scratch_bytes(in.T, in.H, in.E, in.grid, xbytes));
+    if (region > budget) return false;
     out->nr = nr;
     out->na = na;
-    out->nb = nb;
     out->raw_stride = raw;
     out->bslot = bslot;
     out->n16max = n16max;
-    out->rings = rings();
-    out->smem = (size_t)1024 + rings() + PL.total;
+    out->rings = region;
+    out->smem = (size_t)1024 + region + PL.total;
     return true;
 }
 
@@ -1284,7 +1397,6 @@ cudaError_t launch_tail(const TailCall &t, const TailLaunch &L, int grid, int pd
     a.cnt_out = t.ws->cnt;
     a.nr = L.nr;
     a.na = L.na;
-    a.nb = L.nb;
     a.raw_stride = L.raw_stride;
     a.bslot = L.bslot;
     a.n16max = L.n16max;
@@ -1307,8 +1419,7 @@ cudaError_t launch_tail(const TailCall &t, const TailLaunch &L, int grid, int pd
     }
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const DecodeTcMaps &m = *t.maps;
-    return cudaLaunchKernelEx(&cfg, tl_pick(t.gu->fmt, t.dn->fmt), m.xg, m.h, a);
+    return cudaLaunchKernelEx(&cfg, tl_pick(t.gu->fmt, t.dn->fmt), a);
 }
 
 }  // namespace moe
