@@ -150,7 +150,7 @@ def kernel_traffic(stage, wl_name):
         return None
     if not rec:
         return None
-    if rec.get("source_sha") != kernel_source_sha():
+    if rec.get("source_sha") != kernel_source_sha(rec.get("source_files")):
         return None
     return rec.get("bytes_per_launch")
 
@@ -162,20 +162,23 @@ def traffic_source(stage, wl_name):
         rec = json.load(open(path)).get(f"{stage}:{wl_name}")
     except Exception:
         rec = None
-    cur = kernel_source_sha()
     if not rec:
-        return {"status": f"no ncu capture recorded for {stage}:{wl_name}", "kernel_source_sha": cur}
+        return {"status": f"no ncu capture recorded for {stage}:{wl_name}", "kernel_source_sha": kernel_source_sha()}
+    cur = kernel_source_sha(rec.get("source_files"))
     same = rec.get("source_sha") == cur
     return {"status": "captured on this kernel source" if same
             else "kernel source changed since the capture: null until it is retaken",
-            "captured_sha": rec.get("source_sha"), "kernel_source_sha": cur, "command": rec.get("command")}
+            "captured_sha": rec.get("source_sha"), "kernel_source_sha": cur, "source_files": rec.get("source_files"),
+            "kernel": rec.get("kernel"), "command": rec.get("command")}
 
 
-def kernel_source_sha():
+def kernel_source_sha(files=None):
+    """Hash of the kernel sources a capture depends on: the given .cu files (all of
+    them when None) and every shared header."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_quantized_expert_moe_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
+        if f.endswith(".cuh") or (f.endswith(".cu") and (files is None or f in files)):
             h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -418,8 +421,13 @@ def measure(a, bq, torch, wl, layers, T, dist, world, dev, e2e=True):
         # timed graph's time per layer
         launch_us, launch_src = layer_us, "timed graph: ms_per_step / layers (one launch per layer)"
     else:
-        launch_us, launch_src = stage_us[dom], ("event-bracketed replay of the same graph (kernel times of a "
-                                                "multi-launch forward; their sum is profiled_layer_us)")
+        # several launches per layer: the event-bracketed replay (no overlap between
+        # launches) gives each kernel's share; scaled so that the shares add up to the
+        # timed graph's time per layer
+        prof_sum = sum(stage_us.values())
+        launch_us = stage_us[dom] * layer_us / prof_sum
+        launch_src = (f"timed graph share: event-bracketed {stage_us[dom]:.2f} us of {prof_sum:.2f} us per "
+                      f"layer, scaled to the timed {layer_us:.2f} us per layer")
     if dom == "prefill":
         kind = "fp4" if wl.fmt_gate_up == synth.FMT_NVFP4 else "bf16"
         tpk, tsrc = tensor_peak(kind)

@@ -82,6 +82,8 @@ def _load():
     L.moe_debug_wait_timeout.argtypes = [vp, vp]
     L.moe_debug_act_quant_nvfp4.restype = i32
     L.moe_debug_act_quant_nvfp4.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
+    L.moe_debug_dequant_rows.restype = i32
+    L.moe_debug_dequant_rows.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp]
     L.moe_debug_fail_alloc_after.restype = i32
     L.moe_debug_fail_alloc_after.argtypes = [i32]
     L.moe_read_routing.restype = i32
@@ -264,6 +266,19 @@ def moe_debug_act_quant_nvfp4(x, stream=None):
     _check(lib.moe_debug_act_quant_nvfp4(px, _dtype_code(x), rows, cols, pc, ps, pr, _stream_ptr(stream)),
            "moe_debug_act_quant_nvfp4")
     return codes, scales, row_scale
+
+
+def moe_debug_dequant_rows(pack, proj, slot, row0, nrows, kind, cols, stream=None):
+    """Tests only: the block decoders on rows of a packed projection (proj 0 gate/up,
+    1 down; kind 0: the tensor-core decode's fp16 expansion, returned as float16;
+    kind 1: the bf16-dequantising prefill's fp32 values).  cols: the projection's
+    row length (H for gate/up, I for down).  Returns a CUDA tensor [nrows, cols]."""
+    import torch
+    dt = torch.float16 if kind == 0 else torch.float32
+    out = torch.empty(nrows, cols, dtype=dt, device=f"cuda:{pack.device}")
+    _check(lib.moe_debug_dequant_rows(pack.handle, proj, slot, row0, nrows, kind, out.data_ptr(), _stream_ptr(stream)),
+           "moe_debug_dequant_rows")
+    return out
 
 
 def moe_route_workspace_bytes(n_tokens, n_experts):

@@ -20,6 +20,8 @@ cudaError_t route_set_attributes();
 cudaError_t matvec_set_attributes();
 cudaError_t debug_act_quant(const void *x, bool bf16, int rows, int cols, uint8_t *codes, uint8_t *sf_atoms,
                             float *row_scale, int32_t *scratch, cudaStream_t s);
+cudaError_t debug_dequant(const DevProj &w, const CodeTable &tab, int slot, int row0, int nrows, int kind, void *out,
+                          cudaStream_t s);
 }  // namespace moe
 
 // kernel-stage slots of the profiling API (moe_profile_end's ms[])
@@ -1269,6 +1271,18 @@ moe_status moe_debug_act_quant_nvfp4(const void *x, moe_dtype x_dtype, int rows,
     if (atoms) cudaFree(atoms);
     if (scratch) cudaFree(scratch);
     return st;
+}
+
+moe_status moe_debug_dequant_rows(const moe_pack *p, int proj, int slot, int row0, int nrows, int kind, void *out,
+                                  void *stream)
+{
+    if (!p || (proj != 0 && proj != 1) || (kind != 0 && kind != 1) || !out || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    const DevProj &w = proj == 0 ? p->gu : p->dn;
+    if (slot < 0 || slot >= p->n_local + p->has_shared || row0 < 0 || nrows < 1 || row0 > w.rows - nrows)
+        return MOE_ERR_INVALID_ARG;
+    DeviceGuard g(p->device);
+    return check_launch(debug_dequant(w, proj == 0 ? p->ct_gu : p->ct_dn, slot, row0, nrows, kind, out,
+                                      static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_get_device_error(const moe_pack *p)

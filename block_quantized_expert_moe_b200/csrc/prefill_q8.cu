@@ -440,4 +440,56 @@ cudaError_t prefill_q8_forward(const PrefillNvArgs &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
+// ---- diagnostic: the block decoders on rows of a packed projection ---------------
+// One thread per 32-block: kind 0 writes the fp16 expansion of the tensor-core
+// decode (dq::blk_f16), kind 1 the fp32 values of the bf16-dequantising
+// prefill's decoder (dq::blk_values) before their bf16 rounding; NVFP4 values
+// are twice E2M1 x E4M3, the matrix scale left to the callers' epilogues.
+template <int FMT>
+__global__ void debug_dequant_kernel(DevProj w, CodeTable tab, int slot, int row0, int nrows, int kind, void *out)
+{
+    const int nb = w.cols / 32;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= nrows * nb) return;
+    const int r = i / nb, b = i - r * nb, row = row0 + r;
+    const uint8_t *qrow = w.qs + (int64_t)slot * w.qs_stride + (int64_t)row * w.qs_row;
+    const uint8_t *srow = w.sr + (int64_t)slot * w.sr_stride + (int64_t)row * w.sr_row;
+    const uint8_t *hrow = w.qh ? w.qh + (int64_t)slot * w.qh_stride + (int64_t)row * w.qh_row : nullptr;
+    const dq::Blk<FMT> blk = dq::load_blk<FMT>(qrow, srow, hrow, b);
+    if (kind == 0) {
+        uint32_t q[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) q[j] = j < (FMT == MOE_FMT_Q8_0 ? 8 : 4) ? (&blk.q[0].x)[j] : 0u;
+        uint4 o4[4];
+        dq::blk_f16<FMT>(q, blk.s, blk.h, tab, o4);
+        uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + ((size_t)r * w.cols + b * 32));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[c] = o4[c];
+    } else {
+        float v[32];
+        dq::blk_values<FMT>(blk, tab, v);
+        float *o = static_cast<float *>(out) + ((size_t)r * w.cols + b * 32);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = v[j];
+    }
+}
+
+cudaError_t debug_dequant(const DevProj &w, const CodeTable &tab, int slot, int row0, int nrows, int kind, void *out,
+                          cudaStream_t s)
+{
+    const int n = nrows * (w.cols / 32), grid = (n + 255) / 256;
+    switch (w.fmt) {
+    case MOE_FMT_Q8_0: debug_dequant_kernel<MOE_FMT_Q8_0><<<grid, 256, 0, s>>>(w, tab, slot, row0, nrows, kind, out); break;
+    case MOE_FMT_Q5_1: debug_dequant_kernel<MOE_FMT_Q5_1><<<grid, 256, 0, s>>>(w, tab, slot, row0, nrows, kind, out); break;
+    case MOE_FMT_IQ4_NL:
+        debug_dequant_kernel<MOE_FMT_IQ4_NL><<<grid, 256, 0, s>>>(w, tab, slot, row0, nrows, kind, out);
+        break;
+    case MOE_FMT_NVFP4:
+        debug_dequant_kernel<MOE_FMT_NVFP4><<<grid, 256, 0, s>>>(w, tab, slot, row0, nrows, kind, out);
+        break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace moe

@@ -724,7 +724,9 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const RouteArgs a)
         topk_phase(a, smem, t0, min(a.T, t0 + a.rt), small && NB == 1 ? idx_s : nullptr);
     __syncthreads();
     route_event(a.stamps, 3);
-    route_clock(a.stamps, 3, tb == 0);
+    // SM clocks are per SM: with several token blocks the plan may run on another
+    // CTA's SM, so the selection's end is recorded only when one CTA does both
+    route_clock(a.stamps, 3, tb == 0 && NB == 1);
     if (threadIdx.x == 0) {
         a.ticket[2 + tb] = 0;
         if (NB > 1) {  // one block group: this CTA is already the last

@@ -355,6 +355,26 @@ moe_status moe_debug_wait_timeout(const moe_pack *pack, void *stream);
 moe_status moe_debug_act_quant_nvfp4(const void *x, moe_dtype x_dtype, int rows, int cols, uint8_t *codes,
                                      uint8_t *scales, float *row_scale, void *stream);
 
+/* Diagnostic for tests of the block decoders (the formats of the Unsloth
+ * dynamic-quantisation page, "Quantization types", and of the UD-IQ2_XS model
+ * card, "What was changed"): decodes rows [row0, row0 + nrows) of expert slot
+ * `slot` of one projection of `pack` (proj 0: gate/up, rows 0 .. 2I - 1 the
+ * gate rows then the up rows; 1: down, rows 0 .. H - 1; slot e - expert_begin
+ * for routed expert e, the shared expert after the routed ones) with the
+ * decoders the kernels use, from the pack's own planes:
+ *   kind 0  fp16 bits of the tensor-core decode's expansion (one rounding of
+ *           each weight to fp16)
+ *   kind 1  fp32 values of the bf16-dequantising prefill's decoder (before
+ *           its rounding to bf16)
+ * NVFP4 weights come out as 2 x E2M1 x E4M3: the per-expert matrix scale (and
+ * the halving) stay with the kernels' epilogues.
+ *   out  device [nrows x cols] (cols: H for gate/up, I for down), uint16 for
+ *        kind 0, float for kind 1, 16-byte aligned
+ * Enqueued on `stream`, no synchronisation.  MOE_ERR_INVALID_ARG for a bad
+ * projection, slot, row range, kind or pointer. */
+moe_status moe_debug_dequant_rows(const moe_pack *pack, int proj, int slot, int row0, int nrows, int kind, void *out,
+                                  void *stream);
+
 /* Sticky device-side error of the pack (synchronises its device), then clears it. */
 moe_status moe_get_device_error(const moe_pack *pack);
 

@@ -80,6 +80,7 @@ def test_pack_requires_tables_scales_and_shared_blocks():
 
 def test_forward_and_route_reject_null_and_misaligned_pointers():
     assert bq.lib.moe_layer_forward(None, 1, None, None, 0, 1, 1, None, None) == bq.MOE_ERR_INVALID_ARG
+    assert bq.lib.moe_debug_dequant_rows(None, 0, 0, 0, 1, 0, None, None) == bq.MOE_ERR_INVALID_ARG
     buf = np.zeros(4096, np.uint8)
     p = buf.ctypes.data + 8 if buf.ctypes.data % 16 == 0 else buf.ctypes.data
     assert bq.lib.moe_route_topk(p, 2, p, 1, 64, 4, 2, p, p, p, 4096, None) == bq.MOE_ERR_INVALID_ARG

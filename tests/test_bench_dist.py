@@ -92,17 +92,22 @@ def test_traffic_is_reported_only_for_the_captured_kernel_source(monkeypatch):
     rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
     key, entry = next(iter(rec.items()))
     stage, wl_name = key.split(":")
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda: entry["source_sha"])
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda files=None: entry["source_sha"])
     assert bench.kernel_traffic(stage, wl_name) == entry["bytes_per_launch"]
     assert entry["bytes_per_launch"] == entry["dram_read"] + entry["dram_write"]
     assert bench.traffic_source(stage, wl_name)["status"] == "captured on this kernel source"
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "0" * 16)
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda files=None: "0" * 16)
     assert bench.kernel_traffic(stage, wl_name) is None
     src = bench.traffic_source(stage, wl_name)
     assert src["captured_sha"] == entry["source_sha"] and src["kernel_source_sha"] == "0" * 16
     assert "changed" in src["status"] and src["command"] == entry["command"]
     assert bench.kernel_traffic(stage, "no_such_workload") is None
     assert "no ncu capture" in bench.traffic_source(stage, "no_such_workload")["status"]
+    # each record names the kernel source files its sha covers (with every shared header)
+    monkeypatch.undo()
+    for k, e in rec.items():
+        assert e["source_files"] and all(f.endswith(".cu") for f in e["source_files"]), k
+        assert e["bytes_per_launch"] == e["dram_read"] + e["dram_write"], k
 
 
 def test_reference_arm_under_torchrun_prints_once_from_rank_0(repo_tmp):
