@@ -893,6 +893,7 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
         tc.tab_gu = p->ct_gu;
         tc.tab_dn = p->ct_dn;
         tc.ws = &p->ws;
+        tc.maps = &pm->dtc_maps;
         tc.out = out;
         int pbase = -1;
         if (pm->prof_on && (size_t)pm->prof_used + 2 <= pm->prof_ev.size()) {

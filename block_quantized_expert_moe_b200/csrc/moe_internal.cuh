@@ -294,7 +294,7 @@ struct TailPlanIn {
     int T, max_tokens, H, E, I, k, x_dtype, fmt_gu, fmt_dn, grid;
 };
 struct TailLaunch {
-    int nr, na, raw_stride, bslot, n16max, rings;
+    int nr, na, nb, raw_stride, bslot, n16max, rings;
     size_t smem;
 };
 struct TailCall {
@@ -306,6 +306,7 @@ struct TailCall {
     const DevProj *gu, *dn;
     CodeTable tab_gu, tab_dn;
     const Workspace *ws;
+    const DecodeTcMaps *maps;  // the x and h slot-row maps (16-row boxes) of the tensor-core decode
     float *out;
     long long *stamps;
 };

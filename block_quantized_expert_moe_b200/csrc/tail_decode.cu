@@ -33,19 +33,22 @@
 //             in the layer's order
 //
 // The tensor-core tile is M = 128 weight rows, N = the group's tokens (padded
-// to 16), K = 64 per shared-memory stage, fp16 x fp16 -> fp32 in tensor memory:
-// the weights are expanded from their blocks to fp16 in shared memory once per
-// unit (one rounding each, exact for the 4-bit codes), the slot rows of x are
-// exact fp16 after the token's power-of-two scale, h is rounded to fp16.
+// to 16), K = 64 per stage, fp16 x fp16 -> fp32 in tensor memory: the weights
+// are expanded from their blocks to fp16 straight into tensor memory (the MMA's
+// A operand; one rounding each, exact for the 4-bit codes), the slot rows of x
+// (the B operand, shared memory) are exact fp16 after the token's power-of-two
+// scale, h is rounded to fp16.  Tensor memory: columns 0-255 two accumulator
+// buffers, 256-511 four A stages of 64 columns (two tiles of 32).
 //
 //   warps 0-3   epilogue: tensor-memory lanes 32w .. 32w + 31 (tile rows)
 //   warp 4      MMA issuer (one elected thread)
 //   warp 5      raw producer (two bulk copies a unit from the tiled planes)
-//   warps 6-13  expanders: each thread both 32-blocks of one row per slice,
-//               and up to two 16-byte chunks of the slice's B rows (the
-//               group's slot rows of x or h, read from L2 once the group's
-//               readiness counter is full), stored beside the A tiles of the
-//               same operand stage: the MMA issuer waits on one barrier a slice
+//   warp 6      B producer: once the group's readiness counter is full, TMA
+//               loads (16-row boxes) of the group's slot rows of x or h, one
+//               ring slot per slice
+//   warps 7-14  expanders: warp 7 + i expands tile i / 4, lanes 32 (warp % 4)
+//               .. + 31 (the lanes a warp may store to), both 32-blocks of
+//               its row per slice
 //
 // Every wait is bounded (~1 s): a wait that runs out records MOE_ERR_TIMEOUT,
 // raises the CTA's abort flag and the CTA drains what it issued before it
@@ -61,6 +64,7 @@
 #include "dequant.cuh"
 #include "moe_internal.cuh"
 #include "tc_common.cuh"
+#include "tma_maps.cuh"
 
 namespace moe {
 
@@ -68,15 +72,15 @@ namespace {
 
 using namespace tc;
 
-constexpr int kTlEpiWarps = 4, kTlMmaWarp = 4, kTlRawWarp = 5, kTlDeqWarp0 = 6, kTlDeqWarps = 8;
-constexpr int kTlWarps = kTlDeqWarp0 + kTlDeqWarps;  // 14
+constexpr int kTlEpiWarps = 4, kTlMmaWarp = 4, kTlRawWarp = 5, kTlBWarp = 6, kTlDeqWarp0 = 7, kTlDeqWarps = 8;
+constexpr int kTlWarps = kTlDeqWarp0 + kTlDeqWarps;  // 15
 constexpr int kTlThreads = 32 * kTlWarps;
-constexpr int kTlDeqThreads = 32 * kTlDeqWarps;      // 256: one per row of the unit's two tiles
 constexpr int kTlWriters = 32 * (kTlEpiWarps + kTlDeqWarps);  // the warps that write the x slot rows
-constexpr int kTlMaxRaw = 4, kTlMaxA = 4;
-constexpr int kTlA = 128 * 128;           // one 128-row tile x 64 fp16 of K
-constexpr int kTlAStage = 2 * kTlA;       // a unit's two tiles (the slice's B rows follow in the stage)
-constexpr int kTlTmemCols = 256;          // two accumulator buffers of 128 columns
+constexpr int kTlMaxRaw = 4, kTlMaxB = 8;
+constexpr int kTlTmemCols = 512;          // two accumulator buffers of 128 columns, then the A stages
+constexpr int kTlAcc = 256;               // first tensor-memory column of the A stages
+constexpr int kTlAStageCols = 64;         // a stage: the unit's two 128-row tiles x 64 fp16 of K (32 columns each)
+constexpr int kTlNA = 4;                  // A stages (the rest of tensor memory)
 constexpr long long kTlSpin = 1ll << 31;  // clocks
 
 __host__ __device__ inline int tl_cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -195,8 +199,8 @@ struct TailArgs {
     int32_t *idx_out;            // routing readback, written by CTA 0
     float *gate_out;
     int32_t *cnt_out;
-    int nr, na;                  // ring depths
-    int raw_stride, bslot, n16max;  // B slots (na + 2 of them, after the A stages): n16max rows of 128 bytes
+    int nr, na, nb;              // ring depths: raw stages, A stages (tensor memory), B slots
+    int raw_stride, bslot, n16max;  // a B slot: n16max rows of 128 bytes
     int rings;                   // bytes of the rings (the plan follows)
     long long *stamps;           // profiling only: grid events {2^62 - first, last} at words 10..19
 };
@@ -225,14 +229,29 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
                  : "memory");
 }
 
-// 16-byte asynchronous copy global -> shared (L2 only), in the thread's current group.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+// Tensor memory: one thread's 16 consecutive 32-bit columns of its lane (the warp's 32 lanes at once).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+                 "%13, %14, %15, %16};" ::"r"(taddr),
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+                 "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+                 : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// f16 x f16 -> f32 MMA with A in tensor memory (M = 128: row m in lane m, K packed two
+// fp16 per 32-bit column), B a shared-memory descriptor.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 
 __device__ __forceinline__ void grid_event(long long *st, int ev)
 {
@@ -428,111 +447,59 @@ __device__ __forceinline__ void load_slice(const uint8_t *st, int r, int tile, i
     }
 }
 
-// fp16 of both blocks into row r of tile `tile` of the operand stage (128-byte
-// swizzle, K-major): 16-byte chunk c of the slice's 64 values at c ^ (r % 8).
+// fp16 of both blocks of the thread's row into its tensor-memory lane: block
+// bsel of the slice at columns col + 16 bsel .. + 15 (two fp16 of K per column,
+// in K order), the layout the MMA reads A from.
 template <int FMT>
-__device__ __forceinline__ void store_slice(const SliceRaw<FMT> &R, uint8_t *a_stage, int r, int tile,
-                                            const CodeTable &tab)
+__device__ __forceinline__ void store_slice(const SliceRaw<FMT> &R, uint32_t taddr, const CodeTable &tab)
 {
-    uint8_t *a_row = a_stage + tile * kTlA + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
     for (int bsel = 0; bsel < 2; ++bsel) {
         uint4 o4[4];
         dq::blk_f16<FMT>(R.q[bsel], R.s[bsel], R.h[bsel], tab, o4);
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            const int c = 4 * bsel + cc;
-            *reinterpret_cast<uint4 *>(a_row + ((c ^ (r & 7)) << 4)) = o4[cc];
-        }
+        const uint32_t w[16] = {o4[0].x, o4[0].y, o4[0].z, o4[0].w, o4[1].x, o4[1].y, o4[1].z, o4[1].w,
+                                o4[2].x, o4[2].y, o4[2].z, o4[2].w, o4[3].x, o4[3].y, o4[3].z, o4[3].w};
+        tmem_st16(taddr + 16 * bsel, w);
     }
 }
 
 // The expanding warps' walk over their rings, kept across the two phases.
 struct ExpState {
-    Ring ra, rr;     // operand stages, raw stages
-    int bs = 0;      // B slot of the current slice (slices in order, na + 2 slots)
-    bool pre = false;  // the current slice's B was issued during the previous slice
-    int ready_g = -1;
+    Ring ra, rr;  // A stages (tensor memory), raw stages
 };
 
 // Everything the expanding warps read of the kernel's state.
 struct ExpCtx {
     const TailArgs *a;
     const Geo *q;
-    const TlCtr *C;
-    const int16_t *grp_n;
-    const int *grp_off;
     const uint8_t *raw;
-    uint8_t *atile, *bring;
+    uint32_t tmem;  // the CTA's tensor memory
     uint64_t *rf, *re, *fa, *ae;
     volatile int *abort_flag;
-    int G, c, n, lane, slots;
+    int c, lane, warp;
 };
 
 // One phase (0 gate/up, FMT = the gate/up format; 1 down) of the expanding
-// warps; false when a wait ran out or the CTA aborted.  Thread n (0 .. 255)
-// expands row n % 128 of tile n / 128, and copies B chunks n and n + 256 of
-// each slice: B row j (slot off + j of the group) holds K values kc * 256 +
-// 64 d .. + 63 of x (gate/up) or h (down), 8 chunks of 16 bytes, chunk
-// 8 j + cc at the 128-byte swizzled place of row j in its B slot.  A slice's B
-// is issued one slice ahead, before the wait on the operand stage, when the
-// MMAs up to slice - 1 - na are known complete: na + 2 slots keep it clear of
-// any slice still read.
+// warps; false when a wait ran out or the CTA aborted.  Expanding warp w
+// (0 .. 7) expands tile w / 4, rows 32 (warp % 4) .. + 31 (the tensor-memory
+// lanes its warp may write), one row per lane, into the A stage in tensor
+// memory; the next slice's raw bytes are loaded before the current slice's
+// expansion.
 template <int FMT>
 __device__ bool expand_phase(const ExpCtx &x, int p, ExpState &es, const CodeTable &tab)
 {
     const TailArgs &a = *x.a;
     const Geo &q = *x.q;
-    const int n = x.n, r = n & 127, tile = n >> 7, nbs = a.na + 2;
-    const int bld = p == 0 ? a.H : a.I;
-    const __half *bbase = p == 0 ? a.xg : a.h;
-    // this thread's B chunks: destination in a slot, source from a row's start
-    int bdst[2], bsrc[2], bch[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int ch = n + kTlDeqThreads * i, j = ch >> 3, cc = ch & 7;
-        bch[i] = ch;
-        bdst[i] = (j >> 3) * 1024 + (j & 7) * 128 + ((cc ^ (j & 7)) << 4);
-        bsrc[i] = j * bld + cc * 8;
-    }
-    auto issue_b = [&](const __half *src, int nch, int slot) {
-        uint8_t *b_s = x.bring + slot * a.bslot;
-#pragma unroll
-        for (int i = 0; i < 2; ++i)
-            if (bch[i] < nch) cp_async16(b_s + bdst[i], src + bsrc[i]);
-    };
+    const int r = 32 * (x.warp & 3) + x.lane, tile = (x.warp - kTlDeqWarp0) >> 2;
+    // this thread's lane and tile in an A stage (the stage's columns are added per slice)
+    const uint32_t t_row = x.tmem + ((uint32_t)(32 * (x.warp & 3)) << 16) + kTlAcc + tile * 32;
     for (int u = q.lo[p]; u < q.hi[p]; ++u, es.rr.next(a.nr)) {
         if (*x.abort_flag) return false;
-        const Unit un = unit_at(q, p, u);
-        const int gn = x.grp_n[un.g], goff = x.grp_off[un.g], nch = gn * 8;
-        if (un.g != es.ready_g) {
-            // the group's B rows: gate/up, its x slot rows written by the CTAs
-            // that own them; down, all of its h tiles finished.  Lane 0 waits,
-            // then every lane takes its own acquire of the (full) count
-            const unsigned *cp = a.ctr + (p == 0 ? x.C->grp_x : x.C->grp_h) + un.g;
-            bool w_ok = true;
-            if (x.lane == 0)
-                w_ok = wait_count(cp, p == 0 ? (unsigned)owners(goff, gn, x.slots, x.G) : (unsigned)q.NB[0]);
-            w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-            if (!w_ok) {
-                if (x.lane == 0) atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
-                *x.abort_flag = 1;
-                return false;
-            }
-            (void)ld_acq(cp);
-            es.ready_g = un.g;
-        }
-        const __half *bsrc_u = bbase + (size_t)goff * bld + un.kc * 256;
-        const __half *bsrc_n = nullptr;  // the next unit's B, when its rows are the same group's
-        if (u + 1 < q.hi[p]) {
-            const Unit nx = unit_at(q, p, u + 1);
-            if (nx.g == un.g) bsrc_n = bbase + (size_t)goff * bld + nx.kc * 256;
-        }
         if (!mbar_wait(&x.rf[es.rr.s], es.rr.u & 1)) {
             *x.abort_flag = 1;
             return false;
         }
-        if (a.stamps && x.c == 0 && n == 0) {  // profiling: CTA 0's first units, raw stage landed
+        if (a.stamps && x.c == 0 && x.warp == kTlDeqWarp0 && x.lane == 0) {  // profiling: CTA 0's first units
             const int ui = (p == 0 ? u - q.lo[0] : q.hi[0] - q.lo[0] + u - q.lo[1]);
             if (ui < 4) a.stamps[24 + ui] = clock64();
         }
@@ -541,27 +508,19 @@ __device__ bool expand_phase(const ExpCtx &x, int p, ExpState &es, const CodeTab
         load_slice<FMT>(st, r, tile, 0, R);
 #pragma unroll 1
         for (int d = 0; d < 4; ++d, es.ra.next(a.na)) {
-            const int bn = es.bs + 1 == nbs ? 0 : es.bs + 1;
-            if (!es.pre) {
-                issue_b(bsrc_u + d * 64, nch, es.bs);
-                cp_async_commit();
-            }
-            es.pre = d < 3 || bsrc_n != nullptr;
-            if (es.pre) issue_b(d < 3 ? bsrc_u + (d + 1) * 64 : bsrc_n, nch, bn);
-            cp_async_commit();
             SliceRaw<FMT> Rn;
             if (d < 3) load_slice<FMT>(st, r, tile, d + 1, Rn);
             if (es.ra.u > 0 && !__all_sync(0xffffffffu, mbar_wait(&x.ae[es.ra.s], (es.ra.u - 1) & 1))) {
                 *x.abort_flag = 1;
                 return false;
             }
-            store_slice<FMT>(R, x.atile + es.ra.s * kTlAStage, r, tile, tab);
-            cp_async_wait_prev();  // this slice's B has landed (the next one may be in flight)
-            fence_proxy_async_smem();
+            tc_fence_after_sync();  // the MMAs that read this stage are complete
+            store_slice<FMT>(R, t_row + es.ra.s * kTlAStageCols, tab);
+            tmem_wait_st();
+            tc_fence_before_sync();
             __syncwarp();
             if (x.lane == 0) mbar_arrive(&x.fa[es.ra.s]);
             if (d < 3) R = Rn;
-            es.bs = bn;
         }
         __syncwarp();
         if (x.lane == 0) mbar_arrive(&x.re[es.rr.s]);
@@ -577,11 +536,11 @@ __host__ __device__ constexpr uint32_t tl_idesc(int N)
 
 template <int FG, int FD>
 __global__ void __launch_bounds__(kTlThreads, 1)
-    tail_kernel(const __grid_constant__ TailArgs a)
+    tail_kernel(const __grid_constant__ CUtensorMap mXg, const __grid_constant__ CUtensorMap mH, const TailArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t rf_bar[kTlMaxRaw], re_bar[kTlMaxRaw], fa_bar[kTlMaxA], ae_bar[kTlMaxA],
-        accf_bar[2], acce_bar[2], dr_bar, wr_bar;
+    __shared__ __align__(8) uint64_t rf_bar[kTlMaxRaw], re_bar[kTlMaxRaw], fa_bar[kTlNA], ae_bar[kTlNA],
+        fb_bar[kTlMaxB], be_bar[kTlMaxB], accf_bar[2], acce_bar[2], dr_bar, wr_bar;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
     __shared__ volatile int s_epi_abort;  // the four epilogue warps leave together
@@ -619,6 +578,10 @@ __global__ void __launch_bounds__(kTlThreads, 1)
         for (int s = 0; s < a.na; ++s) {
             mbar_init(&fa_bar[s], kTlDeqWarps);
             mbar_init(&ae_bar[s], 1);
+        }
+        for (int s = 0; s < a.nb; ++s) {
+            mbar_init(&fb_bar[s], 1);
+            mbar_init(&be_bar[s], 1);
         }
         for (int s = 0; s < a.nr; ++s) {
             mbar_init(&rf_bar[s], 1);
@@ -894,8 +857,8 @@ __global__ void __launch_bounds__(kTlThreads, 1)
         q.lo[p] = range_lo(q.U[p], c, G);
         q.hi[p] = range_lo(q.U[p], c + 1, G);
     }
-    uint8_t *raw = smem, *atile = smem + a.nr * a.raw_stride;
-    int raw_issued = 0;
+    uint8_t *raw = smem, *bring = smem + a.nr * a.raw_stride;
+    int raw_issued = 0, b_issued = 0;
 
     // ---- this CTA's share of the fp16 slot rows of x (slots [s0, s1)), by the
     // epilogue and expanding warps while the raw producer and the MMA issuer
@@ -986,11 +949,49 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                 }
             raw_issued = rr.u * a.nr + rr.s;
         }
+    } else if (run && warp == kTlBWarp) {
+        if (lane == 0) {
+            prefetch_tmap(&mXg);
+            prefetch_tmap(&mH);
+            Ring rb;
+            int ready_g = -1, ready_p = -1;
+            for (int p = 0; p < 2 && !abort_flag; ++p)
+                for (int u = q.lo[p]; u < q.hi[p] && !abort_flag; ++u) {
+                    const Unit x = unit_at(q, p, u);
+                    const int n = p_grp_n[x.g], off = p_grp_off[x.g], n16 = (n + 15) >> 4;
+                    if (x.g != ready_g || p != ready_p) {
+                        // gate/up: the group's x slot rows written by the CTAs that own
+                        // them; down: all of the group's h tiles finished.  The rows were
+                        // written with generic stores: the acquire of the full count, then
+                        // a proxy fence, before the TMA reads them
+                        const unsigned *cp = a.ctr + (p == 0 ? C.grp_x : C.grp_h) + x.g;
+                        if (!wait_count(cp, p == 0 ? (unsigned)owners(off, n, s_misc[1], G) : (unsigned)q.NB[0])) {
+                            abort_flag = 1;
+                            atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
+                            break;
+                        }
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        ready_g = x.g;
+                        ready_p = p;
+                    }
+                    for (int sl = 0; sl < 4; ++sl, rb.next(a.nb)) {
+                        if (rb.u > 0 && !mbar_wait_idle(&be_bar[rb.s], (rb.u - 1) & 1)) {
+                            abort_flag = 1;
+                            break;
+                        }
+                        uint8_t *b_s = bring + rb.s * a.bslot;
+                        mbar_arrive_expect_tx(&fb_bar[rb.s], (uint32_t)n16 * 2048u);
+                        for (int jj = 0; jj < n16; ++jj)
+                            tma_load_2d(b_s + jj * 2048, p == 0 ? &mXg : &mH, &fb_bar[rb.s], x.kc * 256 + sl * 64,
+                                        off + 16 * jj);
+                    }
+                }
+            b_issued = rb.u * a.nb + rb.s;
+        }
     } else if (run && warp == kTlMmaWarp) {
         if (lane == 0) {
-            Ring ra;
-            int seg = 0, gs = 0;
-            const uint8_t *bring = atile + a.na * kTlAStage;
+            Ring ra, rbm;
+            int seg = 0;
             for (int p = 0; p < 2 && !abort_flag; ++p)
                 for (int u = q.lo[p]; u < q.hi[p] && !abort_flag; ++u) {
                     const Unit x = unit_at(q, p, u);
@@ -1001,23 +1002,23 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                     }
                     tc_fence_after_sync();
                     const uint32_t idesc = tl_idesc((p_grp_n[x.g] + 15) & ~15);
-                    for (int sl = 0; sl < 4; ++sl, ra.next(a.na), ++gs) {
-                        if (!mbar_wait(&fa_bar[ra.s], ra.u & 1)) {
+                    for (int sl = 0; sl < 4; ++sl, ra.next(a.na), rbm.next(a.nb)) {
+                        if (!mbar_wait(&fa_bar[ra.s], ra.u & 1) || !mbar_wait(&fb_bar[rbm.s], rbm.u & 1)) {
                             abort_flag = 1;
                             break;
                         }
                         tc_fence_after_sync();
-                        const uint8_t *a_s = atile + ra.s * kTlAStage;
-                        const uint64_t bd = desc_kmajor_sw128(bring + (gs % (a.na + 2)) * a.bslot);
+                        const uint32_t a_t = tmem + kTlAcc + ra.s * kTlAStageCols;
+                        const uint64_t bd = desc_kmajor_sw128(bring + rbm.s * a.bslot);
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
-                            const uint64_t ad = desc_kmajor_sw128(a_s + hh * kTlA);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
-                                mma_f16(tmem + ab * 128 + hh * 64, ad + 2 * kk, bd + 2 * kk, idesc,
-                                        !(x.first && sl == 0 && kk == 0));
+                                mma_f16_ts(tmem + ab * 128 + hh * 64, a_t + hh * 32 + kk * 8, bd + 2 * kk, idesc,
+                                           !(x.first && sl == 0 && kk == 0));
                         }
                         mma_commit(&ae_bar[ra.s]);
+                        mma_commit(&be_bar[rbm.s]);
                     }
                     if (a.stamps && c == 0) {  // profiling: CTA 0's first units, MMAs issued
                         const int ui = (p == 0 ? u - q.lo[0] : q.hi[0] - q.lo[0] + u - q.lo[1]);
@@ -1033,28 +1034,19 @@ __global__ void __launch_bounds__(kTlThreads, 1)
         ExpCtx xc;
         xc.a = &a;
         xc.q = &q;
-        xc.C = &C;
-        xc.grp_n = p_grp_n;
-        xc.grp_off = p_grp_off;
         xc.raw = raw;
-        xc.atile = atile;
-        xc.bring = atile + a.na * kTlAStage;
+        xc.tmem = tmem;
         xc.rf = rf_bar;
         xc.re = re_bar;
         xc.fa = fa_bar;
         xc.ae = ae_bar;
         xc.abort_flag = &abort_flag;
-        xc.G = G;
         xc.c = c;
-        xc.n = tid - 32 * kTlDeqWarp0;
         xc.lane = lane;
-        xc.slots = s_misc[1];
+        xc.warp = warp;
         ExpState es;
-        if (expand_phase<FG>(xc, 0, es, a.tab_gu)) {
-            es.ready_g = -1;  // the down phase waits on the groups' h counters
-            expand_phase<FD>(xc, 1, es, a.tab_dn);
-        }
-        cp_async_wait_all();  // no copy into shared memory outlives the loop (abort included)
+        if (expand_phase<FG>(xc, 0, es, a.tab_gu)) expand_phase<FD>(xc, 1, es, a.tab_dn);
+        tmem_wait_st();  // no store into tensor memory outlives the loop (abort included)
     } else if (run && warp < kTlEpiWarps) {
         // ---- epilogue: one tensor-memory lane (tile row) per thread --------------------
         const int r = warp * 32 + lane;
@@ -1193,6 +1185,7 @@ __global__ void __launch_bounds__(kTlThreads, 1)
     if (abort_flag) {  // block-uniform after the barrier: drain what was issued, then release
         if (tid == 0 && router_cta && e1 > e0) mbar_wait(&wr_bar, 0);  // the router rows' bulk copy
         if (lane == 0 && warp == kTlRawWarp) drain_ring(rf_bar, a.nr, raw_issued);
+        if (lane == 0 && warp == kTlBWarp) drain_ring(fb_bar, a.nb, b_issued);
         if (lane == 0 && warp == kTlMmaWarp) drain_mma(&dr_bar);
         if (tid == 0) atomicExch(a.err, (int)MOE_ERR_TIMEOUT);
         tc_fence_before_sync();
@@ -1273,7 +1266,7 @@ __global__ void __launch_bounds__(kTlThreads, 1)
     }
 }
 
-using TlKernel = void (*)(const TailArgs);
+using TlKernel = void (*)(const CUtensorMap, const CUtensorMap, const TailArgs);
 
 template <int FG>
 TlKernel tl_pick_dn(int fd)
@@ -1314,23 +1307,25 @@ bool tail_plan(const TailPlanIn &in, TailLaunch *out)
     const int raw = std::max(tl_raw_bytes(in.fmt_gu), tl_raw_bytes(in.fmt_dn));
     const int bslot = n16max * 128;  // a multiple of 2048
     const int budget = kTlSmemMax - 1024 - PL.total;
-    // two of each ring at least; then raw stages (HBM latency) and operand
-    // stages (a round trip to the MMA issuer each slice), in turn, while they
-    // fit; na + 2 B slots
-    int nr = 2, na = 2;
-    auto rings = [&] { return nr * raw + na * kTlAStage + (na + 2) * bslot; };
+    // the A stages live in tensor memory (kTlNA of them); shared memory holds
+    // the raw stages and the B slots: two raw stages and four slots at least,
+    // then more of each, in turn, while they fit
+    int nr = 2, nb = 4;
+    const int na = kTlNA;
+    auto rings = [&] { return nr * raw + nb * bslot; };
     if (rings() > budget) return false;
     bool grown = true;
     while (grown) {
         grown = false;
         if (nr < kTlMaxRaw && rings() + raw <= budget) { ++nr; grown = true; }
-        if (na < kTlMaxA && rings() + kTlAStage + bslot <= budget) { ++na; grown = true; }
+        if (nb < kTlMaxB && rings() + bslot <= budget) { ++nb; grown = true; }
     }
     // the routing and planning scratch is overlaid on the rings: the region is the larger of the two
     const int region = std::max(rings(), tl_scratch_bytes(in.T, in.H, in.E, in.grid, xbytes));
     if (region > budget) return false;
     out->nr = nr;
     out->na = na;
+    out->nb = nb;
     out->raw_stride = raw;
     out->bslot = bslot;
     out->n16max = n16max;
@@ -1397,6 +1392,7 @@ cudaError_t launch_tail(const TailCall &t, const TailLaunch &L, int grid, int pd
     a.cnt_out = t.ws->cnt;
     a.nr = L.nr;
     a.na = L.na;
+    a.nb = L.nb;
     a.raw_stride = L.raw_stride;
     a.bslot = L.bslot;
     a.n16max = L.n16max;
@@ -1419,7 +1415,8 @@ cudaError_t launch_tail(const TailCall &t, const TailLaunch &L, int grid, int pd
     }
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, tl_pick(t.gu->fmt, t.dn->fmt), a);
+    const DecodeTcMaps &m = *t.maps;
+    return cudaLaunchKernelEx(&cfg, tl_pick(t.gu->fmt, t.dn->fmt), m.xg, m.h, a);
 }
 
 }  // namespace moe
