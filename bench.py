@@ -381,7 +381,8 @@ def measure(a, bq, torch, wl, layers, T, dist, world, dev, e2e=True):
     launches_per_fwd = 1 if stage_ms[4] > 0 else (prefill_kernels if stage_ms[5] > 0 else (5 if tc_path else 4))
     stage_us = {s: float(stage_ms[i] / nf * 1e3) for i, s in enumerate(STAGES) if stage_ms[i] > 0}
     phase_names = ["stage_x", "router", "logit_poll_topk", "issue", "gate_up", "h_poll", "down", "-", "tail"]
-    one_launch_tail = stage_ms[4] > 0 and a.path == "tail"
+    # the one-launch tail: chosen explicitly, or by the automatic path for 2-64 tokens
+    one_launch_tail = stage_ms[4] > 0 and (a.path == "tail" or (a.path == "auto" and T >= 2))
     if one_launch_tail:
         # CTA 0's steps in the one-launch tail
         fused_phase_us = {n: float(stage_ms[6 + i] / nf * 1e3) for i, n in enumerate(
@@ -391,7 +392,7 @@ def measure(a, bq, torch, wl, layers, T, dist, world, dev, e2e=True):
     else:
         fused_phase_us = None
     grid_names = (["last_start", "first_router", "last_router", "first_issue", "last_issue",
-                   "first_gate_up", "last_gate_up", "first_end", "last_end"] if a.path != "tail" else
+                   "first_gate_up", "last_gate_up", "first_end", "last_end"] if not one_launch_tail else
                   # the one-launch tail: routed (grid barrier reached), planned, units done, combined
                   ["last_start", "first_routed", "last_routed", "first_planned", "last_planned",
                    "first_units_done", "last_units_done", "first_end", "last_end"])
@@ -411,7 +412,7 @@ def measure(a, bq, torch, wl, layers, T, dist, world, dev, e2e=True):
     dom = max(stage_us, key=lambda s: stage_us[s])
     kname = KERNEL_NAMES[dom]
     if dom == "fused":
-        kname = ("tail_kernel" if a.path == "tail" else "stream1_kernel" if T == 1 else "fused_decode_kernel")
+        kname = ("tail_kernel" if one_launch_tail else "stream1_kernel" if T == 1 else "fused_decode_kernel")
     if a.path in ("auto", "staged") and T >= 2 and dom in ("gate_up", "down"):
         kname = f"dtc_kernel<{dom.replace('_', '/')}>" if tc_path else f"sgm_kernel<{dom.replace('_', '/')}>"
     hbm, peak_src = peaks()

@@ -859,9 +859,9 @@ moe_status moe_layer_forward_ex(const void *x, moe_dtype x_dtype, const uint16_t
     }
     // 2..64 tokens: the one-launch tail when it fits, else the tensor-core
     // grouped decode in separate launches, when the pack's weights are
-    // fp16-representable
+    // fp16-representable (one token: the single-token streaming kernel)
     bool use_tail = false;
-    if (path == MOE_PATH_TAIL) {
+    if (path == MOE_PATH_TAIL || (path == MOE_PATH_DECODE && T >= 2)) {
         const int xb = x_dtype == MOE_DT_BF16 ? 1 : 0;
         int &ok = pm->tail_ok[T][xb];
         if (ok < 0) {

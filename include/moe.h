@@ -102,12 +102,13 @@ typedef enum { MOE_DT_F32 = 1, MOE_DT_BF16 = 2 } moe_dtype;
  * to bf16 for bf16 MMA; hidden and inter multiples of 256, bf16 activations,
  * top_k <= 32; its buffers are sized at pack time when max_tokens > 64), else
  * GROUPED.  DECODE: one token runs the single-token streaming kernel; 2 to 64
- * tokens run the tensor-core grouped decode as separate launches (route and
- * plan, x gather, gate/up, down, combine; weights expanded to fp16, fp32
+ * tokens run the tensor-core decode (weights expanded to fp16, fp32
  * accumulation; hidden and inter multiples of 256 and every weight an fp16
- * normal number or zero, checked at pack time), else the CUDA-core grouped
- * kernels.  TAIL runs the same layer as one launch (the device-planned tail);
- * packs holding an expert window always take it.  DENSE is the dense-batched comparison variant (pack created with
+ * normal number or zero, checked at pack time) as one launch, the
+ * device-planned tail (TAIL, when its plan fits: top_k <= 16, the pack built
+ * for at most 64 tokens), else as separate launches (DECODE_STAGED: route and
+ * plan, x gather, gate/up, down, combine), else the CUDA-core grouped
+ * kernels.  Packs holding an expert window always take the tail.  DENSE is the dense-batched comparison variant (pack created with
  * MOE_PACK_DENSE, n_tokens <= 64): every active expert multiplies the whole
  * batch, with a zero gate for the tokens not routed to it. */
 typedef enum {

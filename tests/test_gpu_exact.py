@@ -44,7 +44,7 @@ def _bitwise(li, x, path=None, max_tokens=None, h_max=2048):
 @pytest.mark.parametrize("fmt_gu,fmt_dn", PAIRS)
 @pytest.mark.parametrize("T", [1, 5, 64])
 def test_decode_default_path_is_bitwise_exact(fmt_gu, fmt_dn, T):
-    """One token: the single-token streaming kernel; 2-64: the tensor-core grouped decode."""
+    """One token: the single-token streaming kernel; 2-64: the one-launch tail."""
     li = exact_layer(fmt_gu, fmt_dn, seed=10 * fmt_gu + fmt_dn)
     info = _bitwise(li, exact_tokens(li, T, seed=T))
     if synth.FMT_IQ4_NL in (fmt_gu, fmt_dn):

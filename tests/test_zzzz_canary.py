@@ -34,7 +34,9 @@ def _sentinels_intact(full, pad, sentinel):
 @pytest.mark.parametrize("name,T,path,flags", [
     ("tiny_q8", 1, "auto", 0),          # single-token streaming kernel
     ("model_decode", 1, "auto", 0),     # single-token streaming kernel, shared expert
-    ("spec_verify", 8, "auto", 0),      # router + tensor-core grouped decode + combine
+    ("spec_verify", 8, "auto", 0),      # the one-launch tail (route, plan, tensor-core units, combine)
+    ("zipf_batch", 64, "auto", 0),      # the one-launch tail at its largest token count
+    ("spec_verify", 8, "staged", 0),    # router + tensor-core grouped decode + combine as separate launches
     ("tiny_q8", 5, "grouped", 0),       # plain grouped kernels
     ("zipf_batch", 16, "dense", 1),     # dense-batched comparison variant
     ("prefill_nvfp4", 300, "auto", 0),  # tensor-core prefill (output accumulated in place)
@@ -49,7 +51,8 @@ def test_forward_writes_exactly_its_rows(name, T, path, flags):
     pack = bq.pack_layer(li, max_tokens=T, max_top_k=wl.top_k, flags=flags)
     try:
         full, out, pad = _padded(T, wl.hidden, torch.float32, float("nan"), -7.0)
-        p = {"auto": bq.MOE_PATH_AUTO, "grouped": bq.MOE_PATH_GROUPED, "dense": bq.MOE_PATH_DENSE}[path]
+        p = {"auto": bq.MOE_PATH_AUTO, "grouped": bq.MOE_PATH_GROUPED, "dense": bq.MOE_PATH_DENSE,
+             "staged": bq.MOE_PATH_DECODE_STAGED}[path]
         bq.moe_layer_forward_ex(x, wr, pack, bq.MOE_FMT_FROM_PACK, wl.top_k, out, p)
         torch.cuda.synchronize()
         assert bq.moe_get_device_error(pack) == bq.MOE_OK
