@@ -1098,9 +1098,11 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                     tc_fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acce_bar[ab]);
-                    __threadfence();
+                    // the four warps' piece stores, then one release by the leader (the
+                    // named barrier orders them before its fence)
                     epi_sync();
                     if (r == 0) {
+                        __threadfence();
                         const unsigned prev = atomicAdd(a.ctr + (p == 0 ? C.gu_tile : C.dn_tile) + x.tile, 1u);
                         s_misc[3] = prev + 1 == (unsigned)owners(t0u, q.KC[p], q.U[p], G);
                         __threadfence();
@@ -1117,25 +1119,55 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                 // acquire of the group's (full) readiness count orders their reads
                 if (p == 0) (void)ld_acq(a.ctr + C.grp_x + x.g);
                 for (int c0 = 0; c0 < n16; ++c0) {
-                    float v0[16], v1[16];
+                    float v0[16], v1[16], ssc[16];
+                    if (p == 0) {  // the slots' scales, requested with the pieces
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) ssc[j] = c0 * 16 + j < n ? __ldcg(a.slot_scale + off + c0 * 16 + j) : 0.f;
+                    }
                     if (whole) {
                         tmem_ld16(tb0 + c0 * 16, v0);
                         tmem_ld16(tb0 + 64 + c0 * 16, v1);
                     } else {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) v0[j] = v1[j] = 0.f;
-                        int prev = -1;
-                        for (int uu = t0u; uu < t0u + q.KC[p]; ++uu) {
-                            const int cu = cta_of(uu, q.U[p], G);
-                            if (cu == prev) continue;
-                            prev = cu;
-                            const float *ps = piece(a, q, p, cu, x.tile, G);
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                if (c0 * 16 + j < n) {
-                                    v0[j] += __ldcg(ps + (size_t)(c0 * 16 + j) * 256 + r);
-                                    v1[j] += __ldcg(ps + (size_t)(c0 * 16 + j) * 256 + 128 + r);
+                        // the owners of the tile's units in CTA order, two at a time: both
+                        // pieces requested before either is added (the sum keeps CTA order)
+                        int uu = t0u, prev = -1;
+                        auto next_owner = [&]() {
+                            while (uu < t0u + q.KC[p]) {
+                                const int cu = cta_of(uu++, q.U[p], G);
+                                if (cu != prev) {
+                                    prev = cu;
+                                    return cu;
                                 }
+                            }
+                            return -1;
+                        };
+                        for (int oa = next_owner(); oa >= 0; oa = next_owner()) {
+                            const int ob = next_owner();
+                            const float *pa = piece(a, q, p, oa, x.tile, G);
+                            const float *pb = ob >= 0 ? piece(a, q, p, ob, x.tile, G) : pa;
+                            float a0[16], a1[16], b0[16], b1[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const bool in = c0 * 16 + j < n;
+                                const size_t o = (size_t)(c0 * 16 + j) * 256 + r;
+                                a0[j] = in ? __ldcg(pa + o) : 0.f;
+                                a1[j] = in ? __ldcg(pa + o + 128) : 0.f;
+                                b0[j] = in && ob >= 0 ? __ldcg(pb + o) : 0.f;
+                                b1[j] = in && ob >= 0 ? __ldcg(pb + o + 128) : 0.f;
+                            }
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                v0[j] += a0[j];
+                                v1[j] += a1[j];
+                            }
+                            if (ob < 0) break;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                v0[j] += b0[j];
+                                v1[j] += b1[j];
+                            }
                         }
                     }
                     if (p == 0) {
@@ -1144,7 +1176,7 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                             const int jj = c0 * 16 + j;
                             if (jj < n) {
                                 const int slot = off + jj;
-                                const float sc = __ldcg(a.slot_scale + slot) * hts;
+                                const float sc = ssc[j] * hts;
                                 const float gv = v0[j] * sc, uv = v1[j] * sc;
                                 const float hv = gv / (1.f + expf(-gv)) * uv;
                                 range_ok = range_ok && fabsf(hv) <= 65504.f;
@@ -1168,9 +1200,9 @@ __global__ void __launch_bounds__(kTlThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acce_bar[ab]);
                 }
-                __threadfence();
                 epi_sync();
                 if (r == 0) {
+                    __threadfence();  // the four warps' h / y stores, released by the leader
                     if (p == 0) {
                         atomicAdd(a.ctr + C.grp_h + x.g, 1u);
                     } else {
