@@ -84,6 +84,8 @@ def _load():
     L.moe_debug_act_quant_nvfp4.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
     L.moe_debug_dequant_rows.restype = i32
     L.moe_debug_dequant_rows.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp]
+    L.moe_debug_tail_plan.restype = i32
+    L.moe_debug_tail_plan.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, i32, vp]
     L.moe_debug_fail_alloc_after.restype = i32
     L.moe_debug_fail_alloc_after.argtypes = [i32]
     L.moe_read_routing.restype = i32
@@ -279,6 +281,20 @@ def moe_debug_dequant_rows(pack, proj, slot, row0, nrows, kind, cols, stream=Non
     _check(lib.moe_debug_dequant_rows(pack.handle, proj, slot, row0, nrows, kind, out.data_ptr(), _stream_ptr(stream)),
            "moe_debug_dequant_rows")
     return out
+
+
+def moe_debug_tail_plan(n_tokens, max_tokens, hidden, n_experts, inter, top_k, x_dtype, fmt_gate_up, fmt_down,
+                        grid):
+    """Tests only (no device): the one-launch tail's shared-memory plan, a dict (fits False
+    when the tail does not take the shape)."""
+    out = (ctypes.c_int64 * 8)()
+    _check(lib.moe_debug_tail_plan(n_tokens, max_tokens, hidden, n_experts, inter, top_k, x_dtype, fmt_gate_up,
+                                   fmt_down, grid, out), "moe_debug_tail_plan")
+    keys = ("fits", "raw_stages", "b_slots", "raw_stage_bytes", "b_slot_bytes", "rings_bytes", "smem_bytes",
+            "a_stages")
+    d = dict(zip(keys, list(out)))
+    d["fits"] = bool(d["fits"])
+    return d
 
 
 def moe_route_workspace_bytes(n_tokens, n_experts):

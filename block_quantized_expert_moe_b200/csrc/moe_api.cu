@@ -1286,6 +1286,20 @@ moe_status moe_debug_dequant_rows(const moe_pack *p, int proj, int slot, int row
                                       static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_debug_tail_plan(int n_tokens, int max_tokens, int hidden, int n_experts, int inter, int top_k,
+                               moe_dtype x_dtype, moe_fmt fmt_gate_up, moe_fmt fmt_down, int grid, int64_t *out)
+{
+    if (!out || !valid_fmt(fmt_gate_up) || !valid_fmt(fmt_down) || (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16))
+        return MOE_ERR_INVALID_ARG;
+    TailPlanIn in{n_tokens, max_tokens, hidden, n_experts, inter, top_k, x_dtype, device_fmt(fmt_gate_up),
+                  device_fmt(fmt_down), grid};
+    TailLaunch L{};
+    const bool fits = tail_plan(in, &L);
+    const int64_t v[8] = {fits ? 1 : 0, L.nr, L.nb, L.raw_stride, L.bslot, L.rings, (int64_t)L.smem, L.na};
+    for (int i = 0; i < 8; ++i) out[i] = fits ? v[i] : 0;
+    return MOE_OK;
+}
+
 moe_status moe_get_device_error(const moe_pack *p)
 {
     if (!p) return MOE_ERR_INVALID_ARG;

@@ -376,6 +376,16 @@ moe_status moe_debug_act_quant_nvfp4(const void *x, moe_dtype x_dtype, int rows,
 moe_status moe_debug_dequant_rows(const moe_pack *pack, int proj, int slot, int row0, int nrows, int kind, void *out,
                                   void *stream);
 
+/* Diagnostic for tests of the one-launch tail's host planner; touches no
+ * device.  For a launch of n_tokens tokens on a pack built for max_tokens
+ * (device formats: a Q5_0 projection is planned as Q5_1) over `grid` CTAs,
+ * writes out[0..7] = {1 if the tail fits else 0, raw stages, B slots, bytes of
+ * a raw stage, bytes of a B slot, bytes of the rings region (the routing and
+ * planning scratch overlaid on it), dynamic shared memory per CTA, tensor-memory
+ * A stages}.  MOE_ERR_INVALID_ARG for a NULL out or an unknown format or dtype. */
+moe_status moe_debug_tail_plan(int n_tokens, int max_tokens, int hidden, int n_experts, int inter, int top_k,
+                               moe_dtype x_dtype, moe_fmt fmt_gate_up, moe_fmt fmt_down, int grid, int64_t *out);
+
 /* Sticky device-side error of the pack (synchronises its device), then clears it. */
 moe_status moe_get_device_error(const moe_pack *pack);
 
